@@ -1,0 +1,415 @@
+"""Benchmark of the TokenGate gated-prefill hot path on B200.
+
+One step = gate score (all N tokens) -> top-K select -> gather/compaction ->
+one token-gated decoder layer on the M kept rows, on the Qwen3-1.7B-shaped
+single-layer workload (N = 16384 tokens of which the last 64 are the question,
+d_model 2048, GQA 16/8 x 128, gate MLP 2048 -> 256 -> 1, K = 2000, bf16).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  Multi-GPU runs are independent replicas (one
+request per GPU, no collective on the data path): value = all tokens / the
+slowest rank's time.  `--impl reference` times the CPU oracle on the host
+cores instead (bounded sample per step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "gated-prefill tokens/s & TTFT ms at N=16K/128K; attention % bf16 peak"
+L2_FLUSH_BYTES = 256 << 20   # > the 126 MB L2
+
+
+# ----------------------------------------------------------------------------- helpers (host only)
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def workload_work(w, m):
+    """Algorithmic bytes / flops of each call of one step ('roofline')."""
+    n, dm, h, D, hq, hkv, dff = w.n, w.d_model, w.gate_hidden, w.head_dim, w.hq, w.hkv, w.d_ff
+    es = 2 if w.dtype == "bf16" else 4
+    qkv = (hq + 2 * hkv) * D
+    return {
+        "gate_score": {"bytes": n * dm * es + n * 1 + n * 4 + h * dm * es, "flops": 2 * n * dm * h},
+        "topk_select": {"bytes": n * 4 + n * 1 + m * 4},
+        "gather": {"bytes": 2 * m * dm * es + m * 4 * 5},
+        "attention": {"flops": 2 * D * hq * m * (m + 1)},
+        "linear_qkv": {"flops": 2 * m * dm * qkv},
+        "linear_o": {"flops": 2 * m * hq * D * dm},
+        "linear_gate_up_swiglu": {"flops": 2 * m * dm * 2 * dff},
+        "linear_down": {"flops": 2 * m * dff * dm},
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", gpu_id], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    import torch.distributed as dist
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws <= 1:
+        return 0, 1, None
+    rank = int(os.environ["RANK"])
+    import datetime
+    import torch
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if backend == "nccl":
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, ws, dist
+
+
+def max_over_ranks(x: float, dist, device=None) -> float:
+    """Largest value of x over all ranks (host float in, host float out)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+
+def oracle_step_seconds(w, gate_rows: int = 2048):
+    """Time the oracle on a bounded sample of one step and scale it to the whole step.
+
+    Sample: gate scores of `gate_rows` tokens (scaled by N / gate_rows), the
+    selector on all N scores, the gather and the decoder layer on all M kept
+    rows.  Returns (seconds per full step, description, threads).
+    """
+    from oracle import tokengate_oracle as O
+    from learned_token_pruning_b200 import synth
+    gate = synth.gate_inputs(w)
+    layer = synth.layer_weights(w)
+    hp = synth.head_params(w)
+    t0 = time.perf_counter()
+    s_part = O.gate_scores(gate["hidden"][:gate_rows], gate["norm_w"], 1e-6, gate["w1"], gate["b1"], gate["w2"],
+                           gate["b2"], gate["prunable"][:gate_rows])
+    t_gate = (time.perf_counter() - t0) * (w.n / gate_rows)
+    # full score array for the selector: sampled rows plus the rest drawn from their distribution
+    rng = np.random.default_rng(0)
+    s = rng.normal(float(np.mean(s_part)), float(np.std(s_part) + 1e-12), size=w.n)
+    s[:gate_rows] = s_part
+    s[gate["prunable"] == 0] = 0.0
+    s32 = s.astype(np.float32)
+    t0 = time.perf_counter()
+    idx = O.select_kept(s32, gate["prunable"], w.k)
+    g = O.gather(gate["hidden"], idx, s32, gate["prunable"], 1e-6)
+    t_sel = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.decoder_layer(g["hidden_kept"], layer, hq=w.hq, hkv=w.hkv, head_dim=w.head_dim, pos=g["pos"], bias=g["bias"],
+                    ratio=g["ratio"], head_gain=hp["head_gain"], head_temp=hp["head_temp"],
+                    rope_theta=w.rope_theta, qk_norm=w.qk_norm)
+    t_layer = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    desc = (f"oracle (numpy fp64): gate MLP on {gate_rows} of {w.n} tokens scaled x{w.n / gate_rows:g}, "
+            f"selector + gather on all {w.n}, decoder layer on all {idx.size} kept rows")
+    return t_gate + t_sel + t_layer, desc, threads
+
+
+def run_reference(args, w):
+    rank, world, dist = dist_setup()
+    if rank != 0:
+        return
+    times = []
+    desc, threads = "", 1
+    for i in range(args.warmup + args.steps):
+        sec, desc, threads = oracle_step_seconds(w)
+        if i >= args.warmup:
+            times.append(sec)
+    step_s = sum(times) / len(times)
+    value = w.n / step_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w, world),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(w, world):
+    return {"workload": w.name, "n_tokens": w.n, "question_tokens": w.n_question, "k_budget": w.k,
+            "kept_rows": w.m, "d_model": w.d_model, "heads": f"{w.hq}/{w.hkv}x{w.head_dim}",
+            "gate_mlp": f"{w.d_model}->{w.gate_hidden}->1", "d_ff": w.d_ff, "layers_above_gate": 1,
+            "parallelism": f"replicas x{world}", "l2": "flushed (256 MiB write) before every timed step"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, w):
+    import torch
+    from learned_token_pruning_b200 import pipeline, tokengate as tg
+
+    rank, world, dist = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
+    step = pipeline.GatedPrefillStep(w, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    m = step.m
+
+    def one_step():
+        step.run()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        one_step()
+    torch.cuda.synchronize(dev)
+    tg.tg_check_device_error()
+
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_id = visible.split(",")[dev.index].strip() if visible else str(dev.index)
+    sampler = ClockSampler(gpu_id) if rank == 0 else None
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        one_step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    wall = time.perf_counter() - t_wall
+    clocks = sampler.stop() if sampler else None
+    tg.tg_check_device_error()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_s = sum(step_ms) / 1e3
+    total_s = max_over_ranks(total_s, dist, dev)
+    ms_per_step = total_s * 1e3 / args.steps
+    value = world * w.n * args.steps / total_s
+
+    # ---- per-call breakdown (same inputs, each library call bracketed by events on the stream)
+    work = workload_work(w, m)
+    br = breakdown(step, w, args, stream, flush)
+    kernels = {}
+    for name, ms in br.items():
+        wk = work.get(name, {})
+        entry = {"us": ms * 1e3}
+        if "flops" in wk and name != "gate_score":
+            tf = wk["flops"] / (ms * 1e-3) / 1e12
+            entry.update({"tflops": tf, "frac_bf16_peak": tf / peaks["bf16_tflops"]})
+        if "bytes" in wk:
+            gbs = wk["bytes"] / (ms * 1e-3) / 1e9
+            entry.update({"gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"]})
+        if name == "gate_score":
+            entry["tflops"] = wk["flops"] / (ms * 1e-3) / 1e12
+        kernels[name] = entry
+    dom = max((k for k in kernels if k != "layer_total"), key=lambda k: kernels[k]["us"])
+    wk = work[dom]
+    if "flops" in wk and dom != "gate_score":
+        roof = {"kernel": dom, "bound": "tensor", "achieved": kernels[dom]["tflops"], "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": kernels[dom]["tflops"] / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": peaks["source"] + " (burst bf16)"}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["gbs"], "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": kernels[dom]["gbs"] / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": peaks["source"]}
+
+    # ---- end to end through the public API: pinned host inputs in, result back to the host
+    e2e = end_to_end(step, w, args, stream, flush, dist, dev, world)
+
+    launches_per_step = 11  # gate(1) + select(1) + gather(1) + layer(rmsnorm, qkv, rope, attn, o, rmsnorm, mlp-up, down)
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        sec, desc, threads = oracle_step_seconds(w)
+        cpu = {"value": w.n / sec, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) hidden, N(0,0.02) weights)",
+        "config": config_dict(w, world),
+        "ttft_ms": {"gated_layer_step": ms_per_step},
+        "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks, "wall_s": wall,
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def breakdown(step, w, args, stream, flush):
+    """Average duration (ms) of each library call of the step, on the step's own inputs."""
+    import torch
+    from learned_token_pruning_b200 import tokengate as tg
+    D, hq, hkv = w.head_dim, w.hq, w.hkv
+    m = step.m
+    dt = step.dt
+    qkv_w = (hq + 2 * hkv) * D
+    # layer intermediates in their own buffers (the layer call keeps them in its workspace)
+    xn = torch.randn(m, w.d_model, device=stream.device).to(dt)
+    qkv = torch.randn(m, qkv_w, device=stream.device).to(dt)
+    att = torch.empty(m, hq * D, dtype=dt, device=stream.device)
+    act = torch.empty(m, w.d_ff, dtype=dt, device=stream.device)
+    hres = torch.randn(m, w.d_model, device=stream.device).to(dt)
+    L = step.layer
+    calls = {
+        "gate_score": step.gate_score,
+        "topk_select": step.select,
+        "gather": step.gather,
+        "attention": lambda: tg.tg_gated_attention(qkv[:, :hq * D], qkv[:, hq * D:(hq + hkv) * D],
+                                                   qkv[:, (hq + hkv) * D:], D, step.bias, L["head_gain"],
+                                                   L["head_temp"], step.ratio, 1.0 / math.sqrt(D), att),
+        "linear_qkv": lambda: tg.tg_linear(xn, L["w_qkv"], qkv),
+        "linear_o": lambda: tg.tg_linear(att, L["w_o"], hres, tg.TG_EPI_RESIDUAL),
+        "linear_gate_up_swiglu": lambda: tg.tg_linear(xn, L["w_gate_up"], act, tg.TG_EPI_SWIGLU),
+        "linear_down": lambda: tg.tg_linear(act, L["w_down"], hres, tg.TG_EPI_RESIDUAL),
+        "layer_total": step.layer_above,
+    }
+    step.run()
+    torch.cuda.synchronize()
+    reps = max(5, min(args.steps, 50))
+    out = {}
+    for name, fn in calls.items():
+        fn()
+        ms = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms += a.elapsed_time(b)
+        out[name] = ms / reps
+    return out
+
+
+def end_to_end(step, w, args, stream, flush, dist, dev, world):
+    """Same metric through the public API with the inputs in pinned host memory:
+    every step copies the hidden states and the prunable mask in, runs the
+    four calls and copies the kept-row output back."""
+    import torch
+    h_host = step.hidden.cpu().pin_memory()
+    m_host = step.prunable.cpu().pin_memory()
+    out_host = torch.empty(step.hidden_kept.shape, dtype=step.hidden_kept.dtype).pin_memory()
+    steps = max(3, min(args.steps, 30))
+
+    def one():
+        step.hidden.copy_(h_host, non_blocking=True)
+        step.prunable.copy_(m_host, non_blocking=True)
+        step.run()
+        out_host.copy_(step.hidden_kept, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    barrier(dist, dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    sec = max_over_ranks(a.elapsed_time(b) / 1e3, dist, dev)
+    return {"value": world * w.n * steps / sec, "unit": "tokens/s",
+            "h2d_bytes_per_step": h_host.numel() * h_host.element_size() + m_host.numel(),
+            "d2h_bytes_per_step": out_host.numel() * out_host.element_size(), "steps": steps}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    from learned_token_pruning_b200 import synth
+    w = synth.qwen3_1p7b_16k()
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

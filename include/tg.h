@@ -1,0 +1,248 @@
+/*
+ * tg.h -- C ABI of the TokenGate pruned-prefill library (libtokengate.so).
+ *
+ * The library implements, as CUDA kernels for NVIDIA B200 (sm_100a), the
+ * inference hot path of TokenGate learned token pruning:
+ *
+ *   gate layer L:  score every prunable token with a small MLP  (tg_gate_score)
+ *                  keep the top-K document tokens + every question token
+ *                                                                (tg_topk_select)
+ *                  compact the kept rows in their original order (tg_gather)
+ *   layers > L:    token-gated causal GQA attention over the kept rows
+ *                                                                (tg_gated_attention)
+ *                  one whole decoder layer on the kept rows      (tg_pruned_prefill_layer)
+ *
+ * The method is described on the TokenGate pages; citations below name the
+ * page and its section:
+ *   [R] "TokenGate and T2Quant: a close reading" (MessageDaily blog)
+ *   [K] "Stanford-Berkeley TokenGate" explainer (kg.zhiyong.dev)
+ *   [M] MarkTechPost TokenGate article (farwalk translation)
+ *
+ * Conventions shared by every entry point
+ *   - Pointers marked "device" are caller-owned device memory on the current
+ *     CUDA device; the library never frees them.  Pointers marked "host" are
+ *     host memory.  Scratch memory, where an op needs any, is passed in as a
+ *     workspace (size from tg_workspace_bytes); the library allocates nothing.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call only enqueues work on it and returns without synchronising, except
+ *     tg_check_device_error.
+ *   - Matrices are row-major and contiguous unless a leading dimension (in
+ *     elements) is given.  bf16 operands and their leading dimensions must be
+ *     16-byte aligned (TG_ERR_ALIGN otherwise).
+ *   - Argument and shape errors are detected on the host before anything is
+ *     enqueued and return a status without touching the stream.  A failed
+ *     launch returns TG_ERR_CUDA.  Conditions only the device can see (a
+ *     prunable mask whose count disagrees with n_prunable, a bounded wait that
+ *     expired) set a sticky device error word instead of faulting; read it
+ *     with tg_check_device_error.
+ *   - tg_last_error() returns a human-readable detail string for the last
+ *     failing call on the calling host thread.
+ */
+#ifndef TG_H_
+#define TG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TG_OK = 0,
+  TG_ERR_INVALID_ARG = 1,     /* null pointer, negative size or budget, bad enum   */
+  TG_ERR_SHAPE = 2,           /* inconsistent sizes (e.g. m != min(k, np) + n - np) */
+  TG_ERR_ALIGN = 3,           /* pointer or leading dimension not 16-byte aligned   */
+  TG_ERR_UNSUPPORTED = 4,     /* valid but not implemented (e.g. head_dim 96)       */
+  TG_ERR_WORKSPACE = 5,       /* workspace missing or smaller than required         */
+  TG_ERR_CUDA = 6,            /* a CUDA runtime call or kernel launch failed        */
+  TG_ERR_DEVICE_TIMEOUT = 7,  /* a bounded device-side wait expired                 */
+  TG_ERR_DEVICE_CHECK = 8     /* a device-side consistency check failed             */
+} tg_status;
+
+typedef enum { TG_F32 = 0, TG_BF16 = 1 } tg_dtype;
+
+/* Static description of a status code. */
+const char* tg_status_string(int status);
+
+/* Detail text for the last failing call on this host thread ("" if none). */
+const char* tg_last_error(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  Returns TG_OK, TG_ERR_DEVICE_TIMEOUT, TG_ERR_DEVICE_CHECK or
+ * TG_ERR_CUDA (if the synchronisation itself failed).  `detail` (host, may be
+ * NULL) receives the raw word: bits 0-7 the failing site, bits 8-31 a payload.
+ */
+int tg_check_device_error(void* stream, uint32_t* detail);
+
+/*
+ * Gate scores ([R] §4.1 "Gate module"; [M] "how does learned token pruning
+ * work"): for every token j,
+ *     x_j = RMSNorm(h_j) * norm_w            (eps = norm_eps)
+ *     s_j = w2 . SiLU(W1 x_j + b1) + b2      if prunable[j]
+ *     s_j = 0                                otherwise (question tokens)
+ * and sumsq = sum over prunable j of s_j^2 (fp32, summed in a fixed order,
+ * so it is deterministic), used by tg_gather for the sequence-wise RMS norm.
+ *
+ *   hidden   device, dtype [n][d_model]   post-attention residual of layer L
+ *   norm_w   device, fp32 [d_model] or NULL (all ones)
+ *   w1       device, dtype [h][d_model]   (nn.Linear layout: one row per unit)
+ *   b1       device, fp32 [h] or NULL (zeros)
+ *   w2       device, fp32 [h]
+ *   prunable device, uint8 [n]            1 = document token, 0 = question token
+ *   scores   device, fp32 [n]  out
+ *   sumsq    device, fp32 [1]  out
+ *   ws       device workspace (16-byte aligned) of at least
+ *            tg_workspace_bytes(TG_OP_GATE_SCORE, n, 0, d_model, h, NULL)
+ *            bytes; its contents on entry do not matter.
+ * bf16 with d_model % 8 == 0 and h % 16 == 0, h <= 256 runs on the tcgen05
+ * tensor cores (a non-NULL norm_w is folded into W1 in bf16 first); other
+ * shapes and fp32 run on CUDA cores (h <= 1024) and do not use ws.
+ */
+int tg_gate_score(const void* hidden, int dtype, int64_t n, int32_t d_model,
+                  const float* norm_w, float norm_eps,
+                  const void* w1, const float* b1, const float* w2, float b2, int32_t h,
+                  const uint8_t* prunable, float* scores, float* sumsq,
+                  void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Masked top-K selection ([R] §4.1 "Top-K selector": S = top-K(b) U N).
+ * Keeps exactly k' = min(k, n_prunable) prunable tokens -- those with the
+ * largest score, where equal scores (and -0 == +0) are broken towards the
+ * lower index and NaN ranks below -inf -- plus every non-prunable token.
+ * The kept indices are written in ascending order, so the compacted sequence
+ * keeps the original causal order.  Integer-exact and deterministic.
+ *
+ *   scores     device, fp32 [n]   (selection is on the raw scores; the
+ *              sequence RMS norm is a positive scale and does not change it)
+ *   prunable   device, uint8 [n]
+ *   n_prunable number of nonzero entries of prunable (known to the caller from
+ *              the prompt layout; checked on the device, a mismatch sets the
+ *              device error word and the output is then unspecified but never
+ *              written past m entries)
+ *   k          budget, >= 0 (k >= n_prunable keeps everything)
+ *   kept_idx   device, int32 [m] out, m = min(k, n_prunable) + n - n_prunable
+ * Needs no workspace: the whole selection runs in one thread-block cluster.
+ */
+int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int64_t n_prunable,
+                   int64_t k, int32_t* kept_idx, int64_t m, void* stream);
+
+/*
+ * Compaction of the kept rows ([R] §4.1 three-stage forward: pruned tokens
+ * never enter the layers above L) plus the per-row inputs of gated attention:
+ *     hidden_kept[r] = hidden[kept_idx[r]]            (bit-exact copy)
+ *     pos[r]         = kept_idx[r]                    (original position)
+ *     bias[r]        = s[kept_idx[r]] / rms           (importance b_j, [R] §4.1;
+ *                      rms = sqrt(sumsq / n_prunable + seq_eps); 0 for question tokens)
+ *     ratio[r]       = log(r + 1) / log(max(2, kept_idx[r] + 1))
+ *                      (the log m_i / log max(2, p_i) factor of the temperature,
+ *                       [R] §4.1 "temperature scaling")
+ *   hidden      device, dtype [n][d_model];  hidden_kept device, dtype [m][d_model] out
+ *   kept_idx    device, int32 [m], ascending, values in [0, n)
+ *   scores      device, fp32 [n];  sumsq device, fp32 [1] (from tg_gate_score)
+ *   pos/bias/ratio  device, int32/fp32/fp32 [m] out (any may be NULL to skip)
+ */
+int tg_gather(const void* hidden, int dtype, int64_t n, int32_t d_model,
+              const int32_t* kept_idx, int64_t m,
+              const float* scores, const float* sumsq, int64_t n_prunable, float seq_eps,
+              void* hidden_kept, int32_t* pos, float* bias, float* ratio, void* stream);
+
+/*
+ * Token-gated causal GQA attention over the m kept rows ([R] §4.1 "token-gated
+ * attention", "head-wise gain", "temperature scaling"; [K]; [M]).  For query
+ * head h, KV head g = h / (hq / hkv), kept row r and key c <= r:
+ *     l_rc = head_temp[h] * ratio[r] * sm_scale * (q_r . k_c) + head_gain[h] * bias[c]
+ *     out_r = sum_c softmax_c(l_r.) v_c
+ * (the gate value g_j = softmax(b_j) multiplies exp(z_ij) in the attention
+ * weights, which is the same as adding b_j to the logits; the gain acts on
+ * that log-space term; the temperature rescales the content logit).
+ *
+ *   q    device, dtype, row r of head h at q + r*ldq + h*head_dim
+ *   k, v device, dtype, row r of KV head g at k + r*ldk + g*head_dim (same for v/ldv)
+ *   out  device, dtype, row r of head h at out + r*ldo + h*head_dim
+ *   bias device fp32 [m] or NULL (0);  ratio device fp32 [m] or NULL (1)
+ *   head_gain, head_temp  device fp32 [hq] (values after softplus)
+ *   lse  device fp32 [hq][m] out (natural-log sum of exp of l) or NULL
+ * head_dim in {64, 128}; hq % hkv == 0.  bf16 runs on the tcgen05 tensor cores
+ * (fp32 softmax and accumulation); fp32 runs on CUDA cores in full fp32.
+ */
+int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk,
+                       const void* v, int64_t ldv, int dtype, int64_t m,
+                       int32_t hq, int32_t hkv, int32_t head_dim,
+                       const float* bias, const float* head_gain, const float* head_temp,
+                       const float* ratio, float sm_scale,
+                       void* out, int64_t ldo, float* lse, void* stream);
+
+/* Weights of one Qwen3-style decoder layer (device pointers). */
+typedef struct {
+  const float* w_in_norm;    /* fp32 [d_model]                                  */
+  const void* w_qkv;         /* dtype [(hq + 2*hkv)*head_dim][d_model]: q rows, then k, then v */
+  const float* w_q_norm;     /* fp32 [head_dim] (used when qk_norm != 0)        */
+  const float* w_k_norm;     /* fp32 [head_dim] (used when qk_norm != 0)        */
+  const void* w_o;           /* dtype [d_model][hq*head_dim]                    */
+  const float* w_post_norm;  /* fp32 [d_model]                                  */
+  const void* w_gate_up;     /* dtype [2*d_ff][d_model]: gate rows, then up rows */
+  const void* w_down;        /* dtype [d_model][d_ff]                           */
+  const float* head_gain;    /* fp32 [hq]  softplus(gamma), per head            */
+  const float* head_temp;    /* fp32 [hq]  softplus(sigma), per head            */
+} tg_layer_weights;
+
+typedef struct {
+  int32_t dtype;             /* TG_F32 or TG_BF16 */
+  int32_t d_model, hq, hkv, head_dim, d_ff;
+  int32_t qk_norm;           /* per-head RMSNorm of q and k before RoPE (Qwen3) */
+  float rope_theta;          /* rotate-half RoPE base */
+  float norm_eps;            /* RMSNorm epsilon */
+} tg_layer_shape;
+
+/*
+ * One decoder layer above the gate, run on the m kept rows only ([R] §4.1
+ * three-stage forward; [M]: the layers above L process only the kept tokens
+ * and never create KV for pruned ones):
+ *   x = RMSNorm(h) ; q,k,v = x Wqkv^T ; (q,k per-head RMSNorm) ;
+ *   RoPE(q,k) at the ORIGINAL positions pos ; a = gated attention (see above,
+ *   sm_scale = 1/sqrt(head_dim)) ; h += a Wo^T ; y = RMSNorm(h) ;
+ *   h += (SiLU(y Wg^T) * (y Wu^T)) Wd^T
+ * Intermediates are rounded to the layer dtype between steps.
+ *   hidden_kept device dtype [m][d_model], updated in place
+ *   pos  device int32 [m];  bias/ratio device fp32 [m] or NULL (0 / 1)
+ *   ws   device workspace of tg_workspace_bytes(TG_OP_LAYER, 0, m, 0, 0, shape) bytes
+ * With bias = NULL, ratio = NULL and pos = 0..m-1 this is the plain unpruned
+ * layer (used for the layers below the gate).
+ */
+int tg_pruned_prefill_layer(const tg_layer_weights* weights, const tg_layer_shape* shape,
+                            void* hidden_kept, const int32_t* pos, const float* bias,
+                            const float* ratio, int64_t m, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Row-wise linear layer of the decoder layer above, exported so that each of
+ * its GEMMs can be called (and timed) on its own:
+ *   epilogue TG_EPI_STORE     y = x W^T
+ *   epilogue TG_EPI_RESIDUAL  y = y + x W^T          (y holds the residual on entry)
+ *   epilogue TG_EPI_SWIGLU    y = SiLU(x Wg^T) * (x Wu^T), where W is [2*n_out][k_in]
+ *                             with the gate rows first and the up rows after them
+ *   x device dtype, row r at x + r*ldx, k_in columns
+ *   w device dtype [n_out or 2*n_out][k_in] (nn.Linear layout)
+ *   y device dtype, row r at y + r*ldy, n_out columns
+ * bf16 runs on the tcgen05 tensor cores (k_in % 8 == 0; n_out % 32 == 0, or
+ * n_out % 128 == 0 for SwiGLU); fp32 and other bf16 shapes run on CUDA cores,
+ * where SwiGLU is not offered (TG_ERR_UNSUPPORTED).
+ */
+enum { TG_EPI_STORE = 0, TG_EPI_RESIDUAL = 1, TG_EPI_SWIGLU = 2 };
+int tg_linear(const void* x, int64_t ldx, const void* w, void* y, int64_t ldy, int dtype,
+              int64_t m, int32_t n_out, int32_t k_in, int epilogue, void* stream);
+
+enum { TG_OP_GATE_SCORE = 0, TG_OP_LAYER = 1 };
+
+/* Workspace bytes needed by an op: TG_OP_GATE_SCORE uses n, d_model and h;
+ * TG_OP_LAYER uses m and shape.  Returns 0 for an invalid request. */
+size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t h, const tg_layer_shape* shape);
+
+/* Library version string. */
+const char* tg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TG_H_ */

@@ -1,0 +1,535 @@
+// TokenGate pruned-prefill library: the C ABI declared in include/tg.h.
+//
+// Host code validates every argument before anything is enqueued, builds TMA
+// descriptors for the tensor-core kernels and launches the kernels on the
+// caller's stream.  Nothing here allocates device memory or synchronises,
+// except tg_check_device_error.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/tg.h"
+#include "attn_tc.cuh"
+#include "common.cuh"
+#include "gather.cuh"
+#include "gemm_tc.cuh"
+#include "select.cuh"
+#include "simt.cuh"
+
+#define TG_VERSION "tokengate-b200 0.1.0"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return status;
+}
+
+int check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(TG_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return TG_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// ---------------------------------------------------------------------------
+// TMA descriptor encoding through the driver entry point (no -lcuda needed).
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][inner] with a row stride in bytes; box {64, box_rows}, 128-byte swizzle.
+int make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride_bytes,
+             uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(TG_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return TG_OK;
+}
+
+template <typename Kern>
+int set_smem(Kern k, size_t bytes) {
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e != cudaSuccess) return fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+  return TG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05 GEMM launch
+// ---------------------------------------------------------------------------
+constexpr int kGemmStages = 4;
+
+template <int BN, int EPI>
+int launch_gemm_tc(const void* A, int64_t lda, const void* B, int64_t b_rows, int M, int K, const tg::GemmParams& p0,
+                   int grid_n, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  int rc = make_map(&ta, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(lda) * 2, 128);
+  if (rc) return rc;
+  rc = make_map(&tb, B, static_cast<uint64_t>(K), static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K) * 2,
+                tg::GemmCfg<BN>::kBBox);
+  if (rc) return rc;
+  auto kern = tg::k_gemm_tc<BN, kGemmStages, EPI>;
+  const size_t smem = tg::gemm_smem_bytes<BN, kGemmStages>();
+  rc = set_smem(kern, smem);
+  if (rc) return rc;
+  tg::GemmParams p = p0;
+  p.M = M;
+  p.K = K;
+  dim3 grid(grid_n, (M + tg::kGemmBM - 1) / tg::kGemmBM);
+  kern<<<grid, tg::kGemmThreads, smem, st>>>(ta, tb, p);
+  return check_launch("k_gemm_tc");
+}
+
+int dtype_size(int dtype) { return dtype == TG_BF16 ? 2 : (dtype == TG_F32 ? 4 : 0); }
+
+// workspace layout of tg_gate_score (256-byte aligned pieces):
+//   [per-CTA partial sums of s^2][completion counter][W1 scaled by the norm weight, bf16 [h][d]]
+size_t gate_partials_bytes(int64_t n) { return ((static_cast<size_t>((n + 127) / 128) * 4 + 255) / 256) * 256; }
+size_t gate_ws_bytes(int64_t n, int32_t d, int32_t h) {
+  return gate_partials_bytes(n) + 256 + ((static_cast<size_t>(d) * h * 2 + 255) / 256) * 256;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tg_version(void) { return TG_VERSION; }
+
+const char* tg_status_string(int status) {
+  switch (status) {
+    case TG_OK: return "ok";
+    case TG_ERR_INVALID_ARG: return "invalid argument";
+    case TG_ERR_SHAPE: return "inconsistent shape";
+    case TG_ERR_ALIGN: return "misaligned pointer or leading dimension";
+    case TG_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TG_ERR_WORKSPACE: return "workspace missing or too small";
+    case TG_ERR_CUDA: return "CUDA error";
+    case TG_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case TG_ERR_DEVICE_CHECK: return "device-side consistency check failed";
+    default: return "unknown status";
+  }
+}
+
+const char* tg_last_error(void) { return g_last_error; }
+
+int tg_check_device_error(void* stream, uint32_t* detail) {
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return fail(TG_ERR_CUDA, "stream synchronize: %s", cudaGetErrorString(e));
+  uint32_t word = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&word, tg::g_error_word, sizeof(word));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(tg::g_error_word, &zero, sizeof(zero));
+  if (e != cudaSuccess) return fail(TG_ERR_CUDA, "error word: %s", cudaGetErrorString(e));
+  if (detail) *detail = word;
+  if (word == 0) return TG_OK;
+  const uint32_t site = word & 0xffu;
+  if (site >= tg::kErrTimeoutFirst && site <= tg::kErrTimeoutLast)
+    return fail(TG_ERR_DEVICE_TIMEOUT, "device wait timed out at site %u", site);
+  return fail(TG_ERR_DEVICE_CHECK, "device check failed at site %u (payload %u)", site, word >> 8);
+}
+
+size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t h, const tg_layer_shape* shape) {
+  if (op == TG_OP_GATE_SCORE) return (n > 0 && d_model > 0 && h > 0) ? gate_ws_bytes(n, d_model, h) : 0;
+  if (op == TG_OP_LAYER) {
+    if (!shape || m <= 0) return 0;
+    const int es = dtype_size(shape->dtype);
+    if (!es) return 0;
+    const size_t qkv = static_cast<size_t>(shape->hq + 2 * shape->hkv) * shape->head_dim;
+    const size_t rows = static_cast<size_t>(m);
+    auto al = [](size_t b) { return (b + 255) / 256 * 256; };
+    // x (normed rows), qkv, attention output, MLP activation (room for the
+    // un-fused gate/up product, twice as wide as the fused SwiGLU output)
+    const size_t act = static_cast<size_t>(shape->d_ff) * 2;
+    return al(rows * shape->d_model * es) + al(rows * qkv * es) + al(rows * shape->hq * shape->head_dim * es) +
+           al(rows * act * es);
+  }
+  return 0;
+}
+
+int tg_gate_score(const void* hidden, int dtype, int64_t n, int32_t d_model, const float* norm_w, float norm_eps,
+                  const void* w1, const float* b1, const float* w2, float b2, int32_t h, const uint8_t* prunable,
+                  float* scores, float* sumsq, void* ws, size_t ws_bytes, void* stream) {
+  if (!hidden || !w1 || !w2 || !prunable || !scores || !sumsq) return fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (n <= 0 || d_model <= 0 || h <= 0) return fail(TG_ERR_INVALID_ARG, "n, d_model and h must be positive");
+  if (n >= (int64_t(1) << 31)) return fail(TG_ERR_UNSUPPORTED, "n must be < 2^31");
+  if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "dtype");
+  cudaStream_t st = as_stream(stream);
+  const bool tc = dtype == TG_BF16 && d_model % 8 == 0 && h <= 256 && h % 16 == 0 && aligned16(hidden) &&
+                  aligned16(w1);
+  if (tc) {
+    const size_t need = gate_ws_bytes(n, d_model, h);
+    if (!ws || ws_bytes < need) return fail(TG_ERR_WORKSPACE, "gate score needs %zu workspace bytes", need);
+    if (!aligned16(ws)) return fail(TG_ERR_ALIGN, "workspace must be 16-byte aligned");
+    float* partials = static_cast<float*>(ws);
+    uint32_t* counter = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + gate_partials_bytes(n));
+    cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(uint32_t), st);
+    if (e != cudaSuccess) return fail(TG_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+    const void* w1_eff = w1;
+    if (norm_w) {
+      // RMSNorm(h) * w_n feeds W1, so (h * w_n) W1^T = h (W1 diag(w_n))^T: fold the weight into W1
+      __nv_bfloat16* w1f = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + gate_partials_bytes(n) + 256);
+      const int64_t total = int64_t(h) * d_model;
+      tg::k_fold_norm<<<unsigned((total + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w1), norm_w,
+                                                                   w1f, total, d_model);
+      int rc = check_launch("k_fold_norm");
+      if (rc) return rc;
+      w1_eff = w1f;
+    }
+    tg::GemmParams p{};
+    p.N = h;
+    p.b1 = b1;
+    p.w2 = w2;
+    p.b2 = b2;
+    p.norm_eps = norm_eps;
+    p.prunable = prunable;
+    p.scores = scores;
+    p.partials = partials;
+    p.counter = counter;
+    p.sumsq = sumsq;
+    const int nn = static_cast<int>(n);
+    if (h <= 64) return launch_gemm_tc<64, tg::kEpiGateScore>(hidden, d_model, w1_eff, h, nn, d_model, p, 1, st);
+    if (h <= 128) return launch_gemm_tc<128, tg::kEpiGateScore>(hidden, d_model, w1_eff, h, nn, d_model, p, 1, st);
+    return launch_gemm_tc<256, tg::kEpiGateScore>(hidden, d_model, w1_eff, h, nn, d_model, p, 1, st);
+  }
+  if (h > 1024) return fail(TG_ERR_UNSUPPORTED, "h > 1024");
+  const unsigned blocks = static_cast<unsigned>((n + 7) / 8);
+  if (dtype == TG_F32)
+    tg::k_gate_score_simt<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(hidden), n, d_model, norm_w,
+                                                          norm_eps, static_cast<const float*>(w1), b1, w2, b2, h,
+                                                          prunable, scores);
+  else
+    tg::k_gate_score_simt<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(hidden), n, d_model, norm_w, norm_eps,
+        static_cast<const __nv_bfloat16*>(w1), b1, w2, b2, h, prunable, scores);
+  int rc = check_launch("k_gate_score_simt");
+  if (rc) return rc;
+  tg::k_sumsq_ordered<<<1, 1024, 0, st>>>(scores, prunable, n, sumsq);
+  return check_launch("k_sumsq_ordered");
+}
+
+int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int64_t n_prunable, int64_t k,
+                   int32_t* kept_idx, int64_t m, void* stream) {
+  if (!scores || !prunable || !kept_idx) return fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (n <= 0 || n_prunable < 0 || n_prunable > n) return fail(TG_ERR_INVALID_ARG, "bad n / n_prunable");
+  if (k < 0) return fail(TG_ERR_INVALID_ARG, "k must be >= 0");
+  if (n >= (int64_t(1) << 31)) return fail(TG_ERR_UNSUPPORTED, "n must be < 2^31");
+  const int64_t want = (k < n_prunable ? k : n_prunable) + (n - n_prunable);
+  if (m != want) return fail(TG_ERR_SHAPE, "m = %lld but min(k, n_prunable) + n - n_prunable = %lld",
+                             static_cast<long long>(m), static_cast<long long>(want));
+  tg::SelectParams p{};
+  p.scores = scores;
+  p.prunable = prunable;
+  p.n = n;
+  p.n_prunable = n_prunable;
+  p.k = k;
+  p.out = kept_idx;
+  p.m = m;
+  p.slice = (n + tg::kSelCluster - 1) / tg::kSelCluster;
+  const size_t cache = static_cast<size_t>(p.slice) * 5;
+  p.cached = cache <= tg::kSelCacheBytes ? 1 : 0;
+  const size_t smem = p.cached ? ((cache + 15) / 16) * 16 : 0;
+  int rc = set_smem(tg::k_topk_select, smem > 0 ? smem : 16);
+  if (rc) return rc;
+  tg::k_topk_select<<<tg::kSelCluster, tg::kSelThreads, smem, as_stream(stream)>>>(p);
+  return check_launch("k_topk_select");
+}
+
+int tg_gather(const void* hidden, int dtype, int64_t n, int32_t d_model, const int32_t* kept_idx, int64_t m,
+              const float* scores, const float* sumsq, int64_t n_prunable, float seq_eps, void* hidden_kept,
+              int32_t* pos, float* bias, float* ratio, void* stream) {
+  if (!hidden || !kept_idx || !hidden_kept) return fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (bias && (!scores || !sumsq)) return fail(TG_ERR_INVALID_ARG, "bias needs scores and sumsq");
+  if (n <= 0 || m <= 0 || m > n || d_model <= 0) return fail(TG_ERR_INVALID_ARG, "bad sizes");
+  if (bias && n_prunable <= 0) return fail(TG_ERR_INVALID_ARG, "n_prunable must be > 0 for bias");
+  const int es = dtype_size(dtype);
+  if (!es) return fail(TG_ERR_INVALID_ARG, "dtype");
+  const int64_t row_bytes = static_cast<int64_t>(d_model) * es;
+  if (row_bytes % 16 != 0 || !aligned16(hidden) || !aligned16(hidden_kept))
+    return fail(TG_ERR_ALIGN, "rows must be 16-byte multiples on 16-byte aligned buffers");
+  tg::GatherParams p{};
+  p.hidden = static_cast<const uint8_t*>(hidden);
+  p.n = n;
+  p.row_bytes = row_bytes;
+  p.idx = kept_idx;
+  p.m = m;
+  p.scores = scores;
+  p.sumsq = sumsq;
+  p.n_prunable = n_prunable;
+  p.eps = seq_eps;
+  p.out = static_cast<uint8_t*>(hidden_kept);
+  p.pos = pos;
+  p.bias = bias;
+  p.ratio = ratio;
+  const unsigned blocks = static_cast<unsigned>((m + tg::kGatherRows - 1) / tg::kGatherRows);
+  tg::k_gather<<<blocks, tg::kGatherThreads, 0, as_stream(stream)>>>(p);
+  return check_launch("k_gather");
+}
+
+int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk, const void* v, int64_t ldv, int dtype,
+                       int64_t m, int32_t hq, int32_t hkv, int32_t head_dim, const float* bias,
+                       const float* head_gain, const float* head_temp, const float* ratio, float sm_scale, void* out,
+                       int64_t ldo, float* lse, void* stream) {
+  if (!q || !k || !v || !out || !head_gain || !head_temp) return fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (m <= 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0) return fail(TG_ERR_INVALID_ARG, "bad m / heads");
+  if (m >= (int64_t(1) << 31)) return fail(TG_ERR_UNSUPPORTED, "m must be < 2^31");
+  if (head_dim != 64 && head_dim != 128) return fail(TG_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (ldq < int64_t(hq) * head_dim || ldk < int64_t(hkv) * head_dim || ldv < int64_t(hkv) * head_dim ||
+      ldo < int64_t(hq) * head_dim)
+    return fail(TG_ERR_SHAPE, "leading dimension smaller than the heads it holds");
+  if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "dtype");
+  cudaStream_t st = as_stream(stream);
+  const int group = hq / hkv;
+  if (dtype == TG_BF16) {
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || ldq % 8 || ldk % 8 || ldv % 8 ||
+        ldo % 8)
+      return fail(TG_ERR_ALIGN, "bf16 attention operands need 16-byte alignment");
+  }
+  if (dtype == TG_BF16 && group % 2 == 0) {
+    tg::AttnTcParams p{};
+    p.m = static_cast<int>(m);
+    p.hq = hq;
+    p.hkv = hkv;
+    p.group = group;
+    p.num_qtiles = static_cast<int>((m + 127) / 128);
+    p.bias = bias;
+    p.gain = head_gain;
+    p.temp = head_temp;
+    p.ratio = ratio;
+    p.scale_log2 = sm_scale * 1.4426950408889634f;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.ldo = ldo;
+    p.lse = lse;
+    CUtensorMap tq, tk, tv;
+    int rc = make_map(&tq, q, uint64_t(hq) * head_dim, uint64_t(m), uint64_t(ldq) * 2, 128);
+    if (!rc) rc = make_map(&tk, k, uint64_t(hkv) * head_dim, uint64_t(m), uint64_t(ldk) * 2, 128);
+    if (!rc) rc = make_map(&tv, v, uint64_t(hkv) * head_dim, uint64_t(m), uint64_t(ldv) * 2, 128);
+    if (rc) return rc;
+    const unsigned blocks = static_cast<unsigned>(p.num_qtiles * hkv * (group / 2));
+    if (head_dim == 128) {
+      rc = set_smem(tg::k_attn_tc<128>, tg::AttnCfg<128>::kSmem);
+      if (rc) return rc;
+      tg::k_attn_tc<128><<<blocks, tg::kAttnThreads, tg::AttnCfg<128>::kSmem, st>>>(tq, tk, tv, p);
+    } else {
+      rc = set_smem(tg::k_attn_tc<64>, tg::AttnCfg<64>::kSmem);
+      if (rc) return rc;
+      tg::k_attn_tc<64><<<blocks, tg::kAttnThreads, tg::AttnCfg<64>::kSmem, st>>>(tq, tk, tv, p);
+    }
+    return check_launch("k_attn_tc");
+  }
+  tg::AttnSimtParams p{};
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.ldq = ldq;
+  p.ldk = ldk;
+  p.ldv = ldv;
+  p.ldo = ldo;
+  p.m = static_cast<int>(m);
+  p.hq = hq;
+  p.hkv = hkv;
+  p.bias = bias;
+  p.gain = head_gain;
+  p.temp = head_temp;
+  p.ratio = ratio;
+  p.sm_scale = sm_scale;
+  p.out = out;
+  p.lse = lse;
+  dim3 grid(static_cast<unsigned>((m + 15) / 16), static_cast<unsigned>(hq));
+  if (dtype == TG_F32) {
+    if (head_dim == 128) tg::k_attn_simt<float, 128><<<grid, 128, 0, st>>>(p);
+    else tg::k_attn_simt<float, 64><<<grid, 128, 0, st>>>(p);
+  } else {
+    if (head_dim == 128) tg::k_attn_simt<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(p);
+    else tg::k_attn_simt<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(p);
+  }
+  return check_launch("k_attn_simt");
+}
+
+int tg_linear(const void* x, int64_t ldx, const void* w, void* y, int64_t ldy, int dtype, int64_t m, int32_t n_out,
+              int32_t k_in, int epilogue, void* stream) {
+  if (!x || !w || !y) return fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (m <= 0 || n_out <= 0 || k_in <= 0 || ldx < k_in || ldy < n_out) return fail(TG_ERR_INVALID_ARG, "bad sizes");
+  if (epilogue < TG_EPI_STORE || epilogue > TG_EPI_SWIGLU) return fail(TG_ERR_INVALID_ARG, "epilogue");
+  if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "dtype");
+  if (m >= (int64_t(1) << 31)) return fail(TG_ERR_UNSUPPORTED, "m must be < 2^31");
+  cudaStream_t st = as_stream(stream);
+  const int mm = static_cast<int>(m);
+  if (dtype == TG_BF16) {
+    if (!aligned16(x) || !aligned16(w) || !aligned16(y) || ldx % 8 || ldy % 8 || k_in % 8)
+      return fail(TG_ERR_ALIGN, "bf16 linear operands need 16-byte alignment");
+    tg::GemmParams p{};
+    p.N = n_out;
+    p.out = static_cast<__nv_bfloat16*>(y);
+    p.ldo = ldy;
+    if (epilogue == TG_EPI_SWIGLU) {
+      if (n_out % 128 != 0) return fail(TG_ERR_UNSUPPORTED, "SwiGLU epilogue needs n_out %% 128 == 0");
+      p.up_row0 = n_out;
+      return launch_gemm_tc<256, tg::kEpiSwiGLU>(x, ldx, w, 2 * int64_t(n_out), mm, k_in, p, n_out / 128, st);
+    }
+    if (n_out % 32 == 0) {
+      const int gn = (n_out + 255) / 256;
+      if (epilogue == TG_EPI_RESIDUAL)
+        return launch_gemm_tc<256, tg::kEpiResidual>(x, ldx, w, n_out, mm, k_in, p, gn, st);
+      return launch_gemm_tc<256, tg::kEpiStore>(x, ldx, w, n_out, mm, k_in, p, gn, st);
+    }
+  }
+  if (epilogue == TG_EPI_SWIGLU) return fail(TG_ERR_UNSUPPORTED, "SwiGLU epilogue needs bf16");
+  const bool res = epilogue == TG_EPI_RESIDUAL;
+  dim3 grid(static_cast<unsigned>((n_out + 63) / 64), static_cast<unsigned>((m + 63) / 64));
+  if (dtype == TG_F32) {
+    const float* xa = static_cast<const float*>(x);
+    const float* wa = static_cast<const float*>(w);
+    float* ya = static_cast<float*>(y);
+    if (res) tg::k_gemm_simt<float, true><<<grid, 256, 0, st>>>(xa, ldx, wa, ya, ldy, mm, n_out, k_in);
+    else tg::k_gemm_simt<float, false><<<grid, 256, 0, st>>>(xa, ldx, wa, ya, ldy, mm, n_out, k_in);
+  } else {
+    using B = __nv_bfloat16;
+    const B* xa = static_cast<const B*>(x);
+    const B* wa = static_cast<const B*>(w);
+    B* ya = static_cast<B*>(y);
+    if (res) tg::k_gemm_simt<B, true><<<grid, 256, 0, st>>>(xa, ldx, wa, ya, ldy, mm, n_out, k_in);
+    else tg::k_gemm_simt<B, false><<<grid, 256, 0, st>>>(xa, ldx, wa, ya, ldy, mm, n_out, k_in);
+  }
+  return check_launch("k_gemm_simt");
+}
+
+int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden_kept,
+                            const int32_t* pos, const float* bias, const float* ratio, int64_t m, void* ws,
+                            size_t ws_bytes, void* stream) {
+  if (!W || !S || !hidden_kept) return fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (!W->w_in_norm || !W->w_qkv || !W->w_o || !W->w_post_norm || !W->w_gate_up || !W->w_down || !W->head_gain ||
+      !W->head_temp)
+    return fail(TG_ERR_INVALID_ARG, "null weight pointer");
+  if (S->qk_norm && (!W->w_q_norm || !W->w_k_norm)) return fail(TG_ERR_INVALID_ARG, "qk_norm needs its weights");
+  if (m <= 0 || S->d_model <= 0 || S->hq <= 0 || S->hkv <= 0 || S->hq % S->hkv || S->d_ff <= 0)
+    return fail(TG_ERR_INVALID_ARG, "bad layer shape");
+  if (S->head_dim != 64 && S->head_dim != 128) return fail(TG_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  const int es = dtype_size(S->dtype);
+  if (!es) return fail(TG_ERR_INVALID_ARG, "dtype");
+  const size_t need = tg_workspace_bytes(TG_OP_LAYER, 0, m, 0, 0, S);
+  if (!ws || ws_bytes < need) return fail(TG_ERR_WORKSPACE, "layer needs %zu workspace bytes", need);
+  cudaStream_t st = as_stream(stream);
+  const int d = S->d_model, D = S->head_dim, hq = S->hq, hkv = S->hkv, dff = S->d_ff;
+  const int64_t qkv_w = int64_t(hq + 2 * hkv) * D;
+  auto al = [](size_t b) { return (b + 255) / 256 * 256; };
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  void* xn = base;
+  base += al(size_t(m) * d * es);
+  void* qkv = base;
+  base += al(size_t(m) * qkv_w * es);
+  void* att = base;
+  base += al(size_t(m) * hq * D * es);
+  void* act = base;
+  const bool bf = S->dtype == TG_BF16;
+  int rc;
+  // 1. x = RMSNorm(h)
+  if (bf)
+    tg::k_rmsnorm<__nv_bfloat16><<<unsigned(m), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(hidden_kept),
+                                                                static_cast<__nv_bfloat16*>(xn), W->w_in_norm, d,
+                                                                S->norm_eps);
+  else
+    tg::k_rmsnorm<float><<<unsigned(m), 256, 0, st>>>(static_cast<const float*>(hidden_kept),
+                                                       static_cast<float*>(xn), W->w_in_norm, d, S->norm_eps);
+  if ((rc = check_launch("k_rmsnorm"))) return rc;
+  // 2. qkv = x Wqkv^T
+  if ((rc = tg_linear(xn, d, W->w_qkv, qkv, qkv_w, S->dtype, m, int32_t(qkv_w), d, TG_EPI_STORE, stream))) return rc;
+  // 3. per-head q/k norm and RoPE at the original positions
+  {
+    const int64_t items = m * (hq + hkv);
+    const unsigned blocks = unsigned((items + 7) / 8);
+    if (bf) {
+      if (D == 128)
+        tg::k_qk_norm_rope<__nv_bfloat16, 128><<<blocks, 256, 0, st>>>(
+            static_cast<__nv_bfloat16*>(qkv), qkv_w, int(m), hq, hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm,
+            S->norm_eps, S->rope_theta);
+      else
+        tg::k_qk_norm_rope<__nv_bfloat16, 64><<<blocks, 256, 0, st>>>(
+            static_cast<__nv_bfloat16*>(qkv), qkv_w, int(m), hq, hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm,
+            S->norm_eps, S->rope_theta);
+    } else {
+      if (D == 128)
+        tg::k_qk_norm_rope<float, 128><<<blocks, 256, 0, st>>>(static_cast<float*>(qkv), qkv_w, int(m), hq, hkv, pos,
+                                                              W->w_q_norm, W->w_k_norm, S->qk_norm, S->norm_eps,
+                                                              S->rope_theta);
+      else
+        tg::k_qk_norm_rope<float, 64><<<blocks, 256, 0, st>>>(static_cast<float*>(qkv), qkv_w, int(m), hq, hkv, pos,
+                                                             W->w_q_norm, W->w_k_norm, S->qk_norm, S->norm_eps,
+                                                             S->rope_theta);
+    }
+    if ((rc = check_launch("k_qk_norm_rope"))) return rc;
+  }
+  // 4. token-gated attention
+  {
+    const uint8_t* qb = static_cast<const uint8_t*>(qkv);
+    if ((rc = tg_gated_attention(qb, qkv_w, qb + int64_t(hq) * D * es, qkv_w, qb + int64_t(hq + hkv) * D * es, qkv_w,
+                                 S->dtype, m, hq, hkv, D, bias, W->head_gain, W->head_temp, ratio,
+                                 1.0f / sqrtf(float(D)), att, int64_t(hq) * D, nullptr, stream)))
+      return rc;
+  }
+  // 5. h += a Wo^T
+  if ((rc = tg_linear(att, int64_t(hq) * D, W->w_o, hidden_kept, d, S->dtype, m, d, hq * D, TG_EPI_RESIDUAL, stream)))
+    return rc;
+  // 6. y = RMSNorm(h)
+  if (bf)
+    tg::k_rmsnorm<__nv_bfloat16><<<unsigned(m), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(hidden_kept),
+                                                                static_cast<__nv_bfloat16*>(xn), W->w_post_norm, d,
+                                                                S->norm_eps);
+  else
+    tg::k_rmsnorm<float><<<unsigned(m), 256, 0, st>>>(static_cast<const float*>(hidden_kept),
+                                                       static_cast<float*>(xn), W->w_post_norm, d, S->norm_eps);
+  if ((rc = check_launch("k_rmsnorm"))) return rc;
+  // 7. act = SiLU(y Wg^T) * (y Wu^T)
+  if (bf && dff % 128 == 0) {
+    if ((rc = tg_linear(xn, d, W->w_gate_up, act, dff, S->dtype, m, dff, d, TG_EPI_SWIGLU, stream))) return rc;
+  } else {
+    // un-fused: gate/up product into the activation buffer, then SiLU(g) * u
+    // written over the gate half of each row (every element reads only its
+    // own gate/up pair), and the down projection reads rows of stride 2*d_ff
+    void* gu = act;
+    if ((rc = tg_linear(xn, d, W->w_gate_up, gu, 2 * int64_t(dff), S->dtype, m, 2 * dff, d, TG_EPI_STORE, stream)))
+      return rc;
+    const int64_t total = m * dff;
+    const unsigned blocks = unsigned((total + 255) / 256);
+    if (bf)
+      tg::k_swiglu<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<__nv_bfloat16*>(gu), m, dff);
+    else
+      tg::k_swiglu<float><<<blocks, 256, 0, st>>>(static_cast<float*>(gu), m, dff);
+    if ((rc = check_launch("k_swiglu"))) return rc;
+    return tg_linear(gu, 2 * int64_t(dff), W->w_down, hidden_kept, d, S->dtype, m, d, dff, TG_EPI_RESIDUAL, stream);
+  }
+  // 8. h += act Wd^T
+  return tg_linear(act, dff, W->w_down, hidden_kept, d, S->dtype, m, d, dff, TG_EPI_RESIDUAL, stream);
+}
+
+}  // extern "C"

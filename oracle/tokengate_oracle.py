@@ -223,16 +223,18 @@ def rope(x, pos, theta: float) -> np.ndarray:
 
 def decoder_layer(hidden, weights: Dict[str, np.ndarray], *, hq: int, hkv: int, head_dim: int,
                   pos, bias, ratio, head_gain, head_temp, rope_theta: float, qk_norm: bool,
-                  norm_eps: float = 1e-6, rows_attn: Optional[Sequence[int]] = None) -> np.ndarray:
+                  norm_eps: float = 1e-6, rows: Optional[Sequence[int]] = None) -> np.ndarray:
     """One Qwen3-shaped decoder layer run on the kept rows only.
 
     RMSNorm -> QKV projection -> (per-head q/k RMSNorm) -> RoPE at the original
     positions -> token-gated attention -> O projection + residual -> RMSNorm ->
     SwiGLU MLP + residual.  Linear weights are [out, in]; w_gate_up stacks the
-    gate rows over the up rows.  All float64.
+    gate rows over the up rows.  All float64.  With `rows`, only those output
+    rows are produced (keys and values still come from every row).
     """
     h = np.asarray(hidden, dtype=F64)
     mrows = h.shape[0]
+    sel = np.arange(mrows) if rows is None else np.asarray(rows, dtype=np.int64)
     x = rms_norm(h, weights["w_in_norm"], norm_eps)
     qkv = x @ np.asarray(weights["w_qkv"], dtype=F64).T
     q = qkv[:, : hq * head_dim].reshape(mrows, hq, head_dim)
@@ -243,8 +245,8 @@ def decoder_layer(hidden, weights: Dict[str, np.ndarray], *, hq: int, hkv: int, 
         k = rms_norm(k, weights["w_k_norm"], norm_eps)
     q = rope(q, pos, rope_theta)
     k = rope(k, pos, rope_theta)
-    a = gated_attention(q, k, v, bias, head_gain, head_temp, ratio, 1.0 / math.sqrt(head_dim))
-    h1 = h + a.reshape(mrows, hq * head_dim) @ np.asarray(weights["w_o"], dtype=F64).T
+    a = gated_attention(q, k, v, bias, head_gain, head_temp, ratio, 1.0 / math.sqrt(head_dim), rows=sel)
+    h1 = h[sel] + a.reshape(sel.size, hq * head_dim) @ np.asarray(weights["w_o"], dtype=F64).T
     y = rms_norm(h1, weights["w_post_norm"], norm_eps)
     gu = y @ np.asarray(weights["w_gate_up"], dtype=F64).T
     d_ff = gu.shape[1] // 2

@@ -1,0 +1,80 @@
+"""CPU-only checks of the C ABI: the library builds, loads, exports every entry
+point the header declares, and rejects bad arguments on the host before any
+CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from learned_token_pruning_b200 import build, tokengate as tg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return tg.lib()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "tg.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tg_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_hot_path_entry_points():
+    names = header_functions()
+    for n in ("tg_gate_score", "tg_topk_select", "tg_gather", "tg_gated_attention", "tg_pruned_prefill_layer"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = header_functions()
+    assert names
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in tg.SIGNATURES, f"binding lacks {n}"
+
+
+def test_version_and_status_strings(L):
+    assert tg.tg_version().startswith("tokengate-b200")
+    assert L.tg_status_string(0) == b"ok"
+    assert L.tg_status_string(7) == b"device-side wait timed out"
+
+
+P = ctypes.c_void_p(256)  # a non-null dummy: validation fails before it is ever dereferenced
+
+
+def test_select_validation(L):
+    assert L.tg_topk_select(None, P, 10, 5, 3, P, 8, None) == 1
+    assert L.tg_topk_select(P, P, 10, 5, -1, P, 5, None) == 1           # k < 0
+    assert L.tg_topk_select(P, P, 10, 11, 3, P, 8, None) == 1           # n_prunable > n
+    assert L.tg_topk_select(P, P, 10, 5, 3, P, 7, None) == 2            # m mismatch
+    assert b"m = 7" in L.tg_last_error()
+    assert L.tg_topk_select(P, P, 1 << 31, 5, 3, P, (1 << 31) - 2, None) == 4
+
+
+def test_attention_validation(L):
+    g = ctypes.c_void_p(256)
+    assert L.tg_gated_attention(g, 2048, g, 1024, g, 1024, 1, 100, 16, 8, 96, None, g, g, None, 0.1, g, 2048, None, None) == 4
+    assert L.tg_gated_attention(g, 2048, g, 1024, g, 1024, 1, 100, 16, 6, 128, None, g, g, None, 0.1, g, 2048, None, None) == 1
+    assert L.tg_gated_attention(g, 100, g, 1024, g, 1024, 1, 100, 16, 8, 128, None, g, g, None, 0.1, g, 2048, None, None) == 2
+    assert L.tg_gated_attention(ctypes.c_void_p(258), 2048, g, 1024, g, 1024, 1, 100, 16, 8, 128, None, g, g, None,
+                                0.1, g, 2048, None, None) == 3
+
+
+def test_gather_and_gate_validation(L):
+    assert L.tg_gather(P, 1, 10, 2048, P, 11, P, P, 5, 1e-6, P, None, None, None, None) == 1   # m > n
+    assert L.tg_gather(P, 1, 10, 20, P, 5, P, P, 5, 1e-6, P, None, None, None, None) == 3      # 40-byte rows
+    assert L.tg_gate_score(P, 1, 100, 256, None, 1e-6, P, None, P, 0.0, 64, P, P, P, None, 0, None) == 5
+
+
+def test_workspace_sizes(L):
+    S = tg.LayerShape(1, 2048, 16, 8, 128, 6144, 1, 1e6, 1e-6)
+    m = 2064
+    want = sum((b + 255) // 256 * 256 for b in (m * 2048 * 2, m * 4096 * 2, m * 2048 * 2, m * 2 * 6144 * 2))
+    assert tg.tg_workspace_bytes(tg.TG_OP_LAYER, m=m, shape=S) == want
+    assert tg.tg_workspace_bytes(tg.TG_OP_GATE_SCORE, n=16384, d_model=2048, h=256) >= 16384 // 128 * 4 + 256 * 2048 * 2
+    assert tg.tg_workspace_bytes(99) == 0
