@@ -261,13 +261,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       logits(s3, 96);
       // lazy rescaling: the reference maximum only moves when the row maximum
       // exceeds it by more than 8 (so every p stays <= 2^8)
+      // (per row: the branch below is divergent, so it holds no warp-collective op)
       float sc = 1.0f;
-      bool rescale = false;
       if (mx > m_run + 8.0f) {
-        if (j > 0) {
-          sc = exp2f(m_run - mx);
-          rescale = true;
-        }
+        if (j > 0) sc = exp2f(m_run - mx);
         m_run = mx;
       }
       float sum = 0.0f;
@@ -288,7 +285,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       emit_p(s2, 64);
       emit_p(s3, 96);
       l_run = l_run * sc + sum;
-      if (rescale) {
+      // tcgen05.ld/st are warp-collective (.sync.aligned): the whole warp
+      // rescales its 32 rows if any of them needs it, the others with sc = 1
+      if (__any_sync(0xffffffffu, sc != 1.0f)) {
         // O_i holds the sum over earlier tiles (its last PV finished before
         // s_full fired) and no PV into it is issued before p_full below
 #pragma unroll 1
@@ -336,6 +335,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   if (warp == 9) {
     tc_fence_after();
+    __syncwarp();  // the .sync.aligned dealloc needs the whole warp converged
     tmem_dealloc(tmem, 512);
   }
 }

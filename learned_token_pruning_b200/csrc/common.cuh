@@ -94,11 +94,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   }
 }
 
-// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast.
+// Warp-uniform bounded wait: every lane waits on the barrier itself (so each
+// one acquires what the barrier guards) and the verdict is agreed on by vote,
+// so a warp never splits over a later warp-collective instruction.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t site) {
-  bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, site);
-  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  const bool ok = mbar_wait(bar, parity, site);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // ---------------------------------------------------------------------------

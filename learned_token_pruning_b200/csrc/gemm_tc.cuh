@@ -183,6 +183,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ss = fmaf(hi, hi, ss);
           }
         }
+        // order these generic-proxy reads before the TMA (async proxy) refill of the stage
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
       }
@@ -305,6 +307,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
+    __syncwarp();  // the .sync.aligned dealloc needs the whole warp converged
     tmem_dealloc(tmem, Cfg::kTmemCols);
   }
 }

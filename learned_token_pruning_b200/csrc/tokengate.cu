@@ -240,7 +240,7 @@ int tg_gate_score(const void* hidden, int dtype, int64_t n, int32_t d_model, con
 
 int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int64_t n_prunable, int64_t k,
                    int32_t* kept_idx, int64_t m, void* stream) {
-  if (!scores || !prunable || !kept_idx) return fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (!scores || !prunable || (!kept_idx && m > 0)) return fail(TG_ERR_INVALID_ARG, "null pointer");
   if (n <= 0 || n_prunable < 0 || n_prunable > n) return fail(TG_ERR_INVALID_ARG, "bad n / n_prunable");
   if (k < 0) return fail(TG_ERR_INVALID_ARG, "k must be >= 0");
   if (n >= (int64_t(1) << 31)) return fail(TG_ERR_UNSUPPORTED, "n must be < 2^31");
