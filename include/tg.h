@@ -239,6 +239,38 @@ enum { TG_OP_GATE_SCORE = 0, TG_OP_LAYER = 1 };
  * TG_OP_LAYER uses m and shape.  Returns 0 for an invalid request. */
 size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t h, const tg_layer_shape* shape);
 
+/*
+ * tg_gate_score without a workspace argument, for callers that cannot
+ * allocate device memory when they score a prompt (a serving runtime that owns
+ * all of HBM through its own pool and passes the library only the request's
+ * tensors, a plugin interface with no workspace hook, or a latency-critical
+ * path that must avoid cudaMalloc's device-wide synchronisation).  The TokenGate
+ * pages have no counterpart of this call; it computes exactly what
+ * tg_gate_score computes, with the same arguments minus ws / ws_bytes.
+ *
+ * Scratch lives in a fixed array compiled into the library,
+ * tg_gate_score_noalloc_scratch_bytes() bytes (2 MiB + 64 KiB) on every device
+ * that loads the library, held until the process exits.  Sizes whose scratch
+ * would not fit (about n/32 + 2*d_model*h bytes, e.g. n up to 2^20 tokens with
+ * d_model*h up to 2^20) are rejected with TG_ERR_UNSUPPORTED before anything
+ * is enqueued.  The call allocates and frees nothing.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any stream
+ * capture.  All calls on a device share the one array and leave the last
+ * call's contents in it (the part that must start at zero is cleared by each
+ * call on its stream), so calls whose executions overlap on the GPU -- on
+ * different streams, or from several host threads -- race on it and must be
+ * serialised by the caller.
+ */
+int tg_gate_score_noalloc(const void* hidden, int dtype, int64_t n, int32_t d_model,
+                          const float* norm_w, float norm_eps,
+                          const void* w1, const float* b1, const float* w2, float b2, int32_t h,
+                          const uint8_t* prunable, float* scores, float* sumsq, void* stream);
+
+/* Size in bytes of the per-device scratch array used by tg_gate_score_noalloc. */
+size_t tg_gate_score_noalloc_scratch_bytes(void);
+
 /* Library version string. */
 const char* tg_version(void);
 

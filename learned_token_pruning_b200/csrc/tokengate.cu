@@ -11,6 +11,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/tg.h"
 #include "attn_tc.cuh"
@@ -531,5 +532,74 @@ int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, 
   // 8. h += act Wd^T
   return tg_linear(act, dff, W->w_down, hidden_kept, d, S->dtype, m, d, dff, TG_EPI_RESIDUAL, stream);
 }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Gate scores without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they score a
+// prompt: a serving runtime that hands the library only the tensors of the
+// request and owns every other byte of HBM through its own pool, a plugin
+// host whose interface has no workspace argument, or a latency-critical path
+// that must not take cudaMalloc's implicit device-wide synchronisation.  For
+// them tg_gate_score_noalloc keeps its scratch (per-CTA partial sums, the
+// completion counter and the norm-folded W1) in a fixed array compiled into
+// the library instead of in `ws`.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (2u << 20) + (64u << 10);  // 2 MiB + 64 KiB per device
+constexpr int kNoAllocMaxDevices = 64;
+
+// Every GPU that loads the library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_gate_scratch[kNoAllocScratchBytes];
+
+std::mutex g_gate_scratch_mu;
+void* g_gate_scratch_addr[kNoAllocMaxDevices] = {};
+
+// Device address of g_gate_scratch on the current device.  Host code cannot
+// use the symbol itself (on the host it names a stand-in, not device memory),
+// so the address is looked up once per device, with that device current.
+int gate_scratch_address(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(TG_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(TG_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_gate_scratch_mu);
+  if (!g_gate_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_gate_scratch);
+    if (e != cudaSuccess || !p) return fail(TG_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    g_gate_scratch_addr[dev] = p;
+  }
+  *out = g_gate_scratch_addr[dev];
+  return TG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int tg_gate_score_noalloc(const void* hidden, int dtype, int64_t n, int32_t d_model, const float* norm_w,
+                          float norm_eps, const void* w1, const float* b1, const float* w2, float b2, int32_t h,
+                          const uint8_t* prunable, float* scores, float* sumsq, void* stream) {
+  if (n > 0 && d_model > 0 && h > 0) {
+    const size_t need = gate_ws_bytes(n, d_model, h);
+    if (need > kNoAllocScratchBytes)
+      return fail(TG_ERR_UNSUPPORTED,
+                  "tg_gate_score_noalloc: n = %lld, d_model = %d, h = %d need %zu scratch bytes, more than the "
+                  "%zu built into the library (n/32 + 2*d_model*h bytes must stay below it); use tg_gate_score "
+                  "with a workspace",
+                  static_cast<long long>(n), d_model, h, need, kNoAllocScratchBytes);
+  }
+  void* scratch = nullptr;
+  const int rc = gate_scratch_address(&scratch);
+  if (rc) return rc;
+  return tg_gate_score(hidden, dtype, n, d_model, norm_w, norm_eps, w1, b1, w2, b2, h, prunable, scores, sumsq,
+                       scratch, kNoAllocScratchBytes, stream);
+}
+
+size_t tg_gate_score_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 }  // extern "C"

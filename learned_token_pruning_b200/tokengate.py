@@ -57,6 +57,8 @@ SIGNATURES = {
                                        _I64, _P, _SZ, _P]),
     "tg_linear": (_INT, [_P, _I64, _P, _P, _I64, _INT, _I64, _I32, _I32, _INT, _P]),
     "tg_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I32, _I32, ctypes.POINTER(LayerShape)]),
+    "tg_gate_score_noalloc": (_INT, [_P, _INT, _I64, _I32, _P, _F, _P, _P, _P, _F, _I32, _P, _P, _P, _P]),
+    "tg_gate_score_noalloc_scratch_bytes": (_SZ, []),
 }
 
 _lib = None
@@ -129,6 +131,16 @@ def tg_gate_score(hidden, norm_w, norm_eps, w1, b1, w2, b2, prunable, scores, su
                              _ptr(w2), float(b2), h, _ptr(prunable), _ptr(scores), _ptr(sumsq), _ptr(ws),
                              ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream))
     _check("tg_gate_score", rc)
+
+
+def tg_gate_score_noalloc(hidden, norm_w, norm_eps, w1, b1, w2, b2, prunable, scores, sumsq, stream=None):
+    """tg_gate_score for callers that cannot allocate: the scratch is the library's own fixed array."""
+    n, d = hidden.shape
+    h = w1.shape[0]
+    rc = lib().tg_gate_score_noalloc(_ptr(hidden), _dtype(hidden), n, d, _ptr(norm_w), float(norm_eps), _ptr(w1),
+                                     _ptr(b1), _ptr(w2), float(b2), h, _ptr(prunable), _ptr(scores), _ptr(sumsq),
+                                     _stream(stream))
+    _check("tg_gate_score_noalloc", rc)
 
 
 def tg_topk_select(scores, prunable, n_prunable: int, k: int, kept_idx, stream=None):
