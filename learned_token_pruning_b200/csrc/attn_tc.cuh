@@ -5,28 +5,43 @@
 // and kept rows c <= r
 //     l_rc = temp_h * ratio_r * sm_scale * (q_r . k_c) + gain_h * bias_c
 //     o_r  = sum_c softmax_c(l_r.) v_c
-// computed in base 2: x = a_r * S_rc + beta_c with a_r = temp_h * ratio_r *
-// sm_scale * log2(e) (one scale per row) and beta_c = gain_h * log2(e) * bias_c
-// (one offset per key).
+// computed in base 2 with the head gain factored out of the row:
+//     x_rc = g_h * y_rc,   y_rc = (a_r / g_h) * S_rc + bias_c,
+//     a_r = temp_h * ratio_r * sm_scale * log2(e),  g_h = gain_h * log2(e),
+// so the raw per-key bias tile, which TMA brings in with each K tile, serves
+// both query heads of the CTA unchanged; the softmax runs on y (max, then
+// exp2(g_h * (y - max))).
 //
 // One CTA owns a 128-row query block of TWO query heads that share a KV head
-// (GQA), so every K/V tile fetched by TMA feeds two 128x128 score tiles.
-//   warps 0-3  softmax warpgroup 0 (query tile 0), one thread per row
-//   warps 4-7  softmax warpgroup 1 (query tile 1)
-//   warp 8     TMA producer (Q once, then K and V tiles through a 2-stage ring)
+// (GQA), so every K/V tile fetched by TMA feeds two score tiles.  Keys come in
+// tiles of 64.
+//   warps 0-3  softmax warpgroup 0 (query head 0), one thread per row
+//   warps 4-7  softmax warpgroup 1 (query head 1)
+//   warp 8     TMA producer (Q once, then K + bias tiles through a 3-stage
+//              ring and V tiles through a 2-stage ring)
 //   warp 9     TMEM allocator and single-thread tcgen05.mma issuer
-// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 and O1 after them.
-// S_i = Q_i K^T is an SS-MMA (both operands in shared memory, K-major); the
-// softmax warps read S_i with tcgen05.ld, write P_i = exp2(x - m) as packed
-// bf16 over the first 64 columns of S_i, and O_i += P_i V is a TS-MMA with P
-// taken from tensor memory and V (MN-major) from shared memory.  The running
-// row maximum is only moved when it grows by more than 8 (log2 units), and O is
-// then rescaled in tensor memory by the softmax warps themselves; P <= 2^8 in
-// between, which bf16 and the fp32 accumulators hold exactly enough.
-// Every MMA is issued by one thread, so tcgen05 executes them in issue order:
-// QK_i(j+1), which overwrites S_i, is issued after PV_i(j), which reads P_i
-// from the same columns, and the commit after QK_i(j+1) also covers PV_i(j),
-// which is what lets the softmax warps touch O_i after waiting on it.
+// Tensor memory (512 columns): S of each head double-buffered, 4 x 64 columns,
+// then O0 and O1 (D columns each).  S = Q K^T is an SS-MMA into TMEM; P =
+// exp2(x - m) is written as bf16 to shared memory (128-byte swizzle,
+// double-buffered per head) and O += P V is an SS-MMA with V read MN-major.
+// Per key tile j the MMA thread issues P V of tile j for both heads and then
+// Q K^T of tile j + 2, so the scores of the next tile are ready when a
+// softmax finishes and the loop is bounded by the slower of the softmax and
+// the tensor core, not by their sum.
+//
+// The MMA thread is the one serial resource of the CTA: it shares its SM
+// sub-partition with two softmax warps, and every barrier check it makes costs
+// a shared-memory round trip.  So it makes two checks per key tile, each of
+// two barriers at once (their latencies overlap), and three commits: one
+// "P V of tile j done" barrier (a ring of 4) frees the K and V stages for the
+// producer, the P buffer for the softmax and orders the O rescale, and
+// "softmax read S" needs no barrier of its own because the softmax only
+// declares P ready after its S loads have completed.  The softmax does its
+// elementwise arithmetic on packed pairs (fma/add.f32x2, three-input max),
+// which halves its FMA-pipe instructions and leaves issue slots to the MMA
+// thread.  The running row maximum only moves when it grows by more than 8
+// (log2 units); O is then rescaled in tensor memory by the softmax warps after
+// the previous P V into it has completed.
 #pragma once
 
 #include "common.cuh"
@@ -35,23 +50,35 @@
 namespace tg {
 
 constexpr int kAttnThreads = 320;
+constexpr bool kPolyShare = false;  // evaluate a quarter of the exponentials with exp2_poly
 
 template <int D>
 struct AttnCfg {
-  static constexpr int BM = 128, BN = 128;
-  static constexpr int kQBytes = BM * D * 2;   // one query tile
-  static constexpr int kKVBytes = BN * D * 2;  // one K or V tile
-  static constexpr int kBlk = 128 * 128;       // bytes of one 64-column TMA box of 128 rows
-  static constexpr int kStages = 2;
-  static constexpr int kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
-  // Data, barriers and bias tiles; D = 64 is padded so that only one CTA fits
-  // on an SM and its 512-column TMEM allocation never waits on a neighbour.
-  static constexpr size_t kSmemData = 2 * kQBytes + kStages * 2 * kKVBytes;
-  static constexpr size_t kSmem = 1024 + (kSmemData < 120 * 1024 ? 120 * 1024 : kSmemData) + 2048 + 256;
+  static constexpr int BM = 128, BN = 64;
+  static constexpr int kQBytes = BM * D * 2;     // one query tile
+  static constexpr int kKVBytes = BN * D * 2;    // one K or V tile
+  static constexpr int kQBlk = BM * 128;         // one 64-column TMA box of a Q tile
+  static constexpr int kKVBlk = BN * 128;        // one 64-column TMA box of a K or V tile
+  static constexpr int kPBytes = BM * BN * 2;    // one P tile (128 rows x 64 keys, bf16)
+  static constexpr int kKStages = 3, kVStages = 2;
+  static constexpr int kColO0 = 256, kColO1 = 256 + D;
+  static constexpr size_t kOffK = 2 * kQBytes;
+  static constexpr size_t kOffV = kOffK + kKStages * kKVBytes;
+  static constexpr size_t kOffP = kOffV + kVStages * kKVBytes;
+  static constexpr size_t kOffBias = kOffP + 4 * kPBytes;
+  static constexpr size_t kOffBars = kOffBias + kKStages * BN * 4;  // 16 barriers + TMEM slot
+  static constexpr size_t kData = kOffBars + 256;
+  // D = 64 is padded so that only one CTA fits on an SM and its 512-column
+  // TMEM allocation never waits on a neighbour
+  static constexpr size_t kSmem = 1024 + (kData < 120 * 1024 ? 120 * 1024 : kData);
 };
+
+// TMEM column of head h's S buffer b
+__device__ __forceinline__ uint32_t attn_col_s(int h, int b) { return static_cast<uint32_t>((h * 2 + b) * 64); }
 
 struct AttnTcParams {
   int m, hq, hkv, group;
+  int has_bias;
   int num_qtiles;
   const float* bias;
   const float* gain;
@@ -63,28 +90,87 @@ struct AttnTcParams {
   float* lse;
 };
 
+// 2^x by the hardware approximation (ex2.approx.ftz.f32, the MUFU unit).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x on the FMA pipe for x <= 8 (Cody-Waite split x = n + f with n = floor(x)
+// and f in [0, 1); 2^f by the cubic minimax polynomial 1 + c1 f + c2 f^2 + c3 f^3
+// fitted for relative error on [0, 1) (max 8.6e-5); 2^n by adding n to the
+// exponent field).  Inputs below -127 return 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -127.0f);
+  const float n = floorf(x);
+  const float f = x - n;
+  float q = fmaf(f, 0.07706519961357117f, 0.22764700651168823f);
+  q = fmaf(q, f, 0.6951163411140442f);
+  q = fmaf(q, f, 1.0f);
+  return __int_as_float(__float_as_int(q) + (static_cast<int>(n) << 23));
+}
+
+// Packed fp32 pairs (two lanes of one 64-bit register): Blackwell executes
+// fma/add.f32x2 as one instruction with per-lane IEEE round-to-nearest, so the
+// results equal two scalar fmaf/adds.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Two barrier checks issued back to back, so that their shared-memory round
+// trips overlap; falls back to the bounded waits when either is still open.
+__device__ __forceinline__ bool mbar_wait2(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, uint32_t site) {
+  const bool r0 = mbar_try_wait(smem_u32(b0), p0);
+  const bool r1 = mbar_try_wait(smem_u32(b1), p1);
+  if (r0 && r1) return true;
+  return mbar_wait(b0, p0, site) && mbar_wait(b1, p1, site);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, AttnTcParams p) {
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmBias,
+              AttnTcParams p) {
   using Cfg = AttnCfg<D>;
+  constexpr int BN = Cfg::BN;
   constexpr int kDBoxes = D / 64;
   extern __shared__ uint8_t attn_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(attn_smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                                    // [2][kQBytes]
-  uint8_t* sK = sQ + 2 * Cfg::kQBytes;                   // [stages][kKVBytes]
-  uint8_t* sV = sK + Cfg::kStages * Cfg::kKVBytes;       // [stages][kKVBytes]
-  float* sBeta = reinterpret_cast<float*>(smem + (Cfg::kSmem - 1024 - 2048 - 256));  // [2 wg][2 buf][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sBeta + 512);
+  uint8_t* sQ = smem;                     // [2 heads][kQBytes]
+  uint8_t* sK = smem + Cfg::kOffK;        // [3 stages][kKVBytes]
+  uint8_t* sV = smem + Cfg::kOffV;        // [2 stages][kKVBytes]
+  uint8_t* sP = smem + Cfg::kOffP;        // [2 heads][2 buffers][kPBytes]
+  float* sBias = reinterpret_cast<float*>(smem + Cfg::kOffBias);  // [3 stages][BN]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBars);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;      // [2]
-  uint64_t* v_full = bars + 3;      // [2]
-  uint64_t* kv_empty = bars + 5;    // [2]
-  uint64_t* s_full = bars + 7;      // [2]
-  uint64_t* p_full = bars + 9;      // [2]
-  uint64_t* o_final = bars + 11;
-  uint64_t* beta_bar = bars + 12;   // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* k_full = bars + 1;      // [3]  K tile j (stage j % 3) and its bias tile
+  uint64_t* v_full = bars + 4;      // [2]  V tile j (stage j % 2)
+  uint64_t* pv_done = bars + 6;     // [4]  P V of tile j (both heads) complete, slot j % 4
+  uint64_t* s_full = bars + 10;     // [head * 2 + buffer]
+  uint64_t* p_full = bars + 14;     // [head * 2 + buffer]  (128 arrivals: the warpgroup)
+  uint64_t* o_final = bars + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -95,17 +181,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int pair = static_cast<int>(blockIdx.x) % per_tile;
   const int g = pair / pairs_per_kv;
   const int h0 = g * p.group + 2 * (pair % pairs_per_kv);
-  const int nt = t + 1;  // causal: key tiles 0..t
+  // causal: key tiles 0 .. (128t + 127) / 64, and none past the last kept row
+  const int nt = min(2 * t + 2, (p.m + BN - 1) / BN);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
-      mbar_init(&beta_bar[s], 128);
+    for (int s = 0; s < 3; ++s) mbar_init(&k_full[s], 1);
+    for (int s = 0; s < 2; ++s) mbar_init(&v_full[s], 1);
+    for (int s = 0; s < 4; ++s) mbar_init(&pv_done[s], 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
     }
     mbar_init(o_final, 1);
     *abort_flag = 0;
@@ -115,6 +201,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  if (!p.has_bias)
+    for (int i = threadIdx.x; i < Cfg::kKStages * BN; i += kAttnThreads) sBias[i] = 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -126,77 +214,89 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
+      if (p.has_bias) prefetch_tmap(&tmBias);
       mbar_arrive_expect_tx(q_full, 2 * Cfg::kQBytes);
       for (int i = 0; i < 2; ++i)
         for (int b = 0; b < kDBoxes; ++b)
-          tma_load_2d(sQ + i * Cfg::kQBytes + b * Cfg::kBlk, &tmQ, q_full, (h0 + i) * D + 64 * b, t * 128);
+          tma_load_2d(sQ + i * Cfg::kQBytes + b * Cfg::kQBlk, &tmQ, q_full, (h0 + i) * D + 64 * b, t * 128);
       for (int j = 0; j < nt; ++j) {
-        const int s = j & 1;
-        if (*abort_flag || !mbar_wait(&kv_empty[s], ((j >> 1) & 1) ^ 1, kErrWaitAttention)) {
+        // K stage j % 3 held tile j - 3, V stage j % 2 held tile j - 2: both
+        // are free once the P V of that tile has completed
+        if (j >= 3 && !mbar_wait(&pv_done[(j - 3) & 3], ((j - 3) >> 2) & 1, kErrWaitAttention)) {
           *abort_flag = 1;
           break;
         }
-        mbar_arrive_expect_tx(&k_full[s], Cfg::kKVBytes);
+        const int ks = j % 3, vs = j & 1;
+        mbar_arrive_expect_tx(&k_full[ks], Cfg::kKVBytes + (p.has_bias ? BN * 4 : 0));
         for (int b = 0; b < kDBoxes; ++b)
-          tma_load_2d(sK + s * Cfg::kKVBytes + b * Cfg::kBlk, &tmK, &k_full[s], g * D + 64 * b, j * 128);
-        mbar_arrive_expect_tx(&v_full[s], Cfg::kKVBytes);
+          tma_load_2d(sK + ks * Cfg::kKVBytes + b * Cfg::kKVBlk, &tmK, &k_full[ks], g * D + 64 * b, j * BN);
+        if (p.has_bias) tma_load_1d(sBias + ks * BN, &tmBias, &k_full[ks], j * BN);
+        if (j >= 2 && !mbar_wait(&pv_done[(j - 2) & 3], ((j - 2) >> 2) & 1, kErrWaitAttention)) {
+          *abort_flag = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[vs], Cfg::kKVBytes);
         for (int b = 0; b < kDBoxes; ++b)
-          tma_load_2d(sV + s * Cfg::kKVBytes + b * Cfg::kBlk, &tmV, &v_full[s], g * D + 64 * b, j * 128);
+          tma_load_2d(sV + vs * Cfg::kKVBytes + b * Cfg::kKVBlk, &tmV, &v_full[vs], g * D + 64 * b, j * BN);
       }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-      auto issue_qk = [&](int i, int s) {
-        const uint32_t qa = smem_u32(sQ + i * Cfg::kQBytes), kb = smem_u32(sK + s * Cfg::kKVBytes);
+      // descriptors of every operand's first 16-element K slice; a later
+      // slice adds its byte offset / 16 to the start-address field
+      const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dp0 = sdesc_sw128(smem_u32(sP), 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(sV), Cfg::kKVBlk, 1024);
+      auto issue_qk = [&](int h, int j) {
+        const uint64_t da = dq0 + (h * Cfg::kQBytes >> 4), db = dk0 + ((j % 3) * Cfg::kKVBytes >> 4);
+        const uint32_t d_tmem = tmem + attn_col_s(h, j & 1);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Cfg::kBlk + (kk & 3) * 32;
-          umma_ss(tmem + (i ? Cfg::kColS1 : Cfg::kColS0), sdesc_sw128(qa + off, 16, 1024),
-                  sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk != 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss(d_tmem, da + (((kk >> 2) * Cfg::kQBlk + (kk & 3) * 32) >> 4),
+                  db + (((kk >> 2) * Cfg::kKVBlk + (kk & 3) * 32) >> 4), idesc_qk, kk != 0 ? 1u : 0u);
+        umma_commit(&s_full[2 * h + (j & 1)]);
       };
-      auto issue_pv = [&](int i, int s, int j) {
-        const uint32_t vb = smem_u32(sV + s * Cfg::kKVBytes);
+      auto issue_pv = [&](int h, int j) {
+        const uint64_t da = dp0 + ((2 * h + (j & 1)) * Cfg::kPBytes >> 4), db = dv0 + ((j & 1) * Cfg::kKVBytes >> 4);
+        const uint32_t d_tmem = tmem + (h ? Cfg::kColO1 : Cfg::kColO0);
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk) {
-          umma_ts(tmem + (i ? Cfg::kColO1 : Cfg::kColO0), tmem + (i ? Cfg::kColS1 : Cfg::kColS0) + kk * 8,
-                  sdesc_sw128(vb + kk * 16 * 128, Cfg::kBlk, 1024), idesc_pv, (j | kk) != 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ss(d_tmem, da + ((kk * 32) >> 4), db + ((kk * 16 * 128) >> 4), idesc_pv, (j | kk) != 0 ? 1u : 0u);
       };
-      bool ok = mbar_wait(q_full, 0, kErrWaitAttention) && mbar_wait(&k_full[0], 0, kErrWaitAttention);
+      // the scores of tiles 0 and 1 first
+      bool ok = mbar_wait2(q_full, 0, &k_full[0], 0, kErrWaitAttention);
       if (ok) {
         tc_fence_after();
         issue_qk(0, 0);
-        umma_commit(&s_full[0]);
         issue_qk(1, 0);
-        umma_commit(&s_full[1]);
       }
+      if (ok && nt > 1 && (ok = mbar_wait(&k_full[1], 0, kErrWaitAttention))) {
+        tc_fence_after();
+        issue_qk(0, 1);
+        issue_qk(1, 1);
+      }
+      // per tile j: P V of tile j for head 0, then head 1, then the scores of
+      // tile j + 2 into the S buffers whose tile j the softmax has read (its
+      // p_full arrival comes after its S loads completed)
       for (int j = 0; ok && j < nt; ++j) {
-        const int s = j & 1;
         const uint32_t ph = (j >> 1) & 1;
-        ok = !*abort_flag && mbar_wait(&v_full[s], ph, kErrWaitAttention) &&
-             mbar_wait(&p_full[0], j & 1, kErrWaitAttention);
+        if (!(ok = mbar_wait2(&v_full[j & 1], ph, &p_full[j & 1], ph, kErrWaitAttention))) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        const bool next = j + 2 < nt;
+        ok = next ? mbar_wait2(&p_full[2 + (j & 1)], ph, &k_full[(j + 2) % 3], ((j + 2) / 3) & 1, kErrWaitAttention)
+                  : mbar_wait(&p_full[2 + (j & 1)], ph, kErrWaitAttention);
         if (!ok) break;
         tc_fence_after();
-        issue_pv(0, s, j);
-        if (j + 1 < nt) {
-          ok = mbar_wait(&k_full[s ^ 1], ((j + 1) >> 1) & 1, kErrWaitAttention);
-          if (!ok) break;
-          tc_fence_after();
-          issue_qk(0, s ^ 1);
-          umma_commit(&s_full[0]);
-        }
-        ok = mbar_wait(&p_full[1], j & 1, kErrWaitAttention);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(1, s, j);
-        umma_commit(&kv_empty[s]);
-        if (j + 1 < nt) {
-          issue_qk(1, s ^ 1);
-          umma_commit(&s_full[1]);
+        issue_pv(1, j);
+        umma_commit(&pv_done[j & 3]);
+        if (next) {
+          issue_qk(0, j + 2);
+          issue_qk(1, j + 2);
         }
       }
       if (ok) umma_commit(o_final);
@@ -204,92 +304,124 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroups
-    const int wg = warp >> 2;           // 0 or 1: which query tile
+    const int wg = warp >> 2;           // 0 or 1: which query head
     const int q4 = warp & 3;            // TMEM lane quarter
     const int row = q4 * 32 + lane;     // row inside the query tile
     const int grow = t * 128 + row;
     const int h = h0 + wg;
-    const int wtid = threadIdx.x & 127;
-    const uint32_t colS = wg ? Cfg::kColS1 : Cfg::kColS0;
     const uint32_t colO = wg ? Cfg::kColO1 : Cfg::kColO0;
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const float a_row = grow < p.m ? p.temp[h] * (p.ratio ? p.ratio[grow] : 1.0f) * p.scale_log2 : 0.0f;
-    const float gb = p.gain[h] * kLog2e;
-    float* beta_wg = sBeta + wg * 256;
-    float m_run = -INFINITY, l_run = 0.0f;
+    // g > 0 always (a zero gain leaves the bias term at 1e-20 * bias, i.e. nothing)
+    const float gg = fmaxf(p.gain[h] * kLog2e, 1e-20f);
+    const float a_y = a_row / gg;
+    const uint64_t ay2 = f2_pack(a_y, a_y), gg2 = f2_pack(gg, gg);
+    float m_run = -INFINITY, l_run = 0.0f;  // running max of y, running sum of exp2(g * (y - m_run))
     bool ok = true;
+    // this thread's 128-byte row of head wg's first P buffer; 16-byte chunk c sits at c ^ (row & 7)
+    uint8_t* prow0 = sP + (2 * wg) * Cfg::kPBytes + row * 128;
+    const int sw = row & 7;
 
     for (int j = 0; j < nt; ++j) {
-      // this tile's key offsets: one per thread, exchanged through shared memory
-      {
-        const int c = j * 128 + wtid;
-        beta_wg[(j & 1) * 128 + wtid] = (p.bias && c < p.m) ? gb * p.bias[c] : 0.0f;
-        mbar_arrive(&beta_bar[wg]);
-      }
-      if (*abort_flag || !warp_wait(&beta_bar[wg], j & 1, kErrWaitAttention) ||
-          !warp_wait(&s_full[wg], j & 1, kErrWaitAttention)) {
+      const int b = j & 1;
+      const uint32_t ph = (j >> 1) & 1;
+      // S of tile j, its bias tile (it rides with K) and, from tile 2 on, P
+      // buffer b back from the P V of tile j - 2
+      bool rdy = !*abort_flag && mbar_wait2(&s_full[2 * wg + b], ph, &k_full[j % 3], (j / 3) & 1, kErrWaitAttention);
+      if (rdy && j >= 2) rdy = mbar_wait(&pv_done[(j - 2) & 3], ((j - 2) >> 2) & 1, kErrWaitAttention);
+      if (!__all_sync(0xffffffffu, rdy)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float* beta = beta_wg + (j & 1) * 128;
-      uint32_t s0[32], s1[32], s2[32], s3[32];
-      tmem_ld32(tmem + lane_base + colS + 0, s0);
-      tmem_ld32(tmem + lane_base + colS + 32, s1);
-      tmem_ld32(tmem + lane_base + colS + 64, s2);
-      tmem_ld32(tmem + lane_base + colS + 96, s3);
+      uint32_t s0[32], s1[32];
+      tmem_ld32(tmem + lane_base + attn_col_s(wg, b), s0);
+      tmem_ld32(tmem + lane_base + attn_col_s(wg, b) + 32, s1);
       tmem_ld_wait();
-      const bool diag = (j == t);
-      float mx = -INFINITY;
-      auto logits = [&](uint32_t(&r)[32], int c0) {
+      const float* bias = sBias + (j % 3) * BN;
+      // Pass 1: y = a_y * S + bias on pairs, and the row maximum (four
+      // independent chains); the causal mask only touches the key tiles that
+      // cross the diagonal.
+      uint64_t y2[BN / 2];
+      const int key0 = j * BN;
+      const bool diag = key0 + BN - 1 > t * 128;  // warp-uniform
+      float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      auto logits = [&](const uint32_t(&r)[32], int c0) {
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          const float4 b4 = *reinterpret_cast<const float4*>(beta + c0 + e);
-          const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+          const float4 b4 = *reinterpret_cast<const float4*>(bias + c0 + e);
+          const int i = (c0 + e) >> 1;
+          y2[i] = f2_fma(ay2, f2_pack(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), f2_pack(b4.x, b4.y));
+          y2[i + 1] = f2_fma(ay2, f2_pack(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])), f2_pack(b4.z, b4.w));
+          if (diag) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            float x = fmaf(a_row, __uint_as_float(r[e + u]), bb[u]);
-            if (diag && c0 + e + u > row) x = -INFINITY;
-            r[e + u] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
+            for (int u = 0; u < 2; ++u) {
+              float lo, hi;
+              f2_unpack(y2[i + u], lo, hi);
+              const int c = key0 + c0 + e + 2 * u;
+              if (c > grow) lo = -INFINITY;
+              if (c + 1 > grow) hi = -INFINITY;
+              y2[i + u] = f2_pack(lo, hi);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            float lo, hi;
+            f2_unpack(y2[i + u], lo, hi);
+            mxv[(i + u) & 3] = fmax3(mxv[(i + u) & 3], lo, hi);
           }
         }
       };
       logits(s0, 0);
       logits(s1, 32);
-      logits(s2, 64);
-      logits(s3, 96);
+      const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
       // lazy rescaling: the reference maximum only moves when the row maximum
-      // exceeds it by more than 8 (so every p stays <= 2^8)
-      // (per row: the branch below is divergent, so it holds no warp-collective op)
+      // exceeds it by more than 8 in log2 units, so every p stays <= 2^8
+      // (per row: the branch is divergent, so it holds no warp-collective op)
       float sc = 1.0f;
-      if (mx > m_run + 8.0f) {
-        if (j > 0) sc = exp2f(m_run - mx);
+      if (gg * (mx - m_run) > 8.0f) {
+        if (j > 0) sc = ex2_approx(gg * (m_run - mx));
         m_run = mx;
       }
-      float sum = 0.0f;
-      auto emit_p = [&](const uint32_t(&r)[32], int c0) {
-        uint32_t pk[16];
+      const float nm = -gg * m_run;
+      const uint64_t nm2 = f2_pack(nm, nm);
+      // Pass 2: p = 2^(g*y - g*m), partial sums on pairs, P as bf16 into shared memory
+      uint64_t sum2[2] = {0, 0};
+      uint8_t* prow = prow0 + b * Cfg::kPBytes;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = exp2f(__uint_as_float(r[2 * e]) - m_run);
-          const float p1 = exp2f(__uint_as_float(r[2 * e + 1]) - m_run);
-          sum += p0 + p1;
+      for (int c = 0; c < BN / 8; ++c) {  // 16-byte chunks of 8 keys
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float x0, x1;
+          f2_unpack(f2_fma(gg2, y2[4 * c + e], nm2), x0, x1);
+          float p0, p1;
+          if (kPolyShare && e == 3) {
+            p0 = exp2_poly(x0);
+            p1 = exp2_poly(x1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          sum2[e & 1] = f2_add(sum2[e & 1], f2_pack(p0, p1));
           pk[e] = pack_bf16x2(p0, p1);
         }
-        // P overwrites the first 64 columns of S as packed bf16 pairs
-        tmem_st16(tmem + lane_base + colS + c0 / 2, pk);
-      };
-      emit_p(s0, 0);
-      emit_p(s1, 32);
-      emit_p(s2, 64);
-      emit_p(s3, 96);
-      l_run = l_run * sc + sum;
+        *reinterpret_cast<uint4*>(prow + ((c ^ sw) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      float sa, sb, sc2, sd;
+      f2_unpack(sum2[0], sa, sb);
+      f2_unpack(sum2[1], sc2, sd);
+      l_run = l_run * sc + ((sa + sb) + (sc2 + sd));
       // tcgen05.ld/st are warp-collective (.sync.aligned): the whole warp
       // rescales its 32 rows if any of them needs it, the others with sc = 1
       if (__any_sync(0xffffffffu, sc != 1.0f)) {
-        // O_i holds the sum over earlier tiles (its last PV finished before
-        // s_full fired) and no PV into it is issued before p_full below
+        // O holds the sum over tiles < j once the P V of tile j - 1 is done;
+        // the P V of tile j is not issued before p_full below
+        if (!warp_wait(&pv_done[(j - 1) & 3], ((j - 1) >> 2) & 1, kErrWaitAttention)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
@@ -299,10 +431,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * sc);
           tmem_st32(tmem + lane_base + colO + c0, o);
         }
+        tmem_st_wait();
       }
-      tmem_st_wait();
+      // S loads (and any O rescale) are complete; make the generic-proxy P
+      // stores visible to the tensor core (async proxy), then hand P over
       tc_fence_before();
-      mbar_arrive(&p_full[wg]);
+      fence_proxy_async_smem();
+      mbar_arrive(&p_full[2 * wg + b]);
     }
     if (ok && !*abort_flag) ok = warp_wait(o_final, 0, kErrWaitAttention);
     if (ok) {
@@ -326,7 +461,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
       }
-      if (p.lse && grow < p.m) p.lse[static_cast<int64_t>(h) * p.m + grow] = (m_run + log2f(l_run)) * kLn2;
+      if (p.lse && grow < p.m) p.lse[static_cast<int64_t>(h) * p.m + grow] = (gg * m_run + log2f(l_run)) * kLn2;
     } else {
       *abort_flag = 1;
     }

@@ -16,13 +16,16 @@ namespace tg {
 // ---------------------------------------------------------------------------
 enum DeviceErrorSite : uint32_t {
   kErrNone = 0,
+  // consistency checks
   kErrMaskCount = 1,        // prunable-mask count disagrees with n_prunable
-  kErrWaitGemm = 2,         // bounded wait expired in the GEMM kernel
-  kErrWaitAttention = 3,    // bounded wait expired in the attention kernel
-  kErrGatherIndex = 4,      // kept index out of range in the gather kernel
-  kErrSelectOverflow = 5,   // selector produced more than m rows
+  kErrGatherIndex = 2,      // kept index out of range in the gather kernel
+  kErrSelectOverflow = 3,   // selector produced more than m rows
+  // bounded waits that expired
+  kErrWaitGemm = 8,         // GEMM / gate-score kernels
+  kErrWaitAttention = 9,    // attention kernel
+  kErrWaitGather = 10,      // gather kernel
   kErrTimeoutFirst = kErrWaitGemm,
-  kErrTimeoutLast = kErrWaitAttention,
+  kErrTimeoutLast = kErrWaitGather,
 };
 
 __device__ uint32_t g_error_word;
@@ -111,6 +114,39 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
       "[%2];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Prefetch a tile into L2 only (no shared-memory destination, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
+}
+
+// Untiled bulk copies (both addresses 16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst_smem)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* dst, const void* src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src_smem)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_1d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x) {
+  asm volatile(
+      "cp.async.bulk.tensor.1d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(x)
       : "memory");
 }
 

@@ -6,8 +6,11 @@
 // i is log m_i / log max(2, p_i) with m_i = i + 1 (rank among kept tokens) and
 // p_i = idx_i + 1 (original position).
 //
-// Each CTA copies kGatherRows rows with 16-byte vector loads, all loads of a
-// thread issued before its stores so several are in flight per thread.
+// k_gather_bulk moves whole rows with the bulk-copy (TMA) engine: one thread
+// per CTA streams batches of rows global -> shared -> global through two
+// shared-memory halves (loads of batch b+1 overlap the stores of batch b)
+// while the other threads write the per-row side outputs.  k_gather (16-byte
+// vector copies by every thread) handles rows too large for the staging buffer.
 #pragma once
 
 #include "common.cuh"
@@ -87,6 +90,76 @@ __global__ void __launch_bounds__(kGatherThreads) k_gather(GatherParams p) {
       if (dst[u] >= 0) *reinterpret_cast<uint4*>(p.out + dst[u]) = v[u];
     }
   }
+}
+
+constexpr int kGatherBulkThreads = 128;
+constexpr int kGatherBatch = 8;                    // rows per bulk batch
+constexpr size_t kGatherStageBytes = 96 * 1024;    // both halves of the staging buffer
+
+__device__ __forceinline__ void gather_side_outputs(const GatherParams& p, int64_t r, int64_t j) {
+  if (p.pos) p.pos[r] = static_cast<int32_t>(j);
+  if (p.bias) {
+    const float rms = sqrtf(p.sumsq[0] / static_cast<float>(p.n_prunable) + p.eps);
+    p.bias[r] = p.scores[j] / rms;
+  }
+  if (p.ratio) {
+    const double lm = log(static_cast<double>(r + 1));
+    const double lp = log(fmax(2.0, static_cast<double>(j) + 1.0));
+    p.ratio[r] = static_cast<float>(lm / lp);
+  }
+}
+
+// rows_per_batch * row_bytes * 2 <= dynamic shared memory; rows [r_begin, r_end) per CTA.
+__global__ void __launch_bounds__(kGatherBulkThreads) k_gather_bulk(GatherParams p, int rows_per_batch) {
+  extern __shared__ __align__(128) uint8_t gbuf[];
+  __shared__ uint64_t bar[2];
+  const int64_t per = (p.m + gridDim.x - 1) / gridDim.x;
+  const int64_t r_begin = static_cast<int64_t>(blockIdx.x) * per;
+  const int64_t r_end = min(p.m, r_begin + per);
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // per-row side outputs (every thread but the copy issuer)
+  for (int64_t r = r_begin + threadIdx.x - 1; threadIdx.x > 0 && r < r_end; r += kGatherBulkThreads - 1) {
+    const int64_t j = p.idx[r];
+    if (j < 0 || j >= p.n) {
+      raise_error(kErrGatherIndex, static_cast<uint32_t>(r & 0xffffff));
+      continue;
+    }
+    gather_side_outputs(p, r, j);
+  }
+  if (threadIdx.x != 0) return;
+  // the copy issuer
+  const uint32_t rb = static_cast<uint32_t>(p.row_bytes);
+  int batch = 0;
+  bool ok = true;
+  for (int64_t r0 = r_begin; r0 < r_end && ok; r0 += rows_per_batch, ++batch) {
+    const int b = batch & 1;
+    const int cnt = static_cast<int>(min(static_cast<int64_t>(rows_per_batch), r_end - r0));
+    uint8_t* half = gbuf + static_cast<size_t>(b) * rows_per_batch * rb;
+    // this half was last read by the stores of batch - 2: keep at most the
+    // newest group (batch - 1) in flight
+    bulk_wait_read<1>();
+    int64_t src[kGatherBatch];
+    uint32_t bytes = 0;
+    for (int i = 0; i < cnt; ++i) {
+      const int64_t j = p.idx[r0 + i];
+      src[i] = (j >= 0 && j < p.n) ? j : -1;  // a bad index was reported above; its row is skipped
+      if (src[i] >= 0) bytes += rb;
+    }
+    mbar_arrive_expect_tx(&bar[b], bytes);
+    for (int i = 0; i < cnt; ++i)
+      if (src[i] >= 0) bulk_load(half + static_cast<size_t>(i) * rb, p.hidden + src[i] * p.row_bytes, rb, &bar[b]);
+    ok = mbar_wait(&bar[b], (batch >> 1) & 1, kErrWaitGather);
+    if (!ok) break;
+    for (int i = 0; i < cnt; ++i)
+      if (src[i] >= 0) bulk_store(p.out + (r0 + i) * p.row_bytes, half + static_cast<size_t>(i) * rb, rb);
+    bulk_commit();
+  }
+  bulk_wait_all();
 }
 
 }  // namespace tg

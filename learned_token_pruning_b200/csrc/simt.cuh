@@ -229,18 +229,26 @@ __global__ void __launch_bounds__(256) k_gemm_simt(const T* __restrict__ A, int6
 }
 
 // ---------------------------------------------------------------------------
-// Row RMSNorm: y = x / sqrt(mean(x^2) + eps) * w; one block per row.
+// Row RMSNorm: y = x / sqrt(mean(x^2) + eps) * w; one block per row, 16-byte
+// vector accesses (the row is read twice; the second read hits L1).
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ x, T* __restrict__ y,
                                                  const float* __restrict__ w, int d, float eps) {
+  constexpr int V = 16 / sizeof(T);  // elements per 16-byte vector
   __shared__ float part[8];
   const T* xr = x + static_cast<int64_t>(blockIdx.x) * d;
   T* yr = y + static_cast<int64_t>(blockIdx.x) * d;
+  const int nv = d / V;  // d % V == 0 (checked by the caller)
   float ss = 0.0f;
-  for (int i = threadIdx.x; i < d; i += 256) {
-    const float v = to_f32(xr[i]);
-    ss += v * v;
+  for (int c = threadIdx.x; c < nv; c += 256) {
+    const uint4 v = reinterpret_cast<const uint4*>(xr)[c];
+    const T* e = reinterpret_cast<const T*>(&v);
+#pragma unroll
+    for (int t = 0; t < V; ++t) {
+      const float f = to_f32(e[t]);
+      ss = fmaf(f, f, ss);
+    }
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -250,15 +258,24 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ x, T* __r
 #pragma unroll
   for (int i = 0; i < 8; ++i) tot += part[i];
   const float inv = 1.0f / sqrtf(tot / static_cast<float>(d) + eps);
-  for (int i = threadIdx.x; i < d; i += 256) yr[i] = from_f32<T>(to_f32(xr[i]) * inv * (w ? w[i] : 1.0f));
+  for (int c = threadIdx.x; c < nv; c += 256) {
+    const uint4 v = reinterpret_cast<const uint4*>(xr)[c];
+    const T* e = reinterpret_cast<const T*>(&v);
+    uint4 o;
+    T* oe = reinterpret_cast<T*>(&o);
+#pragma unroll
+    for (int t = 0; t < V; ++t) oe[t] = from_f32<T>(to_f32(e[t]) * inv * (w ? w[c * V + t] : 1.0f));
+    reinterpret_cast<uint4*>(yr)[c] = o;
+  }
 }
 
 // ---------------------------------------------------------------------------
 // Per-head q/k RMSNorm (optional) and rotate-half RoPE at the original token
-// positions, in place on the fused qkv rows.  One warp per (row, head) of the
-// hq + hkv rotated heads; lane l holds dims l*E .. l*E+E-1 of the first half
-// and the matching dims of the second half, so each pair is in one thread.
-// Angles are formed in double precision (positions reach 2^17).
+// positions, in place on the fused qkv rows.  A block takes 256/(D/2) rows:
+// first one thread per (row, frequency) forms cos/sin of pos * theta^(-2i/D)
+// in double precision (positions reach 2^17) into shared memory, then each
+// warp walks the (row, head) items of the hq + hkv rotated heads; lane l holds
+// dims l*E .. l*E+E-1 of the first half and the matching dims of the second.
 // ---------------------------------------------------------------------------
 template <typename T, int D>
 __global__ void __launch_bounds__(256) k_qk_norm_rope(T* __restrict__ qkv, int64_t ld, int m, int hq, int hkv,
@@ -266,48 +283,57 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope(T* __restrict__ qkv, int64
                                                       const float* __restrict__ wq, const float* __restrict__ wk,
                                                       int qk_norm, float eps, float theta) {
   constexpr int H2 = D / 2;
-  constexpr int E = H2 / 32;  // first-half dims per lane
-  const int lane = threadIdx.x & 31;
-  const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int heads = hq + hkv;
-  if (item >= static_cast<int64_t>(m) * heads) return;
-  const int64_t r = item / heads;
-  const int hh = static_cast<int>(item - r * heads);
-  T* x = qkv + r * ld + static_cast<int64_t>(hh) * D;
-  const bool is_q = hh < hq;
-  float a[E], b[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    a[e] = to_f32(x[lane * E + e]);
-    b[e] = to_f32(x[H2 + lane * E + e]);
+  constexpr int E = H2 / 32;
+  constexpr int ROWS = 256 / H2;
+  __shared__ float2 cs[ROWS][H2];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r0 = blockIdx.x * ROWS;
+  {
+    const int rr = threadIdx.x / H2, i = threadIdx.x % H2;
+    const int r = r0 + rr;
+    float2 v = make_float2(1.0f, 0.0f);
+    if (r < m) {
+      const double p = static_cast<double>(pos ? pos[r] : r);
+      const double ang = p * exp(-2.0 * static_cast<double>(i) / static_cast<double>(D) * log(static_cast<double>(theta)));
+      double sn, cn;
+      sincos(ang, &sn, &cn);
+      v = make_float2(static_cast<float>(cn), static_cast<float>(sn));
+    }
+    cs[rr][i] = v;
   }
-  if (qk_norm) {
-    float ss = 0.0f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) ss += a[e] * a[e] + b[e] * b[e];
-#pragma unroll
-    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float inv = 1.0f / sqrtf(ss / static_cast<float>(D) + eps);
-    const float* w = is_q ? wq : wk;
+  __syncthreads();
+  const int heads = hq + hkv;
+  for (int item = warp; item < ROWS * heads; item += 8) {
+    const int rr = item / heads, hh = item - rr * heads;
+    const int r = r0 + rr;
+    if (r >= m) continue;  // warp-uniform
+    T* x = qkv + static_cast<int64_t>(r) * ld + static_cast<int64_t>(hh) * D;
+    float a[E], b[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      a[e] *= inv * w[lane * E + e];
-      b[e] *= inv * w[H2 + lane * E + e];
+      a[e] = to_f32(x[lane * E + e]);
+      b[e] = to_f32(x[H2 + lane * E + e]);
     }
-  }
-  const double p = static_cast<double>(pos ? pos[r] : static_cast<int32_t>(r));
-  const double ltheta = log(static_cast<double>(theta));
+    if (qk_norm) {
+      float ss = 0.0f;
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const int i = lane * E + e;
-    const double ang = p * exp(-2.0 * static_cast<double>(i) / static_cast<double>(D) * ltheta);
-    double s, c;
-    sincos(ang, &s, &c);
-    const float cf = static_cast<float>(c), sf = static_cast<float>(s);
-    const float na = a[e] * cf - b[e] * sf;
-    const float nb = b[e] * cf + a[e] * sf;
-    x[i] = from_f32<T>(na);
-    x[H2 + i] = from_f32<T>(nb);
+      for (int e = 0; e < E; ++e) ss += a[e] * a[e] + b[e] * b[e];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float inv = 1.0f / sqrtf(ss / static_cast<float>(D) + eps);
+      const float* w = hh < hq ? wq : wk;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        a[e] *= inv * w[lane * E + e];
+        b[e] *= inv * w[H2 + lane * E + e];
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float2 c = cs[rr][lane * E + e];
+      x[lane * E + e] = from_f32<T>(a[e] * c.x - b[e] * c.y);
+      x[H2 + lane * E + e] = from_f32<T>(b[e] * c.x + a[e] * c.y);
+    }
   }
 }
 

@@ -10,12 +10,16 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "../../include/tg.h"
 #include "attn_tc.cuh"
 #include "common.cuh"
+#include "gate_tc.cuh"
 #include "gather.cuh"
 #include "gemm_tc.cuh"
 #include "select.cuh"
@@ -64,53 +68,120 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [rows][inner] with a row stride in bytes; box {64, box_rows}, 128-byte swizzle.
+// 2-D bf16 tensor [rows][inner] with a row stride in bytes; box {box_inner, box_rows}.  Operand
+// tiles use a 64-column box with the 128-byte swizzle; L2-prefetch maps use wider unswizzled boxes.
 int make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t row_stride_bytes,
-             uint32_t box_rows) {
+             uint32_t box_rows, uint32_t box_inner = 64, bool swizzle = true) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(TG_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {row_stride_bytes};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(TG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return TG_OK;
 }
 
+// 1-D fp32 vector of n elements, box of `box` elements, no swizzle (bounds fill: zeros).
+int make_map_1d_f32(CUtensorMap* map, const void* base, uint64_t n, uint32_t box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(TG_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[1] = {n};
+  cuuint64_t strides[1] = {0};
+  cuuint32_t bx[1] = {box};
+  cuuint32_t estr[1] = {1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, const_cast<void*>(base), dims, strides, bx, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TG_ERR_CUDA, "cuTensorMapEncodeTiled (1-D) failed (%d)", static_cast<int>(r));
+  return TG_OK;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device): the
+// attribute call is host work that would otherwise repeat on every launch.
+std::mutex g_smem_mu;
+std::map<std::pair<const void*, int>, size_t> g_smem_set;
+
 template <typename Kern>
 int set_smem(Kern k, size_t bytes) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const auto key = std::make_pair(reinterpret_cast<const void*>(k), dev);
+  {
+    std::lock_guard<std::mutex> lock(g_smem_mu);
+    auto it = g_smem_set.find(key);
+    if (it != g_smem_set.end() && it->second >= bytes) return TG_OK;
+  }
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
   if (e != cudaSuccess) return fail(TG_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+  std::lock_guard<std::mutex> lock(g_smem_mu);
+  size_t& v = g_smem_set[key];
+  if (bytes > v) v = bytes;
   return TG_OK;
 }
 
 // ---------------------------------------------------------------------------
-// tcgen05 GEMM launch
+// tcgen05 launches
 // ---------------------------------------------------------------------------
 constexpr int kGemmStages = 4;
 
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+// Persistent GEMM: grid = min(tiles, SMs); B has b_rows rows of K elements.
 template <int BN, int EPI>
-int launch_gemm_tc(const void* A, int64_t lda, const void* B, int64_t b_rows, int M, int K, const tg::GemmParams& p0,
-                   int grid_n, cudaStream_t st) {
+int launch_gemm_tc(const void* A, int64_t lda, const void* B, int64_t b_rows, int M, int K, int tiles_n,
+                   const tg::GemmParams& p0, cudaStream_t st) {
+  using Cfg = tg::GemmCfg<BN, kGemmStages>;
   CUtensorMap ta, tb;
   int rc = make_map(&ta, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(lda) * 2, 128);
   if (rc) return rc;
   rc = make_map(&tb, B, static_cast<uint64_t>(K), static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K) * 2,
-                tg::GemmCfg<BN>::kBBox);
+                Cfg::kBBox);
   if (rc) return rc;
   auto kern = tg::k_gemm_tc<BN, kGemmStages, EPI>;
-  const size_t smem = tg::gemm_smem_bytes<BN, kGemmStages>();
-  rc = set_smem(kern, smem);
+  rc = set_smem(kern, Cfg::kSmem);
   if (rc) return rc;
   tg::GemmParams p = p0;
   p.M = M;
   p.K = K;
-  dim3 grid(grid_n, (M + tg::kGemmBM - 1) / tg::kGemmBM);
-  kern<<<grid, tg::kGemmThreads, smem, st>>>(ta, tb, p);
+  p.tiles_m = (M + tg::kGemmBM - 1) / tg::kGemmBM;
+  p.tiles_n = tiles_n;
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int grid = tiles < sm_count() ? tiles : sm_count();
+  kern<<<grid, tg::kGemmThreads, Cfg::kSmem, st>>>(ta, tb, p);
   return check_launch("k_gemm_tc");
+}
+
+template <int BN>
+int launch_gate_tc(const void* A, const void* W1, int M, int K, const tg::GateParams& p0, cudaStream_t st) {
+  using Cfg = tg::GateCfg<BN>;
+  CUtensorMap ta, tb;
+  int rc = make_map(&ta, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, 128);
+  if (rc) return rc;
+  rc = make_map(&tb, W1, static_cast<uint64_t>(K), static_cast<uint64_t>(p0.N), static_cast<uint64_t>(K) * 2,
+                Cfg::kBBox);
+  if (rc) return rc;
+  rc = set_smem(tg::k_gate_tc<BN>, Cfg::kSmem);
+  if (rc) return rc;
+  tg::GateParams p = p0;
+  p.M = M;
+  p.K = K;
+  p.hidden = static_cast<const __nv_bfloat16*>(A);
+  tg::k_gate_tc<BN><<<(M + tg::kGateBM - 1) / tg::kGateBM, tg::kGateThreads, Cfg::kSmem, st>>>(ta, tb, p);
+  return check_launch("k_gate_tc");
 }
 
 int dtype_size(int dtype) { return dtype == TG_BF16 ? 2 : (dtype == TG_F32 ? 4 : 0); }
@@ -207,7 +278,7 @@ int tg_gate_score(const void* hidden, int dtype, int64_t n, int32_t d_model, con
       if (rc) return rc;
       w1_eff = w1f;
     }
-    tg::GemmParams p{};
+    tg::GateParams p{};
     p.N = h;
     p.b1 = b1;
     p.w2 = w2;
@@ -219,9 +290,9 @@ int tg_gate_score(const void* hidden, int dtype, int64_t n, int32_t d_model, con
     p.counter = counter;
     p.sumsq = sumsq;
     const int nn = static_cast<int>(n);
-    if (h <= 64) return launch_gemm_tc<64, tg::kEpiGateScore>(hidden, d_model, w1_eff, h, nn, d_model, p, 1, st);
-    if (h <= 128) return launch_gemm_tc<128, tg::kEpiGateScore>(hidden, d_model, w1_eff, h, nn, d_model, p, 1, st);
-    return launch_gemm_tc<256, tg::kEpiGateScore>(hidden, d_model, w1_eff, h, nn, d_model, p, 1, st);
+    if (h <= 64) return launch_gate_tc<64>(hidden, w1_eff, nn, d_model, p, st);
+    if (h <= 128) return launch_gate_tc<128>(hidden, w1_eff, nn, d_model, p, st);
+    return launch_gate_tc<256>(hidden, w1_eff, nn, d_model, p, st);
   }
   if (h > 1024) return fail(TG_ERR_UNSUPPORTED, "h > 1024");
   const unsigned blocks = static_cast<unsigned>((n + 7) / 8);
@@ -256,13 +327,59 @@ int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int6
   p.k = k;
   p.out = kept_idx;
   p.m = m;
-  p.slice = (n + tg::kSelCluster - 1) / tg::kSelCluster;
+  if (n <= tg::kSelSmallMax) {
+    // short prompt: one CTA, keys resident in shared memory
+    const int need = static_cast<int>((n + tg::kSelSmallThreads - 1) / tg::kSelSmallThreads);
+    const int kpt = need <= 4 ? 4 : (need <= 8 ? 8 : (need <= 16 ? 16 : 32));
+    const size_t smem = static_cast<size_t>(kpt) * tg::kSelSmallStride * 5 + 16;
+    const int vec = (aligned16(scores) && (reinterpret_cast<uintptr_t>(prunable) & 3u) == 0) ? 1 : 0;
+    cudaStream_t st = as_stream(stream);
+    int rc;
+    switch (kpt) {
+      case 4:
+        if ((rc = set_smem(tg::k_topk_select_cta<4>, smem))) return rc;
+        tg::k_topk_select_cta<4><<<1, tg::kSelSmallThreads, smem, st>>>(p, vec);
+        break;
+      case 8:
+        if ((rc = set_smem(tg::k_topk_select_cta<8>, smem))) return rc;
+        tg::k_topk_select_cta<8><<<1, tg::kSelSmallThreads, smem, st>>>(p, vec);
+        break;
+      case 16:
+        if ((rc = set_smem(tg::k_topk_select_cta<16>, smem))) return rc;
+        tg::k_topk_select_cta<16><<<1, tg::kSelSmallThreads, smem, st>>>(p, vec);
+        break;
+      default:
+        if ((rc = set_smem(tg::k_topk_select_cta<32>, smem))) return rc;
+        tg::k_topk_select_cta<32><<<1, tg::kSelSmallThreads, smem, st>>>(p, vec);
+        break;
+    }
+    return check_launch("k_topk_select_cta");
+  }
+  // cluster of 2, 4 or 8 CTAs: about 4096 tokens per CTA, and slices that fit the key cache
+  int csize = 1;
+  while (csize < tg::kSelCluster &&
+         ((n + csize - 1) / csize > 4096 || static_cast<size_t>((n + csize - 1) / csize) * 5 > tg::kSelCacheBytes))
+    csize *= 2;
+  p.slice = (n + csize - 1) / csize;
   const size_t cache = static_cast<size_t>(p.slice) * 5;
   p.cached = cache <= tg::kSelCacheBytes ? 1 : 0;
   const size_t smem = p.cached ? ((cache + 15) / 16) * 16 : 0;
   int rc = set_smem(tg::k_topk_select, smem > 0 ? smem : 16);
   if (rc) return rc;
-  tg::k_topk_select<<<tg::kSelCluster, tg::kSelThreads, smem, as_stream(stream)>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(csize);
+  cfg.blockDim = dim3(tg::kSelThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = as_stream(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, tg::k_topk_select, p);
+  if (e != cudaSuccess) return fail(TG_ERR_CUDA, "k_topk_select launch: %s", cudaGetErrorString(e));
   return check_launch("k_topk_select");
 }
 
@@ -292,6 +409,19 @@ int tg_gather(const void* hidden, int dtype, int64_t n, int32_t d_model, const i
   p.pos = pos;
   p.bias = bias;
   p.ratio = ratio;
+  const int rows_per_batch =
+      static_cast<int>(std::min<int64_t>(tg::kGatherBatch, static_cast<int64_t>(tg::kGatherStageBytes / 2) / row_bytes));
+  if (rows_per_batch >= 1) {
+    // bulk copies: about eight rows per CTA, at most three CTAs per SM
+    const int64_t want = (m + 7) / 8;
+    const int64_t cap = 3 * static_cast<int64_t>(sm_count());
+    const unsigned blocks = static_cast<unsigned>(want < cap ? want : cap);
+    const size_t smem = static_cast<size_t>(2) * rows_per_batch * row_bytes;
+    int rc = set_smem(tg::k_gather_bulk, smem);
+    if (rc) return rc;
+    tg::k_gather_bulk<<<blocks, tg::kGatherBulkThreads, smem, as_stream(stream)>>>(p, rows_per_batch);
+    return check_launch("k_gather_bulk");
+  }
   const unsigned blocks = static_cast<unsigned>((m + tg::kGatherRows - 1) / tg::kGatherRows);
   tg::k_gather<<<blocks, tg::kGatherThreads, 0, as_stream(stream)>>>(p);
   return check_launch("k_gather");
@@ -331,20 +461,27 @@ int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk, c
     p.out = static_cast<__nv_bfloat16*>(out);
     p.ldo = ldo;
     p.lse = lse;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, tb;
+    std::memset(&tb, 0, sizeof(tb));
     int rc = make_map(&tq, q, uint64_t(hq) * head_dim, uint64_t(m), uint64_t(ldq) * 2, 128);
-    if (!rc) rc = make_map(&tk, k, uint64_t(hkv) * head_dim, uint64_t(m), uint64_t(ldk) * 2, 128);
-    if (!rc) rc = make_map(&tv, v, uint64_t(hkv) * head_dim, uint64_t(m), uint64_t(ldv) * 2, 128);
+    // keys and values come in tiles of 64 rows (AttnCfg::BN)
+    if (!rc) rc = make_map(&tk, k, uint64_t(hkv) * head_dim, uint64_t(m), uint64_t(ldk) * 2, 64);
+    if (!rc) rc = make_map(&tv, v, uint64_t(hkv) * head_dim, uint64_t(m), uint64_t(ldv) * 2, 64);
     if (rc) return rc;
+    p.has_bias = bias != nullptr;
+    if (bias) {
+      if (!aligned16(bias)) return fail(TG_ERR_ALIGN, "bias must be 16-byte aligned");
+      if ((rc = make_map_1d_f32(&tb, bias, uint64_t(m), 64))) return rc;
+    }
     const unsigned blocks = static_cast<unsigned>(p.num_qtiles * hkv * (group / 2));
     if (head_dim == 128) {
       rc = set_smem(tg::k_attn_tc<128>, tg::AttnCfg<128>::kSmem);
       if (rc) return rc;
-      tg::k_attn_tc<128><<<blocks, tg::kAttnThreads, tg::AttnCfg<128>::kSmem, st>>>(tq, tk, tv, p);
+      tg::k_attn_tc<128><<<blocks, tg::kAttnThreads, tg::AttnCfg<128>::kSmem, st>>>(tq, tk, tv, tb, p);
     } else {
       rc = set_smem(tg::k_attn_tc<64>, tg::AttnCfg<64>::kSmem);
       if (rc) return rc;
-      tg::k_attn_tc<64><<<blocks, tg::kAttnThreads, tg::AttnCfg<64>::kSmem, st>>>(tq, tk, tv, p);
+      tg::k_attn_tc<64><<<blocks, tg::kAttnThreads, tg::AttnCfg<64>::kSmem, st>>>(tq, tk, tv, tb, p);
     }
     return check_launch("k_attn_tc");
   }
@@ -396,13 +533,13 @@ int tg_linear(const void* x, int64_t ldx, const void* w, void* y, int64_t ldy, i
     if (epilogue == TG_EPI_SWIGLU) {
       if (n_out % 128 != 0) return fail(TG_ERR_UNSUPPORTED, "SwiGLU epilogue needs n_out %% 128 == 0");
       p.up_row0 = n_out;
-      return launch_gemm_tc<256, tg::kEpiSwiGLU>(x, ldx, w, 2 * int64_t(n_out), mm, k_in, p, n_out / 128, st);
+      return launch_gemm_tc<256, tg::kEpiSwiGLU>(x, ldx, w, 2 * int64_t(n_out), mm, k_in, n_out / 128, p, st);
     }
     if (n_out % 32 == 0) {
       const int gn = (n_out + 255) / 256;
       if (epilogue == TG_EPI_RESIDUAL)
-        return launch_gemm_tc<256, tg::kEpiResidual>(x, ldx, w, n_out, mm, k_in, p, gn, st);
-      return launch_gemm_tc<256, tg::kEpiStore>(x, ldx, w, n_out, mm, k_in, p, gn, st);
+        return launch_gemm_tc<256, tg::kEpiResidual>(x, ldx, w, n_out, mm, k_in, gn, p, st);
+      return launch_gemm_tc<256, tg::kEpiStore>(x, ldx, w, n_out, mm, k_in, gn, p, st);
     }
   }
   if (epilogue == TG_EPI_SWIGLU) return fail(TG_ERR_UNSUPPORTED, "SwiGLU epilogue needs bf16");
@@ -438,6 +575,7 @@ int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, 
   if (S->head_dim != 64 && S->head_dim != 128) return fail(TG_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
   const int es = dtype_size(S->dtype);
   if (!es) return fail(TG_ERR_INVALID_ARG, "dtype");
+  if ((S->d_model * es) % 16 != 0) return fail(TG_ERR_UNSUPPORTED, "d_model rows must be a multiple of 16 bytes");
   const size_t need = tg_workspace_bytes(TG_OP_LAYER, 0, m, 0, 0, S);
   if (!ws || ws_bytes < need) return fail(TG_ERR_WORKSPACE, "layer needs %zu workspace bytes", need);
   cudaStream_t st = as_stream(stream);
@@ -467,8 +605,8 @@ int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, 
   if ((rc = tg_linear(xn, d, W->w_qkv, qkv, qkv_w, S->dtype, m, int32_t(qkv_w), d, TG_EPI_STORE, stream))) return rc;
   // 3. per-head q/k norm and RoPE at the original positions
   {
-    const int64_t items = m * (hq + hkv);
-    const unsigned blocks = unsigned((items + 7) / 8);
+    const int rows_per_block = 256 / (D / 2);
+    const unsigned blocks = unsigned((m + rows_per_block - 1) / rows_per_block);
     if (bf) {
       if (D == 128)
         tg::k_qk_norm_rope<__nv_bfloat16, 128><<<blocks, 256, 0, st>>>(

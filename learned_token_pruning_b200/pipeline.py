@@ -85,3 +85,22 @@ class GatedPrefillStep:
         self.gather(stream)
         self.layer_above(stream)
         return self.hidden_kept
+
+    def capture(self):
+        """Record run() once into a CUDA graph, so a step costs one graph launch
+        (the TMA descriptors and launch parameters are baked into the graph).
+        One eager step runs first to set the kernels' attributes up."""
+        self.run()
+        torch.cuda.synchronize(self.device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.run()
+        self._graph = graph
+        return graph
+
+    def replay(self):
+        """One step by replaying the captured graph on the current stream."""
+        if getattr(self, "_graph", None) is None:
+            self.capture()
+        self._graph.replay()
+        return self.hidden_kept

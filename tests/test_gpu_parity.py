@@ -441,3 +441,12 @@ def test_step_qwen3_16k_full_size_sampled():
     rng = np.random.default_rng(0)
     rows = np.unique(np.r_[0, 1, 8191, 8192, 8200, 16319, 16320, 16383, rng.integers(0, w.n, 200)])
     _check_step(w, dict(score=1e-3, layer=LAYER_BF16), sample_rows=rows)
+
+
+def test_attention_bf16_zero_gain_ignores_bias():
+    q, k, v, bias, ratio, gain, temp = _attn_case(260, 4, 2, 128, "bf16", seed=21)
+    gain[[0, 3]] = 0.0
+    got, lse = _gpu_attn(q, k, v, 128, bias, ratio, gain, temp, "bf16")
+    want, wlse = _oracle_attn(q, k, v, 128, bias, ratio, gain, temp)
+    assert_close(got, want, what="out", **ATTN_BF16)
+    assert_close(lse, wlse, 2e-2, 1e-3, "lse")
