@@ -332,13 +332,16 @@ def breakdown(step, w, args, stream, flush):
     act = torch.empty(m, w.d_ff, dtype=dt, device=stream.device)
     hres = torch.randn(m, w.d_model, device=stream.device).to(dt)
     L = step.layer
+    aws_n = tg.attention_workspace_bytes(m, hq, hkv, D, dt)
+    aws = torch.empty(max(aws_n, 16), dtype=torch.uint8, device=stream.device) if aws_n else None
     calls = {
         "gate_score": step.gate_score,
         "topk_select": step.select,
         "gather": step.gather,
         "attention": lambda: tg.tg_gated_attention(qkv[:, :hq * D], qkv[:, hq * D:(hq + hkv) * D],
                                                    qkv[:, (hq + hkv) * D:], D, step.bias, L["head_gain"],
-                                                   L["head_temp"], step.ratio, 1.0 / math.sqrt(D), att),
+                                                   L["head_temp"], step.ratio, 1.0 / math.sqrt(D), att,
+                                                   ws=aws),
         "linear_qkv": lambda: tg.tg_linear(xn, L["w_qkv"], qkv),
         "linear_o": lambda: tg.tg_linear(att, L["w_o"], hres, tg.TG_EPI_RESIDUAL),
         "linear_gate_up_swiglu": lambda: tg.tg_linear(xn, L["w_gate_up"], act, tg.TG_EPI_SWIGLU),
@@ -422,9 +425,12 @@ def ncu_case():
     m, hq, hkv, D = 2064, 16, 8, 128
     qkv = torch.randn(m, (hq + 2 * hkv) * D, device=dev).to(torch.bfloat16)
     out = torch.empty(m, hq * D, dtype=torch.bfloat16, device=dev)
+    aws_n = tg.attention_workspace_bytes(m, hq, hkv, D, torch.bfloat16)
+    aws = torch.empty(max(aws_n, 16), dtype=torch.uint8, device=dev) if aws_n else None
     tg.tg_gated_attention(qkv[:, :hq * D], qkv[:, hq * D:(hq + hkv) * D], qkv[:, (hq + hkv) * D:], D,
                           torch.randn(m, device=dev), torch.rand(hq, device=dev) + 0.5,
-                          torch.rand(hq, device=dev) * 0.4 + 0.8, torch.rand(m, device=dev), 1 / math.sqrt(D), out)
+                          torch.rand(hq, device=dev) * 0.4 + 0.8, torch.rand(m, device=dev), 1 / math.sqrt(D), out,
+                          ws=aws)
     x = torch.randn(m, 2048, device=dev).to(torch.bfloat16)
     wgu = (torch.randn(2 * 6144, 2048, device=dev) * 0.02).to(torch.bfloat16)
     act = torch.empty(m, 6144, dtype=torch.bfloat16, device=dev)

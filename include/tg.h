@@ -164,15 +164,22 @@ int tg_gather(const void* hidden, int dtype, int64_t n, int32_t d_model,
  *   bias device fp32 [m] or NULL (0);  ratio device fp32 [m] or NULL (1)
  *   head_gain, head_temp  device fp32 [hq] (values after softplus)
  *   lse  device fp32 [hq][m] out (natural-log sum of exp of l) or NULL
- * head_dim in {64, 128}; hq % hkv == 0.  bf16 runs on the tcgen05 tensor cores
- * (fp32 softmax and accumulation); fp32 runs on CUDA cores in full fp32.
+ *   ws   device workspace of tg_workspace_bytes(TG_OP_ATTENTION, 0, m, 0, 0, shape)
+ *        bytes (shape gives dtype, hq, hkv, head_dim), 16-byte aligned, or NULL.
+ *        When the causal work is about one wave of the GPU, the longest query
+ *        blocks are split over two CTAs whose partial results meet in ws; with
+ *        ws NULL (or smaller than required) nothing is split.  The size depends
+ *        on the SM count of the current device and is 0 when no split is made.
+ * head_dim in {64, 128}; hq % hkv == 0.  bf16 with an even hq / hkv runs on the
+ * tcgen05 tensor cores (fp32 softmax and accumulation); fp32 and odd groups
+ * run on CUDA cores in full fp32.
  */
 int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk,
                        const void* v, int64_t ldv, int dtype, int64_t m,
                        int32_t hq, int32_t hkv, int32_t head_dim,
                        const float* bias, const float* head_gain, const float* head_temp,
                        const float* ratio, float sm_scale,
-                       void* out, int64_t ldo, float* lse, void* stream);
+                       void* out, int64_t ldo, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* Weights of one Qwen3-style decoder layer (device pointers). */
 typedef struct {
@@ -233,10 +240,12 @@ enum { TG_EPI_STORE = 0, TG_EPI_RESIDUAL = 1, TG_EPI_SWIGLU = 2 };
 int tg_linear(const void* x, int64_t ldx, const void* w, void* y, int64_t ldy, int dtype,
               int64_t m, int32_t n_out, int32_t k_in, int epilogue, void* stream);
 
-enum { TG_OP_GATE_SCORE = 0, TG_OP_LAYER = 1 };
+enum { TG_OP_GATE_SCORE = 0, TG_OP_LAYER = 1, TG_OP_ATTENTION = 2 };
 
 /* Workspace bytes needed by an op: TG_OP_GATE_SCORE uses n, d_model and h;
- * TG_OP_LAYER uses m and shape.  Returns 0 for an invalid request. */
+ * TG_OP_LAYER and TG_OP_ATTENTION use m and shape (TG_OP_ATTENTION reads its
+ * dtype, hq, hkv and head_dim).  Returns 0 for an invalid request, and 0 for
+ * TG_OP_ATTENTION when the attention needs no workspace. */
 size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t h, const tg_layer_shape* shape);
 
 /*

@@ -88,6 +88,22 @@ struct AttnTcParams {
   __nv_bfloat16* out;
   int64_t ldo;
   float* lse;
+  // Key-range split of the longest query blocks (see AttnWork): query blocks
+  // t >= ts run as two CTAs each; their partial results meet in `part`.
+  int use_table;  // blocks take their work item from AttnWork (else: block b -> query block T-1-b/per_tile, whole)
+  int ts;
+  float4* part;   // [slot][half][head][D/4][128 rows] unnormalised O
+  float2* part_ml;  // [slot][half][head][128 rows] (running max of y, running sum)
+  unsigned* counters;  // [slot], zero on entry
+};
+
+// Work items of the CTAs in launch order, longest first: item i covers the
+// blocks i*per_tile .. i*per_tile + per_tile - 1 (one per head pair) and
+// encodes the query block in bits 2.. and the part in bits 0-1 (0 the whole
+// key range, 1 the first half of the key tiles, 2 the second half).
+constexpr int kAttnWorkCap = 1920;
+struct AttnWork {
+  uint16_t item[kAttnWorkCap];
 };
 
 // 2^x by the hardware approximation (ex2.approx.ftz.f32, the MUFU unit).
@@ -151,7 +167,7 @@ template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmBias,
-              AttnTcParams p) {
+              const __grid_constant__ CUtensorMap tmO, AttnTcParams p, const __grid_constant__ AttnWork work) {
   using Cfg = AttnCfg<D>;
   constexpr int BN = Cfg::BN;
   constexpr int kDBoxes = D / 64;
@@ -173,20 +189,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
+  __shared__ int s_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // longest query blocks first: the last row block has the most causal work
+  // longest work first (the last row block has the most causal work)
   const int pairs_per_kv = p.group / 2;
   const int per_tile = p.hkv * pairs_per_kv;
-  const int t = p.num_qtiles - 1 - static_cast<int>(blockIdx.x) / per_tile;
+  int t, part_code = 0;
+  if (p.use_table) {
+    const int it = work.item[blockIdx.x / per_tile];
+    t = it >> 2;
+    part_code = it & 3;
+  } else {
+    t = p.num_qtiles - 1 - static_cast<int>(blockIdx.x) / per_tile;
+  }
   const int pair = static_cast<int>(blockIdx.x) % per_tile;
   const int g = pair / pairs_per_kv;
   const int h0 = g * p.group + 2 * (pair % pairs_per_kv);
-  // causal: key tiles 0 .. (128t + 127) / 64, and none past the last kept row
-  const int nt = min(2 * t + 2, (p.m + BN - 1) / BN);
+  // causal: key tiles 0 .. (128t + 127) / 64, and none past the last kept row;
+  // a split block takes the first or the second half of them
+  const int nt_all = min(2 * t + 2, (p.m + BN - 1) / BN);
+  const int j0 = part_code == 2 ? nt_all / 2 : 0;
+  const int j1 = part_code == 1 ? nt_all / 2 : nt_all;
+  const int nt = j1 - j0;  // key tiles of this CTA; local tile i is global tile j0 + i
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 3; ++s) mbar_init(&k_full[s], 1);
+    for (int s = 0; s < Cfg::kKStages; ++s) mbar_init(&k_full[s], 1);
     for (int s = 0; s < 2; ++s) mbar_init(&v_full[s], 1);
     for (int s = 0; s < 4; ++s) mbar_init(&pv_done[s], 1);
     for (int i = 0; i < 4; ++i) {
@@ -229,15 +257,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int ks = j % 3, vs = j & 1;
         mbar_arrive_expect_tx(&k_full[ks], Cfg::kKVBytes + (p.has_bias ? BN * 4 : 0));
         for (int b = 0; b < kDBoxes; ++b)
-          tma_load_2d(sK + ks * Cfg::kKVBytes + b * Cfg::kKVBlk, &tmK, &k_full[ks], g * D + 64 * b, j * BN);
-        if (p.has_bias) tma_load_1d(sBias + ks * BN, &tmBias, &k_full[ks], j * BN);
+          tma_load_2d(sK + ks * Cfg::kKVBytes + b * Cfg::kKVBlk, &tmK, &k_full[ks], g * D + 64 * b, (j0 + j) * BN);
+        if (p.has_bias) tma_load_1d(sBias + ks * BN, &tmBias, &k_full[ks], (j0 + j) * BN);
         if (j >= 2 && !mbar_wait(&pv_done[(j - 2) & 3], ((j - 2) >> 2) & 1, kErrWaitAttention)) {
           *abort_flag = 1;
           break;
         }
         mbar_arrive_expect_tx(&v_full[vs], Cfg::kKVBytes);
         for (int b = 0; b < kDBoxes; ++b)
-          tma_load_2d(sV + vs * Cfg::kKVBytes + b * Cfg::kKVBlk, &tmV, &v_full[vs], g * D + 64 * b, j * BN);
+          tma_load_2d(sV + vs * Cfg::kKVBytes + b * Cfg::kKVBlk, &tmV, &v_full[vs], g * D + 64 * b, (j0 + j) * BN);
       }
     }
   } else if (warp == 9) {
@@ -343,7 +371,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // independent chains); the causal mask only touches the key tiles that
       // cross the diagonal.
       uint64_t y2[BN / 2];
-      const int key0 = j * BN;
+      const int key0 = (j0 + j) * BN;
       const bool diag = key0 + BN - 1 > t * 128;  // warp-uniform
       float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       auto logits = [&](const uint32_t(&r)[32], int c0) {
@@ -440,30 +468,101 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(&p_full[2 * wg + b]);
     }
     if (ok && !*abort_flag) ok = warp_wait(o_final, 0, kErrWaitAttention);
-    if (ok) {
+    // every softmax thread ends here, so the named barriers below see all 256
+    if (!ok) *abort_flag = 1;
+    float mm = m_run, inv = 0.0f, s_me = 1.0f, s_ot = 0.0f;
+    const float4* other = nullptr;
+    bool own_first = true;  // merge as fma(O_second, s_second, O_first * s_first) whichever half merges
+    bool write_out = ok;
+    if (part_code != 0) {
+      // half of a split row block: publish the unnormalised O and (max, sum);
+      // the half that finishes second merges both and writes the output
+      const int slot = (t - p.ts) * per_tile + pair;
+      const int half = part_code - 1;
+      float4* mine = p.part + ((static_cast<size_t>(slot) * 2 + half) * 2 + wg) * (D / 4) * 128;
+      if (ok) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + colO + c0, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            mine[(c0 / 4 + v) * 128 + row] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                                         __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+        }
+        p.part_ml[((static_cast<size_t>(slot) * 2 + half) * 2 + wg) * 128 + row] = make_float2(m_run, l_run);
+      }
+      __threadfence();
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (threadIdx.x == 0) s_last = (!*abort_flag && atomicAdd(&p.counters[slot], 1u) == 1u) ? 1 : 0;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      write_out = ok && s_last;
+      if (write_out) {
+        __threadfence();
+        const size_t ob = (static_cast<size_t>(slot) * 2 + (1 - half)) * 2 + wg;
+        const float2 oml = __ldcg(&p.part_ml[ob * 128 + row]);
+        other = p.part + ob * (D / 4) * 128;
+        own_first = half == 0;
+        mm = fmaxf(m_run, oml.x);
+        s_me = ex2_approx(gg * (m_run - mm));
+        s_ot = ex2_approx(gg * (oml.x - mm));
+        // the same rounding whichever half merges: fma(l_second, s_second, l_first * s_first)
+        inv = 1.0f / (own_first ? fmaf(oml.y, s_ot, l_run * s_me) : fmaf(l_run, s_me, oml.y * s_ot));
+        s_me *= inv;
+        s_ot *= inv;
+        if (threadIdx.x == 0) p.counters[slot] = 0u;  // ready for the next launch
+      }
+    } else if (ok) {
+      inv = 1.0f / l_run;
+      s_me = inv;
+    }
+    if (write_out) {
+      // O as bf16 into the P buffers (free once o_final has completed), in the
+      // 128-byte-swizzled layout of the output tensor map: box b holds columns
+      // 64b..64b+63, row r at 128 r, 16-byte chunk c at c ^ (r & 7)
+      uint8_t* stage = sP + wg * (Cfg::kPBytes * 2);
       tc_fence_after();
-      const float inv = 1.0f / l_run;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
         tmem_ld32(tmem + lane_base + colO + c0, o);
         tmem_ld_wait();
-        if (grow < p.m) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(grow) * p.ldo + h * D + c0);
+        float f[32];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
-            dst[v] = w;
+        for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(o[e]) * s_me;
+        if (other) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const float4 w4 = __ldcg(&other[(c0 / 4 + v) * 128 + row]);
+            const float w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float own = __uint_as_float(o[4 * v + u]);
+              f[4 * v + u] = own_first ? fmaf(w[u], s_ot, own * s_me) : fmaf(own, s_me, w[u] * s_ot);
+            }
           }
         }
+        uint8_t* box = stage + (c0 / 64) * (128 * 128) + row * 128;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int chunk = (c0 % 64) / 8 + v;
+          *reinterpret_cast<uint4*>(box + ((chunk ^ sw) << 4)) =
+              make_uint4(pack_bf16x2(f[8 * v], f[8 * v + 1]), pack_bf16x2(f[8 * v + 2], f[8 * v + 3]),
+                         pack_bf16x2(f[8 * v + 4], f[8 * v + 5]), pack_bf16x2(f[8 * v + 6], f[8 * v + 7]));
+        }
       }
-      if (p.lse && grow < p.m) p.lse[static_cast<int64_t>(h) * p.m + grow] = (gg * m_run + log2f(l_run)) * kLn2;
-    } else {
-      *abort_flag = 1;
+      // the warpgroup's tile is staged: one thread stores it (rows past m are clipped)
+      fence_proxy_async_smem();
+      if (wg == 0) asm volatile("bar.sync 2, 128;" ::: "memory");
+      else asm volatile("bar.sync 3, 128;" ::: "memory");
+      if (row == 0) {
+        for (int b = 0; b < kDBoxes; ++b) tma_store_2d(&tmO, stage + b * (128 * 128), h * D + 64 * b, t * 128);
+        bulk_commit();
+        bulk_wait_all();  // written out before the CTA (and its shared memory) goes away
+      }
+      if (p.lse && grow < p.m) p.lse[static_cast<int64_t>(h) * p.m + grow] = (gg * mm - log2f(inv)) * kLn2;
     }
   }
   tc_fence_before();

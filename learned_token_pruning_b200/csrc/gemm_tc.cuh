@@ -2,12 +2,18 @@
 // epilogues: C[M][N] = A[M][K] * B[N][K]^T (both operands K-major, the
 // nn.Linear layout), fp32 accumulation in tensor memory.
 //
-// One CTA per SM walks the 128 x BN output tiles (m fastest, so the weight
-// block of a column of tiles is fetched from HBM about once).  TMA streams
-// 128x64 A tiles and BNx64 B tiles (128-byte swizzle) through a STAGES-deep
-// shared-memory ring; a single thread issues tcgen05.mma (M=128, N=BN, K=16).
-// The accumulator is double-buffered in tensor memory (2 x BN columns), so the
-// four epilogue warps drain tile i while the MMAs of tile i+1 run.
+// One CTA per SM walks the (128 MH) x BN output tiles (m fastest, so the
+// weight block of a column of tiles is fetched from HBM about once).  TMA
+// streams MH 128x64 A tiles and a BNx64 B tile (128-byte swizzle) through a
+// STAGES-deep shared-memory ring; a single thread issues tcgen05.mma (M=128,
+// N=BN, K=16) for each of the MH row halves, which share the B tile.
+//   MH = 1: the accumulator is double-buffered in tensor memory (2 x BN
+//           columns), so the epilogue drains tile i while tile i+1 runs.
+//   MH = 2: a 256 x BN tile reads half as many B bytes per FLOP (the operand
+//           feed from L2 is what bounds these GEMMs); its two 128 x BN
+//           accumulators fill tensor memory, so the MMAs of tile i+1 wait for
+//           the epilogue of tile i.
+// A GEMM whose 256-row tiles would leave SMs idle keeps MH = 1.
 // Epilogues:
 //   kEpiStore     C = acc                                (bf16)
 //   kEpiResidual  C = C + acc                            (bf16, in place)
@@ -15,17 +21,16 @@
 //                 output block f is the 128 gate rows of those features
 //                 followed by their 128 up rows, so the MLP activation is
 //                 formed in registers and the [M][2*d_ff] product is never stored.
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
-// issuer, warps 2-5 epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps
+// 2 .. 2+4MH-1 epilogue (warp w reads TMEM lanes 32*(w%4)..+31 of row half
+// (w-2)/4).
 #pragma once
 
 #include "common.cuh"
 
 namespace tg {
 
-constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 64;
-constexpr int kGemmThreads = 192;
 
 enum GemmEpilogue { kEpiStore = 0, kEpiResidual = 1, kEpiSwiGLU = 2 };
 
@@ -37,28 +42,33 @@ struct GemmParams {
   int up_row0;  // SwiGLU: first B row of the up block (= d_ff)
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int MH>
 struct GemmCfg {
-  static constexpr int kABytes = kGemmBM * kGemmBK * 2;
+  static constexpr int kBM = 128 * MH;
+  static constexpr int kABytes = kBM * kGemmBK * 2;  // MH boxes of 128 rows
   static constexpr int kBBytes = BN * kGemmBK * 2;
   static constexpr int kBBox = BN < 128 ? BN : 128;  // rows per B TMA box
   static constexpr int kAccCols = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
-  static constexpr int kTmemCols = 2 * kAccCols;
+  static constexpr int kBufCols = MH * kAccCols;     // one accumulator buffer: every row half
+  static constexpr int kBufs = 2 * kBufCols <= 512 ? 2 : 1;
+  static constexpr int kTmemCols = kBufs * kBufCols;
+  static constexpr int kEpiWarps = 4 * MH;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr size_t kSmem = 1024 + STAGES * (kABytes + kBBytes) + 256;
 };
 
-template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+template <int BN, int STAGES, int EPI, int MH>
+__global__ void __launch_bounds__(GemmCfg<BN, STAGES, MH>::kThreads, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
-  using Cfg = GemmCfg<BN, STAGES>;
+  using Cfg = GemmCfg<BN, STAGES, MH>;
   extern __shared__ uint8_t gemm_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * Cfg::kABytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * Cfg::kBBytes);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;   // [2]
-  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint64_t* acc_full = empty + STAGES;   // [kBufs]
+  uint64_t* acc_empty = acc_full + 2;    // [kBufs]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
@@ -71,9 +81,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < Cfg::kBufs; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+      mbar_init(&acc_empty[b], Cfg::kEpiWarps);  // one arrival per epilogue warp
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -95,7 +105,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t it = 0;
       for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
         const int mb = tile % p.tiles_m;
-        const int m0 = mb * kGemmBM;
+        const int m0 = mb * Cfg::kBM;
         const int nb = tile / p.tiles_m;
         // tiles that share an A row block or a B column block walk K from
         // different starts, so concurrent CTAs do not all read the same L2 lines
@@ -109,7 +119,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const int kx = ((kt + kofs) % num_k) * kGemmBK;
           mbar_arrive_expect_tx(&full[s], Cfg::kABytes + Cfg::kBBytes);
-          tma_load_2d(sA + s * Cfg::kABytes, &tmA, &full[s], kx, m0);
+#pragma unroll
+          for (int mh = 0; mh < MH; ++mh)
+            tma_load_2d(sA + s * Cfg::kABytes + mh * (128 * 128), &tmA, &full[s], kx, m0 + mh * 128);
 #pragma unroll
           for (int hb = 0; hb < BN / Cfg::kBBox; ++hb) {
             const int brow = (EPI == kEpiSwiGLU) ? (hb * p.up_row0 + nb * 128) : (nb * BN + hb * Cfg::kBBox);
@@ -125,15 +137,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kGemmBM, BN, false, false);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false, false);
       uint32_t it = 0;
       int i = 0;
       for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++i) {
-        const uint32_t b = i & 1;
-        bool ok = !*abort_flag && mbar_wait(&acc_empty[b], ((i >> 1) & 1) ^ 1, kErrWaitGemm);
+        const uint32_t b = i % Cfg::kBufs;
+        bool ok = !*abort_flag && mbar_wait(&acc_empty[b], ((i / Cfg::kBufs) & 1) ^ 1, kErrWaitGemm);
         if (ok) {
           tc_fence_after();
-          const uint32_t d_tmem = tmem + b * Cfg::kAccCols;
+          const uint32_t d_tmem = tmem + b * Cfg::kBufCols;
           for (int kt = 0; kt < num_k; ++kt, ++it) {
             const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
             if (*abort_flag || !mbar_wait(&full[s], ph, kErrWaitGemm)) {
@@ -144,9 +156,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t a0 = smem_u32(sA + s * Cfg::kABytes);
             const uint32_t b0 = smem_u32(sB + s * Cfg::kBBytes);
 #pragma unroll
-            for (int kk = 0; kk < kGemmBK / 16; ++kk)
-              umma_ss(d_tmem, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), idesc,
-                      (kt | kk) != 0 ? 1u : 0u);
+            for (int mh = 0; mh < MH; ++mh)
+#pragma unroll
+              for (int kk = 0; kk < kGemmBK / 16; ++kk)
+                umma_ss(d_tmem + mh * Cfg::kAccCols, sdesc_sw128(a0 + mh * (128 * 128) + kk * 32, 16, 1024),
+                        sdesc_sw128(b0 + kk * 32, 16, 1024), idesc, (kt | kk) != 0 ? 1u : 0u);
             umma_commit(&empty[s]);
           }
         }
@@ -160,19 +174,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue warps
     const int q = warp & 3;
-    const int row = q * 32 + lane;
+    const int mh = (warp - 2) >> 2;
+    const int row = mh * 128 + q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     int i = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++i) {
-      const uint32_t b = i & 1;
-      if (*abort_flag || !warp_wait(&acc_full[b], (i >> 1) & 1, kErrWaitGemm)) {
+      const uint32_t b = i % Cfg::kBufs;
+      if (*abort_flag || !warp_wait(&acc_full[b], (i / Cfg::kBufs) & 1, kErrWaitGemm)) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const int grow = (tile % p.tiles_m) * kGemmBM + row;
+      const int grow = (tile % p.tiles_m) * Cfg::kBM + row;
       const int nb = tile / p.tiles_m;
-      const uint32_t t_row = tmem + lane_base + b * Cfg::kAccCols;
+      const uint32_t t_row = tmem + lane_base + b * Cfg::kBufCols + mh * Cfg::kAccCols;
       if (EPI == kEpiStore || EPI == kEpiResidual) {
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 32) {

@@ -12,9 +12,12 @@
 #include <cstdio>
 #include <algorithm>
 #include <cstring>
+#include <functional>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
+#include <vector>
 
 #include "../../include/tg.h"
 #include "attn_tc.cuh"
@@ -141,28 +144,40 @@ int sm_count() {
 }
 
 // Persistent GEMM: grid = min(tiles, SMs); B has b_rows rows of K elements.
-template <int BN, int EPI>
+// MH = 2 takes 256-row tiles (half the B traffic per FLOP) when they still
+// give every SM a tile; otherwise 128-row tiles keep all SMs busy.
+template <int BN, int EPI, int MH>
 int launch_gemm_tc(const void* A, int64_t lda, const void* B, int64_t b_rows, int M, int K, int tiles_n,
                    const tg::GemmParams& p0, cudaStream_t st) {
-  using Cfg = tg::GemmCfg<BN, kGemmStages>;
+  constexpr int kStages = MH == 2 ? 3 : kGemmStages;
+  using Cfg = tg::GemmCfg<BN, kStages, MH>;
   CUtensorMap ta, tb;
   int rc = make_map(&ta, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(lda) * 2, 128);
   if (rc) return rc;
   rc = make_map(&tb, B, static_cast<uint64_t>(K), static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K) * 2,
                 Cfg::kBBox);
   if (rc) return rc;
-  auto kern = tg::k_gemm_tc<BN, kGemmStages, EPI>;
+  auto kern = tg::k_gemm_tc<BN, kStages, EPI, MH>;
   rc = set_smem(kern, Cfg::kSmem);
   if (rc) return rc;
   tg::GemmParams p = p0;
   p.M = M;
   p.K = K;
-  p.tiles_m = (M + tg::kGemmBM - 1) / tg::kGemmBM;
+  p.tiles_m = (M + Cfg::kBM - 1) / Cfg::kBM;
   p.tiles_n = tiles_n;
   const int tiles = p.tiles_m * p.tiles_n;
   const int grid = tiles < sm_count() ? tiles : sm_count();
-  kern<<<grid, tg::kGemmThreads, Cfg::kSmem, st>>>(ta, tb, p);
+  kern<<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(ta, tb, p);
   return check_launch("k_gemm_tc");
+}
+
+template <int BN, int EPI>
+int launch_gemm_auto(const void* A, int64_t lda, const void* B, int64_t b_rows, int M, int K, int tiles_n,
+                     const tg::GemmParams& p0, cudaStream_t st) {
+  const int64_t tiles256 = int64_t((M + 255) / 256) * tiles_n;
+  if (tiles256 >= sm_count() - sm_count() / 16)
+    return launch_gemm_tc<BN, EPI, 2>(A, lda, B, b_rows, M, K, tiles_n, p0, st);
+  return launch_gemm_tc<BN, EPI, 1>(A, lda, B, b_rows, M, K, tiles_n, p0, st);
 }
 
 template <int BN>
@@ -231,6 +246,117 @@ int tg_check_device_error(void* stream, uint32_t* detail) {
   return fail(TG_ERR_DEVICE_CHECK, "device check failed at site %u (payload %u)", site, word >> 8);
 }
 
+// Schedule of the tensor-core attention kernel.  A CTA owns one 128-row query
+// block of two query heads; its causal work is the number of 64-key tiles up
+// to the diagonal, which grows with the block index, and every CTA also pays a
+// fixed cost (start-up, first loads, epilogue) worth about kAttnCtaFixed tiles.
+// When the launch is about a wave of the GPU, the longest blocks set its
+// length; splitting a block into two CTAs (first and second half of its key
+// tiles, merged by the CTA that finishes second) shortens them but adds a
+// fixed cost.  The plan splits the k longest blocks for the k whose simulated
+// longest-first schedule on the SMs ends first (k = 0: no split), and launches
+// the CTAs longest first.
+constexpr int kAttnCtaFixed = 4;
+
+struct AttnPlan {
+  int T = 0, per_tile = 0, ts = 0;
+  bool table = false;
+  std::vector<uint16_t> items;  // AttnWork encoding, longest first
+  size_t part_off = 0, ml_off = 0, ctr_off = 0, bytes = 0;  // workspace layout
+};
+
+struct AttnItem {
+  int size, t, code;
+};
+
+// items of the schedule that splits blocks t >= ts, longest first
+std::vector<AttnItem> attn_items(int T, int kt, int ts) {
+  std::vector<AttnItem> it;
+  it.reserve(2 * T);
+  for (int t = 0; t < T; ++t) {
+    const int u = std::min(2 * t + 2, kt);
+    if (t >= ts) {
+      it.push_back({u / 2, t, 1});
+      it.push_back({u - u / 2, t, 2});
+    } else {
+      it.push_back({u, t, 0});
+    }
+  }
+  std::stable_sort(it.begin(), it.end(), [](const AttnItem& a, const AttnItem& b) {
+    if (a.size != b.size) return a.size > b.size;
+    if (a.t != b.t) return a.t > b.t;
+    return a.code > b.code;
+  });
+  return it;
+}
+
+// end of the greedy in-order schedule of `per_tile` copies of each item on `sms` SMs
+int64_t attn_makespan(const std::vector<AttnItem>& it, int per_tile, int sms) {
+  std::vector<int64_t> busy(static_cast<size_t>(sms), 0);  // min-heap of SM finish times
+  for (const AttnItem& x : it)
+    for (int r = 0; r < per_tile; ++r) {
+      std::pop_heap(busy.begin(), busy.end(), std::greater<int64_t>());
+      busy.back() += x.size + kAttnCtaFixed;
+      std::push_heap(busy.begin(), busy.end(), std::greater<int64_t>());
+    }
+  return *std::max_element(busy.begin(), busy.end());
+}
+
+AttnPlan attn_plan_compute(int64_t m, int hkv, int group, int head_dim, int sms) {
+  AttnPlan pl;
+  pl.T = static_cast<int>((m + 127) / 128);
+  pl.per_tile = hkv * (group / 2);
+  pl.ts = pl.T;
+  const int kt = static_cast<int>((m + 63) / 64);
+  sms = std::max(sms, 1);
+  // only short launches gain from splitting: at most about two waves of CTAs,
+  // and blocks of at least 4 tiles (each half keeps a visible key per row)
+  if (int64_t(pl.T) * pl.per_tile > 2 * int64_t(sms) || 2 * pl.T > tg::kAttnWorkCap || pl.T >= (1 << 14)) return pl;
+  int64_t best = attn_makespan(attn_items(pl.T, kt, pl.T), pl.per_tile, sms);
+  int best_ts = pl.T;
+  for (int ts = pl.T - 1; ts >= 1 && std::min(2 * ts + 2, kt) >= 4; --ts) {
+    const int64_t span = attn_makespan(attn_items(pl.T, kt, ts), pl.per_tile, sms);
+    if (span < best) {
+      best = span;
+      best_ts = ts;
+    }
+  }
+  if (best_ts == pl.T) return pl;
+  pl.ts = best_ts;
+  const std::vector<AttnItem> it = attn_items(pl.T, kt, pl.ts);
+  pl.table = true;
+  pl.items.reserve(it.size());
+  for (const AttnItem& x : it) pl.items.push_back(static_cast<uint16_t>((x.t << 2) | x.code));
+  const size_t slots = size_t(pl.T - pl.ts) * pl.per_tile;
+  auto al = [](size_t b) { return (b + 255) / 256 * 256; };
+  pl.part_off = 0;
+  pl.ml_off = al(slots * 2 * 2 * 128 * size_t(head_dim) * 4);
+  pl.ctr_off = pl.ml_off + al(slots * 2 * 2 * 128 * 8);
+  pl.bytes = pl.ctr_off + al(slots * 4);
+  return pl;
+}
+
+// The plan depends only on the shape and the SM count; it is computed once
+// per key (the schedule simulation costs tens of microseconds of host time).
+const AttnPlan& attn_plan(int64_t m, int hkv, int group, int head_dim, int sms) {
+  static std::mutex mu;
+  static std::map<std::tuple<int64_t, int, int, int, int>, AttnPlan> cache;
+  const auto key = std::make_tuple(m, hkv, group, head_dim, sms);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it == cache.end()) {
+    if (cache.size() > 4096) cache.clear();
+    it = cache.emplace(key, attn_plan_compute(m, hkv, group, head_dim, sms)).first;
+  }
+  return it->second;
+}
+
+// workspace of tg_gated_attention (0 when the launch is long enough to need no split)
+size_t attn_ws_bytes(int64_t m, int hq, int hkv, int head_dim, int dtype) {
+  if (dtype != TG_BF16 || m <= 0 || hq <= 0 || hkv <= 0 || hq % hkv || (hq / hkv) % 2) return 0;
+  return attn_plan(m, hkv, hq / hkv, head_dim, sm_count()).bytes;
+}
+
 size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t h, const tg_layer_shape* shape) {
   if (op == TG_OP_GATE_SCORE) return (n > 0 && d_model > 0 && h > 0) ? gate_ws_bytes(n, d_model, h) : 0;
   if (op == TG_OP_LAYER) {
@@ -244,7 +370,11 @@ size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t
     // un-fused gate/up product, twice as wide as the fused SwiGLU output)
     const size_t act = static_cast<size_t>(shape->d_ff) * 2;
     return al(rows * shape->d_model * es) + al(rows * qkv * es) + al(rows * shape->hq * shape->head_dim * es) +
-           al(rows * act * es);
+           al(rows * act * es) + attn_ws_bytes(m, shape->hq, shape->hkv, shape->head_dim, shape->dtype);
+  }
+  if (op == TG_OP_ATTENTION) {
+    if (!shape || m <= 0) return 0;
+    return attn_ws_bytes(m, shape->hq, shape->hkv, shape->head_dim, shape->dtype);
   }
   return 0;
 }
@@ -430,7 +560,7 @@ int tg_gather(const void* hidden, int dtype, int64_t n, int32_t d_model, const i
 int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk, const void* v, int64_t ldv, int dtype,
                        int64_t m, int32_t hq, int32_t hkv, int32_t head_dim, const float* bias,
                        const float* head_gain, const float* head_temp, const float* ratio, float sm_scale, void* out,
-                       int64_t ldo, float* lse, void* stream) {
+                       int64_t ldo, float* lse, void* ws, size_t ws_bytes, void* stream) {
   if (!q || !k || !v || !out || !head_gain || !head_temp) return fail(TG_ERR_INVALID_ARG, "null pointer");
   if (m <= 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0) return fail(TG_ERR_INVALID_ARG, "bad m / heads");
   if (m >= (int64_t(1) << 31)) return fail(TG_ERR_UNSUPPORTED, "m must be < 2^31");
@@ -461,9 +591,11 @@ int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk, c
     p.out = static_cast<__nv_bfloat16*>(out);
     p.ldo = ldo;
     p.lse = lse;
-    CUtensorMap tq, tk, tv, tb;
+    CUtensorMap tq, tk, tv, tb, to;
     std::memset(&tb, 0, sizeof(tb));
     int rc = make_map(&tq, q, uint64_t(hq) * head_dim, uint64_t(m), uint64_t(ldq) * 2, 128);
+    // the output tile of a head is stored by TMA from shared memory, 128 rows x 64 columns per box
+    if (!rc) rc = make_map(&to, out, uint64_t(hq) * head_dim, uint64_t(m), uint64_t(ldo) * 2, 128);
     // keys and values come in tiles of 64 rows (AttnCfg::BN)
     if (!rc) rc = make_map(&tk, k, uint64_t(hkv) * head_dim, uint64_t(m), uint64_t(ldk) * 2, 64);
     if (!rc) rc = make_map(&tv, v, uint64_t(hkv) * head_dim, uint64_t(m), uint64_t(ldv) * 2, 64);
@@ -473,15 +605,33 @@ int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk, c
       if (!aligned16(bias)) return fail(TG_ERR_ALIGN, "bias must be 16-byte aligned");
       if ((rc = make_map_1d_f32(&tb, bias, uint64_t(m), 64))) return rc;
     }
-    const unsigned blocks = static_cast<unsigned>(p.num_qtiles * hkv * (group / 2));
+    // key-range split of the longest row blocks when a workspace is given
+    const AttnPlan& pl = attn_plan(m, hkv, group, head_dim, sm_count());
+    static thread_local tg::AttnWork work;  // 3.75 KiB: passed by value as a kernel parameter
+    p.ts = p.num_qtiles;
+    if (pl.table && ws && ws_bytes >= pl.bytes) {
+      if (!aligned16(ws)) return fail(TG_ERR_ALIGN, "attention workspace must be 16-byte aligned");
+      uint8_t* wb = static_cast<uint8_t*>(ws);
+      p.use_table = 1;
+      p.ts = pl.ts;
+      p.part = reinterpret_cast<float4*>(wb + pl.part_off);
+      p.part_ml = reinterpret_cast<float2*>(wb + pl.ml_off);
+      p.counters = reinterpret_cast<unsigned*>(wb + pl.ctr_off);
+      std::fill(std::begin(work.item), std::end(work.item), uint16_t(0));
+      std::copy(pl.items.begin(), pl.items.end(), work.item);
+      if (cudaMemsetAsync(p.counters, 0, pl.bytes - pl.ctr_off, st) != cudaSuccess)
+        return fail(TG_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(cudaGetLastError()));
+    }
+    const int items = p.use_table ? static_cast<int>(pl.items.size()) : p.num_qtiles;
+    const unsigned blocks = static_cast<unsigned>(items * hkv * (group / 2));
     if (head_dim == 128) {
       rc = set_smem(tg::k_attn_tc<128>, tg::AttnCfg<128>::kSmem);
       if (rc) return rc;
-      tg::k_attn_tc<128><<<blocks, tg::kAttnThreads, tg::AttnCfg<128>::kSmem, st>>>(tq, tk, tv, tb, p);
+      tg::k_attn_tc<128><<<blocks, tg::kAttnThreads, tg::AttnCfg<128>::kSmem, st>>>(tq, tk, tv, tb, to, p, work);
     } else {
       rc = set_smem(tg::k_attn_tc<64>, tg::AttnCfg<64>::kSmem);
       if (rc) return rc;
-      tg::k_attn_tc<64><<<blocks, tg::kAttnThreads, tg::AttnCfg<64>::kSmem, st>>>(tq, tk, tv, tb, p);
+      tg::k_attn_tc<64><<<blocks, tg::kAttnThreads, tg::AttnCfg<64>::kSmem, st>>>(tq, tk, tv, tb, to, p, work);
     }
     return check_launch("k_attn_tc");
   }
@@ -533,13 +683,13 @@ int tg_linear(const void* x, int64_t ldx, const void* w, void* y, int64_t ldy, i
     if (epilogue == TG_EPI_SWIGLU) {
       if (n_out % 128 != 0) return fail(TG_ERR_UNSUPPORTED, "SwiGLU epilogue needs n_out %% 128 == 0");
       p.up_row0 = n_out;
-      return launch_gemm_tc<256, tg::kEpiSwiGLU>(x, ldx, w, 2 * int64_t(n_out), mm, k_in, n_out / 128, p, st);
+      return launch_gemm_auto<256, tg::kEpiSwiGLU>(x, ldx, w, 2 * int64_t(n_out), mm, k_in, n_out / 128, p, st);
     }
     if (n_out % 32 == 0) {
       const int gn = (n_out + 255) / 256;
       if (epilogue == TG_EPI_RESIDUAL)
-        return launch_gemm_tc<256, tg::kEpiResidual>(x, ldx, w, n_out, mm, k_in, gn, p, st);
-      return launch_gemm_tc<256, tg::kEpiStore>(x, ldx, w, n_out, mm, k_in, gn, p, st);
+        return launch_gemm_auto<256, tg::kEpiResidual>(x, ldx, w, n_out, mm, k_in, gn, p, st);
+      return launch_gemm_auto<256, tg::kEpiStore>(x, ldx, w, n_out, mm, k_in, gn, p, st);
     }
   }
   if (epilogue == TG_EPI_SWIGLU) return fail(TG_ERR_UNSUPPORTED, "SwiGLU epilogue needs bf16");
@@ -590,6 +740,9 @@ int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, 
   void* att = base;
   base += al(size_t(m) * hq * D * es);
   void* act = base;
+  base += al(size_t(m) * dff * 2 * es);
+  void* attn_ws = base;
+  const size_t attn_ws_sz = attn_ws_bytes(m, hq, hkv, D, S->dtype);
   const bool bf = S->dtype == TG_BF16;
   int rc;
   // 1. x = RMSNorm(h)
@@ -633,7 +786,8 @@ int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, 
     const uint8_t* qb = static_cast<const uint8_t*>(qkv);
     if ((rc = tg_gated_attention(qb, qkv_w, qb + int64_t(hq) * D * es, qkv_w, qb + int64_t(hq + hkv) * D * es, qkv_w,
                                  S->dtype, m, hq, hkv, D, bias, W->head_gain, W->head_temp, ratio,
-                                 1.0f / sqrtf(float(D)), att, int64_t(hq) * D, nullptr, stream)))
+                                 1.0f / sqrtf(float(D)), att, int64_t(hq) * D, nullptr, attn_ws_sz ? attn_ws : nullptr,
+                                 attn_ws_sz, stream)))
       return rc;
   }
   // 5. h += a Wo^T

@@ -18,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libtokengate.so")
 
 TG_F32, TG_BF16 = 0, 1
-TG_OP_GATE_SCORE, TG_OP_LAYER = 0, 1
+TG_OP_GATE_SCORE, TG_OP_LAYER, TG_OP_ATTENTION = 0, 1, 2
 STATUS = {0: "TG_OK", 1: "TG_ERR_INVALID_ARG", 2: "TG_ERR_SHAPE", 3: "TG_ERR_ALIGN", 4: "TG_ERR_UNSUPPORTED",
           5: "TG_ERR_WORKSPACE", 6: "TG_ERR_CUDA", 7: "TG_ERR_DEVICE_TIMEOUT", 8: "TG_ERR_DEVICE_CHECK"}
 
@@ -52,7 +52,7 @@ SIGNATURES = {
     "tg_topk_select": (_INT, [_P, _P, _I64, _I64, _I64, _P, _I64, _P]),
     "tg_gather": (_INT, [_P, _INT, _I64, _I32, _P, _I64, _P, _P, _I64, _F, _P, _P, _P, _P, _P]),
     "tg_gated_attention": (_INT, [_P, _I64, _P, _I64, _P, _I64, _INT, _I64, _I32, _I32, _I32, _P, _P, _P, _P, _F,
-                                  _P, _I64, _P, _P]),
+                                  _P, _I64, _P, _P, _SZ, _P]),
     "tg_pruned_prefill_layer": (_INT, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerShape), _P, _P, _P, _P,
                                        _I64, _P, _SZ, _P]),
     "tg_linear": (_INT, [_P, _I64, _P, _P, _I64, _INT, _I64, _I32, _I32, _INT, _P]),
@@ -167,9 +167,16 @@ def _row_view(t: torch.Tensor):
     return ctypes.c_void_p(t.data_ptr()), t.stride(0)
 
 
+def attention_workspace_bytes(m: int, hq: int, hkv: int, head_dim: int, dtype: torch.dtype) -> int:
+    """Workspace bytes tg_gated_attention uses on the current device (0: none needed)."""
+    shape = LayerShape(dtype=TG_BF16 if dtype == torch.bfloat16 else TG_F32, hq=hq, hkv=hkv, head_dim=head_dim)
+    return tg_workspace_bytes(TG_OP_ATTENTION, m=m, shape=shape)
+
+
 def tg_gated_attention(q, k, v, head_dim: int, bias, head_gain, head_temp, ratio, sm_scale: float, out, lse=None,
-                       stream=None):
-    """q/k/v/out are 2-D row views [m, heads*head_dim] (rows may be strided)."""
+                       ws=None, stream=None):
+    """q/k/v/out are 2-D row views [m, heads*head_dim] (rows may be strided); ws is a device
+    byte buffer of attention_workspace_bytes(...) bytes or None (no key-range split)."""
     qp, ldq = _row_view(q)
     kp, ldk = _row_view(k)
     vp, ldv = _row_view(v)
@@ -179,6 +186,7 @@ def tg_gated_attention(q, k, v, head_dim: int, bias, head_gain, head_temp, ratio
     hkv = k.shape[1] // head_dim
     rc = lib().tg_gated_attention(qp, ldq, kp, ldk, vp, ldv, _dtype(q), m, hq, hkv, head_dim, _ptr(bias),
                                   _ptr(head_gain), _ptr(head_temp), _ptr(ratio), float(sm_scale), op, ldo, _ptr(lse),
+                                  _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0,
                                   _stream(stream))
     _check("tg_gated_attention", rc)
 

@@ -58,11 +58,11 @@ def test_select_validation(L):
 
 def test_attention_validation(L):
     g = ctypes.c_void_p(256)
-    assert L.tg_gated_attention(g, 2048, g, 1024, g, 1024, 1, 100, 16, 8, 96, None, g, g, None, 0.1, g, 2048, None, None) == 4
-    assert L.tg_gated_attention(g, 2048, g, 1024, g, 1024, 1, 100, 16, 6, 128, None, g, g, None, 0.1, g, 2048, None, None) == 1
-    assert L.tg_gated_attention(g, 100, g, 1024, g, 1024, 1, 100, 16, 8, 128, None, g, g, None, 0.1, g, 2048, None, None) == 2
+    assert L.tg_gated_attention(g, 2048, g, 1024, g, 1024, 1, 100, 16, 8, 96, None, g, g, None, 0.1, g, 2048, None, None, 0, None) == 4
+    assert L.tg_gated_attention(g, 2048, g, 1024, g, 1024, 1, 100, 16, 6, 128, None, g, g, None, 0.1, g, 2048, None, None, 0, None) == 1
+    assert L.tg_gated_attention(g, 100, g, 1024, g, 1024, 1, 100, 16, 8, 128, None, g, g, None, 0.1, g, 2048, None, None, 0, None) == 2
     assert L.tg_gated_attention(ctypes.c_void_p(258), 2048, g, 1024, g, 1024, 1, 100, 16, 8, 128, None, g, g, None,
-                                0.1, g, 2048, None, None) == 3
+                                0.1, g, 2048, None, None, 0, None) == 3
 
 
 def test_gather_and_gate_validation(L):
@@ -75,6 +75,18 @@ def test_workspace_sizes(L):
     S = tg.LayerShape(1, 2048, 16, 8, 128, 6144, 1, 1e6, 1e-6)
     m = 2064
     want = sum((b + 255) // 256 * 256 for b in (m * 2048 * 2, m * 4096 * 2, m * 2048 * 2, m * 2 * 6144 * 2))
-    assert tg.tg_workspace_bytes(tg.TG_OP_LAYER, m=m, shape=S) == want
+    attn = tg.tg_workspace_bytes(tg.TG_OP_ATTENTION, m=m, shape=S)
+    assert tg.tg_workspace_bytes(tg.TG_OP_LAYER, m=m, shape=S) == want + attn
+    # without a GPU the library plans for 148 SMs: 17 row blocks x 8 head pairs are
+    # one wave, so some of the longest blocks are split; each split block keeps two
+    # halves of O (fp32) and of (max, sum) for both heads, plus one counter
+    al = lambda b: (b + 255) // 256 * 256
+    layout = lambda slots: al(slots * 2 * 2 * 128 * 128 * 4) + al(slots * 2 * 2 * 128 * 8) + al(slots * 4)
+    splits = [k for k in range(1, 17) if layout(8 * k) == attn]
+    assert len(splits) == 1, attn
+    # a launch of several waves needs no split and no workspace
+    assert tg.tg_workspace_bytes(tg.TG_OP_ATTENTION, m=8256, shape=S) == 0
+    S32 = tg.LayerShape(0, 2048, 16, 8, 128, 6144, 1, 1e6, 1e-6)  # fp32 runs on CUDA cores: no split
+    assert tg.tg_workspace_bytes(tg.TG_OP_ATTENTION, m=m, shape=S32) == 0
     assert tg.tg_workspace_bytes(tg.TG_OP_GATE_SCORE, n=16384, d_model=2048, h=256) >= 16384 // 128 * 4 + 256 * 2048 * 2
     assert tg.tg_workspace_bytes(99) == 0

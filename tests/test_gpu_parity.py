@@ -244,14 +244,24 @@ def _attn_case(m, hq, hkv, D, dtype, seed):
     return q, k, v, bias, ratio, gain, temp
 
 
-def _gpu_attn(q, k, v, D, bias, ratio, gain, temp, dtype, with_lse=True):
+def _attn_ws(m, hq, hkv, D, dt, split=True):
+    """Workspace for the key-range split (garbage-filled: the call must not rely on its contents)."""
+    nbytes = tg.attention_workspace_bytes(m, hq, hkv, D, dt) if split else 0
+    if nbytes == 0:
+        return None
+    return torch.full((nbytes,), 0xA5, dtype=torch.uint8, device=DEV)
+
+
+def _gpu_attn(q, k, v, D, bias, ratio, gain, temp, dtype, with_lse=True, split=True):
     dt = synth.torch_dtype(dtype)
     m = q.shape[0]
     hq = q.shape[1] // D
     out = torch.empty(m, q.shape[1], dtype=dt, device=DEV)
     lse = torch.empty(hq, m, dtype=torch.float32, device=DEV) if with_lse else None
+    ws = _attn_ws(m, hq, k.shape[1] // D, D, dt, split)
     tg.tg_gated_attention(d(q, dt), d(k, dt), d(v, dt), D, None if bias is None else d(bias), d(gain), d(temp),
-                          None if ratio is None else d(ratio), 1.0 / math.sqrt(D), out, lse)
+                          None if ratio is None else d(ratio), 1.0 / math.sqrt(D), out, lse, ws)
+    assert tg.tg_check_device_error() == 0
     return host(out), (host(lse) if with_lse else None)
 
 
@@ -262,14 +272,34 @@ def _oracle_attn(q, k, v, D, bias, ratio, gain, temp, rows=None):
     return o.reshape(o.shape[0], -1), lse
 
 
+@pytest.mark.parametrize("split", [True, False])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("m", [1, 5, 127, 128, 129, 300, 1000])
-def test_attention_bf16_tensor_cores(m, D):
+def test_attention_bf16_tensor_cores(m, D, split):
     q, k, v, bias, ratio, gain, temp = _attn_case(m, 4, 2, D, "bf16", seed=m + D)
-    got, lse = _gpu_attn(q, k, v, D, bias, ratio, gain, temp, "bf16")
+    got, lse = _gpu_attn(q, k, v, D, bias, ratio, gain, temp, "bf16", split=split)
     want, wlse = _oracle_attn(q, k, v, D, bias, ratio, gain, temp)
     assert_close(got, want, what="out", **ATTN_BF16)
     assert_close(lse, wlse, 2e-2, 1e-3, "lse")
+
+
+@pytest.mark.parametrize("m", [1000, 2064])
+def test_attention_bf16_split_key_range_bench_shapes(m):
+    # about one wave of causal work: the longest row blocks run as two CTAs whose
+    # partial results are merged; every 7th row is compared, ragged tail included
+    q, k, v, bias, ratio, gain, temp = _attn_case(m, 16, 8, 128, "bf16", seed=m)
+    assert tg.attention_workspace_bytes(m, 16, 8, 128, torch.bfloat16) > 0
+    got, lse = _gpu_attn(q, k, v, 128, bias, ratio, gain, temp, "bf16")
+    rows = list(range(0, m, 7)) + [m - 1]
+    want, wlse = _oracle_attn(q, k, v, 128, bias, ratio, gain, temp, rows=rows)
+    assert_close(got[rows], want, what="out", **ATTN_BF16)
+    assert_close(lse[:, rows], wlse, 2e-2, 1e-3, "lse")
+    # a second call with the same (now used) workspace gives the same bits
+    again, _ = _gpu_attn(q, k, v, 128, bias, ratio, gain, temp, "bf16")
+    assert np.array_equal(got, again)
+    # and the unsplit schedule agrees to within the kernel's own rounding
+    whole, _ = _gpu_attn(q, k, v, 128, bias, ratio, gain, temp, "bf16", split=False)
+    assert_close(got, whole, what="split vs whole", **ATTN_BF16)
 
 
 def test_attention_bf16_gqa_16_8_and_no_bias_ratio():
@@ -288,7 +318,8 @@ def test_attention_bf16_strided_qkv_views():
     qkv = torch.cat([d(q, torch.bfloat16), d(k, torch.bfloat16), d(v, torch.bfloat16)], dim=1).contiguous()
     out = torch.empty(m, hq * D, dtype=torch.bfloat16, device=DEV)
     tg.tg_gated_attention(qkv[:, : hq * D], qkv[:, hq * D:(hq + hkv) * D], qkv[:, (hq + hkv) * D:], D, d(bias),
-                          d(gain), d(temp), d(ratio), 1.0 / math.sqrt(D), out)
+                          d(gain), d(temp), d(ratio), 1.0 / math.sqrt(D), out,
+                          ws=_attn_ws(m, hq, hkv, D, torch.bfloat16))
     want, _ = _oracle_attn(q, k, v, D, bias, ratio, gain, temp)
     assert_close(host(out), want, what="out", **ATTN_BF16)
 
@@ -323,10 +354,15 @@ def test_attention_bf16_full_size_sampled_rows():
 
 # ============================================================================ linear / layer
 
+@pytest.mark.parametrize("shape", [(300, 512, 384), (333, 18432, 192), (600, 32768, 128)],
+                         ids=["128-row-tiles", "256-row-tiles-ragged", "256-row-tiles-several-per-cta"])
 @pytest.mark.parametrize("epilogue", [tg.TG_EPI_STORE, tg.TG_EPI_RESIDUAL, tg.TG_EPI_SWIGLU])
-def test_linear_bf16_tensor_cores(epilogue):
+def test_linear_bf16_tensor_cores(epilogue, shape):
+    # the wide shapes have enough column tiles for 256-row tiles (two 128 x 256
+    # accumulators per CTA, no double buffering); (600, 32768) gives each CTA
+    # several tiles, so the accumulators are handed back and reused
     rng = np.random.default_rng(12)
-    m, n_out, k_in = 300, 512, 384
+    m, n_out, k_in = shape
     w_rows = 2 * n_out if epilogue == tg.TG_EPI_SWIGLU else n_out
     x = synth.round_to(rng.standard_normal((m, k_in)).astype(np.float32), "bf16")
     w = synth.round_to(rng.standard_normal((w_rows, k_in)).astype(np.float32) * 0.05, "bf16")
