@@ -351,25 +351,44 @@ def breakdown(step, w, args, stream, flush):
     step.run()
     torch.cuda.synchronize()
     reps = max(5, min(args.steps, 50))
+
+    def graph_of(body):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            body()
+        return g
+
+    def replay_ms(g):
+        # back-to-back replays between one pair of events: the GPU never waits
+        # for the host inside the timed interval
+        g.replay()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    # each call is timed as (L2 flush + call) minus (L2 flush): cold L2 like
+    # the step, without the flush and without launch gaps
+    g_flush = graph_of(lambda: flush.zero_())
+    t_flush = replay_ms(g_flush)
     out = {}
     for name, fn in calls.items():
         fn()
         torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()   # one graph per call: the timing holds no host launch work
-        with torch.cuda.graph(g):
-            fn()
-        ms = 0.0
-        for _ in range(reps):
+
+        def body(fn=fn):
             flush.zero_()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            g.replay()
-            b.record(stream)
-            torch.cuda.synchronize()
-            ms += a.elapsed_time(b)
-        out[name] = ms / reps
+            fn()
+
+        g = graph_of(body)
+        out[name] = max(replay_ms(g) - t_flush, 0.0)
         del g
+    del g_flush
     return out
 
 

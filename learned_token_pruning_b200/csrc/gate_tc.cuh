@@ -3,15 +3,17 @@
 //     s_j = w2 . SiLU(W1 RMSNorm(h_j) + b1) + b2   for prunable j, 0 otherwise
 // with (h_j * w_n) W1^T = h_j (W1 diag(w_n))^T, so the RMSNorm weight is folded
 // into W1 on the host side and the row scale 1/rms(h_j) is applied to the
-// accumulator in the epilogue.  The hidden states are read from HBM once.
+// accumulator in the epilogue.  The hidden states are read from HBM once, and
+// into the SM once.
 //
 // One CTA scores 128 tokens.  TMA streams 128x64 tiles of H and BNx64 tiles of
 // W1 (128-byte swizzle) through a STAGES-deep ring; one thread issues
 // tcgen05.mma (M=128, N=BN, K=16) into an fp32 TMEM accumulator.  While the
-// MMAs run, the eight epilogue warps sum h^2 of the CTA's rows with coalesced
-// global reads (whichever of them and the TMA ring touches a line first
-// brings it into L2 for the other), so the ring is never held up by anything
-// but the tensor core.  Then the eight epilogue warps,
+// MMAs run, the eight epilogue warps sum h^2 of the CTA's rows from the same
+// shared-memory tiles (two threads per row, 64 bytes each per tile: the
+// swizzle only permutes the 16-byte chunks inside a row's 128-byte line, which
+// a sum does not see); a stage goes back to the producer once the MMAs and
+// these warps have both read it.  Then the eight epilogue warps,
 // two per TMEM lane quarter, each take half of a row's BN accumulator
 // columns, apply 1/rms, b1, SiLU and w2, and the halves are added through
 // shared memory.  Sum over prunable rows of s^2 is reduced in a fixed order
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__(kGateThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);  // the MMA commit
+      mbar_init(&empty[s], 1 + 8);  // the MMA commit and the eight row-norm warps
     }
     mbar_init(accbar, 1);
     *abort_flag = 0;
@@ -156,49 +158,35 @@ __global__ void __launch_bounds__(kGateThreads, 1)
     const int grow = m0 + row;
     const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
     {
-      // Row norms: all eight warps, 16 rows each (the two warps of a lane
-      // quarter split its 32 rows), two rows in flight at a time with every
-      // lane holding 16-byte loads of both; the rows stream from HBM in
-      // contiguous 4 KB runs and stay in L2 for the TMA ring.
-      const int nv = p.K / 8;
-      const int rbase = q * 32 + half * 16;
-      for (int rr = 0; rr < 16; rr += 2) {
-        const int r0 = rbase + rr;
-        float s0 = 0.0f, s1 = 0.0f;
-        const bool v0 = m0 + r0 < p.M, v1 = m0 + r0 + 1 < p.M;
-        const uint4* src0 = reinterpret_cast<const uint4*>(p.hidden + static_cast<int64_t>(m0 + r0) * p.K);
-        const uint4* src1 = src0 + nv;
-        for (int c0 = 0; c0 < nv; c0 += 32 * 8) {
-          uint4 a[8], b[8];
+      // Row norms from the ring: thread e = threadIdx.x - 64 owns half e & 1
+      // of row e >> 1 (four 16-byte chunks per tile, rotated by the row so
+      // that a quarter-warp touches four different bank groups).
+      const int e = threadIdx.x - 64;
+      const int nrow = e >> 1, nhalf = e & 1;
+      float ss = 0.0f;
+      for (int kt = 0; kt < num_k; ++kt) {
+        const int s = kt % STAGES;
+        const uint32_t ph = (kt / STAGES) & 1;
+        if (*abort_flag || !warp_wait(&full[s], ph, kErrWaitGemm)) {
+          *abort_flag = 1;
+          break;
+        }
+        const uint8_t* line = sA + s * Cfg::kABytes + nrow * 128 + nhalf * 64;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int c = c0 + u * 32 + lane;
-            a[u] = (v0 && c < nv) ? __ldg(src0 + c) : make_uint4(0, 0, 0, 0);
-            b[u] = (v1 && c < nv) ? __ldg(src1 + c) : make_uint4(0, 0, 0, 0);
-          }
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = *reinterpret_cast<const uint4*>(line + (((i + nrow) & 3) << 4));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const uint32_t wa[4] = {a[u].x, a[u].y, a[u].z, a[u].w};
-            const uint32_t wb[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              s0 = fmaf(bf16_lo(wa[t]), bf16_lo(wa[t]), s0);
-              s0 = fmaf(bf16_hi(wa[t]), bf16_hi(wa[t]), s0);
-              s1 = fmaf(bf16_lo(wb[t]), bf16_lo(wb[t]), s1);
-              s1 = fmaf(bf16_hi(wb[t]), bf16_hi(wb[t]), s1);
-            }
+          for (int t = 0; t < 4; ++t) {
+            ss = fmaf(bf16_lo(w[t]), bf16_lo(w[t]), ss);
+            ss = fmaf(bf16_hi(w[t]), bf16_hi(w[t]), ss);
           }
         }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-          s0 += __shfl_xor_sync(0xffffffffu, s0, o);
-          s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-        }
-        if (lane == 0) {
-          s_ss[r0] = s0;
-          s_ss[r0 + 1] = s1;
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);  // release: the reads above come first
       }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      if (nhalf == 0) s_ss[nrow] = ss;
     }
     bool ok = !*abort_flag && warp_wait(accbar, 0, kErrWaitGemm);
     if (!ok) *abort_flag = 1;

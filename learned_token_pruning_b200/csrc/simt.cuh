@@ -337,6 +337,144 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope(T* __restrict__ qkv, int64
   }
 }
 
+// ---------------------------------------------------------------------------
+// RMSNorm with one warp per row (eight rows per block): the row stays in
+// registers between the sum of squares and the scaling, so it is read once,
+// and all of a lane's 16-byte loads are in flight together.  MAXV bounds the
+// vectors per lane (d <= 32 * MAXV * 16 / sizeof(T)); w, if given, is
+// 16-byte aligned.
+// ---------------------------------------------------------------------------
+template <typename T, int MAXV>
+__global__ void __launch_bounds__(256) k_rmsnorm_warp(const T* __restrict__ x, T* __restrict__ y,
+                                                      const float* __restrict__ w, int64_t m, int d, float eps) {
+  constexpr int V = 16 / sizeof(T);
+  const int lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (r >= m) return;  // warp-uniform
+  const int nv = d / V;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + r * d);
+  uint4* yr = reinterpret_cast<uint4*>(y + r * d);
+  uint4 v[MAXV];
+  float ss = 0.0f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = lane + 32 * i;
+    v[i] = c < nv ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const T* e = reinterpret_cast<const T*>(&v[i]);
+#pragma unroll
+    for (int t = 0; t < V; ++t) {
+      const float f = to_f32(e[t]);
+      ss = fmaf(f, f, ss);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.0f / sqrtf(ss / static_cast<float>(d) + eps);
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = lane + 32 * i;
+    if (c >= nv) continue;
+    float wv[V];
+#pragma unroll
+    for (int t = 0; t < V; t += 4) {
+      const float4 w4 = w ? __ldg(reinterpret_cast<const float4*>(w + c * V + t)) : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+      wv[t] = w4.x;
+      wv[t + 1] = w4.y;
+      wv[t + 2] = w4.z;
+      wv[t + 3] = w4.w;
+    }
+    const T* e = reinterpret_cast<const T*>(&v[i]);
+    uint4 o;
+    T* oe = reinterpret_cast<T*>(&o);
+#pragma unroll
+    for (int t = 0; t < V; ++t) oe[t] = from_f32<T>(to_f32(e[t]) * inv * wv[t]);
+    yr[c] = o;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Per-head q/k RMSNorm (optional) and rotate-half RoPE at the original token
+// positions, one warp per row: lane l owns frequencies l*E .. l*E+E-1 of every
+// rotated head.  The frequencies theta^(-2i/D) come from the host in double
+// precision; the angle pos * f is formed and reduced modulo 2 pi in double
+// (positions reach 2^17), so the float sin/cos of the remainder in [-pi, pi]
+// is accurate to about 4e-7.
+// The hq + hkv heads of the row are processed eight at a time with all their
+// loads in flight.
+// ---------------------------------------------------------------------------
+struct RopeTable {
+  double inv_freq[64];  // D / 2 entries
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_qk_norm_rope_warp(T* __restrict__ qkv, int64_t ld, int m, int hq, int hkv,
+                                                           const int32_t* __restrict__ pos,
+                                                           const float* __restrict__ wq, const float* __restrict__ wk,
+                                                           int qk_norm, float eps,
+                                                           const __grid_constant__ RopeTable tab) {
+  constexpr int H2 = D / 2;
+  constexpr int E = H2 / 32;
+  constexpr int HU = 8;  // heads in flight
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= m) return;  // warp-uniform
+  const double p = static_cast<double>(pos ? pos[r] : r);
+  float cs[E], sn[E], wqa[E], wqb[E], wka[E], wkb[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const double ang = p * tab.inv_freq[lane * E + e];
+    const double turns = rint(ang * 0.15915494309189535);  // 1 / (2 pi)
+    const float red = static_cast<float>(fma(-turns, 6.283185307179586, ang));
+    __sincosf(red, &sn[e], &cs[e]);  // |red| <= pi: absolute error about 4e-7
+    wqa[e] = qk_norm ? wq[lane * E + e] : 1.0f;
+    wqb[e] = qk_norm ? wq[H2 + lane * E + e] : 1.0f;
+    wka[e] = qk_norm ? wk[lane * E + e] : 1.0f;
+    wkb[e] = qk_norm ? wk[H2 + lane * E + e] : 1.0f;
+  }
+  T* row = qkv + static_cast<int64_t>(r) * ld;
+  const int heads = hq + hkv;
+  for (int h0 = 0; h0 < heads; h0 += HU) {
+    float a[HU][E], b[HU][E];
+#pragma unroll
+    for (int u = 0; u < HU; ++u) {
+      const T* x = row + static_cast<int64_t>(h0 + u) * D;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        a[u][e] = h0 + u < heads ? to_f32(x[lane * E + e]) : 0.0f;
+        b[u][e] = h0 + u < heads ? to_f32(x[H2 + lane * E + e]) : 0.0f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < HU; ++u) {
+      const int hh = h0 + u;
+      if (hh >= heads) break;  // warp-uniform
+      const bool isq = hh < hq;
+      if (qk_norm) {
+        float ss = 0.0f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) ss += a[u][e] * a[u][e] + b[u][e] * b[u][e];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float inv = 1.0f / sqrtf(ss / static_cast<float>(D) + eps);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          a[u][e] *= inv * (isq ? wqa[e] : wka[e]);
+          b[u][e] *= inv * (isq ? wqb[e] : wkb[e]);
+        }
+      }
+      T* x = row + static_cast<int64_t>(hh) * D;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        x[lane * E + e] = from_f32<T>(a[u][e] * cs[e] - b[u][e] * sn[e]);
+        x[H2 + lane * E + e] = from_f32<T>(b[u][e] * cs[e] + a[u][e] * sn[e]);
+      }
+    }
+  }
+}
+
 // gu[r][f] <- SiLU(gu[r][f]) * gu[r][d_ff + f]  (rows of 2*d_ff: gate half, then up half)
 template <typename T>
 __global__ void __launch_bounds__(256) k_swiglu(T* __restrict__ gu, int64_t m, int d_ff) {

@@ -210,6 +210,33 @@ size_t gate_ws_bytes(int64_t n, int32_t d, int32_t h) {
 
 }  // namespace
 
+// RMSNorm of m rows: one warp per row when the row fits in a warp's registers
+// (and the weight is 16-byte aligned), else one block per row.
+template <typename T>
+int launch_rmsnorm(const void* x, void* y, const float* w, int64_t m, int d, float eps, cudaStream_t st) {
+  constexpr int V = 16 / sizeof(T);
+  const int nv = d / V;
+  const T* xa = static_cast<const T*>(x);
+  T* ya = static_cast<T*>(y);
+  const unsigned blocks = static_cast<unsigned>((m + 7) / 8);
+  if (!w || aligned16(w)) {
+    if (nv <= 32 * 4) {
+      tg::k_rmsnorm_warp<T, 4><<<blocks, 256, 0, st>>>(xa, ya, w, m, d, eps);
+      return check_launch("k_rmsnorm_warp");
+    }
+    if (nv <= 32 * 8) {
+      tg::k_rmsnorm_warp<T, 8><<<blocks, 256, 0, st>>>(xa, ya, w, m, d, eps);
+      return check_launch("k_rmsnorm_warp");
+    }
+    if (nv <= 32 * 16) {
+      tg::k_rmsnorm_warp<T, 16><<<blocks, 256, 0, st>>>(xa, ya, w, m, d, eps);
+      return check_launch("k_rmsnorm_warp");
+    }
+  }
+  tg::k_rmsnorm<T><<<unsigned(m), 256, 0, st>>>(xa, ya, w, d, eps);
+  return check_launch("k_rmsnorm");
+}
+
 extern "C" {
 
 const char* tg_version(void) { return TG_VERSION; }
@@ -746,40 +773,36 @@ int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, 
   const bool bf = S->dtype == TG_BF16;
   int rc;
   // 1. x = RMSNorm(h)
-  if (bf)
-    tg::k_rmsnorm<__nv_bfloat16><<<unsigned(m), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(hidden_kept),
-                                                                static_cast<__nv_bfloat16*>(xn), W->w_in_norm, d,
-                                                                S->norm_eps);
-  else
-    tg::k_rmsnorm<float><<<unsigned(m), 256, 0, st>>>(static_cast<const float*>(hidden_kept),
-                                                       static_cast<float*>(xn), W->w_in_norm, d, S->norm_eps);
-  if ((rc = check_launch("k_rmsnorm"))) return rc;
+  rc = bf ? launch_rmsnorm<__nv_bfloat16>(hidden_kept, xn, W->w_in_norm, m, d, S->norm_eps, st)
+          : launch_rmsnorm<float>(hidden_kept, xn, W->w_in_norm, m, d, S->norm_eps, st);
+  if (rc) return rc;
   // 2. qkv = x Wqkv^T
   if ((rc = tg_linear(xn, d, W->w_qkv, qkv, qkv_w, S->dtype, m, int32_t(qkv_w), d, TG_EPI_STORE, stream))) return rc;
-  // 3. per-head q/k norm and RoPE at the original positions
+  // 3. per-head q/k norm and RoPE at the original positions (one warp per row)
   {
-    const int rows_per_block = 256 / (D / 2);
-    const unsigned blocks = unsigned((m + rows_per_block - 1) / rows_per_block);
+    tg::RopeTable tab{};
+    for (int i = 0; i < D / 2; ++i) tab.inv_freq[i] = std::pow(static_cast<double>(S->rope_theta), -2.0 * i / D);
+    const unsigned blocks = unsigned((m + 7) / 8);
     if (bf) {
       if (D == 128)
-        tg::k_qk_norm_rope<__nv_bfloat16, 128><<<blocks, 256, 0, st>>>(
+        tg::k_qk_norm_rope_warp<__nv_bfloat16, 128><<<blocks, 256, 0, st>>>(
             static_cast<__nv_bfloat16*>(qkv), qkv_w, int(m), hq, hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm,
-            S->norm_eps, S->rope_theta);
+            S->norm_eps, tab);
       else
-        tg::k_qk_norm_rope<__nv_bfloat16, 64><<<blocks, 256, 0, st>>>(
+        tg::k_qk_norm_rope_warp<__nv_bfloat16, 64><<<blocks, 256, 0, st>>>(
             static_cast<__nv_bfloat16*>(qkv), qkv_w, int(m), hq, hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm,
-            S->norm_eps, S->rope_theta);
+            S->norm_eps, tab);
     } else {
       if (D == 128)
-        tg::k_qk_norm_rope<float, 128><<<blocks, 256, 0, st>>>(static_cast<float*>(qkv), qkv_w, int(m), hq, hkv, pos,
-                                                              W->w_q_norm, W->w_k_norm, S->qk_norm, S->norm_eps,
-                                                              S->rope_theta);
+        tg::k_qk_norm_rope_warp<float, 128><<<blocks, 256, 0, st>>>(static_cast<float*>(qkv), qkv_w, int(m), hq,
+                                                                   hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm,
+                                                                   S->norm_eps, tab);
       else
-        tg::k_qk_norm_rope<float, 64><<<blocks, 256, 0, st>>>(static_cast<float*>(qkv), qkv_w, int(m), hq, hkv, pos,
-                                                             W->w_q_norm, W->w_k_norm, S->qk_norm, S->norm_eps,
-                                                             S->rope_theta);
+        tg::k_qk_norm_rope_warp<float, 64><<<blocks, 256, 0, st>>>(static_cast<float*>(qkv), qkv_w, int(m), hq,
+                                                                  hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm,
+                                                                  S->norm_eps, tab);
     }
-    if ((rc = check_launch("k_qk_norm_rope"))) return rc;
+    if ((rc = check_launch("k_qk_norm_rope_warp"))) return rc;
   }
   // 4. token-gated attention
   {
@@ -794,14 +817,9 @@ int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, 
   if ((rc = tg_linear(att, int64_t(hq) * D, W->w_o, hidden_kept, d, S->dtype, m, d, hq * D, TG_EPI_RESIDUAL, stream)))
     return rc;
   // 6. y = RMSNorm(h)
-  if (bf)
-    tg::k_rmsnorm<__nv_bfloat16><<<unsigned(m), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(hidden_kept),
-                                                                static_cast<__nv_bfloat16*>(xn), W->w_post_norm, d,
-                                                                S->norm_eps);
-  else
-    tg::k_rmsnorm<float><<<unsigned(m), 256, 0, st>>>(static_cast<const float*>(hidden_kept),
-                                                       static_cast<float*>(xn), W->w_post_norm, d, S->norm_eps);
-  if ((rc = check_launch("k_rmsnorm"))) return rc;
+  rc = bf ? launch_rmsnorm<__nv_bfloat16>(hidden_kept, xn, W->w_post_norm, m, d, S->norm_eps, st)
+          : launch_rmsnorm<float>(hidden_kept, xn, W->w_post_norm, m, d, S->norm_eps, st);
+  if (rc) return rc;
   // 7. act = SiLU(y Wg^T) * (y Wu^T)
   if (bf && dff % 128 == 0) {
     if ((rc = tg_linear(xn, d, W->w_gate_up, act, dff, S->dtype, m, dff, d, TG_EPI_SWIGLU, stream))) return rc;
