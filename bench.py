@@ -130,6 +130,12 @@ def max_over_ranks(x: float, dist, device=None) -> float:
     return float(t.item())
 
 
+def replica_value(world: int, units_per_step: int, steps: int, slowest_seconds: float) -> float:
+    """Whole-job throughput of `world` independent replicas: every rank processes
+    units_per_step per step, and the job takes as long as its slowest rank."""
+    return world * units_per_step * steps / slowest_seconds
+
+
 def barrier(dist, device=None):
     if dist is not None:
         if device is not None and device.type == "cuda":
@@ -183,6 +189,8 @@ def oracle_step_seconds(w, gate_rows: int = 2048):
 
 def run_reference(args, w):
     rank, world, dist = dist_setup()
+    if dist is not None:
+        dist.destroy_process_group()  # rank 0 alone times the oracle; no collective follows
     if rank != 0:
         return
     times = []
@@ -261,7 +269,7 @@ def run_gpu(args, w):
     total_s = sum(step_ms) / 1e3
     total_s = max_over_ranks(total_s, dist, dev)
     ms_per_step = total_s * 1e3 / args.steps
-    value = world * w.n * args.steps / total_s
+    value = replica_value(world, w.n, args.steps, total_s)
 
     # ---- per-call breakdown (same inputs, each library call bracketed by events on the stream)
     work = workload_work(w, m)
@@ -420,7 +428,7 @@ def end_to_end(step, w, args, stream, flush, dist, dev, world):
     b.record(stream)
     torch.cuda.synchronize()
     sec = max_over_ranks(a.elapsed_time(b) / 1e3, dist, dev)
-    return {"value": world * w.n * steps / sec, "unit": "tokens/s",
+    return {"value": replica_value(world, w.n, steps, sec), "unit": "tokens/s",
             "h2d_bytes_per_step": h_host.numel() * h_host.element_size() + m_host.numel(),
             "d2h_bytes_per_step": out_host.numel() * out_host.element_size(), "steps": steps}
 
