@@ -16,6 +16,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import types
 import math
 import os
 import statistics
@@ -467,6 +468,115 @@ def ncu_case():
     print("ncu case done")
 
 
+def run_sweep(args):
+    """The other single-layer workloads (budget sweep at N=32768, K in {1024,
+    4096, 8192}; 128K with K=8192): one JSON line each with the step time, the
+    per-call breakdown and the peak HBM in use.  Parity cases, not bench lines."""
+    import torch
+    from learned_token_pruning_b200 import pipeline, synth, tokengate as tg
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for w in [synth.budget_sweep_32k(k) for k in (1024, 4096, 8192)] + [synth.long_128k()]:
+        torch.cuda.reset_peak_memory_stats(dev)
+        step = pipeline.GatedPrefillStep(w, dev)
+        step.capture()
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            step.replay()
+        torch.cuda.synchronize(dev)
+        times = []
+        for _ in range(max(args.steps, 5)):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            step.replay()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            times.append(a.elapsed_time(b))
+        tg.tg_check_device_error()
+        step_ms = sorted(times)[len(times) // 2]
+        work = workload_work(w, step.m)
+        br = breakdown(step, w, types.SimpleNamespace(steps=max(args.steps, 5)), stream, flush)
+        calls = {}
+        for name, ms in br.items():
+            e = {"us": round(ms * 1e3, 2)}
+            wk = work.get(name, {})
+            if "flops" in wk:
+                e["tflops"] = round(wk["flops"] / (ms * 1e-3) / 1e12, 1)
+                if name not in ("gate_score",):
+                    e["frac_bf16_peak"] = round(e["tflops"] / peaks["bf16_tflops"], 3)
+            if "bytes" in wk:
+                e["gbs"] = round(wk["bytes"] / (ms * 1e-3) / 1e9, 1)
+                e["frac_hbm"] = round(e["gbs"] / peaks["hbm_gbs"], 3)
+            calls[name] = e
+        line = {"mode": "sweep", "workload": w.name, "n": w.n, "k": w.k, "kept_rows": step.m,
+                "step_ms": round(step_ms, 4), "tokens_per_s": w.n / (step_ms * 1e-3),
+                "peak_hbm_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 3), "calls": calls,
+                "l2": "flushed before every timed step"}
+        print(json.dumps(line), flush=True)
+        del step
+        torch.cuda.empty_cache()
+
+
+def run_stack(args):
+    """Time to first token of a random-init 28-layer Qwen3-1.7B-shaped stack
+    (gate after layer 13) against the same stack unpruned, at N = 16K, 64K and
+    128K: from the layer-0 hidden states in HBM to the last layer's output for
+    the kept rows (embedding, final norm and LM head are not part of the path).
+    One JSON line per N."""
+    import torch
+    from learned_token_pruning_b200 import pipeline, synth, tokengate as tg
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    sizes = [(16384, 2000), (65536, 4096), (131072, 8192)]
+    if args.stack_n:
+        sizes = [x for x in sizes if x[0] in args.stack_n]
+    for n, k in sizes:
+        w = synth.full_stack_64k(n=n, k=k, name=f"qwen3_1.7b_stack28_n{n}_k{k}")
+        torch.cuda.reset_peak_memory_stats(dev)
+        g = torch.Generator(device=dev)
+        g.manual_seed(w.seed)
+        hidden = torch.randn(n, w.d_model, generator=g, device=dev).to(torch.bfloat16)
+        prunable = torch.ones(n, dtype=torch.uint8, device=dev)
+        prunable[n - w.n_question:] = 0
+        gate = {"w1": (torch.randn(w.gate_hidden, w.d_model, generator=g, device=dev) * 0.02).to(torch.bfloat16),
+                "b1": torch.zeros(w.gate_hidden, device=dev),
+                "w2": torch.randn(w.gate_hidden, generator=g, device=dev) * 0.02, "b2": 0.0, "norm_w": None}
+        layers, heads = pipeline.stack_weights_on_device(w, w.n_layers, dev)
+        st = pipeline.PrunedPrefillStack(w, hidden, prunable, gate, layers, heads, w.gate_after)
+
+        def timed(fn, reps):
+            out = []
+            for _ in range(reps):
+                st.reset()
+                torch.cuda.synchronize(dev)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize(dev)
+                out.append(a.elapsed_time(b))
+            return sorted(out)[len(out) // 2]
+
+        timed(st.run, 1)
+        timed(st.unpruned, 1)
+        tg.tg_check_device_error()
+        reps = max(1, min(args.steps, 3))
+        t_pruned = timed(st.run, reps)
+        t_full = timed(st.unpruned, reps)
+        tg.tg_check_device_error()
+        line = {"mode": "stack", "workload": w.name, "n": n, "k": k, "kept_rows": st.m, "layers": w.n_layers,
+                "gate_after_layer": w.gate_after, "ttft_ms": round(t_pruned, 3),
+                "ttft_unpruned_ms": round(t_full, 3), "speedup": round(t_full / t_pruned, 3),
+                "tokens_per_s": n / (t_pruned * 1e-3), "peak_hbm_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 3),
+                "data": "synthetic (seeded on the device: N(0,1) hidden, N(0,0.02) weights)", "reps": reps}
+        print(json.dumps(line), flush=True)
+        del st, layers, heads, hidden
+        torch.cuda.empty_cache()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -475,9 +585,18 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu-case", action="store_true", help="one launch of each heavy kernel (profiling)")
+    ap.add_argument("--sweep", action="store_true", help="budget-sweep and 128K single-layer workloads")
+    ap.add_argument("--stack", action="store_true", help="28-layer stack TTFT, pruned vs unpruned")
+    ap.add_argument("--stack-n", type=int, nargs="*", default=None, help="stack sizes to run (default all)")
     args = ap.parse_args(argv)
     if args.ncu_case:
         ncu_case()
+        return
+    if args.sweep:
+        run_sweep(args)
+        return
+    if args.stack:
+        run_stack(args)
         return
     from learned_token_pruning_b200 import synth
     w = synth.qwen3_1p7b_16k()

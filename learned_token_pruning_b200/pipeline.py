@@ -104,3 +104,123 @@ class GatedPrefillStep:
             self.capture()
         self._graph.replay()
         return self.hidden_kept
+
+
+class PrunedPrefillStack:
+    """Prefill of one prompt through a decoder stack, the three-stage forward of
+    "TokenGate and T2Quant: a close reading", §4.1: layers 0 .. gate_after run
+    on all N rows; the gate scores the residual stream leaving layer
+    gate_after, the top-K document tokens and every question token are kept
+    and gathered in order; layers gate_after+1 .. run on the kept rows with
+    token-gated attention.  `unpruned()` runs every layer on all rows with no
+    gate.  Every step is a library call on the current stream.
+
+    layers: per layer a dict of device tensors (tg_layer_weights names, without
+    head_gain / head_temp); heads: per layer a dict with device tensors
+    head_gain and head_temp (used by the layers above the gate; the layers on
+    all rows run with no gate bias and unit temperature)."""
+
+    def __init__(self, w: synth.Workload, hidden, prunable, gate: Dict, layers, heads, gate_after: int,
+                 norm_eps: float = 1e-6, eps_s: float = 1e-6):
+        self.w, self.gate_after, self.norm_eps, self.eps_s = w, gate_after, norm_eps, eps_s
+        dev = hidden.device
+        self.dt = hidden.dtype
+        self.hidden0 = hidden
+        self.h = torch.empty_like(hidden)
+        self.prunable = prunable
+        self.n_prunable = int(prunable.sum().item())
+        self.gate = gate
+        self.m = min(w.k, self.n_prunable) + (w.n - self.n_prunable)
+        self.pos_all = torch.arange(w.n, dtype=torch.int32, device=dev)
+        self.scores = torch.empty(w.n, dtype=torch.float32, device=dev)
+        self.sumsq = torch.empty(1, dtype=torch.float32, device=dev)
+        self.ws_gate = torch.empty(max(tg.tg_workspace_bytes(tg.TG_OP_GATE_SCORE, n=w.n, d_model=w.d_model,
+                                                             h=gate["w1"].shape[0]), 16), dtype=torch.uint8,
+                                   device=dev)
+        self.kept = torch.empty(self.m, dtype=torch.int32, device=dev)
+        self.hk = torch.empty(self.m, w.d_model, dtype=self.dt, device=dev)
+        self.pos = torch.empty(self.m, dtype=torch.int32, device=dev)
+        self.bias = torch.empty(self.m, dtype=torch.float32, device=dev)
+        self.ratio = torch.empty(self.m, dtype=torch.float32, device=dev)
+        ones = torch.ones(w.hq, dtype=torch.float32, device=dev)
+        zeros = torch.zeros(w.hq, dtype=torch.float32, device=dev)
+        self._keep = []  # device tensors the structs point to
+        self.full_layers, self.pruned_layers = [], []
+        for l, lw in enumerate(layers):
+            for gated in (False, True):
+                d = dict(lw)
+                d["head_gain"], d["head_temp"] = (heads[l]["head_gain"], heads[l]["head_temp"]) if gated else (zeros, ones)
+                W, S = tg.layer_structs(d, dtype=self.dt, d_model=w.d_model, hq=w.hq, hkv=w.hkv, head_dim=w.head_dim,
+                                        d_ff=w.d_ff, qk_norm=w.qk_norm, rope_theta=w.rope_theta, norm_eps=norm_eps)
+                self._keep.append(d)
+                (self.pruned_layers if gated else self.full_layers).append((W, S))
+        S0 = self.full_layers[0][1]
+        ws = max(tg.tg_workspace_bytes(tg.TG_OP_LAYER, m=w.n, shape=S0),
+                 tg.tg_workspace_bytes(tg.TG_OP_LAYER, m=self.m, shape=S0))
+        self.ws_layer = torch.empty(ws, dtype=torch.uint8, device=dev)
+
+    def reset(self):
+        """Load the layer-0 input (kept out of the timed region by the caller)."""
+        self.h.copy_(self.hidden0)
+
+    def full_part(self):
+        for W, S in self.full_layers[: self.gate_after + 1]:
+            tg.tg_pruned_prefill_layer(W, S, self.h, self.pos_all, None, None, self.ws_layer)
+
+    def gate_select_gather(self):
+        g = self.gate
+        tg.tg_gate_score(self.h, g.get("norm_w"), self.norm_eps, g["w1"], g["b1"], g["w2"], g["b2"], self.prunable,
+                         self.scores, self.sumsq, self.ws_gate)
+        tg.tg_topk_select(self.scores, self.prunable, self.n_prunable, self.w.k, self.kept)
+        tg.tg_gather(self.h, self.kept, self.scores, self.sumsq, self.n_prunable, self.eps_s, self.hk, self.pos,
+                     self.bias, self.ratio)
+
+    def pruned_part(self):
+        for W, S in self.pruned_layers[self.gate_after + 1:]:
+            tg.tg_pruned_prefill_layer(W, S, self.hk, self.pos, self.bias, self.ratio, self.ws_layer)
+
+    def run(self):
+        """Layer-0 input in self.h -> kept-row output of the last layer in self.hk."""
+        self.full_part()
+        self.gate_select_gather()
+        self.pruned_part()
+        return self.hk
+
+    def unpruned(self):
+        """Every layer on all rows (self.h), no gate."""
+        for W, S in self.full_layers:
+            tg.tg_pruned_prefill_layer(W, S, self.h, self.pos_all, None, None, self.ws_layer)
+        return self.h
+
+
+def stack_weights_from_synth(w: synth.Workload, n_layers: int, device="cuda"):
+    """Layer and head parameters of synth.py (the oracle reads the same arrays)."""
+    dt = synth.torch_dtype(w.dtype)
+    layers, heads = [], []
+    for l in range(n_layers):
+        lw = synth.layer_weights(w, layer=l)
+        layers.append({k: to_device(v, torch.float32 if k.endswith("norm") else dt, device) for k, v in lw.items()})
+        hp = synth.head_params(w, seed_offset=100 + l)
+        heads.append({k: to_device(v, torch.float32, device) for k, v in hp.items()})
+    return layers, heads
+
+
+def stack_weights_on_device(w: synth.Workload, n_layers: int, device="cuda"):
+    """The same distributions drawn by a seeded generator on the device (weights
+    N(0, 0.02), norm weights 1, gain U(0.5, 2), temperature U(0.8, 1.2)), for
+    stacks too large to draw on the host."""
+    dt = synth.torch_dtype(w.dtype)
+    d, D, hq, hkv, dff = w.d_model, w.head_dim, w.hq, w.hkv, w.d_ff
+    layers, heads = [], []
+    for l in range(n_layers):
+        g = torch.Generator(device=device)
+        g.manual_seed(w.seed * 1000 + 200 + l)
+        rnd = lambda *shape: (torch.randn(*shape, generator=g, device=device) * 0.02).to(dt)
+        layers.append({
+            "w_in_norm": torch.ones(d, device=device), "w_qkv": rnd((hq + 2 * hkv) * D, d),
+            "w_q_norm": torch.ones(D, device=device), "w_k_norm": torch.ones(D, device=device),
+            "w_o": rnd(d, hq * D), "w_post_norm": torch.ones(d, device=device),
+            "w_gate_up": rnd(2 * dff, d), "w_down": rnd(d, dff)})
+        heads.append({"head_gain": torch.rand(hq, generator=g, device=device) * 1.5 + 0.5,
+                      "head_temp": torch.rand(hq, generator=g, device=device) * 0.4 + 0.8})
+    return layers, heads

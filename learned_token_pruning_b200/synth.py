@@ -47,6 +47,8 @@ class Workload:
     plant_shift: float = 3.0
     question_first: bool = False
     score_mixture: bool = False   # inject Gaussian-mixture scores for the selector
+    n_layers: int = 1             # decoder layers of a whole-stack workload
+    gate_after: int = 0           # the gate scores the residual leaving this layer
 
     @property
     def n_prunable(self) -> int:
@@ -95,6 +97,15 @@ def long_128k(**kw) -> Workload:
     w = Workload(name="qwen3_1.7b_layer_n131072_k8192", seed=4, n=131072, n_question=64,
                  d_model=2048, hq=16, hkv=8, head_dim=128, gate_hidden=256, k=8192, dtype="bf16",
                  d_ff=6144, score_mixture=True)
+    return w.replace(**kw) if kw else w
+
+
+def full_stack_64k(**kw) -> Workload:
+    """Random-init 28-layer Qwen3-1.7B-shaped stack, gate after layer 13,
+    N=65536 with 64 question tokens, K=4096 (TTFT against the unpruned stack)."""
+    w = Workload(name="qwen3_1.7b_stack28_n65536_k4096", seed=5, n=65536, n_question=64,
+                 d_model=2048, hq=16, hkv=8, head_dim=128, gate_hidden=256, k=4096, dtype="bf16",
+                 d_ff=6144, n_layers=28, gate_after=13)
     return w.replace(**kw) if kw else w
 
 

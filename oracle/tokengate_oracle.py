@@ -160,8 +160,8 @@ def gated_attention(q, k, v, bias, head_gain, head_temp, ratio, sm_scale: float,
 
     [R] §4.1: alpha_ij = exp(z_ij) g_j / sum_j' exp(z_ij') g_j' with
     g_j = softmax(b_j).  The softmax normaliser of g is common to every key and
-    cancels, so alpha is a softmax over z_ij + b_j ([K], [M]: "the score becomes
-    a bias on the attention logits").  READINGS: the head-wise gain
+    cancels, so alpha is a softmax over z_ij + b_j ([K] and [M] describe the
+    score acting as a bias on the attention logits).  READINGS: the head-wise gain
     softplus(gamma_h) acts in log space, i.e. the bias term is gain_h * b_j (a
     plain multiplier on g_j would cancel); the temperature
     tau_i = softplus(sigma_h) * log m_i / log max(2, p_i) multiplies the content
@@ -277,3 +277,45 @@ def pruned_prefill_step(hidden, gate: Dict[str, np.ndarray], k: int, layer: Dict
                         bias=g["bias"], ratio=g["ratio"], head_gain=head_gain, head_temp=head_temp,
                         rope_theta=rope_theta, qk_norm=qk_norm, norm_eps=norm_eps)
     return {"scores": s, "kept_idx": idx, **g, "out": out}
+
+
+# ---------------------------------------------------------------------------
+# A whole decoder stack  ([R] §4.1 three-stage forward)
+# ---------------------------------------------------------------------------
+def pruned_prefill_stack(hidden, layers: Sequence[Dict[str, np.ndarray]], heads: Sequence[Dict[str, np.ndarray]],
+                         gate: Dict[str, np.ndarray], k: int, gate_after: int, *, hq: int, hkv: int,
+                         head_dim: int, rope_theta: float, qk_norm: bool, norm_eps: float = 1e-6,
+                         eps_s: float = 1e-6, pruned: bool = True) -> Dict[str, np.ndarray]:
+    """Prefill of one prompt through len(layers) decoder layers.
+
+    [R] §4.1 splits the forward in three: layers below the gate run on every
+    token; the gate scores the tokens, keeps the top-K documents tokens plus
+    the question and compacts them in order; the layers above run on the kept
+    tokens only, with token-gated attention.  Here layers 0 .. gate_after run
+    on all N rows (positions 0..N-1, no gate bias, ratio 1, temperature 1);
+    READING: the gate after layer L scores the residual stream leaving layer L
+    (normalised by gate['norm_w']); layers gate_after+1 .. run on the kept rows
+    with each layer's head gain and temperature (heads[l]).  With pruned=False
+    every layer runs on all rows with no gate: the unpruned stack.
+    """
+    h = np.asarray(hidden, dtype=F64)
+    n = h.shape[0]
+    pos = np.arange(n)
+    n_layers = len(layers)
+    common = dict(hq=hq, hkv=hkv, head_dim=head_dim, rope_theta=rope_theta, qk_norm=qk_norm, norm_eps=norm_eps)
+    n_full = n_layers if not pruned else gate_after + 1
+    for l in range(n_full):
+        h = decoder_layer(h, layers[l], pos=pos, bias=None, ratio=None, head_gain=np.zeros(hq),
+                          head_temp=np.ones(hq), **common)
+    if not pruned:
+        return {"out": h}
+    prunable = gate["prunable"]
+    s = gate_scores(h, gate["norm_w"], norm_eps, gate["w1"], gate["b1"], gate["w2"], gate["b2"], prunable)
+    s32 = s.astype(np.float32)
+    idx = select_kept(s32, prunable, k)
+    g = gather(h, idx, s32, prunable, eps_s)
+    hk = g["hidden_kept"]
+    for l in range(gate_after + 1, n_layers):
+        hk = decoder_layer(hk, layers[l], pos=g["pos"], bias=g["bias"], ratio=g["ratio"],
+                           head_gain=heads[l]["head_gain"], head_temp=heads[l]["head_temp"], **common)
+    return {"gate_input": h, "scores": s, "kept_idx": idx, **g, "out": hk}

@@ -384,6 +384,53 @@ def test_keep_everything_with_zero_gain_reduces_to_unpruned_layer():
     np.testing.assert_allclose(res["out"], full, rtol=1e-12, atol=1e-12)
 
 
+# ----------------------------------------------------------------------------- a whole stack
+
+def _stack_case(n_layers=4):
+    w = _small_layer_workload()
+    layers = [synth.layer_weights(w, layer=l) for l in range(n_layers)]
+    heads = [synth.head_params(w, seed_offset=100 + l) for l in range(n_layers)]
+    return w, synth.gate_inputs(w), layers, heads
+
+
+def _stack(w, g, layers, heads, k, gate_after, pruned=True):
+    return O.pruned_prefill_stack(g["hidden"], layers, heads, g, k, gate_after, hq=w.hq, hkv=w.hkv,
+                                  head_dim=w.head_dim, rope_theta=w.rope_theta, qk_norm=True, pruned=pruned)
+
+
+def test_stack_keeping_everything_with_zero_gain_is_the_unpruned_stack():
+    w, g, layers, heads = _stack_case()
+    flat = [{"head_gain": np.zeros(w.hq), "head_temp": np.ones(w.hq)} for _ in layers]
+    res = _stack(w, g, layers, flat, w.n, gate_after=1)
+    assert list(res["kept_idx"]) == list(range(w.n))
+    full = _stack(w, g, layers, heads, w.n, gate_after=1, pruned=False)
+    np.testing.assert_allclose(res["out"], full["out"], rtol=1e-12, atol=1e-12)
+
+
+def test_stack_gate_at_the_top_gathers_the_unpruned_output():
+    w, g, layers, heads = _stack_case(3)
+    res = _stack(w, g, layers, heads, w.k, gate_after=2)
+    full = _stack(w, g, layers, heads, w.k, gate_after=2, pruned=False)
+    assert len(res["kept_idx"]) == w.k + w.n_question
+    np.testing.assert_array_equal(res["out"], full["out"][res["kept_idx"]])
+
+
+def test_unpruned_stack_matches_a_chain_of_transformers_layers():
+    w, g, layers, heads = _stack_case(3)
+    ours = _stack(w, g, layers, heads, w.k, gate_after=0, pruned=False)["out"]
+    x = torch.from_numpy(np.asarray(g["hidden"], dtype=np.float64))[None]
+    pid = torch.arange(w.n)[None]
+    mask = torch.zeros(w.n, w.n, dtype=torch.float64).masked_fill(
+        ~torch.ones(w.n, w.n, dtype=torch.bool).tril(), float("-inf"))[None, None]
+    with torch.no_grad():
+        for lw in layers:
+            layer, rot = _hf_layer(w, lw, w.n)
+            cos, sin = rot(x, pid)
+            x = layer(x, attention_mask=mask, position_ids=pid, position_embeddings=(cos, sin))
+            x = x[0] if isinstance(x, tuple) else x
+    np.testing.assert_allclose(ours, x[0].numpy(), rtol=1e-5, atol=1e-5)
+
+
 # ----------------------------------------------------------------------------- synthetic inputs
 
 def test_tiny_workload_planted_block_is_kept_by_oracle():
