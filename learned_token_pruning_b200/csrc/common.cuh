@@ -40,6 +40,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the kernel before it in the stream is still
+// running: pdl_wait() blocks until that kernel has completed and its writes
+// are visible (a no-op after a normal launch), so every kernel calls it after
+// its set-up (barriers, TMEM, shared memory) and before its first
+// global-memory access; pdl_launch_dependents() lets the next kernel's CTAs
+// start their own set-up on SMs this kernel leaves idle.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Upper bound of any single wait inside a kernel.  The longest legitimate wait
 // (an epilogue warp waiting for a whole attention row block at 128K tokens) is
 // a few milliseconds, so one second only expires on a genuine bug.

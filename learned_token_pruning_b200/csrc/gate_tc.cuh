@@ -98,17 +98,20 @@ __global__ void __launch_bounds__(kGateThreads, 1)
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_launch_dependents();
   if (threadIdx.x >= 64) {
-    // columns past h (zero rows of W1 from the TMA bounds fill) contribute nothing
+    // columns past h (zero rows of W1 from the TMA bounds fill) contribute
+    // nothing; read by the epilogue after its first named barrier
     for (int i = threadIdx.x - 64; i < BN; i += kGateThreads - 64) {
       s_b1[i] = (i < p.N && p.b1) ? p.b1[i] : 0.0f;
       s_w2[i] = i < p.N ? p.w2[i] : 0.0f;
     }
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) {

@@ -38,6 +38,8 @@ struct GatherParams {
 };
 
 __global__ void __launch_bounds__(kGatherThreads) k_gather(GatherParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ int64_t src_row[kGatherRows];
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kGatherRows;
   const int tid = threadIdx.x;
@@ -111,6 +113,8 @@ __device__ __forceinline__ void gather_side_outputs(const GatherParams& p, int64
 
 // rows_per_batch * row_bytes * 2 <= dynamic shared memory; rows [r_begin, r_end) per CTA.
 __global__ void __launch_bounds__(kGatherBulkThreads) k_gather_bulk(GatherParams p, int rows_per_batch) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(128) uint8_t gbuf[];
   __shared__ uint64_t bar[2];
   const int64_t per = (p.m + gridDim.x - 1) / gridDim.x;

@@ -96,6 +96,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, MH>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer

@@ -81,6 +81,8 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
 }
 
 __global__ void __launch_bounds__(kSelThreads, 1) k_topk_select(SelectParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(16) uint8_t sel_smem[];
   __shared__ uint32_t hist[256];
   __shared__ uint32_t warp_sums[kSelWarps + 1];
@@ -298,6 +300,8 @@ __device__ __forceinline__ uint32_t block_exclusive_scan_1024(uint32_t v, uint32
 // scores and mask are 16- and 4-byte aligned (4 tokens per load).
 template <int KPT>
 __global__ void __launch_bounds__(kSelSmallThreads, 1) k_topk_select_cta(SelectParams p, int vec) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(16) uint32_t skeys[];
   __shared__ uint32_t whist[kSelSmallWarps][256];
   __shared__ uint32_t warp_sums[33];

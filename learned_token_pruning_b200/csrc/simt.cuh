@@ -235,6 +235,8 @@ __global__ void __launch_bounds__(256) k_gemm_simt(const T* __restrict__ A, int6
 template <typename T>
 __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ x, T* __restrict__ y,
                                                  const float* __restrict__ w, int d, float eps) {
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int V = 16 / sizeof(T);  // elements per 16-byte vector
   __shared__ float part[8];
   const T* xr = x + static_cast<int64_t>(blockIdx.x) * d;
@@ -347,6 +349,8 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope(T* __restrict__ qkv, int64
 template <typename T, int MAXV>
 __global__ void __launch_bounds__(256) k_rmsnorm_warp(const T* __restrict__ x, T* __restrict__ y,
                                                       const float* __restrict__ w, int64_t m, int d, float eps) {
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int V = 16 / sizeof(T);
   const int lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
@@ -415,6 +419,8 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope_warp(T* __restrict__ qkv, 
                                                            const float* __restrict__ wq, const float* __restrict__ wk,
                                                            int qk_norm, float eps,
                                                            const __grid_constant__ RopeTable tab) {
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int H2 = D / 2;
   constexpr int E = H2 / 32;
   constexpr int HU = 8;  // heads in flight

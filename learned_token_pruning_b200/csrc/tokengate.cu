@@ -50,6 +50,28 @@ int check_launch(const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel in the stream is finishing, does its set-up, and
+// waits in pdl_wait() (griddepcontrol.wait) before touching global memory.
+// Every kernel launched here calls pdl_wait() before its first global access.
+template <typename... KArgs, typename... Args>
+int launch_pdl(const char* what, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+               Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e != cudaSuccess) return fail(TG_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+  return check_launch(what);
+}
+
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 // ---------------------------------------------------------------------------
@@ -167,8 +189,7 @@ int launch_gemm_tc(const void* A, int64_t lda, const void* B, int64_t b_rows, in
   p.tiles_n = tiles_n;
   const int tiles = p.tiles_m * p.tiles_n;
   const int grid = tiles < sm_count() ? tiles : sm_count();
-  kern<<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(ta, tb, p);
-  return check_launch("k_gemm_tc");
+  return launch_pdl("k_gemm_tc", kern, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmem, st, ta, tb, p);
 }
 
 template <int BN, int EPI>
@@ -195,8 +216,8 @@ int launch_gate_tc(const void* A, const void* W1, int M, int K, const tg::GatePa
   p.M = M;
   p.K = K;
   p.hidden = static_cast<const __nv_bfloat16*>(A);
-  tg::k_gate_tc<BN><<<(M + tg::kGateBM - 1) / tg::kGateBM, tg::kGateThreads, Cfg::kSmem, st>>>(ta, tb, p);
-  return check_launch("k_gate_tc");
+  return launch_pdl("k_gate_tc", tg::k_gate_tc<BN>, dim3((M + tg::kGateBM - 1) / tg::kGateBM), dim3(tg::kGateThreads),
+                    Cfg::kSmem, st, ta, tb, p);
 }
 
 int dtype_size(int dtype) { return dtype == TG_BF16 ? 2 : (dtype == TG_F32 ? 4 : 0); }
@@ -221,20 +242,16 @@ int launch_rmsnorm(const void* x, void* y, const float* w, int64_t m, int d, flo
   const unsigned blocks = static_cast<unsigned>((m + 7) / 8);
   if (!w || aligned16(w)) {
     if (nv <= 32 * 4) {
-      tg::k_rmsnorm_warp<T, 4><<<blocks, 256, 0, st>>>(xa, ya, w, m, d, eps);
-      return check_launch("k_rmsnorm_warp");
+      return launch_pdl("k_rmsnorm_warp", tg::k_rmsnorm_warp<T, 4>, dim3(blocks), dim3(256), 0, st, xa, ya, w, m, d, eps);
     }
     if (nv <= 32 * 8) {
-      tg::k_rmsnorm_warp<T, 8><<<blocks, 256, 0, st>>>(xa, ya, w, m, d, eps);
-      return check_launch("k_rmsnorm_warp");
+      return launch_pdl("k_rmsnorm_warp", tg::k_rmsnorm_warp<T, 8>, dim3(blocks), dim3(256), 0, st, xa, ya, w, m, d, eps);
     }
     if (nv <= 32 * 16) {
-      tg::k_rmsnorm_warp<T, 16><<<blocks, 256, 0, st>>>(xa, ya, w, m, d, eps);
-      return check_launch("k_rmsnorm_warp");
+      return launch_pdl("k_rmsnorm_warp", tg::k_rmsnorm_warp<T, 16>, dim3(blocks), dim3(256), 0, st, xa, ya, w, m, d, eps);
     }
   }
-  tg::k_rmsnorm<T><<<unsigned(m), 256, 0, st>>>(xa, ya, w, d, eps);
-  return check_launch("k_rmsnorm");
+  return launch_pdl("k_rmsnorm", tg::k_rmsnorm<T>, dim3(unsigned(m)), dim3(256), 0, st, xa, ya, w, d, eps);
 }
 
 extern "C" {
@@ -495,22 +512,21 @@ int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int6
     switch (kpt) {
       case 4:
         if ((rc = set_smem(tg::k_topk_select_cta<4>, smem))) return rc;
-        tg::k_topk_select_cta<4><<<1, tg::kSelSmallThreads, smem, st>>>(p, vec);
-        break;
+        return launch_pdl("k_topk_select_cta", tg::k_topk_select_cta<4>, dim3(1), dim3(tg::kSelSmallThreads), smem,
+                          st, p, vec);
       case 8:
         if ((rc = set_smem(tg::k_topk_select_cta<8>, smem))) return rc;
-        tg::k_topk_select_cta<8><<<1, tg::kSelSmallThreads, smem, st>>>(p, vec);
-        break;
+        return launch_pdl("k_topk_select_cta", tg::k_topk_select_cta<8>, dim3(1), dim3(tg::kSelSmallThreads), smem,
+                          st, p, vec);
       case 16:
         if ((rc = set_smem(tg::k_topk_select_cta<16>, smem))) return rc;
-        tg::k_topk_select_cta<16><<<1, tg::kSelSmallThreads, smem, st>>>(p, vec);
-        break;
+        return launch_pdl("k_topk_select_cta", tg::k_topk_select_cta<16>, dim3(1), dim3(tg::kSelSmallThreads), smem,
+                          st, p, vec);
       default:
         if ((rc = set_smem(tg::k_topk_select_cta<32>, smem))) return rc;
-        tg::k_topk_select_cta<32><<<1, tg::kSelSmallThreads, smem, st>>>(p, vec);
-        break;
+        return launch_pdl("k_topk_select_cta", tg::k_topk_select_cta<32>, dim3(1), dim3(tg::kSelSmallThreads), smem,
+                          st, p, vec);
     }
-    return check_launch("k_topk_select_cta");
   }
   // cluster of 2, 4 or 8 CTAs: about 4096 tokens per CTA, and slices that fit the key cache
   int csize = 1;
@@ -528,13 +544,15 @@ int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int6
   cfg.blockDim = dim3(tg::kSelThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = as_stream(stream);
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, tg::k_topk_select, p);
   if (e != cudaSuccess) return fail(TG_ERR_CUDA, "k_topk_select launch: %s", cudaGetErrorString(e));
   return check_launch("k_topk_select");
@@ -576,12 +594,11 @@ int tg_gather(const void* hidden, int dtype, int64_t n, int32_t d_model, const i
     const size_t smem = static_cast<size_t>(2) * rows_per_batch * row_bytes;
     int rc = set_smem(tg::k_gather_bulk, smem);
     if (rc) return rc;
-    tg::k_gather_bulk<<<blocks, tg::kGatherBulkThreads, smem, as_stream(stream)>>>(p, rows_per_batch);
-    return check_launch("k_gather_bulk");
+    return launch_pdl("k_gather_bulk", tg::k_gather_bulk, dim3(blocks), dim3(tg::kGatherBulkThreads), smem,
+                      as_stream(stream), p, rows_per_batch);
   }
   const unsigned blocks = static_cast<unsigned>((m + tg::kGatherRows - 1) / tg::kGatherRows);
-  tg::k_gather<<<blocks, tg::kGatherThreads, 0, as_stream(stream)>>>(p);
-  return check_launch("k_gather");
+  return launch_pdl("k_gather", tg::k_gather, dim3(blocks), dim3(tg::kGatherThreads), 0, as_stream(stream), p);
 }
 
 int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk, const void* v, int64_t ldv, int dtype,
@@ -654,13 +671,14 @@ int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk, c
     if (head_dim == 128) {
       rc = set_smem(tg::k_attn_tc<128>, tg::AttnCfg<128>::kSmem);
       if (rc) return rc;
-      tg::k_attn_tc<128><<<blocks, tg::kAttnThreads, tg::AttnCfg<128>::kSmem, st>>>(tq, tk, tv, tb, to, p, work);
+      return launch_pdl("k_attn_tc", tg::k_attn_tc<128>, dim3(blocks), dim3(tg::kAttnThreads), tg::AttnCfg<128>::kSmem, st, tq, tk,
+                        tv, tb, to, p, work);
     } else {
       rc = set_smem(tg::k_attn_tc<64>, tg::AttnCfg<64>::kSmem);
       if (rc) return rc;
-      tg::k_attn_tc<64><<<blocks, tg::kAttnThreads, tg::AttnCfg<64>::kSmem, st>>>(tq, tk, tv, tb, to, p, work);
+      return launch_pdl("k_attn_tc", tg::k_attn_tc<64>, dim3(blocks), dim3(tg::kAttnThreads), tg::AttnCfg<64>::kSmem, st, tq, tk,
+                        tv, tb, to, p, work);
     }
-    return check_launch("k_attn_tc");
   }
   tg::AttnSimtParams p{};
   p.q = q;
@@ -783,26 +801,21 @@ int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, 
     tg::RopeTable tab{};
     for (int i = 0; i < D / 2; ++i) tab.inv_freq[i] = std::pow(static_cast<double>(S->rope_theta), -2.0 * i / D);
     const unsigned blocks = unsigned((m + 7) / 8);
+    const dim3 g(blocks), b(256);
     if (bf) {
-      if (D == 128)
-        tg::k_qk_norm_rope_warp<__nv_bfloat16, 128><<<blocks, 256, 0, st>>>(
-            static_cast<__nv_bfloat16*>(qkv), qkv_w, int(m), hq, hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm,
-            S->norm_eps, tab);
-      else
-        tg::k_qk_norm_rope_warp<__nv_bfloat16, 64><<<blocks, 256, 0, st>>>(
-            static_cast<__nv_bfloat16*>(qkv), qkv_w, int(m), hq, hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm,
-            S->norm_eps, tab);
+      auto* x = static_cast<__nv_bfloat16*>(qkv);
+      rc = D == 128 ? launch_pdl("k_qk_norm_rope_warp", tg::k_qk_norm_rope_warp<__nv_bfloat16, 128>, g, b, 0, st, x,
+                                 qkv_w, int(m), hq, hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm, S->norm_eps, tab)
+                    : launch_pdl("k_qk_norm_rope_warp", tg::k_qk_norm_rope_warp<__nv_bfloat16, 64>, g, b, 0, st, x,
+                                 qkv_w, int(m), hq, hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm, S->norm_eps, tab);
     } else {
-      if (D == 128)
-        tg::k_qk_norm_rope_warp<float, 128><<<blocks, 256, 0, st>>>(static_cast<float*>(qkv), qkv_w, int(m), hq,
-                                                                   hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm,
-                                                                   S->norm_eps, tab);
-      else
-        tg::k_qk_norm_rope_warp<float, 64><<<blocks, 256, 0, st>>>(static_cast<float*>(qkv), qkv_w, int(m), hq,
-                                                                  hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm,
-                                                                  S->norm_eps, tab);
+      auto* x = static_cast<float*>(qkv);
+      rc = D == 128 ? launch_pdl("k_qk_norm_rope_warp", tg::k_qk_norm_rope_warp<float, 128>, g, b, 0, st, x, qkv_w,
+                                 int(m), hq, hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm, S->norm_eps, tab)
+                    : launch_pdl("k_qk_norm_rope_warp", tg::k_qk_norm_rope_warp<float, 64>, g, b, 0, st, x, qkv_w,
+                                 int(m), hq, hkv, pos, W->w_q_norm, W->w_k_norm, S->qk_norm, S->norm_eps, tab);
     }
-    if ((rc = check_launch("k_qk_norm_rope_warp"))) return rc;
+    if (rc) return rc;
   }
   // 4. token-gated attention
   {
