@@ -312,16 +312,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // per tile j: P V of tile j for head 0, then head 1, then the scores of
       // tile j + 2 into the S buffers whose tile j the softmax has read (its
       // p_full arrival comes after its S loads completed)
+      // Each barrier check of this thread holds back its next MMA issue for a
+      // shared-memory round trip (~150-250 cycles), during which the tensor
+      // core's short queue drains; so all four barriers a tile needs (V, the P
+      // of both heads, K of tile j + 2) are checked at once, and the tile's
+      // twenty-four MMAs then issue back to back.
       for (int j = 0; ok && j < nt; ++j) {
         const uint32_t ph = (j >> 1) & 1;
-        if (!(ok = mbar_wait2(&v_full[j & 1], ph, &p_full[j & 1], ph, kErrWaitAttention))) break;
+        const bool next = j + 2 < nt;
+        {
+          uint64_t* kb = &k_full[(j + 2) % 3];
+          const uint32_t kph = ((j + 2) / 3) & 1;
+          const bool r0 = mbar_try_wait(smem_u32(&v_full[j & 1]), ph);
+          const bool r1 = mbar_try_wait(smem_u32(&p_full[j & 1]), ph);
+          const bool r2 = mbar_try_wait(smem_u32(&p_full[2 + (j & 1)]), ph);
+          const bool r3 = !next || mbar_try_wait(smem_u32(kb), kph);
+          if (!(r0 && r1 && r2 && r3)) {
+            ok = mbar_wait2(&v_full[j & 1], ph, &p_full[j & 1], ph, kErrWaitAttention) &&
+                 mbar_wait(&p_full[2 + (j & 1)], ph, kErrWaitAttention) &&
+                 (!next || mbar_wait(kb, kph, kErrWaitAttention));
+            if (!ok) break;
+          }
+        }
         tc_fence_after();
         issue_pv(0, j);
-        const bool next = j + 2 < nt;
-        ok = next ? mbar_wait2(&p_full[2 + (j & 1)], ph, &k_full[(j + 2) % 3], ((j + 2) / 3) & 1, kErrWaitAttention)
-                  : mbar_wait(&p_full[2 + (j & 1)], ph, kErrWaitAttention);
-        if (!ok) break;
-        tc_fence_after();
         issue_pv(1, j);
         umma_commit(&pv_done[j & 3]);
         if (next) {
