@@ -21,27 +21,24 @@
 //              ring and V tiles through a 2-stage ring)
 //   warp 9     TMEM allocator and single-thread tcgen05.mma issuer
 // Tensor memory (512 columns): S of each head double-buffered, 4 x 64 columns,
-// then O0 and O1 (D columns each).  S = Q K^T is an SS-MMA into TMEM; P =
-// exp2(x - m) is written as bf16 to shared memory (128-byte swizzle,
-// double-buffered per head) and O += P V is an SS-MMA with V read MN-major.
-// Per key tile j the MMA thread issues P V of tile j for both heads and then
-// Q K^T of tile j + 2, so the scores of the next tile are ready when a
-// softmax finishes and the loop is bounded by the slower of the softmax and
-// the tensor core, not by their sum.
+// then O0 and O1 (D columns each).  S = Q K^T is an SS-MMA into TMEM; the
+// softmax reads S with tcgen05.ld and writes P = exp2(x - m) as bf16 pairs
+// back over the first 32 columns of the same S buffer; O += P V is a TS-MMA
+// (P from tensor memory, V MN-major from shared memory), which leaves the
+// shared-memory port to Q, K and V.  Per key tile j the MMA thread issues
+// P V of tile j for both heads and then Q K^T of tile j + 2 into the S
+// buffers tile j used (in issue order, after P V has read P), so the scores
+// of the next tile are ready when a softmax finishes and the loop is bounded
+// by the slower of the softmax and the tensor core, not by their sum.
 //
-// The MMA thread is the one serial resource of the CTA: it shares its SM
-// sub-partition with two softmax warps, and every barrier check it makes costs
-// a shared-memory round trip.  So it makes two checks per key tile, each of
-// two barriers at once (their latencies overlap), and three commits: one
-// "P V of tile j done" barrier (a ring of 4) frees the K and V stages for the
-// producer, the P buffer for the softmax and orders the O rescale, and
-// "softmax read S" needs no barrier of its own because the softmax only
-// declares P ready after its S loads have completed.  The softmax does its
-// elementwise arithmetic on packed pairs (fma/add.f32x2, three-input max),
-// which halves its FMA-pipe instructions and leaves issue slots to the MMA
-// thread.  The running row maximum only moves when it grows by more than 8
-// (log2 units); O is then rescaled in tensor memory by the softmax warps after
-// the previous P V into it has completed.
+// The MMA thread checks the four barriers a tile needs (V, the P of both
+// heads, K of tile j + 2) at once: each mbarrier check holds back its next
+// tcgen05.mma for a shared-memory round trip while the tensor core's short
+// queue drains.  The softmax does its elementwise arithmetic on packed pairs
+// (fma/add.f32x2, three-input max), which halves its FMA-pipe instructions and
+// leaves issue slots to the MMA thread.  The running row maximum only moves
+// when it grows by more than 8 (log2 units); O is then rescaled in tensor
+// memory by the softmax warps after the previous P V into it has completed.
 #pragma once
 
 #include "common.cuh"
@@ -65,7 +62,7 @@ struct AttnCfg {
   static constexpr size_t kOffK = 2 * kQBytes;
   static constexpr size_t kOffV = kOffK + kKStages * kKVBytes;
   static constexpr size_t kOffP = kOffV + kVStages * kKVBytes;
-  static constexpr size_t kOffBias = kOffP + 4 * kPBytes;
+  static constexpr size_t kOffBias = kOffP;  // (P lives in tensor memory, over its S columns)
   static constexpr size_t kOffBars = kOffBias + kKStages * BN * 4;  // 16 barriers + TMEM slot
   static constexpr size_t kData = kOffBars + 256;
   // D = 64 is padded so that only one CTA fits on an SM and its 512-column
@@ -176,7 +173,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* sQ = smem;                     // [2 heads][kQBytes]
   uint8_t* sK = smem + Cfg::kOffK;        // [3 stages][kKVBytes]
   uint8_t* sV = smem + Cfg::kOffV;        // [2 stages][kKVBytes]
-  uint8_t* sP = smem + Cfg::kOffP;        // [2 heads][2 buffers][kPBytes]
   float* sBias = reinterpret_cast<float*>(smem + Cfg::kOffBias);  // [3 stages][BN]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBars);
   uint64_t* q_full = bars + 0;
@@ -279,7 +275,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // slice adds its byte offset / 16 to the start-address field
       const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
-      const uint64_t dp0 = sdesc_sw128(smem_u32(sP), 16, 1024);
       const uint64_t dv0 = sdesc_sw128(smem_u32(sV), Cfg::kKVBlk, 1024);
       auto issue_qk = [&](int h, int j) {
         const uint64_t da = dq0 + (h * Cfg::kQBytes >> 4), db = dk0 + ((j % 3) * Cfg::kKVBytes >> 4);
@@ -291,11 +286,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         umma_commit(&s_full[2 * h + (j & 1)]);
       };
       auto issue_pv = [&](int h, int j) {
-        const uint64_t da = dp0 + ((2 * h + (j & 1)) * Cfg::kPBytes >> 4), db = dv0 + ((j & 1) * Cfg::kKVBytes >> 4);
+        // A = P from tensor memory (two bf16 keys per column, over the S columns of tile j)
+        const uint32_t pa = tmem + attn_col_s(h, j & 1);
+        const uint64_t db = dv0 + ((j & 1) * Cfg::kKVBytes >> 4);
         const uint32_t d_tmem = tmem + (h ? Cfg::kColO1 : Cfg::kColO0);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ss(d_tmem, da + ((kk * 32) >> 4), db + ((kk * 16 * 128) >> 4), idesc_pv, (j | kk) != 0 ? 1u : 0u);
+          umma_ts(d_tmem, pa + kk * 8, db + ((kk * 16 * 128) >> 4), idesc_pv, (j | kk) != 0 ? 1u : 0u);
       };
       // the scores of tiles 0 and 1 first
       bool ok = mbar_wait2(q_full, 0, &k_full[0], 0, kErrWaitAttention);
@@ -362,17 +359,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint64_t ay2 = f2_pack(a_y, a_y), gg2 = f2_pack(gg, gg);
     float m_run = -INFINITY, l_run = 0.0f;  // running max of y, running sum of exp2(g * (y - m_run))
     bool ok = true;
-    // this thread's 128-byte row of head wg's first P buffer; 16-byte chunk c sits at c ^ (row & 7)
-    uint8_t* prow0 = sP + (2 * wg) * Cfg::kPBytes + row * 128;
-    const int sw = row & 7;
+    const int sw = row & 7;  // 16-byte chunk c of a 128-byte swizzled row sits at c ^ (row & 7)
 
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1;
       const uint32_t ph = (j >> 1) & 1;
-      // S of tile j, its bias tile (it rides with K) and, from tile 2 on, P
-      // buffer b back from the P V of tile j - 2
+      // S of tile j and its bias tile (it rides with K); P goes over the S
+      // columns, which the P V of tile j - 2 had read before the Q K^T of
+      // tile j wrote them
       bool rdy = !*abort_flag && mbar_wait2(&s_full[2 * wg + b], ph, &k_full[j % 3], (j / 3) & 1, kErrWaitAttention);
-      if (rdy && j >= 2) rdy = mbar_wait(&pv_done[(j - 2) & 3], ((j - 2) >> 2) & 1, kErrWaitAttention);
       if (!__all_sync(0xffffffffu, rdy)) {
         ok = false;
         break;
@@ -429,29 +424,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       const float nm = -gg * m_run;
       const uint64_t nm2 = f2_pack(nm, nm);
-      // Pass 2: p = 2^(g*y - g*m), partial sums on pairs, P as bf16 into shared memory
+      // Pass 2: p = 2^(g*y - g*m), partial sums on pairs, P as bf16 pairs into
+      // tensor memory over the first 32 columns of this tile's S buffer
       uint64_t sum2[2] = {0, 0};
-      uint8_t* prow = prow0 + b * Cfg::kPBytes;
+      uint32_t pk[BN / 2];
 #pragma unroll
-      for (int c = 0; c < BN / 8; ++c) {  // 16-byte chunks of 8 keys
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float x0, x1;
-          f2_unpack(f2_fma(gg2, y2[4 * c + e], nm2), x0, x1);
-          float p0, p1;
-          if (kPolyShare && e == 3) {
-            p0 = exp2_poly(x0);
-            p1 = exp2_poly(x1);
-          } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
-          sum2[e & 1] = f2_add(sum2[e & 1], f2_pack(p0, p1));
-          pk[e] = pack_bf16x2(p0, p1);
+      for (int i = 0; i < BN / 2; ++i) {
+        float x0, x1;
+        f2_unpack(f2_fma(gg2, y2[i], nm2), x0, x1);
+        float p0, p1;
+        if (kPolyShare && (i & 3) == 3) {
+          p0 = exp2_poly(x0);
+          p1 = exp2_poly(x1);
+        } else {
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
         }
-        *reinterpret_cast<uint4*>(prow + ((c ^ sw) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        sum2[i & 1] = f2_add(sum2[i & 1], f2_pack(p0, p1));
+        pk[i] = pack_bf16x2(p0, p1);
       }
+      tmem_st32(tmem + lane_base + attn_col_s(wg, b), pk);
       float sa, sb, sc2, sd;
       f2_unpack(sum2[0], sa, sb);
       f2_unpack(sum2[1], sc2, sd);
@@ -475,12 +467,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * sc);
           tmem_st32(tmem + lane_base + colO + c0, o);
         }
-        tmem_st_wait();
       }
-      // S loads (and any O rescale) are complete; make the generic-proxy P
-      // stores visible to the tensor core (async proxy), then hand P over
+      // the S loads, the P store and any O rescale are complete: hand P over
+      tmem_st_wait();
       tc_fence_before();
-      fence_proxy_async_smem();
       mbar_arrive(&p_full[2 * wg + b]);
     }
     if (ok && !*abort_flag) ok = warp_wait(o_final, 0, kErrWaitAttention);
@@ -535,10 +525,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       s_me = inv;
     }
     if (write_out) {
-      // O as bf16 into the P buffers (free once o_final has completed), in the
+      // O as bf16 into the K/V stages, in the
       // 128-byte-swizzled layout of the output tensor map: box b holds columns
       // 64b..64b+63, row r at 128 r, 16-byte chunk c at c ^ (r & 7)
-      uint8_t* stage = sP + wg * (Cfg::kPBytes * 2);
+      uint8_t* stage = sK + wg * (128 * D * 2);  // K/V stages are idle once o_final has completed
       tc_fence_after();
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
