@@ -26,7 +26,7 @@ namespace tg {
 
 namespace cg = cooperative_groups;
 
-constexpr int kSelCluster = 8;
+constexpr int kSelCluster = 16;  // 16 needs the non-portable cluster size (the host falls back to 8)
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr size_t kSelCacheBytes = 200 * 1024;  // dynamic smem for the key cache
@@ -264,7 +264,10 @@ namespace tg {
 constexpr int kSelSmallThreads = 1024;
 constexpr int kSelSmallWarps = kSelSmallThreads / 32;
 constexpr int kSelSmallKpt = 32;
-constexpr int kSelSmallMax = kSelSmallThreads * kSelSmallKpt;  // 32768 tokens
+constexpr int kSelSmallMax = kSelSmallThreads * kSelSmallKpt;  // 32768 tokens the CTA can hold
+// above this many tokens a cluster is faster than one CTA (measured on B200:
+// 16K tokens 19 us in one CTA, 22 us in a cluster; 32K 33 us vs 23 us)
+constexpr int kSelSmallBest = 16384;
 constexpr int kSelSmallStride = kSelSmallThreads + 1;
 
 __device__ __forceinline__ uint32_t block_exclusive_scan_1024(uint32_t v, uint32_t* warp_sums, uint32_t* total) {

@@ -254,6 +254,39 @@ int launch_rmsnorm(const void* x, void* y, const float* w, int64_t m, int d, flo
   return launch_pdl("k_rmsnorm", tg::k_rmsnorm<T>, dim3(unsigned(m)), dim3(256), 0, st, xa, ya, w, d, eps);
 }
 
+// Whether a 16-CTA cluster of the selector can be resident on this device
+// (a non-portable cluster size): checked once per device.
+bool select_cluster16_ok() {
+  static std::mutex mu;
+  static std::map<int, bool> ok;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = ok.find(dev);
+  if (it != ok.end()) return it->second;
+  bool good = cudaFuncSetAttribute(tg::k_topk_select, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+  if (good) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16);
+    cfg.blockDim = dim3(tg::kSelThreads);
+    cfg.dynamicSmemBytes = tg::kSelCacheBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 16;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    good = cudaFuncSetAttribute(tg::k_topk_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(tg::kSelCacheBytes)) == cudaSuccess &&
+           cudaOccupancyMaxActiveClusters(&clusters, tg::k_topk_select, &cfg) == cudaSuccess && clusters >= 1;
+  }
+  cudaGetLastError();  // a refused query leaves no sticky error behind
+  ok[dev] = good;
+  return good;
+}
+
 extern "C" {
 
 const char* tg_version(void) { return TG_VERSION; }
@@ -501,7 +534,7 @@ int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int6
   p.k = k;
   p.out = kept_idx;
   p.m = m;
-  if (n <= tg::kSelSmallMax) {
+  if (n <= tg::kSelSmallBest) {
     // short prompt: one CTA, keys resident in shared memory
     const int need = static_cast<int>((n + tg::kSelSmallThreads - 1) / tg::kSelSmallThreads);
     const int kpt = need <= 4 ? 4 : (need <= 8 ? 8 : (need <= 16 ? 16 : 32));
@@ -528,11 +561,12 @@ int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int6
                           st, p, vec);
     }
   }
-  // cluster of 2, 4 or 8 CTAs: about 4096 tokens per CTA, and slices that fit the key cache
+  // cluster of 2 .. 16 CTAs: about 4096 tokens per CTA, and slices that fit the key cache
   int csize = 1;
   while (csize < tg::kSelCluster &&
          ((n + csize - 1) / csize > 4096 || static_cast<size_t>((n + csize - 1) / csize) * 5 > tg::kSelCacheBytes))
     csize *= 2;
+  if (csize > 8 && !select_cluster16_ok()) csize = 8;
   p.slice = (n + csize - 1) / csize;
   const size_t cache = static_cast<size_t>(p.slice) * 5;
   p.cached = cache <= tg::kSelCacheBytes ? 1 : 0;
