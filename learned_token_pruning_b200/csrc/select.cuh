@@ -265,9 +265,11 @@ constexpr int kSelSmallThreads = 1024;
 constexpr int kSelSmallWarps = kSelSmallThreads / 32;
 constexpr int kSelSmallKpt = 32;
 constexpr int kSelSmallMax = kSelSmallThreads * kSelSmallKpt;  // 32768 tokens the CTA can hold
-// above this many tokens a cluster is faster than one CTA (measured on B200:
-// 16K tokens 19 us in one CTA, 22 us in a cluster; 32K 33 us vs 23 us)
-constexpr int kSelSmallBest = 16384;
+// above this many tokens a cluster of 2048-token slices is faster than one
+// CTA (measured on B200: 16K tokens 19.3 us in one CTA, 17.0 us in 8 CTAs;
+// 32K 32.7 us vs 21.4 us in 16 CTAs)
+constexpr int kSelSmallBest = 4096;
+constexpr int kSelSlice = 2048;  // tokens per cluster CTA, until the cluster is at its largest
 constexpr int kSelSmallStride = kSelSmallThreads + 1;
 
 __device__ __forceinline__ uint32_t block_exclusive_scan_1024(uint32_t v, uint32_t* warp_sums, uint32_t* total) {

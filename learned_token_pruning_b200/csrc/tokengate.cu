@@ -561,10 +561,10 @@ int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int6
                           st, p, vec);
     }
   }
-  // cluster of 2 .. 16 CTAs: about 4096 tokens per CTA, and slices that fit the key cache
+  // cluster of 2 .. 16 CTAs: about kSelSlice tokens per CTA, and slices that fit the key cache
   int csize = 1;
-  while (csize < tg::kSelCluster &&
-         ((n + csize - 1) / csize > 4096 || static_cast<size_t>((n + csize - 1) / csize) * 5 > tg::kSelCacheBytes))
+  while (csize < tg::kSelCluster && ((n + csize - 1) / csize > tg::kSelSlice ||
+                                     static_cast<size_t>((n + csize - 1) / csize) * 5 > tg::kSelCacheBytes))
     csize *= 2;
   if (csize > 8 && !select_cluster16_ok()) csize = 8;
   p.slice = (n + csize - 1) / csize;
