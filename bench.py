@@ -20,7 +20,6 @@ import types
 import math
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -32,8 +31,37 @@ sys.path.insert(0, ROOT)
 METRIC = "gated-prefill tokens/s & TTFT ms at N=16K/128K; attention % bf16 peak"
 L2_FLUSH_BYTES = 256 << 20   # > the 126 MB L2
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch, from
+# an ncu capture of `bench.py --ncu-case` (profiles/ncu_full_gate_attention_swiglu_case.md),
+# with the rows that launch processed; scaled to the bench launch by rows.  A
+# record counts only while the SHA-256 of its kernel's sources still matches.
+MEASURED_TRAFFIC = {
+    "linear_gate_up_swiglu": {"bytes": 58862848 + 3024384, "rows": 2064, "sources": ("gemm_tc.cuh", "common.cuh"),
+                              "sha256": "30597d58bc87e803a17aa4f3aafe185f103b91d9c32f257062d507c5fbf53fd0"},
+    "gate_score": {"bytes": 269860096 + 3871232, "rows": 65536, "sources": ("gate_tc.cuh", "common.cuh"),
+                   "sha256": "e0855bc49169ea56c20f12efe9c1845c361cc53fb21c8bedcfa0994059881ec7"},
+    "attention": {"bytes": 16978176 + 676864, "rows": 2064, "sources": ("attn_tc.cuh", "common.cuh"),
+                  "sha256": "d89003aeada09144f9708ccc711a002ff23b2dbd2110d483a110ca39022b99f3"},
+}
+
 
 # ----------------------------------------------------------------------------- helpers (host only)
+
+def measured_traffic(kernel: str, rows: int):
+    """Per-launch DRAM traffic of `kernel` at `rows` rows, or None when no
+    capture exists or its sources changed since the capture."""
+    import hashlib
+    rec = MEASURED_TRAFFIC.get(kernel)
+    if rec is None:
+        return None
+    h = hashlib.sha256()
+    for f in rec["sources"]:
+        with open(os.path.join(ROOT, "learned_token_pruning_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != rec["sha256"]:
+        return None
+    return rec["bytes"] * rows / rec["rows"]
+
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -62,48 +90,67 @@ def workload_work(w, m):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples while the timed region runs."""
+    """SM clock and clock-event (throttle) reasons sampled through NVML every
+    couple of milliseconds from a host thread while the timed region runs (the
+    step is short, so nvidia-smi's 200 ms polling would see none of it)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __init__(self, gpu_id: str):
-        self.proc = None
+    def __init__(self, device_uuid: str, fallback_index: int, period_s: float = 0.002):
+        import threading
+        self.samples, self.reasons, self.max_mhz, self.error = [], set(), None, None
+        self._stop = threading.Event()
+        self._thread = None
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200", "-i", gpu_id], stdout=subprocess.PIPE,
-                                         stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            try:
+                self.h = nv.nvmlDeviceGetHandleByUUID(device_uuid)
+            except nv.NVMLError:
+                self.h = nv.nvmlDeviceGetHandleByIndex(fallback_index)
+            self.nv = nv
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        except Exception as e:             # no NVML: the line says so instead of a clock record
+            self.error = f"{type(e).__name__}: {e}"
+            return
+        self.period = period_s
+        self._thread = threading.Thread(target=self._run, daemon=True)
+
+    def start(self):
+        if self._thread is not None:
+            self._thread.start()
+
+    def sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        for name, const in self.REASONS:
+            if bits & getattr(nv, const, 0):
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.sample()
+            except Exception as e:
+                self.error = f"{type(e).__name__}: {e}"
+                return
+            self._stop.wait(self.period)
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for nm, val in zip(names, f[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if self._thread is None:
+            return {"error": self.error} if self.error else None
+        self._stop.set()
+        self._thread.join(timeout=5)
+        if not self.samples:
+            return {"error": self.error or "no sample"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_min_mhz": min(self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "source": "nvml"}
 
 
 def dist_setup():
@@ -249,13 +296,17 @@ def run_gpu(args, w):
     tg.tg_check_device_error()
 
     visible = os.environ.get("CUDA_VISIBLE_DEVICES")
-    gpu_id = visible.split(",")[dev.index].strip() if visible else str(dev.index)
-    sampler = ClockSampler(gpu_id) if rank == 0 else None
+    gpu_index = int(visible.split(",")[dev.index]) if visible and visible.split(",")[dev.index].strip().isdigit() \
+        else dev.index
+    uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", ""))
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}", gpu_index) if rank == 0 else None
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier(dist, dev)
     torch.cuda.synchronize(dev)
     t_wall = time.perf_counter()
+    if sampler:
+        sampler.start()
     for i in range(args.steps):
         flush.zero_()
         starts[i].record(stream)
@@ -279,6 +330,9 @@ def run_gpu(args, w):
     for name, ms in br.items():
         wk = work.get(name, {})
         entry = {"us": ms * 1e3}
+        if ms <= 0:             # serialised replays (under a profiler) can leave no difference to time
+            kernels[name] = entry
+            continue
         if "flops" in wk and name != "gate_score":
             tf = wk["flops"] / (ms * 1e-3) / 1e12
             entry.update({"tflops": tf, "frac_bf16_peak": tf / peaks["bf16_tflops"]})
@@ -288,15 +342,16 @@ def run_gpu(args, w):
         if name == "gate_score":
             entry["tflops"] = wk["flops"] / (ms * 1e-3) / 1e12
         kernels[name] = entry
-    dom = max((k for k in kernels if k != "layer_total"), key=lambda k: kernels[k]["us"])
+    dom = max((k for k in kernels if k != "layer_total" and kernels[k]["us"] > 0), key=lambda k: kernels[k]["us"])
     wk = work[dom]
+    traffic = measured_traffic(dom, w.n if dom == "gate_score" else m)
     if "flops" in wk and dom != "gate_score":
         roof = {"kernel": dom, "bound": "tensor", "achieved": kernels[dom]["tflops"], "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": kernels[dom]["tflops"] / peaks["bf16_tflops"], "traffic": None,
+                "unit": "TFLOP/s", "frac": kernels[dom]["tflops"] / peaks["bf16_tflops"], "traffic": traffic, "traffic_unit": "bytes per launch (ncu DRAM read+write)",
                 "peak_source": peaks["source"] + " (burst bf16)"}
     else:
         roof = {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["gbs"], "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": kernels[dom]["gbs"] / peaks["hbm_gbs"], "traffic": None,
+                "unit": "GB/s", "frac": kernels[dom]["gbs"] / peaks["hbm_gbs"], "traffic": traffic, "traffic_unit": "bytes per launch (ncu DRAM read+write)",
                 "peak_source": peaks["source"]}
 
     # ---- end to end through the public API: pinned host inputs in, result back to the host
@@ -435,8 +490,9 @@ def end_to_end(step, w, args, stream, flush, dist, dev, world):
 
 
 def ncu_case():
-    """One launch each of the three heaviest kernels at the bench shapes, for
-    profiler captures (the gate score at N = 65536 so its input exceeds L2)."""
+    """One launch each of the path's kernels at the bench shapes, for profiler
+    captures (the gate score at N = 65536 so its input exceeds L2; select and
+    gather on the 16K-token prefix with K = 2048 and 16 question tokens)."""
     import torch
     from learned_token_pruning_b200 import tokengate as tg
     torch.manual_seed(0)
@@ -450,6 +506,15 @@ def ncu_case():
     sc, sq = torch.empty(n, device=dev), torch.empty(1, device=dev)
     ws = torch.empty(tg.tg_workspace_bytes(tg.TG_OP_GATE_SCORE, n=n, d_model=d, h=h), dtype=torch.uint8, device=dev)
     tg.tg_gate_score(hid, None, 1e-6, w1, torch.zeros(h, device=dev), w2, 0.0, mask, sc, sq, ws)
+    n16, nq, k = 16384, 16, 2048
+    mask16 = torch.ones(n16, dtype=torch.uint8, device=dev)
+    mask16[-nq:] = 0
+    kept = torch.empty(k + nq, dtype=torch.int32, device=dev)
+    tg.tg_topk_select(sc[:n16].contiguous(), mask16, n16 - nq, k, kept)
+    hk = torch.empty(k + nq, d, dtype=torch.bfloat16, device=dev)
+    tg.tg_gather(hid[:n16], kept, sc[:n16].contiguous(), sq, n16 - nq, 1e-6, hk,
+                 torch.empty(k + nq, dtype=torch.int32, device=dev), torch.empty(k + nq, device=dev),
+                 torch.empty(k + nq, device=dev))
     m, hq, hkv, D = 2064, 16, 8, 128
     qkv = torch.randn(m, (hq + 2 * hkv) * D, device=dev).to(torch.bfloat16)
     out = torch.empty(m, hq * D, dtype=torch.bfloat16, device=dev)
