@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <algorithm>
 #include <cstring>
 #include <functional>
@@ -192,9 +193,99 @@ int launch_gemm_tc(const void* A, int64_t lda, const void* B, int64_t b_rows, in
   return launch_pdl("k_gemm_tc", kern, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmem, st, ta, tb, p);
 }
 
+// TG_GEMM_SINGLE_SM=1 in the environment selects the single-SM tcgen05 GEMM
+// even where two-SM clusters fit (read at every launch, so a test can run
+// both kernels in one process).
+bool force_single_sm_gemm() {
+  const char* e = std::getenv("TG_GEMM_SINGLE_SM");
+  return e && e[0] == '1';
+}
+
+// Pair GEMM (two-SM clusters, 256 x 256 tiles): the number of clusters that
+// can be resident at once, queried once per (kernel, device); 0 if the pair
+// kernel cannot be launched here.
+constexpr int kGemmPairStages = 3;
+
+template <typename Kern>
+int pair_clusters(Kern kern, int threads, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kern), dev);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int clusters = 0;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) ==
+      cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) clusters = 0;
+  }
+  cudaGetLastError();  // a refused query leaves no sticky error behind
+  cache[key] = clusters;
+  return clusters;
+}
+
+template <int EPI>
+int launch_gemm_pair(const void* A, int64_t lda, const void* B, int64_t b_rows, int M, int K, int tiles_n,
+                     const tg::GemmParams& p0, cudaStream_t st, int clusters) {
+  using Cfg = tg::GemmPairCfg<kGemmPairStages>;
+  CUtensorMap ta, tb;
+  int rc = make_map(&ta, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(lda) * 2, 128);
+  if (rc) return rc;
+  rc = make_map(&tb, B, static_cast<uint64_t>(K), static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K) * 2, 128);
+  if (rc) return rc;
+  auto kern = tg::k_gemm_pair<kGemmPairStages, EPI>;
+  rc = set_smem(kern, Cfg::kSmem);
+  if (rc) return rc;
+  tg::GemmParams p = p0;
+  p.M = M;
+  p.K = K;
+  p.tiles_m = (M + 255) / 256;
+  p.tiles_n = tiles_n;
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int pairs = tiles < clusters ? tiles : clusters;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(Cfg::kThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+  if (e != cudaSuccess) return fail(TG_ERR_CUDA, "k_gemm_pair launch: %s", cudaGetErrorString(e));
+  return check_launch("k_gemm_pair");
+}
+
+// Tile choice: the pair kernel (256 x 256 per two SMs, epilogue overlapped)
+// wherever two-SM clusters can be resident; otherwise 256-row single-SM tiles
+// when they give every SM a tile, else 128-row tiles.
 template <int BN, int EPI>
 int launch_gemm_auto(const void* A, int64_t lda, const void* B, int64_t b_rows, int M, int K, int tiles_n,
                      const tg::GemmParams& p0, cudaStream_t st) {
+  static_assert(BN == 256, "the pair kernel's tile is 256 columns wide");
+  const int clusters = pair_clusters(tg::k_gemm_pair<kGemmPairStages, EPI>, tg::GemmPairCfg<kGemmPairStages>::kThreads,
+                                     tg::GemmPairCfg<kGemmPairStages>::kSmem);
+  if (clusters > 0 && !force_single_sm_gemm())
+    return launch_gemm_pair<EPI>(A, lda, B, b_rows, M, K, tiles_n, p0, st, clusters);
   const int64_t tiles256 = int64_t((M + 255) / 256) * tiles_n;
   if (tiles256 >= sm_count() - sm_count() / 16)
     return launch_gemm_tc<BN, EPI, 2>(A, lda, B, b_rows, M, K, tiles_n, p0, st);

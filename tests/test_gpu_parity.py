@@ -354,27 +354,57 @@ def test_attention_bf16_full_size_sampled_rows():
 
 # ============================================================================ linear / layer
 
-@pytest.mark.parametrize("shape", [(300, 512, 384), (333, 18432, 192), (600, 32768, 128)],
-                         ids=["128-row-tiles", "256-row-tiles-ragged", "256-row-tiles-several-per-cta"])
-@pytest.mark.parametrize("epilogue", [tg.TG_EPI_STORE, tg.TG_EPI_RESIDUAL, tg.TG_EPI_SWIGLU])
-def test_linear_bf16_tensor_cores(epilogue, shape):
-    # the wide shapes have enough column tiles for 256-row tiles (two 128 x 256
-    # accumulators per CTA, no double buffering); (600, 32768) gives each CTA
-    # several tiles, so the accumulators are handed back and reused
-    rng = np.random.default_rng(12)
-    m, n_out, k_in = shape
+def _linear_case(epilogue, m, n_out, k_in, seed):
+    rng = np.random.default_rng(seed)
     w_rows = 2 * n_out if epilogue == tg.TG_EPI_SWIGLU else n_out
     x = synth.round_to(rng.standard_normal((m, k_in)).astype(np.float32), "bf16")
     w = synth.round_to(rng.standard_normal((w_rows, k_in)).astype(np.float32) * 0.05, "bf16")
     y0 = synth.round_to(rng.standard_normal((m, n_out)).astype(np.float32), "bf16")
-    y = d(y0, torch.bfloat16)
-    tg.tg_linear(d(x, torch.bfloat16), d(w, torch.bfloat16), y, epilogue)
+    return x, w, y0
+
+
+def _linear_want(epilogue, x, w, y0, n_out):
     xw = x.astype(np.float64) @ w.astype(np.float64).T
     if epilogue == tg.TG_EPI_SWIGLU:
-        want = O.silu(xw[:, :n_out]) * xw[:, n_out:]
+        return O.silu(xw[:, :n_out]) * xw[:, n_out:]
+    return xw + (y0 if epilogue == tg.TG_EPI_RESIDUAL else 0.0)
+
+
+@pytest.mark.parametrize("kernel", ["pair", "single"])
+@pytest.mark.parametrize("shape", [(300, 512, 384), (257, 128, 200), (333, 18432, 192), (600, 32768, 128)],
+                         ids=["one-wave", "ragged-m-and-k", "ragged-m-wide", "several-tiles-per-cta"])
+@pytest.mark.parametrize("epilogue", [tg.TG_EPI_STORE, tg.TG_EPI_RESIDUAL, tg.TG_EPI_SWIGLU])
+def test_linear_bf16_tensor_cores(epilogue, shape, kernel, monkeypatch):
+    # "pair": two-SM clusters, 256 x 256 tiles, double-buffered accumulators;
+    # "single": the one-SM kernel (128- or 256-row tiles).  The wide shapes give
+    # each CTA or pair several tiles, so accumulators are handed back and reused;
+    # K = 200 ends in a partial 64-column k-step (zero-filled by the copy engine)
+    if kernel == "single":
+        monkeypatch.setenv("TG_GEMM_SINGLE_SM", "1")
     else:
-        want = xw + (y0 if epilogue == tg.TG_EPI_RESIDUAL else 0.0)
-    assert_close(host(y), want, 2e-2, 1e-2, "linear")
+        monkeypatch.delenv("TG_GEMM_SINGLE_SM", raising=False)
+    m, n_out, k_in = shape
+    x, w, y0 = _linear_case(epilogue, m, n_out, k_in, 12)
+    y = d(y0, torch.bfloat16)
+    tg.tg_linear(d(x, torch.bfloat16), d(w, torch.bfloat16), y, epilogue)
+    assert_close(host(y), _linear_want(epilogue, x, w, y0, n_out), 2e-2, 1e-2, "linear")
+
+
+@pytest.mark.parametrize("shape", [(2064, 6144, 2048, tg.TG_EPI_SWIGLU), (2064, 4096, 2048, tg.TG_EPI_STORE),
+                                   (2064, 2048, 2048, tg.TG_EPI_RESIDUAL), (2064, 2048, 6144, tg.TG_EPI_RESIDUAL)],
+                         ids=["gate-up-swiglu", "qkv", "o-proj", "down-proj"])
+def test_linear_bench_shapes_sampled_rows(shape, monkeypatch):
+    # the four projections of the 16K-token step (m = 2064 kept rows), in the
+    # launch configuration the step uses; the oracle product on sampled rows
+    monkeypatch.delenv("TG_GEMM_SINGLE_SM", raising=False)
+    m, n_out, k_in, epilogue = shape
+    x, w, y0 = _linear_case(epilogue, m, n_out, k_in, 21)
+    y = d(y0, torch.bfloat16)
+    tg.tg_linear(d(x, torch.bfloat16), d(w, torch.bfloat16), y, epilogue)
+    rows = [0, 1, 127, 128, 255, 256, 1000, 1791, 1792, 2047, 2048, 2063]
+    got = host(y)[rows]
+    assert_close(got, _linear_want(epilogue, x[rows], w, y0[rows], n_out), 2e-2, 1e-2, "linear")
+    assert np.all(np.isfinite(host(y)))
 
 
 def test_linear_fp32_cuda_cores_ragged():
