@@ -186,6 +186,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   __shared__ int s_last;
+  __shared__ int s_ready;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // longest work first (the last row block has the most causal work)
   const int pairs_per_kv = p.group / 2;
@@ -481,44 +482,72 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     bool own_first = true;  // merge as fma(O_second, s_second, O_first * s_first) whichever half merges
     bool write_out = ok;
     if (part_code != 0) {
-      // half of a split row block: publish the unnormalised O and (max, sum);
-      // the half that finishes second merges both and writes the output
+      // half of a split row block.  The slot's counter decides the roles: the
+      // half that gets there first (even count) publishes its unnormalised O
+      // and (max, sum), then adds 4 (ready); the second (odd count) waits for
+      // the ready value 6 = 1 + 1 + 4, merges both and writes the output, so
+      // only one fp32 partial makes the round trip through L2.
       const int slot = (t - p.ts) * per_tile + pair;
       const int half = part_code - 1;
-      float4* mine = p.part + ((static_cast<size_t>(slot) * 2 + half) * 2 + wg) * (D / 4) * 128;
-      if (ok) {
-        tc_fence_after();
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (threadIdx.x == 0) s_last = (atomicAdd(&p.counters[slot], 1u) & 1u) ? 1 : 0;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (!s_last) {
+        if (ok) {
+          float4* mine = p.part + ((static_cast<size_t>(slot) * 2 + half) * 2 + wg) * (D / 4) * 128;
+          tc_fence_after();
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_base + colO + c0, o);
-          tmem_ld_wait();
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_base + colO + c0, o);
+            tmem_ld_wait();
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            mine[(c0 / 4 + v) * 128 + row] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                                         __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+            for (int v = 0; v < 8; ++v)
+              mine[(c0 / 4 + v) * 128 + row] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                                           __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+          }
+          p.part_ml[((static_cast<size_t>(slot) * 2 + half) * 2 + wg) * 128 + row] = make_float2(m_run, l_run);
         }
-        p.part_ml[((static_cast<size_t>(slot) * 2 + half) * 2 + wg) * 128 + row] = make_float2(m_run, l_run);
-      }
-      __threadfence();
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (threadIdx.x == 0) s_last = (!*abort_flag && atomicAdd(&p.counters[slot], 1u) == 1u) ? 1 : 0;
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      write_out = ok && s_last;
-      if (write_out) {
         __threadfence();
-        const size_t ob = (static_cast<size_t>(slot) * 2 + (1 - half)) * 2 + wg;
-        const float2 oml = __ldcg(&p.part_ml[ob * 128 + row]);
-        other = p.part + ob * (D / 4) * 128;
-        own_first = half == 0;
-        mm = fmaxf(m_run, oml.x);
-        s_me = ex2_approx(gg * (m_run - mm));
-        s_ot = ex2_approx(gg * (oml.x - mm));
-        // the same rounding whichever half merges: fma(l_second, s_second, l_first * s_first)
-        inv = 1.0f / (own_first ? fmaf(oml.y, s_ot, l_run * s_me) : fmaf(l_run, s_me, oml.y * s_ot));
-        s_me *= inv;
-        s_ot *= inv;
-        if (threadIdx.x == 0) p.counters[slot] = 0u;  // ready for the next launch
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (threadIdx.x == 0 && !*abort_flag) atomicAdd(&p.counters[slot], 4u);
+        write_out = false;
+      } else {
+        if (threadIdx.x == 0) {
+          // bounded wait for the first half's ready value (it is resident and
+          // past its own count, so it gets there without this CTA's help)
+          bool ready = false;
+          const uint64_t t0 = globaltimer_ns();
+          for (uint32_t i = 0;; ++i) {
+            if (ld_acquire_gpu(&p.counters[slot]) >= 6u) {
+              ready = true;
+              break;
+            }
+            if ((i & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) break;
+          }
+          if (!ready) {
+            raise_error(kErrWaitAttention, 2);
+            *abort_flag = 1;
+          }
+          s_ready = ready ? 1 : 0;
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        write_out = ok && s_ready;
+        if (write_out) {
+          __threadfence();
+          const size_t ob = (static_cast<size_t>(slot) * 2 + (1 - half)) * 2 + wg;
+          const float2 oml = __ldcg(&p.part_ml[ob * 128 + row]);
+          other = p.part + ob * (D / 4) * 128;
+          own_first = half == 0;
+          mm = fmaxf(m_run, oml.x);
+          s_me = ex2_approx(gg * (m_run - mm));
+          s_ot = ex2_approx(gg * (oml.x - mm));
+          // the same rounding whichever half merges: fma(l_second, s_second, l_first * s_first)
+          inv = 1.0f / (own_first ? fmaf(oml.y, s_ot, l_run * s_me) : fmaf(l_run, s_me, oml.y * s_ot));
+          s_me *= inv;
+          s_ot *= inv;
+          if (threadIdx.x == 0) p.counters[slot] = 0u;  // ready for the next launch
+        }
       }
     } else if (ok) {
       inv = 1.0f / l_run;
@@ -530,8 +559,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // 64b..64b+63, row r at 128 r, 16-byte chunk c at c ^ (r & 7)
       uint8_t* stage = sK + wg * (128 * D * 2);  // K/V stages are idle once o_final has completed
       tc_fence_after();
+      // the partner's partial is read one 32-column chunk ahead of its use
+      float4 wcur[8];
+      if (other) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) wcur[v] = __ldcg(&other[v * 128 + row]);
+      }
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
+        float4 wnext[8];
+        if (other && c0 + 32 < D) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) wnext[v] = __ldcg(&other[((c0 + 32) / 4 + v) * 128 + row]);
+        }
         uint32_t o[32];
         tmem_ld32(tmem + lane_base + colO + c0, o);
         tmem_ld_wait();
@@ -541,7 +581,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (other) {
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
-            const float4 w4 = __ldcg(&other[(c0 / 4 + v) * 128 + row]);
+            const float4 w4 = wcur[v];
             const float w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -549,6 +589,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               f[4 * v + u] = own_first ? fmaf(w[u], s_ot, own * s_me) : fmaf(own, s_me, w[u] * s_ot);
             }
           }
+#pragma unroll
+          for (int v = 0; v < 8; ++v) wcur[v] = wnext[v];
         }
         uint8_t* box = stage + (c0 / 64) * (128 * 128) + row * 128;
 #pragma unroll

@@ -129,6 +129,14 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32
   return __all_sync(0xffffffffu, ok);
 }
 
+// Global-memory flag read with acquire semantics at GPU scope (pairs with a
+// release -- here __threadfence() and an atomic -- by a thread of another CTA).
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // ---------------------------------------------------------------------------
 // TMA (tiled tensor copies, no multicast)
 // ---------------------------------------------------------------------------

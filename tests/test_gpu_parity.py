@@ -201,6 +201,8 @@ def _gpu_scores(w, g, pass_norm):
     (777, 512, 128, "bf16", 1e-3),         # 128-wide MLP, ragged last tile
     (4096 + 77, 2048, 256, "bf16", 1e-3),  # Qwen3-1.7B gate shape
     (300, 200, 48, "bf16", 1e-3),          # K tail (200 = 3*64 + 8) and h padded to 64
+    (300, 200, 200, "bf16", 1e-3),         # K tail and h padded to 256
+    (16384, 2048, 256, "bf16", 1e-3),      # the 16K-token step's gate: 128 CTAs, one wave
 ])
 def test_gate_score_matches_oracle(n, dm, h, dtype, tol):
     w, g = _gate_case(n, dm, h, dtype, seed=n)
