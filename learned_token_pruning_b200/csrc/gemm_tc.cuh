@@ -267,6 +267,27 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, MH>::kThreads, 1)
   }
 }
 
+// Epilogue output staging of one warp: its 32 rows x 64 bf16 columns in the
+// 128-byte-swizzled layout of a {64, 32} TMA box (row r at 128 r, 16-byte
+// chunk c at c ^ (r & 7), so the 32 lanes' row writes spread over the banks),
+// written out by one TMA store per 64 columns (rows and columns past the
+// tensor's extent are clipped by the copy engine).
+__device__ __forceinline__ void stage_wait_free(uint8_t* stage, int lane) {
+  if (lane == 0) bulk_wait_read<0>();  // the previous store has read the buffer
+  __syncwarp();
+}
+__device__ __forceinline__ void stage_put(uint8_t* stage, int lane, int chunk, uint4 v) {
+  *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = v;
+}
+__device__ __forceinline__ void stage_store(uint8_t* stage, int lane, const CUtensorMap* map, int col, int row) {
+  fence_proxy_async_smem();  // the generic-proxy writes above, before the copy engine reads them
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, stage, col, row);
+    bulk_commit();
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Pair GEMM: a cluster of two CTAs (two SMs) computes one 256 x 256 output
 // tile with the M = 256 pair form of tcgen05.mma.  Each CTA streams its own
@@ -297,12 +318,14 @@ struct GemmPairCfg {
   static constexpr int kTmemCols = kBufs * kAccCols;
   static constexpr int kEpiWarps = 8;
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
-  static constexpr size_t kSmem = 1024 + STAGES * (kABytes + kBBytes) + 256;
+  static constexpr int kEpiStage = 32 * 128;  // per epilogue warp: 32 rows x 64 bf16 columns, 128-byte swizzle
+  static constexpr size_t kSmem = 1024 + STAGES * (kABytes + kBBytes) + kEpiWarps * kEpiStage + 256;
 };
 
 template <int STAGES, int EPI>
 __global__ void __launch_bounds__(GemmPairCfg<STAGES>::kThreads, 1)
-    k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+    k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmO, GemmParams p) {
   using Cfg = GemmPairCfg<STAGES>;
   extern __shared__ uint8_t gemm_smem_raw[];
   // every CTA of the cluster gets the same dynamic shared-memory offset, so the
@@ -311,7 +334,8 @@ __global__ void __launch_bounds__(GemmPairCfg<STAGES>::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * Cfg::kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * Cfg::kBBytes);
+  uint8_t* sEpi = sB + STAGES * Cfg::kBBytes;  // output staging, one 4 KB buffer per epilogue warp
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + Cfg::kEpiWarps * Cfg::kEpiStage);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;  // [2]
   uint64_t* acc_empty = acc_full + 2;   // [2], used in the even CTA
@@ -469,6 +493,7 @@ __global__ void __launch_bounds__(GemmPairCfg<STAGES>::kThreads, 1)
     const int row = static_cast<int>(rank) * 128 + q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t acc_empty0 = map_to_rank(smem_u32(acc_empty), 0);
+    uint8_t* stage = sEpi + (warp - 2) * Cfg::kEpiStage;
     pdl_wait();  // the residual and the output may belong to the previous kernel
     int i = 0;
     for (int tile = pair; tile < tiles; tile += npairs, ++i) {
@@ -495,6 +520,7 @@ __global__ void __launch_bounds__(GemmPairCfg<STAGES>::kThreads, 1)
       }
       tc_fence_after();
       const uint32_t t_row = tmem + lane_base + b * Cfg::kAccCols;
+      const int srow0 = (tile % p.tiles_m) * 256 + static_cast<int>(rank) * 128 + q * 32;  // the warp's first row
       if (EPI == kEpiStore || EPI == kEpiResidual) {
 #pragma unroll
         for (int c2 = 0; c2 < 4; c2 += 2) {
@@ -502,66 +528,62 @@ __global__ void __launch_bounds__(GemmPairCfg<STAGES>::kThreads, 1)
           tmem_ld32(t_row + ch * 128 + 32 * c2, r[0]);
           tmem_ld32(t_row + ch * 128 + 32 * (c2 + 1), r[1]);
           tmem_ld_wait();
+          stage_wait_free(stage, lane);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int c = c2 + h;
-            if (grow < p.M && gcol0 + 32 * c < p.N) {
-              uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(grow) * p.ldo + gcol0 + 32 * c);
 #pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                float add[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-                if (EPI == kEpiResidual) {
-                  const uint32_t ow[4] = {old[4 * c + v].x, old[4 * c + v].y, old[4 * c + v].z, old[4 * c + v].w};
+            for (int v = 0; v < 4; ++v) {
+              float add[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+              if (EPI == kEpiResidual) {
+                const uint32_t ow[4] = {old[4 * c + v].x, old[4 * c + v].y, old[4 * c + v].z, old[4 * c + v].w};
 #pragma unroll
-                  for (int t = 0; t < 4; ++t) {
-                    add[2 * t] = bf16_lo(ow[t]);
-                    add[2 * t + 1] = bf16_hi(ow[t]);
-                  }
+                for (int t = 0; t < 4; ++t) {
+                  add[2 * t] = bf16_lo(ow[t]);
+                  add[2 * t + 1] = bf16_hi(ow[t]);
                 }
-                const uint32_t* rr = r[h];
-                uint4 o;
-                o.x = pack_bf16x2(__uint_as_float(rr[8 * v + 0]) + add[0], __uint_as_float(rr[8 * v + 1]) + add[1]);
-                o.y = pack_bf16x2(__uint_as_float(rr[8 * v + 2]) + add[2], __uint_as_float(rr[8 * v + 3]) + add[3]);
-                o.z = pack_bf16x2(__uint_as_float(rr[8 * v + 4]) + add[4], __uint_as_float(rr[8 * v + 5]) + add[5]);
-                o.w = pack_bf16x2(__uint_as_float(rr[8 * v + 6]) + add[6], __uint_as_float(rr[8 * v + 7]) + add[7]);
-                dst[v] = o;
               }
+              const uint32_t* rr = r[h];
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(rr[8 * v + 0]) + add[0], __uint_as_float(rr[8 * v + 1]) + add[1]);
+              o.y = pack_bf16x2(__uint_as_float(rr[8 * v + 2]) + add[2], __uint_as_float(rr[8 * v + 3]) + add[3]);
+              o.z = pack_bf16x2(__uint_as_float(rr[8 * v + 4]) + add[4], __uint_as_float(rr[8 * v + 5]) + add[5]);
+              o.w = pack_bf16x2(__uint_as_float(rr[8 * v + 6]) + add[6], __uint_as_float(rr[8 * v + 7]) + add[7]);
+              stage_put(stage, lane, 4 * h + v, o);
             }
           }
+          stage_store(stage, lane, &tmO, gcol0 + 32 * c2, srow0);
         }
       } else {
+        stage_wait_free(stage, lane);
 #pragma unroll 1
-        for (int c0 = ch * 64; c0 < ch * 64 + 64; c0 += 32) {
+        for (int h = 0; h < 2; ++h) {
+          const int c0 = ch * 64 + 32 * h;
           uint32_t g[32], u[32];
           tmem_ld32(t_row + c0, g);
           tmem_ld32(t_row + 128 + c0, u);
           tmem_ld_wait();
-          const int gcol = nb * 128 + c0;
-          if (grow < p.M && gcol < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(grow) * p.ldo + gcol);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              float a[8];
+          for (int v = 0; v < 4; ++v) {
+            float a[8];
 #pragma unroll
-              for (int t = 0; t < 8; ++t) {
-                const float gv = __uint_as_float(g[8 * v + t]);
-                a[t] = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(u[8 * v + t]);
-              }
-              uint4 o;
-              o.x = pack_bf16x2(a[0], a[1]);
-              o.y = pack_bf16x2(a[2], a[3]);
-              o.z = pack_bf16x2(a[4], a[5]);
-              o.w = pack_bf16x2(a[6], a[7]);
-              dst[v] = o;
+            for (int t = 0; t < 8; ++t) {
+              const float gv = __uint_as_float(g[8 * v + t]);
+              a[t] = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(u[8 * v + t]);
             }
+            stage_put(stage, lane, 4 * h + v,
+                      make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                                 pack_bf16x2(a[6], a[7])));
           }
         }
+        stage_store(stage, lane, &tmO, nb * 128 + ch * 64, srow0);
       }
       // this warp's part of accumulator b is drained: release it to the even CTA's MMA thread
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8 * b);
     }
+    if (lane == 0) bulk_wait_all();  // the output stores are complete before the CTA goes away
   }
   tc_fence_before();
   cluster_sync_all();  // neither CTA leaves while the pair still uses its memory

@@ -246,6 +246,10 @@ int launch_gemm_pair(const void* A, int64_t lda, const void* B, int64_t b_rows, 
   if (rc) return rc;
   rc = make_map(&tb, B, static_cast<uint64_t>(K), static_cast<uint64_t>(b_rows), static_cast<uint64_t>(K) * 2, 128);
   if (rc) return rc;
+  // the epilogue writes through TMA: boxes of 32 rows x 64 columns
+  CUtensorMap to;
+  rc = make_map(&to, p0.out, static_cast<uint64_t>(p0.N), static_cast<uint64_t>(M), static_cast<uint64_t>(p0.ldo) * 2, 32);
+  if (rc) return rc;
   auto kern = tg::k_gemm_pair<kGemmPairStages, EPI>;
   rc = set_smem(kern, Cfg::kSmem);
   if (rc) return rc;
@@ -270,7 +274,7 @@ int launch_gemm_pair(const void* A, int64_t lda, const void* B, int64_t b_rows, 
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, to, p);
   if (e != cudaSuccess) return fail(TG_ERR_CUDA, "k_gemm_pair launch: %s", cudaGetErrorString(e));
   return check_launch("k_gemm_pair");
 }
