@@ -458,35 +458,78 @@ def breakdown(step, w, args, stream, flush):
 
 def end_to_end(step, w, args, stream, flush, dist, dev, world):
     """Same metric through the public API with the inputs in pinned host memory:
-    every step copies the hidden states and the prunable mask in, runs the
-    four calls and copies the kept-row output back."""
+    every step copies its hidden states and prunable mask in, runs the four
+    calls and copies the kept-row output back, all inside the timed region.
+    Steps are pipelined the way a server would run consecutive requests: the
+    upload of step i+1 (its own stream, into the other of two device staging
+    buffers) overlaps the compute of step i, and the readback of step i (a
+    third stream, from the other of two output buffers) overlaps step i+1."""
     import torch
     h_host = step.hidden.cpu().pin_memory()
     m_host = step.prunable.cpu().pin_memory()
-    out_host = torch.empty(step.hidden_kept.shape, dtype=step.hidden_kept.dtype).pin_memory()
+    out_host = [torch.empty(step.hidden_kept.shape, dtype=step.hidden_kept.dtype).pin_memory() for _ in range(2)]
+    stage_h = [torch.empty_like(step.hidden) for _ in range(2)]
+    stage_m = [torch.empty_like(step.prunable) for _ in range(2)]
+    stage_o = [torch.empty_like(step.hidden_kept) for _ in range(2)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    copied, used, computed, read = ([ev() for _ in range(2)] for _ in range(4))
     steps = max(3, min(args.steps, 30))
 
-    def one():
-        step.hidden.copy_(h_host, non_blocking=True)
-        step.prunable.copy_(m_host, non_blocking=True)
-        step.replay()
-        out_host.copy_(step.hidden_kept, non_blocking=True)
+    def upload(i):
+        j = i % 2
+        if i >= 2:
+            up.wait_event(used[j])          # step i-2 has taken its inputs out of staging buffer j
+        with torch.cuda.stream(up):
+            stage_h[j].copy_(h_host, non_blocking=True)
+            stage_m[j].copy_(m_host, non_blocking=True)
+            copied[j].record(up)
 
-    for _ in range(2):
-        one()
+    def compute(i):
+        j = i % 2
+        stream.wait_event(copied[j])
+        step.hidden.copy_(stage_h[j], non_blocking=True)
+        step.prunable.copy_(stage_m[j], non_blocking=True)
+        used[j].record(stream)
+        step.replay()
+        if i >= 2:
+            stream.wait_event(read[j])      # the readback of step i-2 is out of output buffer j
+        stage_o[j].copy_(step.hidden_kept, non_blocking=True)
+        computed[j].record(stream)
+
+    def readback(i):
+        j = i % 2
+        down.wait_event(computed[j])
+        with torch.cuda.stream(down):
+            out_host[j].copy_(stage_o[j], non_blocking=True)
+            read[j].record(down)
+
+    def run(n):
+        upload(0)
+        for i in range(n):
+            if i + 1 < n:
+                upload(i + 1)
+            compute(i)
+            readback(i)
+        stream.wait_event(read[(n - 1) % 2])
+
+    run(3)
     torch.cuda.synchronize()
     barrier(dist, dev)
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(steps):
-        one()
+    up.wait_event(a)
+    run(steps)
     b.record(stream)
     torch.cuda.synchronize()
     sec = max_over_ranks(a.elapsed_time(b) / 1e3, dist, dev)
+    out_ok = torch.equal(out_host[(steps - 1) % 2], step.hidden_kept.cpu())
     return {"value": replica_value(world, w.n, steps, sec), "unit": "tokens/s",
             "h2d_bytes_per_step": h_host.numel() * h_host.element_size() + m_host.numel(),
-            "d2h_bytes_per_step": out_host.numel() * out_host.element_size(), "steps": steps}
+            "d2h_bytes_per_step": out_host[0].numel() * out_host[0].element_size(), "steps": steps,
+            "pipelined": "upload of step i+1 and readback of step i-1 overlap the compute of step i",
+            "readback_matches_device": bool(out_ok)}
 
 
 def ncu_case():
