@@ -36,12 +36,12 @@ L2_FLUSH_BYTES = 256 << 20   # > the 126 MB L2
 # with the rows that launch processed; scaled to the bench launch by rows.  A
 # record counts only while the SHA-256 of its kernel's sources still matches.
 MEASURED_TRAFFIC = {
-    "linear_gate_up_swiglu": {"bytes": 58862848 + 3024384, "rows": 2064, "sources": ("gemm_tc.cuh", "common.cuh"),
-                              "sha256": "30597d58bc87e803a17aa4f3aafe185f103b91d9c32f257062d507c5fbf53fd0"},
-    "gate_score": {"bytes": 269860096 + 3871232, "rows": 65536, "sources": ("gate_tc.cuh", "common.cuh"),
-                   "sha256": "e0855bc49169ea56c20f12efe9c1845c361cc53fb21c8bedcfa0994059881ec7"},
-    "attention": {"bytes": 16978176 + 676864, "rows": 2064, "sources": ("attn_tc.cuh", "common.cuh"),
-                  "sha256": "d89003aeada09144f9708ccc711a002ff23b2dbd2110d483a110ca39022b99f3"},
+    "linear_gate_up_swiglu": {"bytes": 58852352 + 7237120, "rows": 2064, "sources": ("gemm_tc.cuh", "common.cuh"),
+                              "sha256": "8d1b356a43a10dd74230fca02bba39aef170ea447c87b34d34d4ade57fcc10bb"},
+    "gate_score": {"bytes": 269859328 + 5020160, "rows": 65536, "sources": ("gate_tc.cuh", "common.cuh"),
+                   "sha256": "182595c9d81cb684ae20b148a60c168d96dd5af5e795460977a043d60dfe59c2"},
+    "attention": {"bytes": 16979200 + 22016, "rows": 2064, "sources": ("attn_tc.cuh", "common.cuh"),
+                  "sha256": "21ae350b717df6dfc56a267bb6fa0b545ef7dec309bd2ae1d29d96743d7d6616"},
 }
 
 
