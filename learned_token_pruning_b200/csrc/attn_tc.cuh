@@ -160,6 +160,155 @@ __device__ __forceinline__ bool mbar_wait2(uint64_t* b0, uint32_t p0, uint64_t* 
   return mbar_wait(b0, p0, site) && mbar_wait(b1, p1, site);
 }
 
+// Epilogue of one softmax warpgroup (128 rows of one query head, O in tensor
+// memory at column colO, complete once o_final has been observed): normalise
+// and store the output tile through shared memory and TMA; for half of a split
+// row block, publish or merge the partial results first (see below).  Shared
+// by the attention kernels; `slot` is the split block's slot in p.part.
+template <int D>
+__device__ __forceinline__ void attn_epilogue(const AttnTcParams& p, const CUtensorMap* tmO, uint8_t* stage_base,
+                                              uint32_t tmem, uint32_t lane_base, uint32_t colO, int wg, int row,
+                                              int grow, int h, int t, int part_code, int slot, bool ok, float m_run,
+                                              float l_run, float gg, volatile uint32_t* abort_flag, int* s_last,
+                                              int* s_ready) {
+  constexpr int kDBoxes = D / 64;
+  const int sw = row & 7;  // 16-byte chunk c of a 128-byte swizzled row sits at c ^ (row & 7)
+  float mm = m_run, inv = 0.0f, s_me = 1.0f, s_ot = 0.0f;
+  const float4* other = nullptr;
+  bool own_first = true;  // merge as fma(O_second, s_second, O_first * s_first) whichever half merges
+  bool write_out = ok;
+  if (part_code != 0) {
+    // half of a split row block.  The slot's counter decides the roles: the
+    // half that gets there first (even count) publishes its unnormalised O
+    // and (max, sum), then adds 4 (ready); the second (odd count) waits for
+    // the ready value 6 = 1 + 1 + 4, merges both and writes the output, so
+    // only one fp32 partial makes the round trip through L2.
+    const int half = part_code - 1;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (threadIdx.x == 0) *s_last = (atomicAdd(&p.counters[slot], 1u) & 1u) ? 1 : 0;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (!*s_last) {
+      if (ok) {
+        float4* mine = p.part + ((static_cast<size_t>(slot) * 2 + half) * 2 + wg) * (D / 4) * 128;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + colO + c0, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            mine[(c0 / 4 + v) * 128 + row] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                                         __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+        }
+        p.part_ml[((static_cast<size_t>(slot) * 2 + half) * 2 + wg) * 128 + row] = make_float2(m_run, l_run);
+      }
+      __threadfence();
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (threadIdx.x == 0 && !*abort_flag) atomicAdd(&p.counters[slot], 4u);
+      write_out = false;
+    } else {
+      if (threadIdx.x == 0) {
+        // bounded wait for the first half's ready value (it is resident and
+        // past its own count, so it gets there without this CTA's help)
+        bool ready = false;
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t i = 0;; ++i) {
+          if (ld_acquire_gpu(&p.counters[slot]) >= 6u) {
+            ready = true;
+            break;
+          }
+          if ((i & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) break;
+        }
+        if (!ready) {
+          raise_error(kErrWaitAttention, 2);
+          *abort_flag = 1;
+        }
+        *s_ready = ready ? 1 : 0;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      write_out = ok && *s_ready;
+      if (write_out) {
+        __threadfence();
+        const size_t ob = (static_cast<size_t>(slot) * 2 + (1 - half)) * 2 + wg;
+        const float2 oml = __ldcg(&p.part_ml[ob * 128 + row]);
+        other = p.part + ob * (D / 4) * 128;
+        own_first = half == 0;
+        mm = fmaxf(m_run, oml.x);
+        s_me = ex2_approx(gg * (m_run - mm));
+        s_ot = ex2_approx(gg * (oml.x - mm));
+        // the same rounding whichever half merges: fma(l_second, s_second, l_first * s_first)
+        inv = 1.0f / (own_first ? fmaf(oml.y, s_ot, l_run * s_me) : fmaf(l_run, s_me, oml.y * s_ot));
+        s_me *= inv;
+        s_ot *= inv;
+        if (threadIdx.x == 0) p.counters[slot] = 0u;  // ready for the next launch
+      }
+    }
+  } else if (ok) {
+    inv = 1.0f / l_run;
+    s_me = inv;
+  }
+  if (write_out) {
+    // O as bf16 into the K/V stages, in the
+    // 128-byte-swizzled layout of the output tensor map: box b holds columns
+    // 64b..64b+63, row r at 128 r, 16-byte chunk c at c ^ (r & 7)
+    uint8_t* stage = stage_base + wg * (128 * D * 2);  // idle once o_final has completed
+    tc_fence_after();
+    // the partner's partial is read one 32-column chunk ahead of its use
+    float4 wcur[8];
+    if (other) {
+#pragma unroll
+      for (int v = 0; v < 8; ++v) wcur[v] = __ldcg(&other[v * 128 + row]);
+    }
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      float4 wnext[8];
+      if (other && c0 + 32 < D) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) wnext[v] = __ldcg(&other[((c0 + 32) / 4 + v) * 128 + row]);
+      }
+      uint32_t o[32];
+      tmem_ld32(tmem + lane_base + colO + c0, o);
+      tmem_ld_wait();
+      float f[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(o[e]) * s_me;
+      if (other) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 w4 = wcur[v];
+          const float w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float own = __uint_as_float(o[4 * v + u]);
+            f[4 * v + u] = own_first ? fmaf(w[u], s_ot, own * s_me) : fmaf(own, s_me, w[u] * s_ot);
+          }
+        }
+#pragma unroll
+        for (int v = 0; v < 8; ++v) wcur[v] = wnext[v];
+      }
+      uint8_t* box = stage + (c0 / 64) * (128 * 128) + row * 128;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int chunk = (c0 % 64) / 8 + v;
+        *reinterpret_cast<uint4*>(box + ((chunk ^ sw) << 4)) =
+            make_uint4(pack_bf16x2(f[8 * v], f[8 * v + 1]), pack_bf16x2(f[8 * v + 2], f[8 * v + 3]),
+                       pack_bf16x2(f[8 * v + 4], f[8 * v + 5]), pack_bf16x2(f[8 * v + 6], f[8 * v + 7]));
+      }
+    }
+    // the warpgroup's tile is staged: one thread stores it (rows past m are clipped)
+    fence_proxy_async_smem();
+    if (wg == 0) asm volatile("bar.sync 2, 128;" ::: "memory");
+    else asm volatile("bar.sync 3, 128;" ::: "memory");
+    if (row == 0) {
+      for (int b = 0; b < kDBoxes; ++b) tma_store_2d(tmO, stage + b * (128 * 128), h * D + 64 * b, t * 128);
+      bulk_commit();
+      bulk_wait_all();  // written out before the CTA (and its shared memory) goes away
+    }
+    if (p.lse && grow < p.m) p.lse[static_cast<int64_t>(h) * p.m + grow] = (gg * mm - log2f(inv)) * kLn2;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -360,7 +509,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint64_t ay2 = f2_pack(a_y, a_y), gg2 = f2_pack(gg, gg);
     float m_run = -INFINITY, l_run = 0.0f;  // running max of y, running sum of exp2(g * (y - m_run))
     bool ok = true;
-    const int sw = row & 7;  // 16-byte chunk c of a 128-byte swizzled row sits at c ^ (row & 7)
 
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1;
@@ -477,141 +625,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (ok && !*abort_flag) ok = warp_wait(o_final, 0, kErrWaitAttention);
     // every softmax thread ends here, so the named barriers below see all 256
     if (!ok) *abort_flag = 1;
-    float mm = m_run, inv = 0.0f, s_me = 1.0f, s_ot = 0.0f;
-    const float4* other = nullptr;
-    bool own_first = true;  // merge as fma(O_second, s_second, O_first * s_first) whichever half merges
-    bool write_out = ok;
-    if (part_code != 0) {
-      // half of a split row block.  The slot's counter decides the roles: the
-      // half that gets there first (even count) publishes its unnormalised O
-      // and (max, sum), then adds 4 (ready); the second (odd count) waits for
-      // the ready value 6 = 1 + 1 + 4, merges both and writes the output, so
-      // only one fp32 partial makes the round trip through L2.
-      const int slot = (t - p.ts) * per_tile + pair;
-      const int half = part_code - 1;
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (threadIdx.x == 0) s_last = (atomicAdd(&p.counters[slot], 1u) & 1u) ? 1 : 0;
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (!s_last) {
-        if (ok) {
-          float4* mine = p.part + ((static_cast<size_t>(slot) * 2 + half) * 2 + wg) * (D / 4) * 128;
-          tc_fence_after();
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_base + colO + c0, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              mine[(c0 / 4 + v) * 128 + row] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                                           __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
-          }
-          p.part_ml[((static_cast<size_t>(slot) * 2 + half) * 2 + wg) * 128 + row] = make_float2(m_run, l_run);
-        }
-        __threadfence();
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (threadIdx.x == 0 && !*abort_flag) atomicAdd(&p.counters[slot], 4u);
-        write_out = false;
-      } else {
-        if (threadIdx.x == 0) {
-          // bounded wait for the first half's ready value (it is resident and
-          // past its own count, so it gets there without this CTA's help)
-          bool ready = false;
-          const uint64_t t0 = globaltimer_ns();
-          for (uint32_t i = 0;; ++i) {
-            if (ld_acquire_gpu(&p.counters[slot]) >= 6u) {
-              ready = true;
-              break;
-            }
-            if ((i & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) break;
-          }
-          if (!ready) {
-            raise_error(kErrWaitAttention, 2);
-            *abort_flag = 1;
-          }
-          s_ready = ready ? 1 : 0;
-        }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        write_out = ok && s_ready;
-        if (write_out) {
-          __threadfence();
-          const size_t ob = (static_cast<size_t>(slot) * 2 + (1 - half)) * 2 + wg;
-          const float2 oml = __ldcg(&p.part_ml[ob * 128 + row]);
-          other = p.part + ob * (D / 4) * 128;
-          own_first = half == 0;
-          mm = fmaxf(m_run, oml.x);
-          s_me = ex2_approx(gg * (m_run - mm));
-          s_ot = ex2_approx(gg * (oml.x - mm));
-          // the same rounding whichever half merges: fma(l_second, s_second, l_first * s_first)
-          inv = 1.0f / (own_first ? fmaf(oml.y, s_ot, l_run * s_me) : fmaf(l_run, s_me, oml.y * s_ot));
-          s_me *= inv;
-          s_ot *= inv;
-          if (threadIdx.x == 0) p.counters[slot] = 0u;  // ready for the next launch
-        }
-      }
-    } else if (ok) {
-      inv = 1.0f / l_run;
-      s_me = inv;
-    }
-    if (write_out) {
-      // O as bf16 into the K/V stages, in the
-      // 128-byte-swizzled layout of the output tensor map: box b holds columns
-      // 64b..64b+63, row r at 128 r, 16-byte chunk c at c ^ (r & 7)
-      uint8_t* stage = sK + wg * (128 * D * 2);  // K/V stages are idle once o_final has completed
-      tc_fence_after();
-      // the partner's partial is read one 32-column chunk ahead of its use
-      float4 wcur[8];
-      if (other) {
-#pragma unroll
-        for (int v = 0; v < 8; ++v) wcur[v] = __ldcg(&other[v * 128 + row]);
-      }
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        float4 wnext[8];
-        if (other && c0 + 32 < D) {
-#pragma unroll
-          for (int v = 0; v < 8; ++v) wnext[v] = __ldcg(&other[((c0 + 32) / 4 + v) * 128 + row]);
-        }
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_base + colO + c0, o);
-        tmem_ld_wait();
-        float f[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(o[e]) * s_me;
-        if (other) {
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const float4 w4 = wcur[v];
-            const float w[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float own = __uint_as_float(o[4 * v + u]);
-              f[4 * v + u] = own_first ? fmaf(w[u], s_ot, own * s_me) : fmaf(own, s_me, w[u] * s_ot);
-            }
-          }
-#pragma unroll
-          for (int v = 0; v < 8; ++v) wcur[v] = wnext[v];
-        }
-        uint8_t* box = stage + (c0 / 64) * (128 * 128) + row * 128;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int chunk = (c0 % 64) / 8 + v;
-          *reinterpret_cast<uint4*>(box + ((chunk ^ sw) << 4)) =
-              make_uint4(pack_bf16x2(f[8 * v], f[8 * v + 1]), pack_bf16x2(f[8 * v + 2], f[8 * v + 3]),
-                         pack_bf16x2(f[8 * v + 4], f[8 * v + 5]), pack_bf16x2(f[8 * v + 6], f[8 * v + 7]));
-        }
-      }
-      // the warpgroup's tile is staged: one thread stores it (rows past m are clipped)
-      fence_proxy_async_smem();
-      if (wg == 0) asm volatile("bar.sync 2, 128;" ::: "memory");
-      else asm volatile("bar.sync 3, 128;" ::: "memory");
-      if (row == 0) {
-        for (int b = 0; b < kDBoxes; ++b) tma_store_2d(&tmO, stage + b * (128 * 128), h * D + 64 * b, t * 128);
-        bulk_commit();
-        bulk_wait_all();  // written out before the CTA (and its shared memory) goes away
-      }
-      if (p.lse && grow < p.m) p.lse[static_cast<int64_t>(h) * p.m + grow] = (gg * mm - log2f(inv)) * kLn2;
-    }
+    attn_epilogue<D>(p, &tmO, sK, tmem, lane_base, colO, wg, row, grow, h, t, part_code, (t - p.ts) * per_tile + pair, ok,
+                     m_run, l_run, gg, abort_flag, &s_last, &s_ready);
   }
   tc_fence_before();
   __syncthreads();

@@ -441,12 +441,13 @@ struct AttnItem {
   int size, t, code;
 };
 
-// items of the schedule that splits blocks t >= ts, longest first
-std::vector<AttnItem> attn_items(int T, int kt, int ts) {
+// items of the schedule that splits blocks t >= ts, longest first; a 128-row
+// block t has (t + 1) * 128 / bn causal key tiles of bn keys (at most kt)
+std::vector<AttnItem> attn_items(int T, int kt, int ts, int bn) {
   std::vector<AttnItem> it;
   it.reserve(2 * T);
   for (int t = 0; t < T; ++t) {
-    const int u = std::min(2 * t + 2, kt);
+    const int u = std::min((t + 1) * (128 / bn), kt);
     if (t >= ts) {
       it.push_back({u / 2, t, 1});
       it.push_back({u - u / 2, t, 2});
@@ -463,31 +464,36 @@ std::vector<AttnItem> attn_items(int T, int kt, int ts) {
 }
 
 // end of the greedy in-order schedule of `per_tile` copies of each item on `sms` SMs
-int64_t attn_makespan(const std::vector<AttnItem>& it, int per_tile, int sms) {
+int64_t attn_makespan(const std::vector<AttnItem>& it, int per_tile, int sms, int fixed) {
   std::vector<int64_t> busy(static_cast<size_t>(sms), 0);  // min-heap of SM finish times
   for (const AttnItem& x : it)
     for (int r = 0; r < per_tile; ++r) {
       std::pop_heap(busy.begin(), busy.end(), std::greater<int64_t>());
-      busy.back() += x.size + kAttnCtaFixed;
+      busy.back() += x.size + fixed;
       std::push_heap(busy.begin(), busy.end(), std::greater<int64_t>());
     }
   return *std::max_element(busy.begin(), busy.end());
 }
 
 AttnPlan attn_plan_compute(int64_t m, int hkv, int group, int head_dim, int sms) {
+  constexpr int bn = 64;  // key-tile width of k_attn_tc
   AttnPlan pl;
   pl.T = static_cast<int>((m + 127) / 128);
   pl.per_tile = hkv * (group / 2);
   pl.ts = pl.T;
-  const int kt = static_cast<int>((m + 63) / 64);
+  const int kt = static_cast<int>((m + bn - 1) / bn);
+  // fixed cost per CTA in key tiles, and the fewest tiles a split block may have
+  // (each half keeps a visible key in every row)
+  const int fixed = kAttnCtaFixed;
+  const int min_split = 4;
   sms = std::max(sms, 1);
   // only short launches gain from splitting: at most about two waves of CTAs,
   // and blocks of at least 4 tiles (each half keeps a visible key per row)
   if (int64_t(pl.T) * pl.per_tile > 2 * int64_t(sms) || 2 * pl.T > tg::kAttnWorkCap || pl.T >= (1 << 14)) return pl;
-  int64_t best = attn_makespan(attn_items(pl.T, kt, pl.T), pl.per_tile, sms);
+  int64_t best = attn_makespan(attn_items(pl.T, kt, pl.T, bn), pl.per_tile, sms, fixed);
   int best_ts = pl.T;
-  for (int ts = pl.T - 1; ts >= 1 && std::min(2 * ts + 2, kt) >= 4; --ts) {
-    const int64_t span = attn_makespan(attn_items(pl.T, kt, ts), pl.per_tile, sms);
+  for (int ts = pl.T - 1; ts >= 1 && std::min((ts + 1) * (128 / bn), kt) >= min_split; --ts) {
+    const int64_t span = attn_makespan(attn_items(pl.T, kt, ts, bn), pl.per_tile, sms, fixed);
     if (span < best) {
       best = span;
       best_ts = ts;
@@ -495,7 +501,7 @@ AttnPlan attn_plan_compute(int64_t m, int hkv, int group, int head_dim, int sms)
   }
   if (best_ts == pl.T) return pl;
   pl.ts = best_ts;
-  const std::vector<AttnItem> it = attn_items(pl.T, kt, pl.ts);
+  const std::vector<AttnItem> it = attn_items(pl.T, kt, pl.ts, bn);
   pl.table = true;
   pl.items.reserve(it.size());
   for (const AttnItem& x : it) pl.items.push_back(static_cast<uint16_t>((x.t << 2) | x.code));

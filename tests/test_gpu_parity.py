@@ -276,7 +276,7 @@ def _oracle_attn(q, k, v, D, bias, ratio, gain, temp, rows=None):
 
 @pytest.mark.parametrize("split", [True, False])
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("m", [1, 5, 127, 128, 129, 300, 1000])
+@pytest.mark.parametrize("m", [1, 5, 127, 128, 129, 255, 256, 257, 300, 1000])
 def test_attention_bf16_tensor_cores(m, D, split):
     q, k, v, bias, ratio, gain, temp = _attn_case(m, 4, 2, D, "bf16", seed=m + D)
     got, lse = _gpu_attn(q, k, v, D, bias, ratio, gain, temp, "bf16", split=split)
