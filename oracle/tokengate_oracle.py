@@ -200,6 +200,63 @@ def gated_attention(q, k, v, bias, head_gain, head_temp, ratio, sm_scale: float,
 
 
 # ---------------------------------------------------------------------------
+# Decode over the gated KV cache  ([R] §4.1 Gate module, temperature scaling,
+# engineering notes)
+# ---------------------------------------------------------------------------
+
+def decode_temperature_ratio(m_kept: int, n_prompt: int, t: int) -> float:
+    """Temperature ratio of the query generated at decode step t (0-based).
+
+    [R] §4.1: tokens produced while decoding are not prunable (their score is
+    fixed at 0), and tau = softplus(sigma) * log m / log max(2, p) with m the
+    number of keys the query sees after pruning and p the number it would see
+    without.  READING: the step-t query is kept row M + t of the cache (after
+    the M kept prompt rows and the t tokens generated before it) and original
+    position N + t, so, as for a kept prompt row i with m_i = i + 1 and
+    p_i = idx_i + 1: m = M + t + 1, p = N + t + 1.
+    """
+    m = float(m_kept + t + 1)
+    p = float(n_prompt + t + 1)
+    return math.log(m) / math.log(max(2.0, p))
+
+
+def gated_decode_attention(q, k_cache, v_cache, bias, head_gain, head_temp, ratio: float, sm_scale: float,
+                           return_lse: bool = False):
+    """Attention of one new query token over the gated KV cache.
+
+    [R] §4.1 engineering notes: at decode time the gate term becomes an
+    additive attention mask, i.e. the same logits as token-gated attention for
+    the newest row, which sees every cached key:
+        l_c = temp_h * ratio * sm_scale * (q_h . k_c) + gain_h * bias_c
+        o_h = sum_c softmax_c(l) v_c,   c = 0 .. L-1 (the cache ends with the
+    query token's own key).  bias_c is the kept prompt token's importance b_c
+    and 0 for generated tokens (the caller passes it that way).
+    q [Hq, D], k/v cache [L, Hkv, D], bias [L] (None = 0).
+    Returns o [Hq, D] float64 (and lse [Hq], natural log).
+    """
+    q = np.asarray(q, dtype=F64)
+    k = np.asarray(k_cache, dtype=F64)
+    v = np.asarray(v_cache, dtype=F64)
+    hq, dh = q.shape
+    length, hkv, _ = k.shape
+    group = hq // hkv
+    bias = np.zeros(length) if bias is None else np.asarray(bias, dtype=F64)
+    gain = np.asarray(head_gain, dtype=F64)
+    temp = np.asarray(head_temp, dtype=F64)
+    out = np.zeros((hq, dh))
+    lse = np.zeros(hq)
+    for h in range(hq):
+        g = h // group
+        logits = temp[h] * ratio * sm_scale * (k[:, g, :] @ q[h]) + gain[h] * bias
+        mx = logits.max()
+        e = np.exp(logits - mx)
+        den = e.sum()
+        out[h] = (e / den) @ v[:, g, :]
+        lse[h] = mx + math.log(den)
+    return (out, lse) if return_lse else out
+
+
+# ---------------------------------------------------------------------------
 # Decoder layer above the gate  ([R] §4.1 three-stage forward; [M])
 # ---------------------------------------------------------------------------
 

@@ -289,6 +289,65 @@ def test_attention_sampled_rows_match_full():
     np.testing.assert_allclose(part, full[rows], rtol=1e-14)
 
 
+# ----------------------------------------------------------------------------- decode over the gated cache
+
+def test_decode_ratio_closed_forms_and_prefill_continuation():
+    # M = 3 kept rows out of N = 10 prompt tokens; step 0 is kept row 3 at position 10
+    assert O.decode_temperature_ratio(3, 10, 0) == pytest.approx(math.log(4) / math.log(11), rel=1e-15)
+    assert O.decode_temperature_ratio(3, 10, 5) == pytest.approx(math.log(9) / math.log(16), rel=1e-15)
+    # nothing pruned (M = N): the ratio is 1 from the second token on
+    assert O.decode_temperature_ratio(7, 7, 2) == pytest.approx(1.0, rel=1e-15)
+    # the first token of an empty prompt sees only itself: log 1 / log 2 = 0
+    assert O.decode_temperature_ratio(0, 0, 0) == 0.0
+    # the decode query continues the kept rows: its ratio is the prefill formula
+    # applied to a kept set extended by the generated positions N .. N + t
+    idx = [0, 4, 9]                 # kept prompt rows of a 10-token prompt
+    ext = idx + [10, 11, 12]        # then three generated tokens
+    pre = O.temperature_ratio(ext)
+    for t in range(3):
+        assert O.decode_temperature_ratio(len(idx), 10, t) == pytest.approx(pre[len(idx) + t], rel=1e-14)
+
+
+def test_decode_attention_is_the_last_row_of_gated_attention():
+    # the query of a decode step is the newest row of the cache: the prefill
+    # attention's last row over the same rows, with the same ratio
+    m, hq, hkv, dh = 19, 4, 2, 8
+    q, k, v, bias, gain, temp, ratio = _rand_attn(m, hq, hkv, dh, 11)
+    full, lse_full = O.gated_attention(q, k, v, bias, gain, temp, ratio, 0.35, return_lse=True)
+    out, lse = O.gated_decode_attention(q[-1], k, v, bias, gain, temp, float(ratio[-1]), 0.35, return_lse=True)
+    np.testing.assert_allclose(out, full[-1], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse, lse_full[:, -1], rtol=1e-13)
+
+
+def test_decode_attention_matches_torch_sdpa_and_closed_forms():
+    rng = np.random.default_rng(12)
+    length, hq, hkv, dh = 33, 6, 2, 16
+    q = rng.standard_normal((hq, dh))
+    k, v = rng.standard_normal((length, hkv, dh)), rng.standard_normal((length, hkv, dh))
+    bias = rng.standard_normal(length)
+    bias[-5:] = 0.0                  # generated tokens carry no gate bias
+    gain, temp = rng.uniform(0.5, 2, hq), rng.uniform(0.8, 1.2, hq)
+    ratio, scale = 0.83, 1.0 / math.sqrt(dh)
+    out = O.gated_decode_attention(q, k, v, bias, gain, temp, ratio, scale)
+    t = torch.from_numpy
+    qs = (t(q) * (t(temp) * ratio)[:, None])[None, :, None, :]              # [1, hq, 1, dh]
+    kk = t(k).transpose(0, 1)[None]                                         # [1, hkv, L, dh]
+    vv = t(v).transpose(0, 1)[None]
+    mask = (t(gain)[:, None] * t(bias)[None, :])[None, :, None, :]          # [1, hq, 1, L]
+    ref = F.scaled_dot_product_attention(qs, kk, vv, attn_mask=mask, scale=scale, enable_gqa=True)[0, :, 0]
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-10, atol=1e-12)
+    # zero content scale: the weights are softmax(gain * bias), written out
+    out0 = O.gated_decode_attention(q, k, v, bias, gain, np.zeros(hq), ratio, scale)
+    for h in range(hq):
+        g = h // (hq // hkv)
+        w = np.exp(gain[h] * bias - np.max(gain[h] * bias))
+        np.testing.assert_allclose(out0[h], (w / w.sum()) @ v[:, g], rtol=1e-12)
+    # a one-row cache returns its value row
+    one = O.gated_decode_attention(q, k[:1], v[:1], bias[:1], gain, temp, ratio, scale)
+    for h in range(hq):
+        np.testing.assert_allclose(one[h], v[0, h // (hq // hkv)], rtol=1e-15)
+
+
 # ----------------------------------------------------------------------------- decoder layer
 
 def _hf_layer(w, lw, n_rows):
