@@ -576,6 +576,74 @@ def ncu_case():
     print("ncu case done")
 
 
+def run_decode(args):
+    """Decode over the gated KV cache (one new token's attention over the kept
+    rows plus the tokens generated so far), per call, L2 flushed before each:
+    one JSON line per cache length with the time, the cache bytes read per call
+    and their rate against the measured HBM copy bandwidth."""
+    import torch
+    from learned_token_pruning_b200 import tokengate as tg
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    hq, hkv, dh = 16, 8, 128
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for name, m_kept, n_prompt, t in (("qwen3_1.7b_decode_n16384_k2000", 2064, 16384, 64),
+                                      ("qwen3_1.7b_decode_n131072_k8192", 8256, 131072, 64),
+                                      ("qwen3_1.7b_decode_unpruned_n131072", 131072, 131072, 64)):
+        length = m_kept + t + 1
+        g = torch.Generator(device=dev).manual_seed(length)
+        k = torch.randn(length, hkv * dh, device=dev, generator=g).to(torch.bfloat16)
+        v = torch.randn(length, hkv * dh, device=dev, generator=g).to(torch.bfloat16)
+        q = torch.randn(hq, dh, device=dev, generator=g).to(torch.bfloat16)
+        bias = torch.randn(length, device=dev, generator=g)
+        bias[m_kept:] = 0.0
+        gain = torch.rand(hq, device=dev, generator=g) + 0.5
+        temp = torch.rand(hq, device=dev, generator=g) * 0.4 + 0.8
+        out = torch.empty(hq, dh, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(tg.decode_workspace_bytes(length, hq, hkv, dh), dtype=torch.uint8, device=dev)
+        ratio = tg.tg_decode_temperature_ratio(m_kept, n_prompt, t)
+        call = lambda: tg.tg_gated_decode_attention(q, k, v, dh, bias, gain, temp, ratio, 1 / math.sqrt(dh), out, ws)
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            call()
+        torch.cuda.synchronize(dev)
+        reps = max(args.steps, 10)
+
+        def graph_of(body):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                body()
+            return gr
+
+        def replay_ms(gr):
+            # back-to-back replays between one pair of events on the replaying stream
+            gr.replay()
+            torch.cuda.synchronize(dev)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                gr.replay()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            return a.elapsed_time(b) / reps
+
+        def flush_and_call():
+            flush.zero_()
+            call()
+
+        # (L2 flush + call) minus (L2 flush), as the step's per-call breakdown
+        ms = replay_ms(graph_of(flush_and_call)) - replay_ms(graph_of(lambda: flush.zero_()))
+        tg.tg_check_device_error()
+        nbytes = 2 * length * hkv * dh * 2 + length * 4
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        print(json.dumps({"mode": "decode", "workload": name, "cache_rows": length, "kept_prompt_rows": m_kept,
+                          "prompt_tokens": n_prompt, "step": t, "us": ms * 1e3, "cache_bytes": nbytes, "gbs": gbs,
+                          "frac_hbm": gbs / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                          "l2": "flushed before every call", "ratio": ratio}), flush=True)
+
+
 def run_sweep(args):
     """The other single-layer workloads (budget sweep at N=32768, K in {1024,
     4096, 8192}; 128K with K=8192): one JSON line each with the step time, the
@@ -695,6 +763,7 @@ def main(argv=None):
     ap.add_argument("--ncu-case", action="store_true", help="one launch of each heavy kernel (profiling)")
     ap.add_argument("--sweep", action="store_true", help="budget-sweep and 128K single-layer workloads")
     ap.add_argument("--stack", action="store_true", help="28-layer stack TTFT, pruned vs unpruned")
+    ap.add_argument("--decode", action="store_true", help="decode attention over the gated KV cache, per call")
     ap.add_argument("--stack-n", type=int, nargs="*", default=None, help="stack sizes to run (default all)")
     args = ap.parse_args(argv)
     if args.ncu_case:
@@ -705,6 +774,9 @@ def main(argv=None):
         return
     if args.stack:
         run_stack(args)
+        return
+    if args.decode:
+        run_decode(args)
         return
     from learned_token_pruning_b200 import synth
     w = synth.qwen3_1p7b_16k()

@@ -181,6 +181,46 @@ int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk,
                        const float* ratio, float sm_scale,
                        void* out, int64_t ldo, float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * One decode step of token-gated attention over the gated KV cache ([R] §4.1
+ * Gate module: tokens produced while decoding are not prunable and score 0;
+ * §4.1 engineering notes: at decode time the gate term is an additive mask on
+ * the attention logits; §4.1 temperature scaling).  The new token's query
+ * attends to all `length` cached rows, the last of which is its own key:
+ *     l_c = head_temp[h] * ratio * sm_scale * (q_h . k_c) + head_gain[h] * bias[c]
+ *     out_h = sum_c softmax_c(l) v_c
+ *   q      device, dtype, [hq][head_dim] (the new token's query rows, after RoPE)
+ *   k, v   device, dtype, cache row c of KV head g at k + c*ldk + g*head_dim
+ *          (same for v / ldv): the kept prompt rows, then the generated ones
+ *   bias   device fp32 [length] or NULL (0): the kept prompt rows' importance
+ *          b_c, 0 for generated rows
+ *   head_gain, head_temp  device fp32 [hq] (values after softplus)
+ *   ratio  the step's temperature ratio (tg_decode_temperature_ratio)
+ *   out    device, dtype, [hq][head_dim];  lse device fp32 [hq] or NULL
+ *   ws     device workspace of tg_workspace_bytes(TG_OP_DECODE, 0, length, 0, 0,
+ *          shape) bytes (shape gives hq, hkv, head_dim), 16-byte aligned;
+ *          required (the cache is split into chunks whose partial results are
+ *          merged in it).  The size depends on the SM count of the device.
+ * head_dim in {64, 128}; hq % hkv == 0 with at most 8 query heads per KV head;
+ * length <= 262144; cache rows 16-byte aligned.  bf16 or fp32 inputs, fp32 arithmetic on the
+ * CUDA cores (the step reads the cache once and is bound by memory).
+ */
+int tg_gated_decode_attention(const void* q, const void* k, int64_t ldk, const void* v, int64_t ldv,
+                              int dtype, int64_t length, int32_t hq, int32_t hkv, int32_t head_dim,
+                              const float* bias, const float* head_gain, const float* head_temp,
+                              float ratio, float sm_scale, void* out, float* lse,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Temperature ratio of the query generated at decode step t (0-based) after a
+ * prompt of n_prompt tokens of which m_kept were kept ([R] §4.1 temperature
+ * scaling, read as for a kept prompt row): the query is kept row m_kept + t at
+ * original position n_prompt + t, so
+ *     ratio = log(m_kept + t + 1) / log(max(2, n_prompt + t + 1)).
+ * Host function; returns 0 for negative arguments.
+ */
+float tg_decode_temperature_ratio(int64_t m_kept, int64_t n_prompt, int64_t t);
+
 /* Weights of one Qwen3-style decoder layer (device pointers). */
 typedef struct {
   const float* w_in_norm;    /* fp32 [d_model]                                  */
@@ -240,11 +280,12 @@ enum { TG_EPI_STORE = 0, TG_EPI_RESIDUAL = 1, TG_EPI_SWIGLU = 2 };
 int tg_linear(const void* x, int64_t ldx, const void* w, void* y, int64_t ldy, int dtype,
               int64_t m, int32_t n_out, int32_t k_in, int epilogue, void* stream);
 
-enum { TG_OP_GATE_SCORE = 0, TG_OP_LAYER = 1, TG_OP_ATTENTION = 2 };
+enum { TG_OP_GATE_SCORE = 0, TG_OP_LAYER = 1, TG_OP_ATTENTION = 2, TG_OP_DECODE = 3 };
 
 /* Workspace bytes needed by an op: TG_OP_GATE_SCORE uses n, d_model and h;
  * TG_OP_LAYER and TG_OP_ATTENTION use m and shape (TG_OP_ATTENTION reads its
- * dtype, hq, hkv and head_dim).  Returns 0 for an invalid request, and 0 for
+ * dtype, hq, hkv and head_dim); TG_OP_DECODE uses m = the cache length and
+ * shape's hq, hkv and head_dim.  Returns 0 for an invalid request, and 0 for
  * TG_OP_ATTENTION when the attention needs no workspace. */
 size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t h, const tg_layer_shape* shape);
 

@@ -24,6 +24,7 @@
 #include "attn_tc.cuh"
 #include "common.cuh"
 #include "gate_tc.cuh"
+#include "decode.cuh"
 #include "gather.cuh"
 #include "gemm_tc.cuh"
 #include "select.cuh"
@@ -535,6 +536,29 @@ size_t attn_ws_bytes(int64_t m, int hq, int hkv, int head_dim, int dtype) {
   return attn_plan(m, hkv, hq / hkv, head_dim, sm_count()).bytes;
 }
 
+// Decode attention: key chunks of a multiple of 64 keys (at most
+// kDecMaxChunk), about two CTAs per SM over all KV heads; the workspace holds
+// each chunk's (O, max, sum) per query head, then one counter per KV head.
+struct DecodePlan {
+  int chunk = 0, nchunks = 0;
+  size_t part_bytes = 0, bytes = 0;
+};
+
+DecodePlan decode_plan(int64_t length, int hkv, int group, int head_dim) {
+  DecodePlan pl;
+  if (length <= 0 || hkv <= 0 || group <= 0) return pl;
+  const int64_t sms = sm_count();
+  int64_t chunk = (length * hkv + 2 * sms - 1) / (2 * sms);
+  chunk = std::max<int64_t>(chunk, (length + tg::kDecMaxChunks - 1) / tg::kDecMaxChunks);  // <= 256 chunks
+  chunk = std::min<int64_t>(std::max<int64_t>((chunk + 63) / 64 * 64, 64), tg::kDecMaxChunk);
+  pl.chunk = static_cast<int>(chunk);
+  pl.nchunks = static_cast<int>((length + chunk - 1) / chunk);
+  auto al = [](size_t b) { return (b + 255) / 256 * 256; };
+  pl.part_bytes = al(static_cast<size_t>(hkv) * pl.nchunks * group * (head_dim + 2) * sizeof(float));
+  pl.bytes = pl.part_bytes + al(static_cast<size_t>(hkv) * sizeof(uint32_t));
+  return pl;
+}
+
 size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t h, const tg_layer_shape* shape) {
   if (op == TG_OP_GATE_SCORE) return (n > 0 && d_model > 0 && h > 0) ? gate_ws_bytes(n, d_model, h) : 0;
   if (op == TG_OP_LAYER) {
@@ -553,6 +577,10 @@ size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t
   if (op == TG_OP_ATTENTION) {
     if (!shape || m <= 0) return 0;
     return attn_ws_bytes(m, shape->hq, shape->hkv, shape->head_dim, shape->dtype);
+  }
+  if (op == TG_OP_DECODE) {
+    if (!shape || m <= 0 || shape->hkv <= 0 || shape->hq % shape->hkv) return 0;
+    return decode_plan(m, shape->hkv, shape->hq / shape->hkv, shape->head_dim).bytes;
   }
   return 0;
 }
@@ -890,6 +918,66 @@ int tg_linear(const void* x, int64_t ldx, const void* w, void* y, int64_t ldy, i
     else tg::k_gemm_simt<B, false><<<grid, 256, 0, st>>>(xa, ldx, wa, ya, ldy, mm, n_out, k_in);
   }
   return check_launch("k_gemm_simt");
+}
+
+float tg_decode_temperature_ratio(int64_t m_kept, int64_t n_prompt, int64_t t) {
+  if (m_kept < 0 || n_prompt < 0 || t < 0) return 0.0f;
+  const double m = static_cast<double>(m_kept + t + 1), p = static_cast<double>(n_prompt + t + 1);
+  return static_cast<float>(std::log(m) / std::log(std::max(2.0, p)));
+}
+
+int tg_gated_decode_attention(const void* q, const void* k, int64_t ldk, const void* v, int64_t ldv, int dtype,
+                              int64_t length, int32_t hq, int32_t hkv, int32_t head_dim, const float* bias,
+                              const float* head_gain, const float* head_temp, float ratio, float sm_scale, void* out,
+                              float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (!q || !k || !v || !out || !head_gain || !head_temp) return fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (length <= 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0) return fail(TG_ERR_INVALID_ARG, "bad length / heads");
+  if (length > int64_t(tg::kDecMaxChunks) * tg::kDecMaxChunk)
+    return fail(TG_ERR_UNSUPPORTED, "cache length must be <= %d", tg::kDecMaxChunks * tg::kDecMaxChunk);
+  if (head_dim != 64 && head_dim != 128) return fail(TG_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (hq / hkv > tg::kDecMaxGroup) return fail(TG_ERR_UNSUPPORTED, "at most %d query heads per KV head", tg::kDecMaxGroup);
+  if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "dtype");
+  if (ldk < int64_t(hkv) * head_dim || ldv < int64_t(hkv) * head_dim)
+    return fail(TG_ERR_SHAPE, "leading dimension smaller than the heads it holds");
+  const int es = dtype_size(dtype);
+  if (!aligned16(k) || !aligned16(v) || (ldk * es) % 16 || (ldv * es) % 16)
+    return fail(TG_ERR_ALIGN, "cache rows need 16-byte alignment");
+  const int group = hq / hkv;
+  const DecodePlan pl = decode_plan(length, hkv, group, head_dim);
+  if (!ws || ws_bytes < pl.bytes) return fail(TG_ERR_WORKSPACE, "decode attention needs %zu workspace bytes", pl.bytes);
+  if (!aligned16(ws)) return fail(TG_ERR_ALIGN, "workspace must be 16-byte aligned");
+  cudaStream_t st = as_stream(stream);
+  tg::DecodeParams p{};
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.ldk = ldk;
+  p.ldv = ldv;
+  p.length = static_cast<int>(length);
+  p.hq = hq;
+  p.hkv = hkv;
+  p.group = group;
+  p.chunk = pl.chunk;
+  p.nchunks = pl.nchunks;
+  p.bias = bias;
+  p.gain = head_gain;
+  p.temp = head_temp;
+  p.ratio_scale_log2 = ratio * sm_scale * tg::kLog2e;
+  p.out = out;
+  p.lse = lse;
+  p.part = static_cast<float*>(ws);
+  p.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + pl.part_bytes);
+  if (cudaMemsetAsync(p.counters, 0, pl.bytes - pl.part_bytes, st) != cudaSuccess)
+    return fail(TG_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(cudaGetLastError()));
+  const dim3 grid(static_cast<unsigned>(hkv * pl.nchunks));
+  if (dtype == TG_BF16) {
+    if (head_dim == 128)
+      return launch_pdl("k_decode_attn", tg::k_decode_attn<__nv_bfloat16, 128>, grid, dim3(tg::kDecThreads), 0, st, p);
+    return launch_pdl("k_decode_attn", tg::k_decode_attn<__nv_bfloat16, 64>, grid, dim3(tg::kDecThreads), 0, st, p);
+  }
+  if (head_dim == 128)
+    return launch_pdl("k_decode_attn", tg::k_decode_attn<float, 128>, grid, dim3(tg::kDecThreads), 0, st, p);
+  return launch_pdl("k_decode_attn", tg::k_decode_attn<float, 64>, grid, dim3(tg::kDecThreads), 0, st, p);
 }
 
 int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden_kept,

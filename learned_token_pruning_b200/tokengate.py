@@ -18,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libtokengate.so")
 
 TG_F32, TG_BF16 = 0, 1
-TG_OP_GATE_SCORE, TG_OP_LAYER, TG_OP_ATTENTION = 0, 1, 2
+TG_OP_GATE_SCORE, TG_OP_LAYER, TG_OP_ATTENTION, TG_OP_DECODE = 0, 1, 2, 3
 STATUS = {0: "TG_OK", 1: "TG_ERR_INVALID_ARG", 2: "TG_ERR_SHAPE", 3: "TG_ERR_ALIGN", 4: "TG_ERR_UNSUPPORTED",
           5: "TG_ERR_WORKSPACE", 6: "TG_ERR_CUDA", 7: "TG_ERR_DEVICE_TIMEOUT", 8: "TG_ERR_DEVICE_CHECK"}
 
@@ -55,6 +55,9 @@ SIGNATURES = {
                                   _P, _I64, _P, _P, _SZ, _P]),
     "tg_pruned_prefill_layer": (_INT, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerShape), _P, _P, _P, _P,
                                        _I64, _P, _SZ, _P]),
+    "tg_gated_decode_attention": (_INT, [_P, _P, _I64, _P, _I64, _INT, _I64, _I32, _I32, _I32, _P, _P, _P, _F, _F,
+                                         _P, _P, _P, _SZ, _P]),
+    "tg_decode_temperature_ratio": (_F, [_I64, _I64, _I64]),
     "tg_linear": (_INT, [_P, _I64, _P, _P, _I64, _INT, _I64, _I32, _I32, _INT, _P]),
     "tg_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I32, _I32, ctypes.POINTER(LayerShape)]),
     "tg_gate_score_noalloc": (_INT, [_P, _INT, _I64, _I32, _P, _F, _P, _P, _P, _F, _I32, _P, _P, _P, _P]),
@@ -189,6 +192,31 @@ def tg_gated_attention(q, k, v, head_dim: int, bias, head_gain, head_temp, ratio
                                   _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0,
                                   _stream(stream))
     _check("tg_gated_attention", rc)
+
+
+def decode_workspace_bytes(length: int, hq: int, hkv: int, head_dim: int) -> int:
+    shape = LayerShape(dtype=TG_BF16, d_model=0, hq=hq, hkv=hkv, head_dim=head_dim, d_ff=0, qk_norm=0,
+                       rope_theta=0.0, norm_eps=0.0)
+    return tg_workspace_bytes(TG_OP_DECODE, m=length, shape=shape)
+
+
+def tg_decode_temperature_ratio(m_kept: int, n_prompt: int, t: int) -> float:
+    return float(lib().tg_decode_temperature_ratio(int(m_kept), int(n_prompt), int(t)))
+
+
+def tg_gated_decode_attention(q, k, v, head_dim: int, bias, head_gain, head_temp, ratio: float, sm_scale: float, out,
+                              ws, lse=None, stream=None):
+    """q/out [hq, head_dim] (contiguous); k/v the cache as 2-D row views [length, hkv*head_dim]
+    (rows may be strided); ws a device byte buffer of decode_workspace_bytes(...) bytes."""
+    kp, ldk = _row_view(k)
+    vp, ldv = _row_view(v)
+    hq = q.numel() // head_dim
+    hkv = k.shape[1] // head_dim
+    rc = lib().tg_gated_decode_attention(_ptr(q), kp, ldk, vp, ldv, _dtype(q), k.shape[0], hq, hkv, head_dim,
+                                         _ptr(bias), _ptr(head_gain), _ptr(head_temp), float(ratio), float(sm_scale),
+                                         _ptr(out), _ptr(lse), _ptr(ws),
+                                         ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream))
+    _check("tg_gated_decode_attention", rc)
 
 
 TG_EPI_STORE, TG_EPI_RESIDUAL, TG_EPI_SWIGLU = 0, 1, 2

@@ -2,6 +2,7 @@
 point the header declares, and rejects bad arguments on the host before any
 CUDA call."""
 import ctypes
+import math
 import os
 import re
 
@@ -90,3 +91,36 @@ def test_workspace_sizes(L):
     assert tg.tg_workspace_bytes(tg.TG_OP_ATTENTION, m=m, shape=S32) == 0
     assert tg.tg_workspace_bytes(tg.TG_OP_GATE_SCORE, n=16384, d_model=2048, h=256) >= 16384 // 128 * 4 + 256 * 2048 * 2
     assert tg.tg_workspace_bytes(99) == 0
+
+
+def test_decode_validation_and_workspace(L):
+    g = ctypes.c_void_p(256)
+    f = L.tg_gated_decode_attention
+    # q, k, ldk, v, ldv, dtype, length, hq, hkv, head_dim, bias, gain, temp, ratio, scale, out, lse, ws, ws_bytes, stream
+    assert f(None, g, 1024, g, 1024, 1, 10, 16, 8, 128, None, g, g, 1.0, 0.1, g, None, g, 1 << 20, None) == 1
+    assert f(g, g, 1024, g, 1024, 1, 0, 16, 8, 128, None, g, g, 1.0, 0.1, g, None, g, 1 << 20, None) == 1   # empty cache
+    assert f(g, g, 1024, g, 1024, 1, 10, 16, 6, 128, None, g, g, 1.0, 0.1, g, None, g, 1 << 20, None) == 1  # hq % hkv
+    assert f(g, g, 1024, g, 1024, 1, 10, 16, 8, 96, None, g, g, 1.0, 0.1, g, None, g, 1 << 20, None) == 4   # head_dim
+    assert f(g, g, 1024, g, 1024, 1, 10, 32, 2, 128, None, g, g, 1.0, 0.1, g, None, g, 1 << 20, None) == 4  # group 16
+    assert f(g, g, 1000, g, 1024, 1, 10, 16, 8, 128, None, g, g, 1.0, 0.1, g, None, g, 1 << 20, None) == 2  # ldk < heads
+    assert f(g, ctypes.c_void_p(258), 1024, g, 1024, 1, 10, 16, 8, 128, None, g, g, 1.0, 0.1, g, None, g, 1 << 20,
+             None) == 3                                                                                        # alignment
+    assert f(g, g, 1028, g, 1024, 1, 10, 16, 8, 128, None, g, g, 1.0, 0.1, g, None, g, 1 << 20, None) == 3  # row stride
+    need = tg.decode_workspace_bytes(10, 16, 8, 128)
+    assert need > 0
+    assert f(g, g, 1024, g, 1024, 1, 10, 16, 8, 128, None, g, g, 1.0, 0.1, g, None, g, need - 1, None) == 5  # workspace
+    assert f(g, g, 1024, g, 1024, 1, 10, 16, 8, 128, None, g, g, 1.0, 0.1, g, None, None, 0, None) == 5
+    # the workspace holds (O, max, sum) of every chunk and query head, then the KV heads' counters
+    for length in (1, 64, 2064, 8256, 131072, 262144):
+        ws = tg.decode_workspace_bytes(length, 16, 8, 128)
+        assert 16 * 130 * 4 * ((length + 1023) // 1024) + 8 * 4 <= ws <= 16 * 130 * 4 * 256 + 256 + 256
+    assert tg.decode_workspace_bytes(2064, 16, 6, 128) == 0   # invalid head split
+    assert f(g, g, 1024, g, 1024, 1, 262145, 16, 8, 128, None, g, g, 1.0, 0.1, g, None, g, 1 << 30, None) == 4
+
+
+def test_decode_temperature_ratio_host_helper(L):
+    # ratio = log(m_kept + t + 1) / log(max(2, n_prompt + t + 1)), in float
+    assert tg.tg_decode_temperature_ratio(3, 10, 0) == pytest.approx(math.log(4) / math.log(11), rel=1e-6)
+    assert tg.tg_decode_temperature_ratio(2064, 16384, 7) == pytest.approx(math.log(2072) / math.log(16392), rel=1e-6)
+    assert tg.tg_decode_temperature_ratio(0, 0, 0) == 0.0
+    assert tg.tg_decode_temperature_ratio(-1, 10, 0) == 0.0

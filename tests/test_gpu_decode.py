@@ -1,0 +1,133 @@
+"""Decode over the gated KV cache: the CUDA kernel against the CPU oracle on the
+same seeded inputs, element by element (small caches, ragged chunk tails, every
+GQA group size the kernel takes, both head dims and dtypes), and at the cache
+lengths of the workloads (kept rows of the 16K and 128K prompts plus generated
+tokens) on every output."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from learned_token_pruning_b200 import synth, tokengate as tg
+from oracle import tokengate_oracle as O
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+ATTN_BF16 = dict(atol=2e-2, rtol=1e-2)
+ATTN_F32 = dict(atol=1e-4, rtol=1e-4)
+
+
+def _case(length, hq, hkv, dh, dtype, seed, generated=3):
+    rng = np.random.default_rng(seed)
+    q = synth.round_to(rng.standard_normal((hq, dh)).astype(np.float32), dtype)
+    k = synth.round_to(rng.standard_normal((length, hkv, dh)).astype(np.float32), dtype)
+    v = synth.round_to(rng.standard_normal((length, hkv, dh)).astype(np.float32), dtype)
+    bias = rng.standard_normal(length).astype(np.float32)
+    bias[max(0, length - generated):] = 0.0   # generated rows carry no gate bias
+    gain = rng.uniform(0.5, 2.0, hq).astype(np.float32)
+    temp = rng.uniform(0.8, 1.2, hq).astype(np.float32)
+    return q, k, v, bias, gain, temp
+
+
+def _gpu(q, k, v, dh, bias, gain, temp, ratio, dtype, kv_buffer=None):
+    dt = synth.torch_dtype(dtype)
+    length, hkv, _ = k.shape
+    hq = q.shape[0]
+    if kv_buffer is None:
+        kd = torch.from_numpy(k.reshape(length, hkv * dh)).to(DEV, dt)
+        vd = torch.from_numpy(v.reshape(length, hkv * dh)).to(DEV, dt)
+    else:
+        kd, vd = kv_buffer
+    qd = torch.from_numpy(q).to(DEV, dt)
+    out = torch.empty(hq, dh, dtype=dt, device=DEV)
+    lse = torch.empty(hq, dtype=torch.float32, device=DEV)
+    ws = torch.full((tg.decode_workspace_bytes(length, hq, hkv, dh),), 0xA5, dtype=torch.uint8, device=DEV)
+    tg.tg_gated_decode_attention(qd, kd, vd, dh, None if bias is None else torch.from_numpy(bias).to(DEV),
+                                 torch.from_numpy(gain).to(DEV), torch.from_numpy(temp).to(DEV), ratio,
+                                 1.0 / math.sqrt(dh), out, ws, lse)
+    assert tg.tg_check_device_error() == 0
+    return out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def _check(length, hq, hkv, dh, dtype, seed, with_bias=True):
+    q, k, v, bias, gain, temp = _case(length, hq, hkv, dh, dtype, seed)
+    ratio = tg.tg_decode_temperature_ratio(max(length - 3, 0), 4 * length, 2)
+    got, lse = _gpu(q, k, v, dh, bias if with_bias else None, gain, temp, ratio, dtype)
+    want, wlse = O.gated_decode_attention(q, k, v, bias if with_bias else None, gain, temp, ratio,
+                                          1.0 / math.sqrt(dh), return_lse=True)
+    tol = ATTN_BF16 if dtype == "bf16" else ATTN_F32
+    np.testing.assert_allclose(got, want, **tol)
+    np.testing.assert_allclose(lse, wlse, rtol=1e-4, atol=1e-4)
+
+
+@pytest.mark.parametrize("length", [1, 2, 63, 64, 65, 127, 300, 1000])
+@pytest.mark.parametrize("dh", [64, 128])
+def test_decode_bf16_small_caches(length, dh):
+    # a single row, one chunk, ragged last chunk, several chunks (64-key multiples)
+    _check(length, 16, 8, dh, "bf16", seed=length + dh)
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (4, 2), (6, 2), (8, 1), (16, 8)])
+def test_decode_group_sizes(hq, hkv):
+    # group 1 .. 8 query heads per KV head (8 is the kernel's limit)
+    _check(517, hq, hkv, 128, "bf16", seed=hq * 10 + hkv)
+
+
+@pytest.mark.parametrize("length,dh", [(1, 64), (200, 64), (777, 128)])
+def test_decode_fp32(length, dh):
+    _check(length, 8, 2, dh, "f32", seed=length)
+
+
+def test_decode_no_bias_is_plain_attention_of_the_last_row():
+    _check(300, 16, 8, 128, "bf16", seed=7, with_bias=False)
+
+
+@pytest.mark.parametrize("length", [2064 + 1, 8256 + 17])
+def test_decode_workload_cache_lengths(length):
+    # the kept rows of the 16K- and 128K-token prompts, then generated tokens;
+    # every output compared (one row of attention is cheap for the oracle)
+    _check(length, 16, 8, 128, "bf16", seed=length)
+
+
+def test_decode_strided_cache_views_and_reruns_are_identical():
+    # the cache as K and V column ranges of one fused [L][(Hq + 2 Hkv) D] buffer
+    length, hq, hkv, dh = 1500, 16, 8, 128
+    q, k, v, bias, gain, temp = _case(length, hq, hkv, dh, "bf16", seed=5)
+    qkv = np.zeros((length, (hq + 2 * hkv) * dh), np.float32)
+    qkv[:, hq * dh:(hq + hkv) * dh] = k.reshape(length, -1)
+    qkv[:, (hq + hkv) * dh:] = v.reshape(length, -1)
+    buf = torch.from_numpy(qkv).to(DEV, torch.bfloat16)
+    views = (buf[:, hq * dh:(hq + hkv) * dh], buf[:, (hq + hkv) * dh:])
+    ratio = 0.9
+    got, _ = _gpu(q, k, v, dh, bias, gain, temp, ratio, "bf16", kv_buffer=views)
+    again, _ = _gpu(q, k, v, dh, bias, gain, temp, ratio, "bf16", kv_buffer=views)
+    assert np.array_equal(got, again)
+    want = O.gated_decode_attention(q, k, v, bias, gain, temp, ratio, 1.0 / math.sqrt(dh))
+    np.testing.assert_allclose(got, want, **ATTN_BF16)
+
+
+def test_decode_continues_prefill_attention():
+    # the decode query is the newest row: decode over the first L rows with the
+    # row's ratio equals the prefill kernel's row L - 1 (two CUDA paths agree)
+    length, hq, hkv, dh = 700, 16, 8, 128
+    rng = np.random.default_rng(9)
+    q = synth.round_to(rng.standard_normal((length, hq * dh)).astype(np.float32), "bf16")
+    k = synth.round_to(rng.standard_normal((length, hkv * dh)).astype(np.float32), "bf16")
+    v = synth.round_to(rng.standard_normal((length, hkv * dh)).astype(np.float32), "bf16")
+    bias = rng.standard_normal(length).astype(np.float32)
+    ratio = rng.uniform(0.2, 1.0, length).astype(np.float32)
+    gain = rng.uniform(0.5, 2.0, hq).astype(np.float32)
+    temp = rng.uniform(0.8, 1.2, hq).astype(np.float32)
+    t = lambda a, dt=torch.float32: torch.from_numpy(a).to(DEV, dt)
+    out = torch.empty(length, hq * dh, dtype=torch.bfloat16, device=DEV)
+    tg.tg_gated_attention(t(q, torch.bfloat16), t(k, torch.bfloat16), t(v, torch.bfloat16), dh, t(bias), t(gain),
+                          t(temp), t(ratio), 1.0 / math.sqrt(dh), out)
+    got, _ = _gpu(q[-1].reshape(hq, dh), k.reshape(length, hkv, dh), v.reshape(length, hkv, dh), dh, bias, gain,
+                  temp, float(ratio[-1]), "bf16")
+    np.testing.assert_allclose(got.reshape(-1), out[-1].float().cpu().numpy(), atol=1e-2, rtol=1e-2)
+
+
+def test_decode_maximum_cache_length():
+    # 262144 rows: 256 chunks of 1024 keys per KV head, the most one call takes
+    _check(262144, 4, 2, 128, "bf16", seed=3)
