@@ -79,9 +79,12 @@ __device__ __forceinline__ void load_f32(const float* src, float (&x)[N]) {
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, int GT>
 __global__ void __launch_bounds__(kDecThreads) k_decode_attn(DecodeParams p) {
   constexpr int Q4 = D / 4;  // head-dimension elements per lane of a key's four lanes
+  // the lane's slice of the group's scaled query rows lives in registers for
+  // groups of up to four heads (else it is read from shared memory per key)
+  constexpr bool kQReg = GT * Q4 <= 128;
   __shared__ float s_q[kDecMaxGroup][D];
   __shared__ float s_x[kDecMaxGroup][kDecMaxChunk];
   __shared__ float s_red[kDecMaxGroup][kDecThreads / 32];
@@ -92,7 +95,8 @@ __global__ void __launch_bounds__(kDecThreads) k_decode_attn(DecodeParams p) {
   pdl_launch_dependents();
   const int g = blockIdx.x / p.nchunks, j = blockIdx.x % p.nchunks;
   const int c0 = j * p.chunk, c1 = min(c0 + p.chunk, p.length), nk = c1 - c0;
-  const int G = p.group, h0 = g * G;
+  constexpr int G = GT;
+  const int h0 = g * G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const T* qp = static_cast<const T*>(p.q);
   const T* kp = static_cast<const T*>(p.k);
@@ -107,31 +111,39 @@ __global__ void __launch_bounds__(kDecThreads) k_decode_attn(DecodeParams p) {
 
   // 2. logits of the chunk's keys: key = pass base + warp * 8 + lane / 4, quarter = lane % 4
   const int qd = (lane & 3) * Q4;
+  float qreg[kQReg ? G : 1][kQReg ? Q4 : 1];
+  if constexpr (kQReg) {
+#pragma unroll
+    for (int u = 0; u < G; ++u)
+#pragma unroll
+      for (int e = 0; e < Q4; ++e) qreg[u][e] = s_q[u][qd + e];
+  }
+  float gbias[G];
+#pragma unroll
+  for (int u = 0; u < G; ++u) gbias[u] = p.gain[h0 + u] * kLog2e;
   for (int base = 0; base < nk; base += kDecKeysPerPass) {
     const int kk = base + warp * 8 + (lane >> 2);
-    float acc[kDecMaxGroup];
+    float acc[G];
 #pragma unroll
-    for (int u = 0; u < kDecMaxGroup; ++u) acc[u] = 0.0f;
+    for (int u = 0; u < G; ++u) acc[u] = 0.0f;
     if (kk < nk) {
       float kv[Q4];
       load_f32<Q4>(kp + static_cast<int64_t>(c0 + kk) * p.ldk + static_cast<int64_t>(g) * D + qd, kv);
 #pragma unroll
       for (int e = 0; e < Q4; ++e) {
 #pragma unroll
-        for (int u = 0; u < kDecMaxGroup; ++u)
-          if (u < G) acc[u] = fmaf(s_q[u][qd + e], kv[e], acc[u]);
+        for (int u = 0; u < G; ++u) acc[u] = fmaf(kQReg ? qreg[kQReg ? u : 0][kQReg ? e : 0] : s_q[u][qd + e], kv[e], acc[u]);
       }
     }
 #pragma unroll
-    for (int u = 0; u < kDecMaxGroup; ++u) {
+    for (int u = 0; u < G; ++u) {
       acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], 1);
       acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], 2);
     }
     if (kk < nk && (lane & 3) == 0) {
       const float b = p.bias ? p.bias[c0 + kk] : 0.0f;
 #pragma unroll
-      for (int u = 0; u < kDecMaxGroup; ++u)
-        if (u < G) s_x[u][kk] = fmaf(p.gain[h0 + u] * kLog2e, b, acc[u]);
+      for (int u = 0; u < G; ++u) s_x[u][kk] = fmaf(gbias[u], b, acc[u]);
     }
   }
   __syncthreads();

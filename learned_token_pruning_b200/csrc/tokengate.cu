@@ -383,6 +383,21 @@ bool select_cluster16_ok() {
   return good;
 }
 
+// decode kernel for a group size (query heads per KV head) fixed at compile time
+template <typename T, int D>
+int launch_decode(int group, dim3 grid, cudaStream_t st, const tg::DecodeParams& p) {
+  switch (group) {
+    case 1: return launch_pdl("k_decode_attn", tg::k_decode_attn<T, D, 1>, grid, dim3(tg::kDecThreads), 0, st, p);
+    case 2: return launch_pdl("k_decode_attn", tg::k_decode_attn<T, D, 2>, grid, dim3(tg::kDecThreads), 0, st, p);
+    case 3: return launch_pdl("k_decode_attn", tg::k_decode_attn<T, D, 3>, grid, dim3(tg::kDecThreads), 0, st, p);
+    case 4: return launch_pdl("k_decode_attn", tg::k_decode_attn<T, D, 4>, grid, dim3(tg::kDecThreads), 0, st, p);
+    case 5: return launch_pdl("k_decode_attn", tg::k_decode_attn<T, D, 5>, grid, dim3(tg::kDecThreads), 0, st, p);
+    case 6: return launch_pdl("k_decode_attn", tg::k_decode_attn<T, D, 6>, grid, dim3(tg::kDecThreads), 0, st, p);
+    case 7: return launch_pdl("k_decode_attn", tg::k_decode_attn<T, D, 7>, grid, dim3(tg::kDecThreads), 0, st, p);
+    default: return launch_pdl("k_decode_attn", tg::k_decode_attn<T, D, 8>, grid, dim3(tg::kDecThreads), 0, st, p);
+  }
+}
+
 extern "C" {
 
 const char* tg_version(void) { return TG_VERSION; }
@@ -970,14 +985,10 @@ int tg_gated_decode_attention(const void* q, const void* k, int64_t ldk, const v
   if (cudaMemsetAsync(p.counters, 0, pl.bytes - pl.part_bytes, st) != cudaSuccess)
     return fail(TG_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(cudaGetLastError()));
   const dim3 grid(static_cast<unsigned>(hkv * pl.nchunks));
-  if (dtype == TG_BF16) {
-    if (head_dim == 128)
-      return launch_pdl("k_decode_attn", tg::k_decode_attn<__nv_bfloat16, 128>, grid, dim3(tg::kDecThreads), 0, st, p);
-    return launch_pdl("k_decode_attn", tg::k_decode_attn<__nv_bfloat16, 64>, grid, dim3(tg::kDecThreads), 0, st, p);
-  }
-  if (head_dim == 128)
-    return launch_pdl("k_decode_attn", tg::k_decode_attn<float, 128>, grid, dim3(tg::kDecThreads), 0, st, p);
-  return launch_pdl("k_decode_attn", tg::k_decode_attn<float, 64>, grid, dim3(tg::kDecThreads), 0, st, p);
+  if (dtype == TG_BF16)
+    return head_dim == 128 ? launch_decode<__nv_bfloat16, 128>(group, grid, st, p)
+                           : launch_decode<__nv_bfloat16, 64>(group, grid, st, p);
+  return head_dim == 128 ? launch_decode<float, 128>(group, grid, st, p) : launch_decode<float, 64>(group, grid, st, p);
 }
 
 int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden_kept,
