@@ -644,6 +644,31 @@ def run_decode(args):
                           "l2": "flushed before every call", "ratio": ratio}), flush=True)
 
 
+def ncu_decode_case():
+    """One decode-attention call on a 131137-row cache (16/8 heads x 128, bf16;
+    the unpruned 128K-token prompt's cache) after a warm-up call, each after an
+    L2 flush, for profiler captures of k_decode_attn."""
+    import torch
+    from learned_token_pruning_b200 import tokengate as tg
+    dev, hq, hkv, dh, length = "cuda", 16, 8, 128, 131137
+    g = torch.Generator(device=dev).manual_seed(1)
+    k = torch.randn(length, hkv * dh, device=dev, generator=g).to(torch.bfloat16)
+    v = torch.randn(length, hkv * dh, device=dev, generator=g).to(torch.bfloat16)
+    q = torch.randn(hq, dh, device=dev, generator=g).to(torch.bfloat16)
+    bias = torch.randn(length, device=dev, generator=g)
+    gain = torch.rand(hq, device=dev, generator=g) + 0.5
+    temp = torch.rand(hq, device=dev, generator=g) * 0.4 + 0.8
+    out = torch.empty(hq, dh, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(tg.decode_workspace_bytes(length, hq, hkv, dh), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        flush.zero_()
+        tg.tg_gated_decode_attention(q, k, v, dh, bias, gain, temp, 0.9, 1 / math.sqrt(dh), out, ws)
+    torch.cuda.synchronize()
+    tg.tg_check_device_error()
+    print("ncu decode case done")
+
+
 def run_sweep(args):
     """The other single-layer workloads (budget sweep at N=32768, K in {1024,
     4096, 8192}; 128K with K=8192): one JSON line each with the step time, the
@@ -764,10 +789,14 @@ def main(argv=None):
     ap.add_argument("--sweep", action="store_true", help="budget-sweep and 128K single-layer workloads")
     ap.add_argument("--stack", action="store_true", help="28-layer stack TTFT, pruned vs unpruned")
     ap.add_argument("--decode", action="store_true", help="decode attention over the gated KV cache, per call")
+    ap.add_argument("--ncu-decode", action="store_true", help="one decode call on a 131137-row cache (profiling)")
     ap.add_argument("--stack-n", type=int, nargs="*", default=None, help="stack sizes to run (default all)")
     args = ap.parse_args(argv)
     if args.ncu_case:
         ncu_case()
+        return
+    if args.ncu_decode:
+        ncu_decode_case()
         return
     if args.sweep:
         run_sweep(args)
