@@ -15,6 +15,7 @@ cores instead (bounded sample per step).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import types
 import math
@@ -723,8 +724,8 @@ def run_sweep(args):
 
 def run_stack(args):
     """Time to first token of a random-init 28-layer Qwen3-1.7B-shaped stack
-    (gate after layer 13) against the same stack unpruned, at N = 16K, 64K and
-    128K: from the layer-0 hidden states in HBM to the last layer's output for
+    (gate after layer 13, or --gate-after L) against the same stack unpruned,
+    at N = 16K, 64K and 128K: from the layer-0 hidden states in HBM to the last layer's output for
     the kept rows (embedding, final norm and LM head are not part of the path).
     One JSON line per N."""
     import torch
@@ -736,6 +737,10 @@ def run_stack(args):
         sizes = [x for x in sizes if x[0] in args.stack_n]
     for n, k in sizes:
         w = synth.full_stack_64k(n=n, k=k, name=f"qwen3_1.7b_stack28_n{n}_k{k}")
+        if args.gate_after is not None:
+            # the gate after layer L (TokenGate's own default is the first layer)
+            w = dataclasses.replace(w, gate_after=args.gate_after,
+                                    name=f"qwen3_1.7b_stack28_gate{args.gate_after}_n{n}_k{k}")
         torch.cuda.reset_peak_memory_stats(dev)
         g = torch.Generator(device=dev)
         g.manual_seed(w.seed)
@@ -791,6 +796,8 @@ def main(argv=None):
     ap.add_argument("--decode", action="store_true", help="decode attention over the gated KV cache, per call")
     ap.add_argument("--ncu-decode", action="store_true", help="one decode call on a 131137-row cache (profiling)")
     ap.add_argument("--stack-n", type=int, nargs="*", default=None, help="stack sizes to run (default all)")
+    ap.add_argument("--gate-after", type=int, default=None,
+                    help="stack: the layer whose output the gate scores (default 13)")
     args = ap.parse_args(argv)
     if args.ncu_case:
         ncu_case()
