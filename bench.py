@@ -670,6 +670,60 @@ def ncu_decode_case():
     print("ncu decode case done")
 
 
+def run_batch(args):
+    """Varlen batching: eight requests of 4K-16K tokens (budget N/8, a 64-token
+    question each) through the gated step as one batch (per-request gate,
+    select and gather, then one layer call over all kept rows with attention
+    per request), against the same eight requests one at a time.  L2 flushed
+    before each timed step; one JSON line."""
+    import torch
+    from learned_token_pruning_b200 import pipeline, synth, tokengate as tg
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    base = synth.qwen3_1p7b_16k()
+    lengths = [16384, 8192, 16384, 4096, 12288, 16384, 8192, 4096]
+    ws = [dataclasses.replace(base, name=f"req{i}", seed=base.seed + 31 * i, n=n, k=n // 8, plant_len=0)
+          for i, n in enumerate(lengths)]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    reps = max(args.steps, 5) if args.steps < 200 else 20
+
+    def timed(replay):
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            replay()
+        torch.cuda.synchronize(dev)
+        total = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            replay()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            total += a.elapsed_time(b)
+        return total / reps
+
+    batch = pipeline.BatchedPrefillStep(ws, dev)
+    batch.capture()
+    t_batch = timed(batch.replay)
+    tg.tg_check_device_error()
+    del batch
+    torch.cuda.empty_cache()
+    singles = [pipeline.GatedPrefillStep(w, dev) for w in ws]
+    for st in singles:
+        st.capture()
+    t_single = timed(lambda: [st.replay() for st in singles])
+    tg.tg_check_device_error()
+    n_tok = sum(lengths)
+    print(json.dumps({"mode": "batch", "workload": "qwen3_1.7b_layer_varlen8_n4k-16k_k_n8",
+                      "requests": len(lengths), "tokens": n_tok, "prompt_lengths": lengths,
+                      "kept_rows": sum(min(w.k, w.n - w.n_question) + w.n_question for w in ws),
+                      "batch_ms": t_batch, "one_at_a_time_ms": t_single,
+                      "tokens_per_s_batch": n_tok / (t_batch * 1e-3),
+                      "tokens_per_s_one_at_a_time": n_tok / (t_single * 1e-3), "speedup": t_single / t_batch,
+                      "l2": "flushed before every timed step", "reps": reps}), flush=True)
+
+
 def run_sweep(args):
     """The other single-layer workloads (budget sweep at N=32768, K in {1024,
     4096, 8192}; 128K with K=8192): one JSON line each with the step time, the
@@ -794,6 +848,7 @@ def main(argv=None):
     ap.add_argument("--sweep", action="store_true", help="budget-sweep and 128K single-layer workloads")
     ap.add_argument("--stack", action="store_true", help="28-layer stack TTFT, pruned vs unpruned")
     ap.add_argument("--decode", action="store_true", help="decode attention over the gated KV cache, per call")
+    ap.add_argument("--batch", action="store_true", help="varlen batch of eight requests vs one at a time")
     ap.add_argument("--ncu-decode", action="store_true", help="one decode call on a 131137-row cache (profiling)")
     ap.add_argument("--stack-n", type=int, nargs="*", default=None, help="stack sizes to run (default all)")
     ap.add_argument("--gate-after", type=int, default=None,
@@ -813,6 +868,9 @@ def main(argv=None):
         return
     if args.decode:
         run_decode(args)
+        return
+    if args.batch:
+        run_batch(args)
         return
     from learned_token_pruning_b200 import synth
     w = synth.qwen3_1p7b_16k()

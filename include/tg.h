@@ -263,6 +263,27 @@ int tg_pruned_prefill_layer(const tg_layer_weights* weights, const tg_layer_shap
                             const float* ratio, int64_t m, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * The same layer over a batch of requests whose kept rows are concatenated
+ * (varlen batching; [R] §4.1 three-stage forward, per request): rows
+ * seg_rows[r] .. seg_rows[r+1]-1 of hidden_kept, pos, bias and ratio belong to
+ * request r.  Every step but attention is row-wise and runs once over all
+ * seg_rows[nseg] rows; attention runs request by request, so a row only sees
+ * keys of its own request (its causal prefix among them).
+ *   seg_rows  host int64 [nseg + 1], seg_rows[0] = 0, non-decreasing (a
+ *             request may have no rows)
+ *   ws        device workspace of tg_layer_varlen_workspace_bytes(shape,
+ *             seg_rows, nseg) bytes, 16-byte aligned
+ * Equals tg_pruned_prefill_layer called on each request's rows on its own.
+ */
+int tg_pruned_prefill_layer_varlen(const tg_layer_weights* weights, const tg_layer_shape* shape,
+                                   void* hidden_kept, const int32_t* pos, const float* bias,
+                                   const float* ratio, const int64_t* seg_rows, int32_t nseg,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes of tg_pruned_prefill_layer_varlen (0 for an invalid request). */
+size_t tg_layer_varlen_workspace_bytes(const tg_layer_shape* shape, const int64_t* seg_rows, int32_t nseg);
+
+/*
  * Row-wise linear layer of the decoder layer above, exported so that each of
  * its GEMMs can be called (and timed) on its own:
  *   epilogue TG_EPI_STORE     y = x W^T

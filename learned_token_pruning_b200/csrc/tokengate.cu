@@ -398,6 +398,23 @@ int launch_decode(int group, dim3 grid, cudaStream_t st, const tg::DecodeParams&
   }
 }
 
+// the layer's own buffers (normed rows, qkv, attention output, MLP activation)
+static size_t layer_buffers_bytes(int64_t m, const tg_layer_shape* S) {
+  const int es = dtype_size(S->dtype);
+  const size_t qkv = static_cast<size_t>(S->hq + 2 * S->hkv) * S->head_dim;
+  const size_t rows = static_cast<size_t>(m);
+  auto al = [](size_t b) { return (b + 255) / 256 * 256; };
+  // x (normed rows), qkv, attention output, MLP activation (room for the
+  // un-fused gate/up product, twice as wide as the fused SwiGLU output)
+  const size_t act = static_cast<size_t>(S->d_ff) * 2;
+  return al(rows * S->d_model * es) + al(rows * qkv * es) + al(rows * S->hq * S->head_dim * es) +
+         al(rows * act * es);
+}
+
+static int prefill_layer_impl(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden_kept, const int32_t* pos,
+                       const float* bias, const float* ratio, int64_t m, const int64_t* seg_rows, int32_t nseg,
+                       void* ws, size_t ws_bytes, void* stream);
+
 extern "C" {
 
 const char* tg_version(void) { return TG_VERSION; }
@@ -577,17 +594,8 @@ DecodePlan decode_plan(int64_t length, int hkv, int group, int head_dim) {
 size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t h, const tg_layer_shape* shape) {
   if (op == TG_OP_GATE_SCORE) return (n > 0 && d_model > 0 && h > 0) ? gate_ws_bytes(n, d_model, h) : 0;
   if (op == TG_OP_LAYER) {
-    if (!shape || m <= 0) return 0;
-    const int es = dtype_size(shape->dtype);
-    if (!es) return 0;
-    const size_t qkv = static_cast<size_t>(shape->hq + 2 * shape->hkv) * shape->head_dim;
-    const size_t rows = static_cast<size_t>(m);
-    auto al = [](size_t b) { return (b + 255) / 256 * 256; };
-    // x (normed rows), qkv, attention output, MLP activation (room for the
-    // un-fused gate/up product, twice as wide as the fused SwiGLU output)
-    const size_t act = static_cast<size_t>(shape->d_ff) * 2;
-    return al(rows * shape->d_model * es) + al(rows * qkv * es) + al(rows * shape->hq * shape->head_dim * es) +
-           al(rows * act * es) + attn_ws_bytes(m, shape->hq, shape->hkv, shape->head_dim, shape->dtype);
+    if (!shape || m <= 0 || !dtype_size(shape->dtype)) return 0;
+    return layer_buffers_bytes(m, shape) + attn_ws_bytes(m, shape->hq, shape->hkv, shape->head_dim, shape->dtype);
   }
   if (op == TG_OP_ATTENTION) {
     if (!shape || m <= 0) return 0;
@@ -994,6 +1002,42 @@ int tg_gated_decode_attention(const void* q, const void* k, int64_t ldk, const v
 int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden_kept,
                             const int32_t* pos, const float* bias, const float* ratio, int64_t m, void* ws,
                             size_t ws_bytes, void* stream) {
+  return prefill_layer_impl(W, S, hidden_kept, pos, bias, ratio, m, nullptr, 0, ws, ws_bytes, stream);
+}
+
+size_t tg_layer_varlen_workspace_bytes(const tg_layer_shape* shape, const int64_t* seg_rows, int32_t nseg) {
+  if (!shape || !seg_rows || nseg <= 0 || seg_rows[0] != 0) return 0;
+  int64_t longest = 0;
+  for (int32_t r = 0; r < nseg; ++r) {
+    if (seg_rows[r + 1] < seg_rows[r]) return 0;
+    longest = std::max(longest, seg_rows[r + 1] - seg_rows[r]);
+  }
+  const int64_t m = seg_rows[nseg];
+  if (m <= 0 || !dtype_size(shape->dtype)) return 0;
+  // + a staging copy of one request's key bias: attention loads the bias with
+  // TMA, which needs a 16-byte aligned start, and a request's rows may begin anywhere
+  return layer_buffers_bytes(m, shape) + attn_ws_bytes(longest, shape->hq, shape->hkv, shape->head_dim, shape->dtype) +
+         (static_cast<size_t>(longest) * sizeof(float) + 255) / 256 * 256;
+}
+
+int tg_pruned_prefill_layer_varlen(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden_kept,
+                                   const int32_t* pos, const float* bias, const float* ratio,
+                                   const int64_t* seg_rows, int32_t nseg, void* ws, size_t ws_bytes, void* stream) {
+  if (!seg_rows || nseg <= 0) return fail(TG_ERR_INVALID_ARG, "segments");
+  if (seg_rows[0] != 0) return fail(TG_ERR_INVALID_ARG, "seg_rows[0] must be 0");
+  for (int32_t r = 0; r < nseg; ++r)
+    if (seg_rows[r + 1] < seg_rows[r]) return fail(TG_ERR_INVALID_ARG, "seg_rows must not decrease");
+  return prefill_layer_impl(W, S, hidden_kept, pos, bias, ratio, seg_rows[nseg], seg_rows, nseg, ws, ws_bytes,
+                            stream);
+}
+
+}  // extern "C"
+
+// One decoder layer over m rows; with seg_rows (host, nseg + 1 offsets) the
+// rows are nseg independent requests and attention runs per request.
+static int prefill_layer_impl(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden_kept, const int32_t* pos,
+                       const float* bias, const float* ratio, int64_t m, const int64_t* seg_rows, int32_t nseg,
+                       void* ws, size_t ws_bytes, void* stream) {
   if (!W || !S || !hidden_kept) return fail(TG_ERR_INVALID_ARG, "null pointer");
   if (!W->w_in_norm || !W->w_qkv || !W->w_o || !W->w_post_norm || !W->w_gate_up || !W->w_down || !W->head_gain ||
       !W->head_temp)
@@ -1005,7 +1049,8 @@ int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, 
   const int es = dtype_size(S->dtype);
   if (!es) return fail(TG_ERR_INVALID_ARG, "dtype");
   if ((S->d_model * es) % 16 != 0) return fail(TG_ERR_UNSUPPORTED, "d_model rows must be a multiple of 16 bytes");
-  const size_t need = tg_workspace_bytes(TG_OP_LAYER, 0, m, 0, 0, S);
+  const size_t need = seg_rows ? tg_layer_varlen_workspace_bytes(S, seg_rows, nseg)
+                               : tg_workspace_bytes(TG_OP_LAYER, 0, m, 0, 0, S);
   if (!ws || ws_bytes < need) return fail(TG_ERR_WORKSPACE, "layer needs %zu workspace bytes", need);
   cudaStream_t st = as_stream(stream);
   const int d = S->d_model, D = S->head_dim, hq = S->hq, hkv = S->hkv, dff = S->d_ff;
@@ -1021,7 +1066,14 @@ int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, 
   void* act = base;
   base += al(size_t(m) * dff * 2 * es);
   void* attn_ws = base;
-  const size_t attn_ws_sz = attn_ws_bytes(m, hq, hkv, D, S->dtype);
+  int64_t longest = m;
+  if (seg_rows) {
+    longest = 0;
+    for (int32_t r = 0; r < nseg; ++r) longest = std::max(longest, seg_rows[r + 1] - seg_rows[r]);
+  }
+  const size_t bias_stage_sz = seg_rows ? (static_cast<size_t>(longest) * sizeof(float) + 255) / 256 * 256 : 0;
+  const size_t attn_ws_sz = need - layer_buffers_bytes(m, S) - bias_stage_sz;
+  float* bias_stage = reinterpret_cast<float*>(static_cast<uint8_t*>(attn_ws) + attn_ws_sz);
   const bool bf = S->dtype == TG_BF16;
   int rc;
   // 1. x = RMSNorm(h)
@@ -1051,13 +1103,23 @@ int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, 
     }
     if (rc) return rc;
   }
-  // 4. token-gated attention
-  {
-    const uint8_t* qb = static_cast<const uint8_t*>(qkv);
+  // 4. token-gated attention, request by request (rows of one request only
+  //    see keys of the same request)
+  for (int32_t r = 0; r < (seg_rows ? nseg : 1); ++r) {
+    const int64_t r0 = seg_rows ? seg_rows[r] : 0, mr = seg_rows ? seg_rows[r + 1] - r0 : m;
+    if (mr == 0) continue;
+    const uint8_t* qb = static_cast<const uint8_t*>(qkv) + r0 * qkv_w * es;
+    uint8_t* ab = static_cast<uint8_t*>(att) + r0 * int64_t(hq) * D * es;
+    const float* br = bias ? bias + r0 : nullptr;
+    if (br && !aligned16(br)) {
+      if (cudaMemcpyAsync(bias_stage, br, size_t(mr) * sizeof(float), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return fail(TG_ERR_CUDA, "bias staging copy: %s", cudaGetErrorString(cudaGetLastError()));
+      br = bias_stage;
+    }
     if ((rc = tg_gated_attention(qb, qkv_w, qb + int64_t(hq) * D * es, qkv_w, qb + int64_t(hq + hkv) * D * es, qkv_w,
-                                 S->dtype, m, hq, hkv, D, bias, W->head_gain, W->head_temp, ratio,
-                                 1.0f / sqrtf(float(D)), att, int64_t(hq) * D, nullptr, attn_ws_sz ? attn_ws : nullptr,
-                                 attn_ws_sz, stream)))
+                                 S->dtype, mr, hq, hkv, D, br, W->head_gain, W->head_temp,
+                                 ratio ? ratio + r0 : nullptr, 1.0f / sqrtf(float(D)), ab, int64_t(hq) * D, nullptr,
+                                 attn_ws_sz ? attn_ws : nullptr, attn_ws_sz, stream)))
       return rc;
   }
   // 5. h += a Wo^T
@@ -1089,8 +1151,6 @@ int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, 
   // 8. h += act Wd^T
   return tg_linear(act, dff, W->w_down, hidden_kept, d, S->dtype, m, d, dff, TG_EPI_RESIDUAL, stream);
 }
-
-}  // extern "C"
 
 // ---------------------------------------------------------------------------
 // Gate scores without a caller-provided workspace.

@@ -106,6 +106,96 @@ class GatedPrefillStep:
         return self.hidden_kept
 
 
+class BatchedPrefillStep:
+    """Several requests through the gated step at once (varlen batching).  Per
+    request: gate score -> top-K select -> gather, into one buffer of kept rows
+    in which request r owns rows seg_rows[r] .. seg_rows[r+1]-1; then one
+    tg_pruned_prefill_layer_varlen call over all rows (every step row-wise,
+    attention per request).  The requests share the model: the gate and layer
+    weights are those of the first workload; each request brings its own
+    hidden states, prunable mask and budget K."""
+
+    def __init__(self, ws, device="cuda", norm_eps: float = 1e-6, eps_s: float = 1e-6):
+        w0 = ws[0]
+        self.w = w0
+        self.device = torch.device(device)
+        dev, dt = self.device, synth.torch_dtype(w0.dtype)
+        self.dt, self.norm_eps, self.eps_s = dt, norm_eps, eps_s
+        gate0 = synth.gate_inputs(w0)
+        self.gate_weights = {k: gate0[k] for k in ("norm_w", "w1", "b1", "w2", "b2")}
+        self.w1 = to_device(gate0["w1"], dt, dev)
+        self.b1 = to_device(gate0["b1"], torch.float32, dev)
+        self.w2 = to_device(gate0["w2"], torch.float32, dev)
+        self.b2 = float(gate0["b2"])
+        self.reqs = []
+        seg = [0]
+        for w in ws:
+            g = synth.gate_inputs(w)
+            n_prunable = int(g["prunable"].sum())
+            m = min(w.k, n_prunable) + (w.n - n_prunable)
+            gws = tg.tg_workspace_bytes(tg.TG_OP_GATE_SCORE, n=w.n, d_model=w.d_model, h=w.gate_hidden)
+            self.reqs.append({
+                "w": w, "k": w.k, "n_prunable": n_prunable, "m": m,
+                "hidden": to_device(g["hidden"], dt, dev), "prunable": to_device(g["prunable"], torch.uint8, dev),
+                "scores": torch.empty(w.n, dtype=torch.float32, device=dev),
+                "sumsq": torch.empty(1, dtype=torch.float32, device=dev),
+                "ws_gate": torch.empty(max(gws, 16), dtype=torch.uint8, device=dev)})
+            seg.append(seg[-1] + m)
+        self.seg_rows = seg
+        total = seg[-1]
+        self.kept = torch.empty(total, dtype=torch.int32, device=dev)
+        self.hidden_kept = torch.empty(total, w0.d_model, dtype=dt, device=dev)
+        self.pos = torch.empty(total, dtype=torch.int32, device=dev)
+        self.bias = torch.empty(total, dtype=torch.float32, device=dev)
+        self.ratio = torch.empty(total, dtype=torch.float32, device=dev)
+        layer = synth.layer_weights(w0)
+        head = synth.head_params(w0)
+        self.layer = {k: to_device(v, torch.float32 if k.endswith("norm") else dt, dev) for k, v in layer.items()}
+        self.layer["head_gain"] = to_device(head["head_gain"], torch.float32, dev)
+        self.layer["head_temp"] = to_device(head["head_temp"], torch.float32, dev)
+        self.W, self.S = tg.layer_structs(self.layer, dtype=dt, d_model=w0.d_model, hq=w0.hq, hkv=w0.hkv,
+                                          head_dim=w0.head_dim, d_ff=w0.d_ff, qk_norm=w0.qk_norm,
+                                          rope_theta=w0.rope_theta, norm_eps=norm_eps)
+        self.ws_layer = torch.empty(tg.tg_layer_varlen_workspace_bytes(self.S, seg), dtype=torch.uint8, device=dev)
+
+    def rows(self, r: int) -> slice:
+        return slice(self.seg_rows[r], self.seg_rows[r + 1])
+
+    def front(self, stream=None):
+        """Gate, select and gather of every request."""
+        for r, q in enumerate(self.reqs):
+            sl = self.rows(r)
+            tg.tg_gate_score(q["hidden"], None, self.norm_eps, self.w1, self.b1, self.w2, self.b2, q["prunable"],
+                             q["scores"], q["sumsq"], q["ws_gate"], stream)
+            tg.tg_topk_select(q["scores"], q["prunable"], q["n_prunable"], q["k"], self.kept[sl], stream)
+            tg.tg_gather(q["hidden"], self.kept[sl], q["scores"], q["sumsq"], q["n_prunable"], self.eps_s,
+                         self.hidden_kept[sl], self.pos[sl], self.bias[sl], self.ratio[sl], stream)
+
+    def layer_above(self, stream=None):
+        tg.tg_pruned_prefill_layer_varlen(self.W, self.S, self.hidden_kept, self.pos, self.bias, self.ratio,
+                                          self.seg_rows, self.ws_layer, stream)
+
+    def run(self, stream=None):
+        self.front(stream)
+        self.layer_above(stream)
+        return self.hidden_kept
+
+    def capture(self):
+        self.run()
+        torch.cuda.synchronize(self.device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.run()
+        self._graph = graph
+        return graph
+
+    def replay(self):
+        if getattr(self, "_graph", None) is None:
+            self.capture()
+        self._graph.replay()
+        return self.hidden_kept
+
+
 class PrunedPrefillStack:
     """Prefill of one prompt through a decoder stack, the three-stage forward of
     "TokenGate and T2Quant: a close reading", §4.1: layers 0 .. gate_after run

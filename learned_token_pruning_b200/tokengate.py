@@ -58,6 +58,9 @@ SIGNATURES = {
     "tg_gated_decode_attention": (_INT, [_P, _P, _I64, _P, _I64, _INT, _I64, _I32, _I32, _I32, _P, _P, _P, _F, _F,
                                          _P, _P, _P, _SZ, _P]),
     "tg_decode_temperature_ratio": (_F, [_I64, _I64, _I64]),
+    "tg_pruned_prefill_layer_varlen": (_INT, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerShape), _P, _P, _P,
+                                              _P, ctypes.POINTER(_I64), _I32, _P, _SZ, _P]),
+    "tg_layer_varlen_workspace_bytes": (_SZ, [ctypes.POINTER(LayerShape), ctypes.POINTER(_I64), _I32]),
     "tg_linear": (_INT, [_P, _I64, _P, _P, _I64, _INT, _I64, _I32, _I32, _INT, _P]),
     "tg_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I32, _I32, ctypes.POINTER(LayerShape)]),
     "tg_gate_score_noalloc": (_INT, [_P, _INT, _I64, _I32, _P, _F, _P, _P, _P, _F, _I32, _P, _P, _P, _P]),
@@ -246,3 +249,23 @@ def tg_pruned_prefill_layer(W: LayerWeights, S: LayerShape, hidden_kept, pos, bi
     rc = lib().tg_pruned_prefill_layer(ctypes.byref(W), ctypes.byref(S), _ptr(hidden_kept), _ptr(pos), _ptr(bias),
                                        _ptr(ratio), m, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check("tg_pruned_prefill_layer", rc)
+
+
+def _seg_array(seg_rows):
+    arr = (_I64 * len(seg_rows))(*[int(x) for x in seg_rows])
+    return arr, len(seg_rows) - 1
+
+
+def tg_layer_varlen_workspace_bytes(S: LayerShape, seg_rows) -> int:
+    arr, nseg = _seg_array(seg_rows)
+    return int(lib().tg_layer_varlen_workspace_bytes(ctypes.byref(S), arr, nseg))
+
+
+def tg_pruned_prefill_layer_varlen(W: LayerWeights, S: LayerShape, hidden_kept, pos, bias, ratio, seg_rows, ws,
+                                   stream=None):
+    """seg_rows: host sequence of nseg + 1 row offsets (0, m_0, m_0 + m_1, ...)."""
+    arr, nseg = _seg_array(seg_rows)
+    rc = lib().tg_pruned_prefill_layer_varlen(ctypes.byref(W), ctypes.byref(S), _ptr(hidden_kept), _ptr(pos),
+                                              _ptr(bias), _ptr(ratio), arr, nseg, _ptr(ws),
+                                              ws.numel() * ws.element_size(), _stream(stream))
+    _check("tg_pruned_prefill_layer_varlen", rc)

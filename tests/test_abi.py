@@ -124,3 +124,29 @@ def test_decode_temperature_ratio_host_helper(L):
     assert tg.tg_decode_temperature_ratio(2064, 16384, 7) == pytest.approx(math.log(2072) / math.log(16392), rel=1e-6)
     assert tg.tg_decode_temperature_ratio(0, 0, 0) == 0.0
     assert tg.tg_decode_temperature_ratio(-1, 10, 0) == 0.0
+
+
+def test_varlen_layer_validation(L):
+    S = tg.LayerShape(1, 2048, 16, 8, 128, 6144, 1, 1e6, 1e-6)
+    al = lambda b: (b + 255) // 256 * 256
+    # attention space and a bias staging copy for the longest request
+    assert tg.tg_layer_varlen_workspace_bytes(S, [0, 100, 300]) - tg.tg_layer_varlen_workspace_bytes(S, [0, 300]) == \
+        tg.tg_workspace_bytes(tg.TG_OP_ATTENTION, m=200, shape=S) - tg.tg_workspace_bytes(tg.TG_OP_ATTENTION, m=300,
+                                                                                          shape=S) \
+        + al(200 * 4) - al(300 * 4)
+    assert tg.tg_layer_varlen_workspace_bytes(S, [1, 100]) == 0                # must start at 0
+    assert tg.tg_layer_varlen_workspace_bytes(S, [0, 100, 50]) == 0            # must not decrease
+    assert tg.tg_layer_varlen_workspace_bytes(S, [0, 0]) == 0                  # no rows
+    assert tg.tg_layer_varlen_workspace_bytes(S, [0, 0, 64]) > 0               # an empty request is fine
+    g = ctypes.c_void_p(256)
+    arr = (ctypes.c_int64 * 3)(0, 100, 50)
+    assert L.tg_pruned_prefill_layer_varlen(None, ctypes.byref(S), g, g, g, g, arr, 2, g, 1 << 30, None) == 1
+    W = tg.LayerWeights(*([g] * 10))
+    assert L.tg_pruned_prefill_layer_varlen(ctypes.byref(W), ctypes.byref(S), g, g, g, g, arr, 2, g, 1 << 30,
+                                            None) == 1                        # decreasing offsets
+    arr0 = (ctypes.c_int64 * 2)(5, 100)
+    assert L.tg_pruned_prefill_layer_varlen(ctypes.byref(W), ctypes.byref(S), g, g, g, g, arr0, 1, g, 1 << 30,
+                                            None) == 1                        # first offset not 0
+    ok = (ctypes.c_int64 * 2)(0, 100)
+    assert L.tg_pruned_prefill_layer_varlen(ctypes.byref(W), ctypes.byref(S), g, g, g, g, ok, 1, g, 16,
+                                            None) == 5                        # workspace too small
