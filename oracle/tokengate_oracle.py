@@ -199,6 +199,60 @@ def gated_attention(q, k, v, bias, head_gain, head_temp, ratio, sm_scale: float,
     return (out, lse) if return_lse else out
 
 
+def gated_attention_backward(q, k, v, bias, head_gain, head_temp, ratio, sm_scale: float, dout):
+    """Gradients of token-gated attention ([R] §4.1 engineering notes: the same
+    attention kernel accumulates the bias gradient back into the scorer; the
+    gate value multiplies exp(z), i.e. the bias adds to the logits).
+
+    With l_rc = temp_h * ratio_r * sm_scale * (q_r . k_c) + gain_h * bias_c for
+    c <= r, P = softmax_c(l), o_r = sum_c P_rc v_c and upstream dO:
+        dP_rc = dO_r . v_c,   dl_rc = P_rc * (dP_rc - dO_r . o_r)
+        dq_r  = sum_c dl_rc * temp_h ratio_r sm_scale * k_c
+        dk_c  = sum over the group's heads and rows of dl_rc * temp_h ratio_r sm_scale * q_r
+        dv_c  = sum over the group's heads and rows of P_rc * dO_r
+        dbias_c = sum over all heads h of gain_h * sum_r dl_rc
+        dgain_h = sum_{r,c} dl_rc * bias_c
+        dtemp_h = sum_{r,c} dl_rc * ratio_r * sm_scale * (q_r . k_c)
+    Shapes as gated_attention; dout [M, Hq, D].  Returns a dict of float64
+    arrays dq [M, Hq, D], dk/dv [M, Hkv, D], dbias [M], dgain/dtemp [Hq].
+    """
+    q = np.asarray(q, dtype=F64)
+    k = np.asarray(k, dtype=F64)
+    v = np.asarray(v, dtype=F64)
+    do = np.asarray(dout, dtype=F64)
+    m, hq, dh = q.shape
+    hkv = k.shape[1]
+    group = hq // hkv
+    bias = np.zeros(m) if bias is None else np.asarray(bias, dtype=F64)
+    ratio = np.ones(m) if ratio is None else np.asarray(ratio, dtype=F64)
+    gain = np.asarray(head_gain, dtype=F64)
+    temp = np.asarray(head_temp, dtype=F64)
+    causal = np.tril(np.ones((m, m), dtype=bool))
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    dbias = np.zeros(m)
+    dgain = np.zeros(hq)
+    dtemp = np.zeros(hq)
+    for h in range(hq):
+        g = h // group
+        z = (q[:, h, :] @ k[:, g, :].T) * sm_scale                  # [M, M]
+        a = temp[h] * ratio                                          # content scale per row
+        logits = np.where(causal, a[:, None] * z + gain[h] * bias[None, :], -np.inf)
+        p = np.exp(logits - logits.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        o = p @ v[:, g, :]
+        dp = do[:, h, :] @ v[:, g, :].T
+        dl = p * (dp - np.sum(do[:, h, :] * o, axis=1, keepdims=True))
+        dq[:, h, :] = (dl * (a * sm_scale)[:, None]) @ k[:, g, :]
+        dk[:, g, :] += (dl * (a * sm_scale)[:, None]).T @ q[:, h, :]
+        dv[:, g, :] += p.T @ do[:, h, :]
+        dbias += gain[h] * dl.sum(axis=0)
+        dgain[h] = np.sum(dl * bias[None, :])
+        dtemp[h] = np.sum(dl * ratio[:, None] * z)
+    return {"dq": dq, "dk": dk, "dv": dv, "dbias": dbias, "dgain": dgain, "dtemp": dtemp}
+
+
 # ---------------------------------------------------------------------------
 # Decode over the gated KV cache  ([R] §4.1 Gate module, temperature scaling,
 # engineering notes)

@@ -348,6 +348,52 @@ def test_decode_attention_matches_torch_sdpa_and_closed_forms():
         np.testing.assert_allclose(one[h], v[0, h // (hq // hkv)], rtol=1e-15)
 
 
+# ----------------------------------------------------------------------------- attention backward
+
+def _loss(q, k, v, bias, gain, temp, ratio, scale, w):
+    return float(np.sum(O.gated_attention(q, k, v, bias, gain, temp, ratio, scale) * w))
+
+
+def test_attention_backward_matches_finite_differences():
+    # central differences of the forward oracle, every input, in fp64
+    m, hq, hkv, dh = 7, 4, 2, 3
+    q, k, v, bias, gain, temp, ratio = _rand_attn(m, hq, hkv, dh, 21)
+    scale = 0.6
+    w = np.random.default_rng(22).standard_normal((m, hq, dh))      # dL/do
+    g = O.gated_attention_backward(q, k, v, bias, gain, temp, ratio, scale, w)
+    eps = 1e-6
+    for name, arr in (("dq", q), ("dk", k), ("dv", v), ("dbias", bias), ("dgain", gain), ("dtemp", temp)):
+        num = np.zeros_like(arr)
+        for i in np.ndindex(arr.shape):
+            old = arr[i]
+            arr[i] = old + eps
+            lp = _loss(q, k, v, bias, gain, temp, ratio, scale, w)
+            arr[i] = old - eps
+            lm = _loss(q, k, v, bias, gain, temp, ratio, scale, w)
+            arr[i] = old
+            num[i] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(g[name], num, rtol=1e-6, atol=1e-8, err_msg=name)
+
+
+def test_attention_backward_matches_torch_autograd():
+    m, hq, hkv, dh = 19, 4, 2, 8
+    q, k, v, bias, gain, temp, ratio = _rand_attn(m, hq, hkv, dh, 23)
+    scale = 1.0 / math.sqrt(dh)
+    w = np.random.default_rng(24).standard_normal((m, hq, dh))
+    g = O.gated_attention_backward(q, k, v, bias, gain, temp, ratio, scale, w)
+    t = lambda a: torch.tensor(a, dtype=torch.float64, requires_grad=True)
+    tq, tk, tv, tb, tgn, ttp = t(q), t(k), t(v), t(bias), t(gain), t(temp)
+    tr = torch.tensor(ratio, dtype=torch.float64)
+    qs = tq * (ttp[None, :, None] * tr[:, None, None])
+    mask = (tgn[:, None, None] * tb[None, None, :]).expand(hq, m, m)
+    mask = mask.masked_fill(~torch.ones(m, m, dtype=torch.bool).tril(), float("-inf"))
+    out = F.scaled_dot_product_attention(qs.transpose(0, 1)[None], tk.transpose(0, 1)[None], tv.transpose(0, 1)[None],
+                                         attn_mask=mask[None], scale=scale, enable_gqa=True)[0].transpose(0, 1)
+    (out * torch.tensor(w)).sum().backward()
+    for name, tt in (("dq", tq), ("dk", tk), ("dv", tv), ("dbias", tb), ("dgain", tgn), ("dtemp", ttp)):
+        np.testing.assert_allclose(g[name], tt.grad.numpy(), rtol=1e-10, atol=1e-12, err_msg=name)
+
+
 # ----------------------------------------------------------------------------- decoder layer
 
 def _hf_layer(w, lw, n_rows):
