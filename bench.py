@@ -645,6 +645,71 @@ def run_decode(args):
                           "l2": "flushed before every call", "ratio": ratio}), flush=True)
 
 
+def run_backward(args):
+    """Backward of token-gated attention at the kept rows of the 16K- and
+    128K-token prompts (Qwen3-1.7B heads, bf16), per call, L2 flushed before
+    each: one JSON line per size with the time, the algorithmic FLOPs (five
+    m x m x D contractions per head over the causal half: S, dP, dV, dK, dQ)
+    and their rate against the fp32 CUDA-core peak the kernels run on
+    (148 SMs x 128 FMA lanes x 2 FLOP x 1965 MHz = 74.4 TFLOP/s)."""
+    import torch
+    from learned_token_pruning_b200 import tokengate as tg
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    hq, hkv, dh = 16, 8, 128
+    simt_peak = 148 * 128 * 2 * 1965e6 / 1e12
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for name, m in (("qwen3_1.7b_attention_backward_k2064", 2064), ("qwen3_1.7b_attention_backward_k8256", 8256)):
+        g = torch.Generator(device=dev).manual_seed(m)
+        rn = lambda *s: torch.randn(*s, device=dev, generator=g)
+        q, k, v, dout = (rn(m, n * dh).to(torch.bfloat16) for n in (hq, hkv, hkv, hq))
+        bias, ratio = rn(m), torch.rand(m, device=dev, generator=g) * 0.8 + 0.2
+        gain = torch.rand(hq, device=dev, generator=g) + 0.5
+        temp = torch.rand(hq, device=dev, generator=g) * 0.4 + 0.8
+        out = torch.empty(m, hq * dh, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(hq, m, device=dev)
+        scale = 1 / math.sqrt(dh)
+        tg.tg_gated_attention(q, k, v, dh, bias, gain, temp, ratio, scale, out, lse)
+        dq = torch.empty(m, hq * dh, device=dev)
+        dk = torch.empty(m, hkv * dh, device=dev)
+        dv = torch.empty(m, hkv * dh, device=dev)
+        dbias, dgain, dtemp = torch.empty(m, device=dev), torch.empty(hq, device=dev), torch.empty(hq, device=dev)
+        ws = torch.empty(tg.attention_backward_workspace_bytes(m, hq, hkv, dh), dtype=torch.uint8, device=dev)
+        call = lambda: tg.tg_gated_attention_backward(q, k, v, out, dout, dh, bias, gain, temp, ratio, scale, lse,
+                                                      dq, dk, dv, ws, dbias=dbias, dgain=dgain, dtemp=dtemp)
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            call()
+        torch.cuda.synchronize(dev)
+        reps = max(min(args.steps, 20), 3)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        total = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            a.record(stream)
+            call()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            total += a.elapsed_time(b)
+        ms = total / reps
+        f0.record(stream)
+        tg.tg_gated_attention(q, k, v, dh, bias, gain, temp, ratio, scale, out, lse)
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        tg.tg_check_device_error()
+        flops = 10.0 * dh * hq * m * (m + 1) / 2
+        tfs = flops / (ms * 1e-3) / 1e12
+        print(json.dumps({"mode": "attention_backward", "workload": name, "rows": m, "hq": hq, "hkv": hkv,
+                          "head_dim": dh, "dtype": "bf16 in, fp32 arithmetic and gradients", "us": ms * 1e3,
+                          "forward_us": f0.elapsed_time(f1) * 1e3, "flops": flops, "tflops": tfs,
+                          "frac_fp32_simt": tfs / simt_peak, "frac_bf16_tensor": tfs / peaks["bf16_tflops"],
+                          "peak_source": peaks["source"], "l2": "flushed before every call"}), flush=True)
+
+
 def ncu_decode_case():
     """One decode-attention call on a 131137-row cache (16/8 heads x 128, bf16;
     the unpruned 128K-token prompt's cache) after a warm-up call, each after an
@@ -850,6 +915,7 @@ def main(argv=None):
     ap.add_argument("--decode", action="store_true", help="decode attention over the gated KV cache, per call")
     ap.add_argument("--batch", action="store_true", help="varlen batch of eight requests vs one at a time")
     ap.add_argument("--ncu-decode", action="store_true", help="one decode call on a 131137-row cache (profiling)")
+    ap.add_argument("--backward", action="store_true", help="backward of gated attention at the kept-row counts")
     ap.add_argument("--stack-n", type=int, nargs="*", default=None, help="stack sizes to run (default all)")
     ap.add_argument("--gate-after", type=int, default=None,
                     help="stack: the layer whose output the gate scores (default 13)")
@@ -871,6 +937,9 @@ def main(argv=None):
         return
     if args.batch:
         run_batch(args)
+        return
+    if args.backward:
+        run_backward(args)
         return
     from learned_token_pruning_b200 import synth
     w = synth.qwen3_1p7b_16k()

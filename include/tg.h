@@ -182,6 +182,35 @@ int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk,
                        void* out, int64_t ldo, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Backward of tg_gated_attention ([R] §4.1 engineering notes: the biased
+ * attention kernel also returns the bias gradient to the scorer).  With
+ * l_rc, P = softmax_c(l) and out as in the forward and upstream dout:
+ *     dP_rc = dout_r . v_c,   dl_rc = P_rc (dP_rc - dout_r . out_r)
+ *     dq_r  = sum_c dl_rc head_temp[h] ratio[r] sm_scale k_c
+ *     dk_c, dv_c: sums over the query heads of c's KV head and over rows
+ *             of dl_rc head_temp[h] ratio[r] sm_scale q_r and of P_rc dout_r
+ *     dbias_c = sum over all heads h of head_gain[h] sum_r dl_rc
+ *     dgain_h = sum_{r,c} dl_rc bias[c];  dtemp_h = sum_{r,c} dl_rc ratio[r] sm_scale (q_r . k_c)
+ *   q, k, v, out, dout  device, dtype, strided rows as in the forward
+ *   lse   device fp32 [hq][m], the forward's (natural-log) log-sum-exp
+ *   dq    device fp32 [m][hq*head_dim];  dk, dv device fp32 [m][hkv*head_dim]
+ *   dbias device fp32 [m] or NULL;  dgain, dtemp device fp32 [hq] or NULL
+ *   ws    device workspace of tg_workspace_bytes(TG_OP_ATTENTION_BWD, 0, m, 0, 0,
+ *         shape) bytes, 16-byte aligned
+ * P is recomputed from lse.  CUDA cores, fp32 arithmetic; deterministic
+ * (every gradient is written by one thread; cross-block sums go through the
+ * workspace in a fixed order).  head_dim in {64, 128}; hq % hkv == 0.
+ */
+int tg_gated_attention_backward(const void* q, int64_t ldq, const void* k, int64_t ldk,
+                                const void* v, int64_t ldv, const void* out, int64_t ldo,
+                                const void* dout, int64_t lddo, int dtype, int64_t m,
+                                int32_t hq, int32_t hkv, int32_t head_dim, const float* bias,
+                                const float* head_gain, const float* head_temp, const float* ratio,
+                                float sm_scale, const float* lse, float* dq, float* dk, float* dv,
+                                float* dbias, float* dgain, float* dtemp,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/*
  * One decode step of token-gated attention over the gated KV cache ([R] §4.1
  * Gate module: tokens produced while decoding are not prunable and score 0;
  * §4.1 engineering notes: at decode time the gate term is an additive mask on
@@ -301,12 +330,12 @@ enum { TG_EPI_STORE = 0, TG_EPI_RESIDUAL = 1, TG_EPI_SWIGLU = 2 };
 int tg_linear(const void* x, int64_t ldx, const void* w, void* y, int64_t ldy, int dtype,
               int64_t m, int32_t n_out, int32_t k_in, int epilogue, void* stream);
 
-enum { TG_OP_GATE_SCORE = 0, TG_OP_LAYER = 1, TG_OP_ATTENTION = 2, TG_OP_DECODE = 3 };
+enum { TG_OP_GATE_SCORE = 0, TG_OP_LAYER = 1, TG_OP_ATTENTION = 2, TG_OP_DECODE = 3, TG_OP_ATTENTION_BWD = 4 };
 
 /* Workspace bytes needed by an op: TG_OP_GATE_SCORE uses n, d_model and h;
  * TG_OP_LAYER and TG_OP_ATTENTION use m and shape (TG_OP_ATTENTION reads its
  * dtype, hq, hkv and head_dim); TG_OP_DECODE uses m = the cache length and
- * shape's hq, hkv and head_dim.  Returns 0 for an invalid request, and 0 for
+ * shape's hq, hkv and head_dim; TG_OP_ATTENTION_BWD uses m and shape's hq and hkv.  Returns 0 for an invalid request, and 0 for
  * TG_OP_ATTENTION when the attention needs no workspace. */
 size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t h, const tg_layer_shape* shape);
 

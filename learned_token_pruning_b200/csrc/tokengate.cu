@@ -21,6 +21,7 @@
 #include <vector>
 
 #include "../../include/tg.h"
+#include "attn_bwd.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
 #include "gate_tc.cuh"
@@ -601,6 +602,12 @@ size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t
     if (!shape || m <= 0) return 0;
     return attn_ws_bytes(m, shape->hq, shape->hkv, shape->head_dim, shape->dtype);
   }
+  if (op == TG_OP_ATTENTION_BWD) {
+    if (!shape || m <= 0 || shape->hq <= 0 || shape->hkv <= 0) return 0;
+    auto al = [](size_t b) { return (b + 255) / 256 * 256; };
+    const size_t nkb = static_cast<size_t>((m + tg::kBwdBlk - 1) / tg::kBwdBlk);
+    return al(size_t(shape->hq) * m * 4) + al(size_t(shape->hkv) * m * 4) + al(size_t(shape->hq) * nkb * 2 * 4);
+  }
   if (op == TG_OP_DECODE) {
     if (!shape || m <= 0 || shape->hkv <= 0 || shape->hq % shape->hkv) return 0;
     return decode_plan(m, shape->hkv, shape->hq / shape->hkv, shape->head_dim).bytes;
@@ -941,6 +948,93 @@ int tg_linear(const void* x, int64_t ldx, const void* w, void* y, int64_t ldy, i
     else tg::k_gemm_simt<B, false><<<grid, 256, 0, st>>>(xa, ldx, wa, ya, ldy, mm, n_out, k_in);
   }
   return check_launch("k_gemm_simt");
+}
+
+int tg_gated_attention_backward(const void* q, int64_t ldq, const void* k, int64_t ldk, const void* v, int64_t ldv,
+                                const void* out, int64_t ldo, const void* dout, int64_t lddo, int dtype, int64_t m,
+                                int32_t hq, int32_t hkv, int32_t head_dim, const float* bias, const float* head_gain,
+                                const float* head_temp, const float* ratio, float sm_scale, const float* lse, float* dq,
+                                float* dk, float* dv, float* dbias, float* dgain, float* dtemp, void* ws,
+                                size_t ws_bytes, void* stream) {
+  if (!q || !k || !v || !out || !dout || !head_gain || !head_temp || !lse || !dq || !dk || !dv)
+    return fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (m <= 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0) return fail(TG_ERR_INVALID_ARG, "bad m / heads");
+  if (m >= (int64_t(1) << 31)) return fail(TG_ERR_UNSUPPORTED, "m must be < 2^31");
+  if (head_dim != 64 && head_dim != 128) return fail(TG_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "dtype");
+  if (ldq < int64_t(hq) * head_dim || ldo < int64_t(hq) * head_dim || lddo < int64_t(hq) * head_dim ||
+      ldk < int64_t(hkv) * head_dim || ldv < int64_t(hkv) * head_dim)
+    return fail(TG_ERR_SHAPE, "leading dimension smaller than the heads it holds");
+  tg_layer_shape sh{};
+  sh.hq = hq;
+  sh.hkv = hkv;
+  sh.head_dim = head_dim;
+  sh.dtype = dtype;
+  const size_t need = tg_workspace_bytes(TG_OP_ATTENTION_BWD, 0, m, 0, 0, &sh);
+  if (!ws || ws_bytes < need) return fail(TG_ERR_WORKSPACE, "attention backward needs %zu workspace bytes", need);
+  if (!aligned16(ws)) return fail(TG_ERR_ALIGN, "workspace must be 16-byte aligned");
+  cudaStream_t st = as_stream(stream);
+  auto al = [](size_t b) { return (b + 255) / 256 * 256; };
+  tg::AttnBwdParams p{};
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = out;
+  p.dout = dout;
+  p.ldq = ldq;
+  p.ldk = ldk;
+  p.ldv = ldv;
+  p.ldo = ldo;
+  p.lddo = lddo;
+  p.m = static_cast<int>(m);
+  p.hq = hq;
+  p.hkv = hkv;
+  p.group = hq / hkv;
+  p.bias = bias;
+  p.gain = head_gain;
+  p.temp = head_temp;
+  p.ratio = ratio;
+  p.lse = lse;
+  p.sm_scale = sm_scale;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.dbias = dbias;
+  p.dgain = dgain;
+  p.dtemp = dtemp;
+  p.nkb = static_cast<int>((m + tg::kBwdBlk - 1) / tg::kBwdBlk);
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  p.rowdot = reinterpret_cast<float*>(wb);
+  wb += al(size_t(hq) * m * 4);
+  p.dbias_part = reinterpret_cast<float*>(wb);
+  wb += al(size_t(hkv) * m * 4);
+  p.dgt_part = reinterpret_cast<float*>(wb);
+  const int nqb = p.nkb;
+  auto run = [&](auto rowdot, auto kv, auto qk, int D) -> int {
+    const size_t DP = size_t(D) + 1;
+    const size_t smem_kv = (4 * tg::kBwdBlk * DP + 3 * tg::kBwdBlk * (tg::kBwdBlk + 1) + tg::kBwdThreads) * 4;
+    const size_t smem_q = (4 * tg::kBwdBlk * DP + tg::kBwdBlk * (tg::kBwdBlk + 1)) * 4;
+    int rc = set_smem(kv, smem_kv);
+    if (!rc) rc = set_smem(qk, smem_q);
+    if (rc) return rc;
+    rowdot<<<unsigned((m * hq + 7) / 8), 256, 0, st>>>(p);
+    if ((rc = check_launch("k_attn_bwd_rowdot"))) return rc;
+    kv<<<unsigned(hkv * p.nkb), tg::kBwdThreads, smem_kv, st>>>(p);
+    if ((rc = check_launch("k_attn_bwd_kv"))) return rc;
+    qk<<<unsigned(hq * nqb), tg::kBwdThreads, smem_q, st>>>(p);
+    if ((rc = check_launch("k_attn_bwd_q"))) return rc;
+    tg::k_attn_bwd_final<<<unsigned((std::max<int64_t>(m, hq) + 255) / 256), 256, 0, st>>>(p);
+    return check_launch("k_attn_bwd_final");
+  };
+  if (dtype == TG_BF16)
+    return head_dim == 128 ? run(tg::k_attn_bwd_rowdot<__nv_bfloat16, 128>, tg::k_attn_bwd_kv<__nv_bfloat16, 128>,
+                                 tg::k_attn_bwd_q<__nv_bfloat16, 128>, 128)
+                           : run(tg::k_attn_bwd_rowdot<__nv_bfloat16, 64>, tg::k_attn_bwd_kv<__nv_bfloat16, 64>,
+                                 tg::k_attn_bwd_q<__nv_bfloat16, 64>, 64);
+  return head_dim == 128 ? run(tg::k_attn_bwd_rowdot<float, 128>, tg::k_attn_bwd_kv<float, 128>,
+                               tg::k_attn_bwd_q<float, 128>, 128)
+                         : run(tg::k_attn_bwd_rowdot<float, 64>, tg::k_attn_bwd_kv<float, 64>,
+                               tg::k_attn_bwd_q<float, 64>, 64);
 }
 
 float tg_decode_temperature_ratio(int64_t m_kept, int64_t n_prompt, int64_t t) {

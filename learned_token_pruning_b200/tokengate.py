@@ -18,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libtokengate.so")
 
 TG_F32, TG_BF16 = 0, 1
-TG_OP_GATE_SCORE, TG_OP_LAYER, TG_OP_ATTENTION, TG_OP_DECODE = 0, 1, 2, 3
+TG_OP_GATE_SCORE, TG_OP_LAYER, TG_OP_ATTENTION, TG_OP_DECODE, TG_OP_ATTENTION_BWD = 0, 1, 2, 3, 4
 STATUS = {0: "TG_OK", 1: "TG_ERR_INVALID_ARG", 2: "TG_ERR_SHAPE", 3: "TG_ERR_ALIGN", 4: "TG_ERR_UNSUPPORTED",
           5: "TG_ERR_WORKSPACE", 6: "TG_ERR_CUDA", 7: "TG_ERR_DEVICE_TIMEOUT", 8: "TG_ERR_DEVICE_CHECK"}
 
@@ -55,6 +55,8 @@ SIGNATURES = {
                                   _P, _I64, _P, _P, _SZ, _P]),
     "tg_pruned_prefill_layer": (_INT, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerShape), _P, _P, _P, _P,
                                        _I64, _P, _SZ, _P]),
+    "tg_gated_attention_backward": (_INT, [_P, _I64, _P, _I64, _P, _I64, _P, _I64, _P, _I64, _INT, _I64, _I32, _I32,
+                                           _I32, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tg_gated_decode_attention": (_INT, [_P, _P, _I64, _P, _I64, _INT, _I64, _I32, _I32, _I32, _P, _P, _P, _F, _F,
                                          _P, _P, _P, _SZ, _P]),
     "tg_decode_temperature_ratio": (_F, [_I64, _I64, _I64]),
@@ -195,6 +197,32 @@ def tg_gated_attention(q, k, v, head_dim: int, bias, head_gain, head_temp, ratio
                                   _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0,
                                   _stream(stream))
     _check("tg_gated_attention", rc)
+
+
+def attention_backward_workspace_bytes(m: int, hq: int, hkv: int, head_dim: int) -> int:
+    shape = LayerShape(dtype=TG_BF16, d_model=0, hq=hq, hkv=hkv, head_dim=head_dim, d_ff=0, qk_norm=0,
+                       rope_theta=0.0, norm_eps=0.0)
+    return tg_workspace_bytes(TG_OP_ATTENTION_BWD, m=m, shape=shape)
+
+
+def tg_gated_attention_backward(q, k, v, out, dout, head_dim: int, bias, head_gain, head_temp, ratio,
+                                sm_scale: float, lse, dq, dk, dv, ws, dbias=None, dgain=None, dtemp=None,
+                                stream=None):
+    """q/k/v/out/dout 2-D row views as in tg_gated_attention; dq/dk/dv fp32 [m, heads*head_dim]."""
+    qp, ldq = _row_view(q)
+    kp, ldk = _row_view(k)
+    vp, ldv = _row_view(v)
+    op, ldo = _row_view(out)
+    gp, lddo = _row_view(dout)
+    m = q.shape[0]
+    hq = q.shape[1] // head_dim
+    hkv = k.shape[1] // head_dim
+    rc = lib().tg_gated_attention_backward(qp, ldq, kp, ldk, vp, ldv, op, ldo, gp, lddo, _dtype(q), m, hq, hkv,
+                                           head_dim, _ptr(bias), _ptr(head_gain), _ptr(head_temp), _ptr(ratio),
+                                           float(sm_scale), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbias),
+                                           _ptr(dgain), _ptr(dtemp), _ptr(ws), ws.numel() * ws.element_size(),
+                                           _stream(stream))
+    _check("tg_gated_attention_backward", rc)
 
 
 def decode_workspace_bytes(length: int, hq: int, hkv: int, head_dim: int) -> int:

@@ -150,3 +150,31 @@ def test_varlen_layer_validation(L):
     ok = (ctypes.c_int64 * 2)(0, 100)
     assert L.tg_pruned_prefill_layer_varlen(ctypes.byref(W), ctypes.byref(S), g, g, g, g, ok, 1, g, 16,
                                             None) == 5                        # workspace too small
+
+
+def test_attention_backward_validation_and_workspace(L):
+    g = ctypes.c_void_p(256)
+    f = L.tg_gated_attention_backward
+
+    def call(m=100, hq=16, hkv=8, dh=128, ldq=2048, ldk=1024, dtype=1, ws=g, ws_bytes=1 << 30, lse=g):
+        # q, ldq, k, ldk, v, ldv, o, ldo, dO, lddo, dtype, m, hq, hkv, head_dim, bias, gain, temp, ratio, scale,
+        # lse, dq, dk, dv, dbias, dgain, dtemp, ws, ws_bytes, stream
+        return f(g, ldq, g, ldk, g, ldk, g, ldq, g, ldq, dtype, m, hq, hkv, dh, None, g, g, None, 0.1, lse, g, g, g,
+                 None, None, None, ws, ws_bytes, None)
+
+    assert call(lse=None) == 1                 # the forward's log-sum-exp is required
+    assert call(m=0) == 1
+    assert call(hkv=6) == 1                    # hq % hkv
+    assert call(dh=96) == 4
+    assert call(dtype=7) == 1
+    assert call(ldq=1000) == 2                 # leading dimension below the heads
+    assert call(ws_bytes=16) == 5
+    assert call(ws=None) == 5
+    assert call(ws=ctypes.c_void_p(260)) == 3  # workspace alignment
+    al = lambda b: (b + 255) // 256 * 256
+    # per query head and row the dO . o row dot, per KV head and key the dbias partial,
+    # per query head and key block of 32 the (dgain, dtemp) partials
+    for m in (1, 31, 32, 33, 2064):
+        nkb = (m + 31) // 32
+        assert tg.attention_backward_workspace_bytes(m, 16, 8, 128) == al(16 * m * 4) + al(8 * m * 4) + al(16 * nkb * 8)
+    assert tg.tg_workspace_bytes(tg.TG_OP_ATTENTION_BWD, m=0) == 0
