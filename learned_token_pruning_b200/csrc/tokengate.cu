@@ -22,6 +22,7 @@
 
 #include "../../include/tg.h"
 #include "attn_bwd.cuh"
+#include "attn_bwd_tc.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
 #include "gate_tc.cuh"
@@ -1010,6 +1011,43 @@ int tg_gated_attention_backward(const void* q, int64_t ldq, const void* k, int64
   wb += al(size_t(hkv) * m * 4);
   p.dgt_part = reinterpret_cast<float*>(wb);
   const int nqb = p.nkb;
+  // bf16 operands that TMA can read go to the tensor cores
+  const bool tc = dtype == TG_BF16 && aligned16(q) && aligned16(k) && aligned16(v) && aligned16(dout) &&
+                  ldq % 8 == 0 && ldk % 8 == 0 && ldv % 8 == 0 && lddo % 8 == 0 && aligned16(dq) &&
+                  aligned16(dk) && aligned16(dv) && (!bias || aligned16(bias));
+  if (tc) {
+    auto run_tc = [&](auto rowdot, auto kv, auto qk, size_t smem_kv, size_t smem_q, int D) -> int {
+      CUtensorMap tq128, tdo128, tk64, tv64, tk128, tv128, tq64, tdo64, tb;
+      std::memset(&tb, 0, sizeof(tb));
+      int rc = make_map(&tq128, q, uint64_t(hq) * D, uint64_t(m), uint64_t(ldq) * 2, 128);
+      if (!rc) rc = make_map(&tdo128, dout, uint64_t(hq) * D, uint64_t(m), uint64_t(lddo) * 2, 128);
+      if (!rc) rc = make_map(&tq64, q, uint64_t(hq) * D, uint64_t(m), uint64_t(ldq) * 2, 64);
+      if (!rc) rc = make_map(&tdo64, dout, uint64_t(hq) * D, uint64_t(m), uint64_t(lddo) * 2, 64);
+      if (!rc) rc = make_map(&tk64, k, uint64_t(hkv) * D, uint64_t(m), uint64_t(ldk) * 2, 64);
+      if (!rc) rc = make_map(&tv64, v, uint64_t(hkv) * D, uint64_t(m), uint64_t(ldv) * 2, 64);
+      if (!rc) rc = make_map(&tk128, k, uint64_t(hkv) * D, uint64_t(m), uint64_t(ldk) * 2, 128);
+      if (!rc) rc = make_map(&tv128, v, uint64_t(hkv) * D, uint64_t(m), uint64_t(ldv) * 2, 128);
+      if (!rc && bias) rc = make_map_1d_f32(&tb, bias, uint64_t(m), 64);
+      if (!rc) rc = set_smem(kv, smem_kv);
+      if (!rc) rc = set_smem(qk, smem_q);
+      if (rc) return rc;
+      const int nqb128 = static_cast<int>((m + 127) / 128);
+      rowdot<<<unsigned((m * hq + 7) / 8), 256, 0, st>>>(p);
+      if ((rc = check_launch("k_attn_bwd_rowdot"))) return rc;
+      kv<<<unsigned(hkv * nqb128), tg::kBwdTcThreads, smem_kv, st>>>(tk128, tv128, tq64, tdo64, p);
+      if ((rc = check_launch("k_attn_bwd_kv_tc"))) return rc;
+      p.nkb = nqb128;  // dgain / dtemp partials per block of 128 rows
+      qk<<<unsigned(hq * nqb128), tg::kBwdTcThreads, smem_q, st>>>(tq128, tdo128, tk64, tv64, tb, p);
+      if ((rc = check_launch("k_attn_bwd_dq_tc"))) return rc;
+      tg::k_attn_bwd_final<<<unsigned((std::max<int64_t>(m, hq) + 255) / 256), 256, 0, st>>>(p);
+      return check_launch("k_attn_bwd_final");
+    };
+    return head_dim == 128
+               ? run_tc(tg::k_attn_bwd_rowdot<__nv_bfloat16, 128>, tg::k_attn_bwd_kv_tc<128>,
+                        tg::k_attn_bwd_dq_tc<128>, tg::BwdKvCfg<128>::kSmem, tg::BwdDqCfg<128>::kSmem, 128)
+               : run_tc(tg::k_attn_bwd_rowdot<__nv_bfloat16, 64>, tg::k_attn_bwd_kv_tc<64>,
+                        tg::k_attn_bwd_dq_tc<64>, tg::BwdKvCfg<64>::kSmem, tg::BwdDqCfg<64>::kSmem, 64);
+  }
   auto run = [&](auto rowdot, auto kv, auto qk, int D) -> int {
     const size_t DP = size_t(D) + 1;
     const size_t smem_kv = (4 * tg::kBwdBlk * DP + 3 * tg::kBwdBlk * (tg::kBwdBlk + 1) + tg::kBwdThreads) * 4;

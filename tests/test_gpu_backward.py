@@ -39,7 +39,7 @@ def _case(m, hq, hkv, dh, dtype, seed, with_bias=True, with_ratio=True):
     return q, k, v, do, bias, ratio, gain, temp
 
 
-def _gpu(q, k, v, do, bias, ratio, gain, temp, dtype, fused=False):
+def _gpu(q, k, v, do, bias, ratio, gain, temp, dtype, fused=False, pad=0):
     dt = synth.torch_dtype(dtype)
     m, hq, dh = q.shape
     hkv = k.shape[1]
@@ -48,13 +48,22 @@ def _gpu(q, k, v, do, bias, ratio, gain, temp, dtype, fused=False):
         # q, k, v as column ranges of one [m][(hq + 2 hkv) dh] buffer, as the layer holds them
         buf = torch.from_numpy(np.concatenate([q.reshape(m, -1), k.reshape(m, -1), v.reshape(m, -1)], 1)).to(DEV, dt)
         qd, kd, vd = buf[:, :hq * dh], buf[:, hq * dh:(hq + hkv) * dh], buf[:, (hq + hkv) * dh:]
+    elif pad:
+        # rows padded by `pad` elements: a row stride TMA cannot take (the CUDA-core path)
+        def padded(a):
+            buf = torch.zeros(m, a.shape[1] * dh + pad, dtype=dt, device=DEV)
+            buf[:, :a.shape[1] * dh] = torch.from_numpy(a.reshape(m, -1)).to(DEV, dt)
+            return buf[:, :a.shape[1] * dh]
+        qd, kd, vd = (padded(a) for a in (q, k, v))
     else:
         qd, kd, vd = (torch.from_numpy(a.reshape(m, -1)).to(DEV, dt) for a in (q, k, v))
     dod = torch.from_numpy(do.reshape(m, -1)).to(DEV, dt)
     out = torch.empty(m, hq * dh, dtype=dt, device=DEV)
     lse = torch.empty(hq, m, dtype=torch.float32, device=DEV)
     scale = 1.0 / math.sqrt(dh)
-    tg.tg_gated_attention(qd, kd, vd, dh, t(bias), t(gain), t(temp), t(ratio), scale, out, lse)
+    # (the forward needs TMA-aligned rows: it reads dense copies of padded views)
+    dense = lambda x: torch.empty(x.shape, dtype=x.dtype, device=DEV).copy_(x)
+    tg.tg_gated_attention(dense(qd), dense(kd), dense(vd), dh, t(bias), t(gain), t(temp), t(ratio), scale, out, lse)
     g = {"dq": torch.full((m, hq * dh), float("nan"), device=DEV),
          "dk": torch.full((m, hkv * dh), float("nan"), device=DEV),
          "dv": torch.full((m, hkv * dh), float("nan"), device=DEV),
@@ -132,3 +141,18 @@ def test_backward_bias_gradient_sums_to_zero_over_keys_per_row():
 def test_backward_workload_kept_rows():
     # the 2064 kept rows of the 16K-token prompt, Qwen3-1.7B attention heads
     _check(2064, 16, 8, 128, "bf16", seed=2064)
+
+
+@pytest.mark.parametrize("m", [1, 70, 300])
+def test_backward_bf16_unaligned_rows_use_the_cuda_core_kernels(m):
+    # a row stride of hq * D + 4 elements is not 16-byte aligned: the CUDA-core
+    # kernels take it, and agree with the oracle and with the tensor-core path
+    hq, hkv, dh = 4, 2, 64
+    q, k, v, do, bias, ratio, gain, temp = _case(m, hq, hkv, dh, "bf16", seed=m + 5)
+    got = _gpu(q, k, v, do, bias, ratio, gain, temp, "bf16", pad=4)
+    want = O.gated_attention_backward(q, k, v, bias, gain, temp, ratio, 1.0 / math.sqrt(dh), do)
+    _compare(got, want, "bf16", m, hq, hkv, dh)
+    tc = _gpu(q, k, v, do, bias, ratio, gain, temp, "bf16")
+    for n in NAMES:
+        scale = max(np.max(np.abs(got[n])), FLOOR)
+        assert np.max(np.abs(tc[n] - got[n])) <= 2 * TOL["bf16"] * scale, n
