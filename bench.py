@@ -709,6 +709,37 @@ def run_backward(args):
                           "peak_source": peaks["source"], "l2": "flushed before every call"}), flush=True)
 
 
+def ncu_backward_case():
+    """One backward call of gated attention at 2064 kept rows (16/8 heads x 128,
+    bf16) after a warm-up call, each after an L2 flush, for profiler captures
+    of k_attn_bwd_kv_tc and k_attn_bwd_dq_tc."""
+    import torch
+    from learned_token_pruning_b200 import tokengate as tg
+    dev, hq, hkv, dh, m = "cuda", 16, 8, 128, 2064
+    g = torch.Generator(device=dev).manual_seed(2)
+    rn = lambda *s: torch.randn(*s, device=dev, generator=g)
+    q, k, v, dout = (rn(m, n * dh).to(torch.bfloat16) for n in (hq, hkv, hkv, hq))
+    bias, ratio = rn(m), torch.rand(m, device=dev, generator=g) * 0.8 + 0.2
+    gain = torch.rand(hq, device=dev, generator=g) + 0.5
+    temp = torch.rand(hq, device=dev, generator=g) * 0.4 + 0.8
+    out = torch.empty(m, hq * dh, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(hq, m, device=dev)
+    scale = 1 / math.sqrt(dh)
+    tg.tg_gated_attention(q, k, v, dh, bias, gain, temp, ratio, scale, out, lse)
+    dq = torch.empty(m, hq * dh, device=dev)
+    dk = torch.empty(m, hkv * dh, device=dev)
+    dv = torch.empty(m, hkv * dh, device=dev)
+    dbias, dgain, dtemp = torch.empty(m, device=dev), torch.empty(hq, device=dev), torch.empty(hq, device=dev)
+    ws = torch.empty(tg.attention_backward_workspace_bytes(m, hq, hkv, dh), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        flush.zero_()
+        tg.tg_gated_attention_backward(q, k, v, out, dout, dh, bias, gain, temp, ratio, scale, lse, dq, dk, dv, ws,
+                                       dbias=dbias, dgain=dgain, dtemp=dtemp)
+    torch.cuda.synchronize()
+    assert tg.tg_check_device_error() == 0
+
+
 def ncu_decode_case():
     """One decode-attention call on a 131137-row cache (16/8 heads x 128, bf16;
     the unpruned 128K-token prompt's cache) after a warm-up call, each after an
@@ -915,6 +946,7 @@ def main(argv=None):
     ap.add_argument("--batch", action="store_true", help="varlen batch of eight requests vs one at a time")
     ap.add_argument("--ncu-decode", action="store_true", help="one decode call on a 131137-row cache (profiling)")
     ap.add_argument("--backward", action="store_true", help="backward of gated attention at the kept-row counts")
+    ap.add_argument("--ncu-backward", action="store_true", help="one backward call at 2064 rows (profiling)")
     ap.add_argument("--stack-n", type=int, nargs="*", default=None, help="stack sizes to run (default all)")
     ap.add_argument("--gate-after", type=int, default=None,
                     help="stack: the layer whose output the gate scores (default 13)")
@@ -924,6 +956,9 @@ def main(argv=None):
         return
     if args.ncu_decode:
         ncu_decode_case()
+        return
+    if args.ncu_backward:
+        ncu_backward_case()
         return
     if args.sweep:
         run_sweep(args)

@@ -50,6 +50,8 @@ struct AttnBwdParams {
   float* dbias_part;   // workspace [hkv][m]
   float* dgt_part;     // workspace [hq][nkb][2]: (dgain, dtemp) partials
   int nkb;             // key blocks
+  float4* rowpar;      // workspace [hq][m_pad] (tensor-core kernels): per-row constants
+  int m_pad;           // m rounded up to 128
 };
 
 template <typename T>

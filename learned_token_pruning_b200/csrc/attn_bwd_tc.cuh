@@ -22,8 +22,11 @@
 //   S^T = K Q^T and dP^T = V dO^T (one thread per key), P^T and dS^T as bf16
 //   pairs over their own columns, then dV += P^T dO and dK += dS^T Q as
 //   TS-MMAs; both accumulators stay in tensor memory over the whole walk.  The
-//   per-row constants of a tile (a_r, lse_r, D_r) are written by the producer
-//   warp into the same stage as the Q / dO tiles and ride on its barrier.
+//   per-row constants of a tile (from k_attn_bwd_prep) come by TMA into the
+//   same stage as the Q / dO tiles.
+// k_attn_bwd_prep: D_r and the per-row constants (a_r sm_scale log2 e,
+//   -lse_r log2 e, D_r, a_r sm_scale) of every head and row, rows past m
+//   masked (P = 0 there), so neither kernel above reads lse or ratio per tile.
 //
 // Warps: 0-7 elementwise (two warpgroups), 8 TMA producer, 9 TMEM allocator
 // and single-thread MMA issuer.  Every wait is bounded (kErrWaitAttention).
@@ -39,7 +42,7 @@ constexpr int kBwdTcThreads = 320;
 
 template <int D>
 struct BwdDqCfg {
-  static constexpr int BM = 128, BN = 64, kStages = 3;
+  static constexpr int BM = 128, BN = 64, kStages = 4;
   static constexpr int kQBytes = BM * D * 2;   // a Q or dO block (128 rows)
   static constexpr int kQBlk = BM * 128;       // one 64-column box of it
   static constexpr int kKVBytes = BN * D * 2;  // a K or V tile (64 keys)
@@ -58,7 +61,7 @@ struct BwdDqCfg {
 
 template <int D>
 struct BwdKvCfg {
-  static constexpr int BK = 128, BR = 64, kStages = 3;
+  static constexpr int BK = 128, BR = 64, kStages = 4;
   static constexpr int kKBytes = BK * D * 2;  // the K or V block (128 keys)
   static constexpr int kKBlk = BK * 128;
   static constexpr int kRBytes = BR * D * 2;  // a Q or dO tile (64 rows)
@@ -66,8 +69,8 @@ struct BwdKvCfg {
   static constexpr size_t kOffV = kKBytes;
   static constexpr size_t kOffQ = 2 * size_t(kKBytes);
   static constexpr size_t kOffDO = kOffQ + kStages * size_t(kRBytes);
-  static constexpr size_t kOffPar = kOffDO + kStages * size_t(kRBytes);  // [stage][4][64] floats
-  static constexpr size_t kOffRed = kOffPar + kStages * 4 * BR * 4;      // [128] floats
+  static constexpr size_t kOffPar = kOffDO + kStages * size_t(kRBytes);  // [stage][64 rows] float4
+  static constexpr size_t kOffRed = kOffPar + kStages * BR * 16;         // [128] floats
   static constexpr size_t kOffBars = kOffRed + BK * 4;
   static constexpr size_t kData = kOffBars + 256;
   static constexpr size_t kSmem = 1024 + (kData < 120 * 1024 ? 120 * 1024 : kData);
@@ -78,6 +81,38 @@ struct BwdKvCfg {
 // whose two 32-wide halves were packed into the first 16 columns of each half
 __device__ __forceinline__ uint32_t bwd_packed_col(int kk) {
   return static_cast<uint32_t>(kk < 2 ? kk * 8 : 32 + (kk - 2) * 8);
+}
+
+// ---------------------------------------------------------------------------
+// Per-row constants: one warp per (row, head), rows m .. m_pad - 1 masked
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) k_attn_bwd_prep(AttnBwdParams p) {
+  const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (w >= p.m_pad * p.hq) return;  // warp-uniform
+  const int r = w / p.hq, h = w % p.hq;
+  float4* dst = p.rowpar + int64_t(h) * p.m_pad + r;
+  if (r >= p.m) {
+    if (lane == 0) *dst = make_float4(0.0f, -INFINITY, 0.0f, 0.0f);
+    return;
+  }
+  const __nv_bfloat16* go = static_cast<const __nv_bfloat16*>(p.dout) + int64_t(r) * p.lddo + h * D;
+  const __nv_bfloat16* oo = static_cast<const __nv_bfloat16*>(p.o) + int64_t(r) * p.ldo + h * D;
+  float s = 0.0f;
+  if constexpr (D == 128) {
+    const uint2 a = reinterpret_cast<const uint2*>(go)[lane], b = reinterpret_cast<const uint2*>(oo)[lane];
+    s = bf16_lo(a.x) * bf16_lo(b.x) + bf16_hi(a.x) * bf16_hi(b.x) + bf16_lo(a.y) * bf16_lo(b.y) +
+        bf16_hi(a.y) * bf16_hi(b.y);
+  } else {
+    const uint32_t a = reinterpret_cast<const uint32_t*>(go)[lane], b = reinterpret_cast<const uint32_t*>(oo)[lane];
+    s = bf16_lo(a) * bf16_lo(b) + bf16_hi(a) * bf16_hi(b);
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (lane == 0) {
+    const float as = p.temp[h] * (p.ratio ? p.ratio[r] : 1.0f) * p.sm_scale;
+    *dst = make_float4(as * kLog2e, -p.lse[int64_t(h) * p.m + r] * kLog2e, s, as);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -101,12 +136,13 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
   float* red = reinterpret_cast<float*>(smem + Cfg::kOffRed);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBars);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;   // [3] K, V and bias tile j (stage j % 3)
-  uint64_t* dq_done = bars + 4;   // [3] dQ += dS K of tile j complete: stage j % 3 free
-  uint64_t* s_full = bars + 7;    // [2] S and dP of tile j in buffer j % 2
-  uint64_t* ds_full = bars + 9;   // [2] dS of tile j written (256 arrivals)
-  uint64_t* o_final = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  constexpr int kS = Cfg::kStages;
+  uint64_t* kv_full = bars + 1;        // [kS] K, V and bias tile j (stage j % kS)
+  uint64_t* dq_done = kv_full + kS;    // [kS] dQ += dS K of tile j complete: stage j % kS free
+  uint64_t* s_full = dq_done + kS;     // [2] S and dP of tile j in buffer j % 2
+  uint64_t* ds_full = s_full + 2;      // [2] dS of tile j written (256 arrivals)
+  uint64_t* o_final = ds_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -120,7 +156,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 3; ++s) {
+    for (int s = 0; s < kS; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&dq_done[s], 1);
     }
@@ -137,7 +173,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     tmem_relinquish();
   }
   if (!has_bias)
-    for (int i = threadIdx.x; i < 3 * BN; i += kBwdTcThreads) sBias[i] = 0.0f;
+    for (int i = threadIdx.x; i < kS * BN; i += kBwdTcThreads) sBias[i] = 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -157,8 +193,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         tma_load_2d(sDO + b * Cfg::kQBlk, &tmDO, q_full, h * D + 64 * b, qb * 128);
       }
       for (int j = 0; j < nt; ++j) {
-        const int s = j % 3;
-        if (j >= 3 && !mbar_wait(&dq_done[s], ((j - 3) / 3) & 1, kErrWaitAttention)) {
+        const int s = j % kS;
+        if (j >= kS && !mbar_wait(&dq_done[s], ((j - kS) / kS) & 1, kErrWaitAttention)) {
           *abort_flag = 1;
           break;
         }
@@ -181,7 +217,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       const uint64_t dv0 = sdesc_sw128(smem_u32(sV), 16, 1024);
       const uint64_t dkmn0 = sdesc_sw128(smem_u32(sK), Cfg::kKVBlk, 1024);
       auto issue_s = [&](int j) {
-        const int b = j & 1, s = j % 3;
+        const int b = j & 1, s = j % kS;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ao = ((kk >> 2) * Cfg::kQBlk + (kk & 3) * 32) >> 4;
@@ -192,7 +228,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         umma_commit(&s_full[b]);
       };
       auto issue_dq = [&](int j) {
-        const int b = j & 1, s = j % 3;
+        const int b = j & 1, s = j % kS;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
           umma_ts(tmem + Cfg::kColDQ, tmem + 64 * b + bwd_packed_col(kk),
@@ -211,7 +247,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       for (int j = 0; ok && j < nt; ++j) {
         const bool next = j + 2 < nt;
         ok = mbar_wait(&ds_full[j & 1], (j >> 1) & 1, kErrWaitAttention) &&
-             (!next || mbar_wait(&kv_full[(j + 2) % 3], ((j + 2) / 3) & 1, kErrWaitAttention));
+             (!next || mbar_wait(&kv_full[(j + 2) % kS], ((j + 2) / kS) & 1, kErrWaitAttention));
         if (!ok) break;
         tc_fence_after();
         issue_dq(j);
@@ -227,17 +263,15 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const bool row_ok = grow < p.m;
     const float ratio_r = row_ok ? (p.ratio ? p.ratio[grow] : 1.0f) : 0.0f;
-    const float as = p.temp[h] * ratio_r * p.sm_scale;      // dl -> dS
-    const float a2 = as * kLog2e;                            // S -> log2 logit
+    const float4 pr = p.rowpar[int64_t(h) * p.m_pad + grow];  // (a2, nl, D_r, as), masked past m
+    const float a2 = pr.x, nl = pr.y, dr = pr.z, as = pr.w;
     const float gg = p.gain[h] * kLog2e;
-    const float nl = row_ok ? -p.lse[int64_t(h) * p.m + grow] * kLog2e : -INFINITY;
-    const float dr = row_ok ? p.rowdot[int64_t(h) * p.m + grow] : 0.0f;
     float dgain_acc = 0.0f, dtz_acc = 0.0f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1;
       bool rdy = !*abort_flag &&
-                 mbar_wait2(&s_full[b], (j >> 1) & 1, &kv_full[j % 3], (j / 3) & 1, kErrWaitAttention);
+                 mbar_wait2(&s_full[b], (j >> 1) & 1, &kv_full[j % kS], (j / kS) & 1, kErrWaitAttention);
       if (!__all_sync(0xffffffffu, rdy)) {
         ok = false;
         break;
@@ -247,7 +281,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       tmem_ld32(tmem + lane_base + 64 * b + 32 * wg, sr);
       tmem_ld32(tmem + lane_base + Cfg::kColDP + 64 * b + 32 * wg, dp);
       tmem_ld_wait();
-      const float* bias = sBias + (j % 3) * BN + 32 * wg;
+      const float* bias = sBias + (j % kS) * BN + 32 * wg;
       const int key0 = j * BN + 32 * wg;
       const bool diag = key0 + 31 > qb * 128;  // warp-uniform
       uint32_t pk[16];
@@ -328,7 +362,7 @@ template <int D>
 __global__ void __launch_bounds__(kBwdTcThreads, 1)
     k_attn_bwd_kv_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
-                     AttnBwdParams p) {
+                     const __grid_constant__ CUtensorMap tmPar, AttnBwdParams p) {
   using Cfg = BwdKvCfg<D>;
   constexpr int BR = Cfg::BR;
   constexpr int kDBoxes = D / 64;
@@ -338,16 +372,17 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
   uint8_t* sV = smem + Cfg::kOffV;
   uint8_t* sQ = smem + Cfg::kOffQ;
   uint8_t* sDO = smem + Cfg::kOffDO;
-  float* sPar = reinterpret_cast<float*>(smem + Cfg::kOffPar);  // [stage][a2, nl, D_r, as][64 rows]
+  const float4* sPar = reinterpret_cast<const float4*>(smem + Cfg::kOffPar);  // [stage][64 rows] (a2, nl, D_r, as)
   float* red = reinterpret_cast<float*>(smem + Cfg::kOffRed);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBars);
-  uint64_t* kv_full = bars + 0;   // the K and V blocks
-  uint64_t* r_full = bars + 1;    // [3] Q, dO tile n and its row constants (stage n % 3; 32 arrivals)
-  uint64_t* mm_done = bars + 4;   // [3] dV, dK MMAs of tile n complete: stage n % 3 free
-  uint64_t* s_full = bars + 7;    // [2] S^T and dP^T of tile n in buffer n % 2
-  uint64_t* p_full = bars + 9;    // [2] P^T and dS^T of tile n written (256 arrivals)
-  uint64_t* o_final = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  constexpr int kS = Cfg::kStages;
+  uint64_t* kv_full = bars + 0;       // the K and V blocks
+  uint64_t* r_full = bars + 1;        // [kS] Q, dO tile n and its row constants (stage n % kS)
+  uint64_t* mm_done = r_full + kS;    // [kS] dV, dK MMAs of tile n complete: stage n % kS free
+  uint64_t* s_full = mm_done + kS;    // [2] S^T and dP^T of tile n in buffer n % 2
+  uint64_t* p_full = s_full + 2;      // [2] P^T and dS^T of tile n written (256 arrivals)
+  uint64_t* o_final = p_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -360,8 +395,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < 3; ++s) {
-      mbar_init(&r_full[s], 32);
+    for (int s = 0; s < kS; ++s) {
+      mbar_init(&r_full[s], 1);
       mbar_init(&mm_done[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -382,48 +417,33 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 8) {
-    // ------------------------------------------------------------ producer warp
-    // lane 0 issues the TMA copies; every lane writes the constants of two rows
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmDO);
+      prefetch_tmap(&tmPar);
       mbar_arrive_expect_tx(kv_full, 2 * Cfg::kKBytes);
       for (int b = 0; b < kDBoxes; ++b) {
         tma_load_2d(sK + b * Cfg::kKBlk, &tmK, kv_full, g * D + 64 * b, key0);
         tma_load_2d(sV + b * Cfg::kKBlk, &tmV, kv_full, g * D + 64 * b, key0);
       }
-    }
-    for (int n = 0; n < nt; ++n) {
-      const int s = n % 3;
-      if (n >= 3 && !warp_wait(&mm_done[s], ((n - 3) / 3) & 1, kErrWaitAttention)) {
-        *abort_flag = 1;
-        break;
-      }
-      const int h = g * p.group + n / ntq;
-      const int row0 = key0 + BR * (n % ntq);
-      float* par = sPar + s * 4 * BR;
-      const float th = p.temp[h] * p.sm_scale;
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int r = lane + 32 * u, gr = row0 + r;
-        const bool ok_r = gr < p.m;
-        const float as = ok_r ? th * (p.ratio ? p.ratio[gr] : 1.0f) : 0.0f;
-        par[r] = as * kLog2e;
-        par[BR + r] = ok_r ? -p.lse[int64_t(h) * p.m + gr] * kLog2e : -INFINITY;
-        par[2 * BR + r] = ok_r ? p.rowdot[int64_t(h) * p.m + gr] : 0.0f;
-        par[3 * BR + r] = as;
-      }
-      // each lane arrives after its own writes; lane 0's arrival carries the transaction count
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&r_full[s], 2 * Cfg::kRBytes);
+      for (int n = 0; n < nt; ++n) {
+        const int s = n % kS;
+        if (n >= kS && !mbar_wait(&mm_done[s], ((n - kS) / kS) & 1, kErrWaitAttention)) {
+          *abort_flag = 1;
+          break;
+        }
+        const int h = g * p.group + n / ntq;
+        const int row0 = key0 + BR * (n % ntq);
+        mbar_arrive_expect_tx(&r_full[s], 2 * Cfg::kRBytes + BR * 16);
         for (int b = 0; b < kDBoxes; ++b) {
           tma_load_2d(sQ + s * Cfg::kRBytes + b * Cfg::kRBlk, &tmQ, &r_full[s], h * D + 64 * b, row0);
           tma_load_2d(sDO + s * Cfg::kRBytes + b * Cfg::kRBlk, &tmDO, &r_full[s], h * D + 64 * b, row0);
         }
-      } else {
-        mbar_arrive(&r_full[s]);
+        tma_load_1d(const_cast<float4*>(sPar) + s * BR, &tmPar, &r_full[s],
+                    static_cast<int32_t>((int64_t(h) * p.m_pad + row0) * 4));
       }
     }
   } else if (warp == 9) {
@@ -438,7 +458,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       const uint64_t dqmn0 = sdesc_sw128(smem_u32(sQ), Cfg::kRBlk, 1024);
       const uint64_t ddomn0 = sdesc_sw128(smem_u32(sDO), Cfg::kRBlk, 1024);
       auto issue_s = [&](int n) {
-        const int b = n & 1, s = n % 3;
+        const int b = n & 1, s = n % kS;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ao = ((kk >> 2) * Cfg::kKBlk + (kk & 3) * 32) >> 4;
@@ -449,7 +469,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         umma_commit(&s_full[b]);
       };
       auto issue_acc = [&](int n) {
-        const int b = n & 1, s = n % 3;
+        const int b = n & 1, s = n % kS;
 #pragma unroll
         for (int kk = 0; kk < BR / 16; ++kk) {
           const uint64_t bo = (s * Cfg::kRBytes + kk * 16 * 128) >> 4;
@@ -471,7 +491,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       for (int n = 0; ok && n < nt; ++n) {
         const bool next = n + 2 < nt;
         ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, kErrWaitAttention) &&
-             (!next || mbar_wait(&r_full[(n + 2) % 3], ((n + 2) / 3) & 1, kErrWaitAttention));
+             (!next || mbar_wait(&r_full[(n + 2) % kS], ((n + 2) / kS) & 1, kErrWaitAttention));
         if (!ok) break;
         tc_fence_after();
         issue_acc(n);
@@ -489,11 +509,11 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     float dbias_acc = 0.0f;
     bool ok = true;
     for (int n = 0; n < nt; ++n) {
-      const int b = n & 1, s = n % 3;
+      const int b = n & 1, s = n % kS;
       const int h = g * p.group + n / ntq;
       const int i = n % ntq;
       bool rdy = !*abort_flag &&
-                 mbar_wait2(&s_full[b], (n >> 1) & 1, &r_full[s], (n / 3) & 1, kErrWaitAttention);
+                 mbar_wait2(&s_full[b], (n >> 1) & 1, &r_full[s], (n / kS) & 1, kErrWaitAttention);
       if (!__all_sync(0xffffffffu, rdy)) {
         ok = false;
         break;
@@ -505,27 +525,22 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       tmem_ld_wait();
       const float gain = p.gain[h];
       const float gb2 = gain * kLog2e * bias_c;
-      const float* par = sPar + s * 4 * BR + 32 * wg;
+      const float4* par = sPar + s * BR + 32 * wg;
       const int r0 = key0 + BR * i + 32 * wg;  // row of column 0 of this half
       const bool diag = i < 2;                 // rows before key0 + 128 meet the causal mask
       uint32_t pp[16], pd[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
-        const float4 a4 = *reinterpret_cast<const float4*>(par + e);
-        const float4 n4 = *reinterpret_cast<const float4*>(par + BR + e);
-        const float4 d4 = *reinterpret_cast<const float4*>(par + 2 * BR + e);
-        const float4 s4 = *reinterpret_cast<const float4*>(par + 3 * BR + e);
-        const float av[4] = {a4.x, a4.y, a4.z, a4.w}, nv[4] = {n4.x, n4.y, n4.z, n4.w};
-        const float dv[4] = {d4.x, d4.y, d4.z, d4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
         float pv[4], dsv[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          float x = fmaf(av[u], __uint_as_float(sr[e + u]), gb2 + nv[u]);
+          const float4 c = par[e + u];  // (a2, nl, D_r, as) of the row
+          float x = fmaf(c.x, __uint_as_float(sr[e + u]), gb2 + c.y);
           if (diag && key > r0 + e + u) x = -INFINITY;
           pv[u] = ex2_approx(x);
-          const float dl = pv[u] * (__uint_as_float(dp[e + u]) - dv[u]);
+          const float dl = pv[u] * (__uint_as_float(dp[e + u]) - c.z);
           dbias_acc = fmaf(gain, dl, dbias_acc);
-          dsv[u] = dl * sv[u];
+          dsv[u] = dl * c.w;
         }
         pp[e >> 1] = pack_bf16x2(pv[0], pv[1]);
         pp[(e >> 1) + 1] = pack_bf16x2(pv[2], pv[3]);

@@ -607,7 +607,9 @@ size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t
     if (!shape || m <= 0 || shape->hq <= 0 || shape->hkv <= 0) return 0;
     auto al = [](size_t b) { return (b + 255) / 256 * 256; };
     const size_t nkb = static_cast<size_t>((m + tg::kBwdBlk - 1) / tg::kBwdBlk);
-    return al(size_t(shape->hq) * m * 4) + al(size_t(shape->hkv) * m * 4) + al(size_t(shape->hq) * nkb * 2 * 4);
+    const size_t m_pad = static_cast<size_t>((m + 127) / 128 * 128);
+    return al(size_t(shape->hq) * m * 4) + al(size_t(shape->hkv) * m * 4) + al(size_t(shape->hq) * nkb * 2 * 4) +
+           al(size_t(shape->hq) * m_pad * 16);
   }
   if (op == TG_OP_DECODE) {
     if (!shape || m <= 0 || shape->hkv <= 0 || shape->hq % shape->hkv) return 0;
@@ -1010,14 +1012,18 @@ int tg_gated_attention_backward(const void* q, int64_t ldq, const void* k, int64
   p.dbias_part = reinterpret_cast<float*>(wb);
   wb += al(size_t(hkv) * m * 4);
   p.dgt_part = reinterpret_cast<float*>(wb);
+  wb += al(size_t(hq) * p.nkb * 2 * 4);
+  p.m_pad = static_cast<int>((m + 127) / 128 * 128);
+  p.rowpar = reinterpret_cast<float4*>(wb);
   const int nqb = p.nkb;
   // bf16 operands that TMA can read go to the tensor cores
   const bool tc = dtype == TG_BF16 && aligned16(q) && aligned16(k) && aligned16(v) && aligned16(dout) &&
-                  ldq % 8 == 0 && ldk % 8 == 0 && ldv % 8 == 0 && lddo % 8 == 0 && aligned16(dq) &&
+                  aligned16(out) && ldq % 8 == 0 && ldk % 8 == 0 && ldv % 8 == 0 && lddo % 8 == 0 &&
+                  ldo % 8 == 0 && aligned16(dq) &&
                   aligned16(dk) && aligned16(dv) && (!bias || aligned16(bias));
   if (tc) {
-    auto run_tc = [&](auto rowdot, auto kv, auto qk, size_t smem_kv, size_t smem_q, int D) -> int {
-      CUtensorMap tq128, tdo128, tk64, tv64, tk128, tv128, tq64, tdo64, tb;
+    auto run_tc = [&](auto prep, auto kv, auto qk, size_t smem_kv, size_t smem_q, int D) -> int {
+      CUtensorMap tq128, tdo128, tk64, tv64, tk128, tv128, tq64, tdo64, tb, tpar;
       std::memset(&tb, 0, sizeof(tb));
       int rc = make_map(&tq128, q, uint64_t(hq) * D, uint64_t(m), uint64_t(ldq) * 2, 128);
       if (!rc) rc = make_map(&tdo128, dout, uint64_t(hq) * D, uint64_t(m), uint64_t(lddo) * 2, 128);
@@ -1028,13 +1034,14 @@ int tg_gated_attention_backward(const void* q, int64_t ldq, const void* k, int64
       if (!rc) rc = make_map(&tk128, k, uint64_t(hkv) * D, uint64_t(m), uint64_t(ldk) * 2, 128);
       if (!rc) rc = make_map(&tv128, v, uint64_t(hkv) * D, uint64_t(m), uint64_t(ldv) * 2, 128);
       if (!rc && bias) rc = make_map_1d_f32(&tb, bias, uint64_t(m), 64);
+      if (!rc) rc = make_map_1d_f32(&tpar, p.rowpar, uint64_t(hq) * p.m_pad * 4, 256);
       if (!rc) rc = set_smem(kv, smem_kv);
       if (!rc) rc = set_smem(qk, smem_q);
       if (rc) return rc;
       const int nqb128 = static_cast<int>((m + 127) / 128);
-      rowdot<<<unsigned((m * hq + 7) / 8), 256, 0, st>>>(p);
-      if ((rc = check_launch("k_attn_bwd_rowdot"))) return rc;
-      kv<<<unsigned(hkv * nqb128), tg::kBwdTcThreads, smem_kv, st>>>(tk128, tv128, tq64, tdo64, p);
+      prep<<<unsigned((int64_t(p.m_pad) * hq + 7) / 8), 256, 0, st>>>(p);
+      if ((rc = check_launch("k_attn_bwd_prep"))) return rc;
+      kv<<<unsigned(hkv * nqb128), tg::kBwdTcThreads, smem_kv, st>>>(tk128, tv128, tq64, tdo64, tpar, p);
       if ((rc = check_launch("k_attn_bwd_kv_tc"))) return rc;
       p.nkb = nqb128;  // dgain / dtemp partials per block of 128 rows
       qk<<<unsigned(hq * nqb128), tg::kBwdTcThreads, smem_q, st>>>(tq128, tdo128, tk64, tv64, tb, p);
@@ -1043,9 +1050,9 @@ int tg_gated_attention_backward(const void* q, int64_t ldq, const void* k, int64
       return check_launch("k_attn_bwd_final");
     };
     return head_dim == 128
-               ? run_tc(tg::k_attn_bwd_rowdot<__nv_bfloat16, 128>, tg::k_attn_bwd_kv_tc<128>,
+               ? run_tc(tg::k_attn_bwd_prep<128>, tg::k_attn_bwd_kv_tc<128>,
                         tg::k_attn_bwd_dq_tc<128>, tg::BwdKvCfg<128>::kSmem, tg::BwdDqCfg<128>::kSmem, 128)
-               : run_tc(tg::k_attn_bwd_rowdot<__nv_bfloat16, 64>, tg::k_attn_bwd_kv_tc<64>,
+               : run_tc(tg::k_attn_bwd_prep<64>, tg::k_attn_bwd_kv_tc<64>,
                         tg::k_attn_bwd_dq_tc<64>, tg::BwdKvCfg<64>::kSmem, tg::BwdDqCfg<64>::kSmem, 64);
   }
   auto run = [&](auto rowdot, auto kv, auto qk, int D) -> int {
