@@ -50,8 +50,11 @@ struct AttnBwdParams {
   float* dbias_part;   // workspace [hkv][m]
   float* dgt_part;     // workspace [hq][nkb][2]: (dgain, dtemp) partials
   int nkb;             // key blocks
-  float4* rowpar;      // workspace [hq][m_pad] (tensor-core kernels): per-row constants
+  float* rowpar;       // workspace [hq][m_pad / 2][8] (tensor-core kernels): per-row constants of row pairs
   int m_pad;           // m rounded up to 128
+  int dbias_nparts;    // rows of dbias_part summed into dbias (hkv here, hq for the tensor-core kernels)
+  float* kv_part;      // workspace [hkv * m_pad / 128][group][128][2 D]: one head's (dV, dK) of a key block
+  unsigned* kv_ctr;    // workspace [2][hkv * m_pad / 128]: tickets, partials published; zero on entry
 };
 
 template <typename T>
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(256) k_attn_bwd_final(AttnBwdParams p) {
   const int i = blockIdx.x * 256 + threadIdx.x;
   if (p.dbias && i < p.m) {
     float s = 0.0f;
-    for (int g = 0; g < p.hkv; ++g) s += p.dbias_part[int64_t(g) * p.m + i];
+    for (int g = 0; g < p.dbias_nparts; ++g) s += p.dbias_part[int64_t(g) * p.m + i];
     p.dbias[i] = s;
   }
   if (i < p.hq) {

@@ -17,16 +17,20 @@
 //   pairs over the first 16 columns of their half of the S buffer, and the
 //   MMA thread accumulates dQ += dS K as a TS-MMA (K MN-major from shared
 //   memory).  The row's dgain / dtemp contributions are summed on the way.
-// k_attn_bwd_kv_tc: one CTA per (KV head g, block of 128 keys), walking the
-//   query tiles of 64 rows from the diagonal on, for every query head of g.
+// k_attn_bwd_kv_tc: one CTA per (query head h, block of 128 keys), walking the
+//   query tiles of 64 rows from the diagonal on.
 //   S^T = K Q^T and dP^T = V dO^T (one thread per key), P^T and dS^T as bf16
 //   pairs over their own columns, then dV += P^T dO and dK += dS^T Q as
 //   TS-MMAs; both accumulators stay in tensor memory over the whole walk.  The
+//   query heads that share a KV head add their (dV, dK) through the workspace
+//   in head order (the last CTA of the group to finish does the sum).  The
 //   per-row constants of a tile (from k_attn_bwd_prep) come by TMA into the
 //   same stage as the Q / dO tiles.
 // k_attn_bwd_prep: D_r and the per-row constants (a_r sm_scale log2 e,
-//   -lse_r log2 e, D_r, a_r sm_scale) of every head and row, rows past m
-//   masked (P = 0 there), so neither kernel above reads lse or ratio per tile.
+//   -lse_r log2 e, -D_r, a_r sm_scale) of every head and row, interleaved by
+//   row pairs so that the elementwise loops read them as packed f32x2 pairs;
+//   rows past m masked (P = 0 there).  The elementwise arithmetic runs on
+//   f32x2 pairs (fma/add/mul.rn.f32x2: per-lane IEEE results).
 //
 // Warps: 0-7 elementwise (two warpgroups), 8 TMA producer, 9 TMEM allocator
 // and single-thread MMA issuer.  Every wait is bounded (kErrWaitAttention).
@@ -83,6 +87,42 @@ __device__ __forceinline__ uint32_t bwd_packed_col(int kk) {
   return static_cast<uint32_t>(kk < 2 ? kk * 8 : 32 + (kk - 2) * 8);
 }
 
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// ---------------------------------------------------------------------------
+// Epilogue staging: a warp holds 32 rows (lane = row) x 32 fp32 columns from a
+// tcgen05.ld; it writes them into a 4 KB swizzled area (16-byte chunk c of row
+// r at c ^ (r & 7): no bank conflicts either way) and reads them back so that
+// eight lanes cover one row's 128 contiguous bytes, four rows per instruction.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float4* stage_slot(float* stage, int row, int chunk) {
+  return reinterpret_cast<float4*>(stage) + row * 8 + (chunk ^ (row & 7));
+}
+
+__device__ __forceinline__ void stage_rows32(float* stage, const uint32_t (&o)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *stage_slot(stage, lane, c) = make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]),
+                                              __uint_as_float(o[4 * c + 2]), __uint_as_float(o[4 * c + 3]));
+  __syncwarp();
+}
+
+// Coalesced write-out of a staged 32 x 32 block: row i goes to dst + (row0 + i) * ld, rows >= nrows skipped.
+__device__ __forceinline__ void stage_store32(float* stage, float* dst, int64_t ld, int row0, int nrows) {
+  const int lane = threadIdx.x & 31, cc = lane & 7;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = (lane >> 3) + 4 * k;
+    if (row0 + r < nrows) reinterpret_cast<float4*>(dst + int64_t(row0 + r) * ld)[cc] = *stage_slot(stage, r, cc);
+  }
+  __syncwarp();  // the area is free for the next block
+}
+
 // ---------------------------------------------------------------------------
 // Per-row constants: one warp per (row, head), rows m .. m_pad - 1 masked
 // ---------------------------------------------------------------------------
@@ -91,9 +131,15 @@ __global__ void __launch_bounds__(256) k_attn_bwd_prep(AttnBwdParams p) {
   const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (w >= p.m_pad * p.hq) return;  // warp-uniform
   const int r = w / p.hq, h = w % p.hq;
-  float4* dst = p.rowpar + int64_t(h) * p.m_pad + r;
+  // rows r and r ^ 1 share 8 floats: (a2, a2', nl, nl', -D, -D', as, as')
+  float* dst = p.rowpar + (int64_t(h) * (p.m_pad / 2) + r / 2) * 8 + (r & 1);
   if (r >= p.m) {
-    if (lane == 0) *dst = make_float4(0.0f, -INFINITY, 0.0f, 0.0f);
+    if (lane == 0) {
+      dst[0] = 0.0f;
+      dst[2] = -INFINITY;
+      dst[4] = 0.0f;
+      dst[6] = 0.0f;
+    }
     return;
   }
   const __nv_bfloat16* go = static_cast<const __nv_bfloat16*>(p.dout) + int64_t(r) * p.lddo + h * D;
@@ -111,7 +157,10 @@ __global__ void __launch_bounds__(256) k_attn_bwd_prep(AttnBwdParams p) {
   for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
   if (lane == 0) {
     const float as = p.temp[h] * (p.ratio ? p.ratio[r] : 1.0f) * p.sm_scale;
-    *dst = make_float4(as * kLog2e, -p.lse[int64_t(h) * p.m + r] * kLog2e, s, as);
+    dst[0] = as * kLog2e;
+    dst[2] = -p.lse[int64_t(h) * p.m + r] * kLog2e;
+    dst[4] = -s;
+    dst[6] = as;
   }
 }
 
@@ -263,10 +312,12 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const bool row_ok = grow < p.m;
     const float ratio_r = row_ok ? (p.ratio ? p.ratio[grow] : 1.0f) : 0.0f;
-    const float4 pr = p.rowpar[int64_t(h) * p.m_pad + grow];  // (a2, nl, D_r, as), masked past m
-    const float a2 = pr.x, nl = pr.y, dr = pr.z, as = pr.w;
+    const float* pr = p.rowpar + (int64_t(h) * (p.m_pad / 2) + grow / 2) * 8 + (grow & 1);  // masked past m
+    const float a2 = pr[0], nl = pr[2], ndr = pr[4], as = pr[6];
     const float gg = p.gain[h] * kLog2e;
-    float dgain_acc = 0.0f, dtz_acc = 0.0f;
+    const uint64_t a2p = f2_pack(a2, a2), nlp = f2_pack(nl, nl), ndrp = f2_pack(ndr, ndr), asp = f2_pack(as, as),
+                   ggp = f2_pack(gg, gg);
+    uint64_t dgain2 = 0, dtz2 = 0;  // (even keys, odd keys) partial sums
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1;
@@ -281,25 +332,27 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       tmem_ld32(tmem + lane_base + 64 * b + 32 * wg, sr);
       tmem_ld32(tmem + lane_base + Cfg::kColDP + 64 * b + 32 * wg, dp);
       tmem_ld_wait();
-      const float* bias = sBias + (j % kS) * BN + 32 * wg;
+      const uint64_t* bias2 = reinterpret_cast<const uint64_t*>(sBias + (j % kS) * BN + 32 * wg);
       const int key0 = j * BN + 32 * wg;
       const bool diag = key0 + 31 > qb * 128;  // warp-uniform
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
-        const float s0 = __uint_as_float(sr[e]), s1 = __uint_as_float(sr[e + 1]);
-        float x0 = fmaf(a2, s0, fmaf(gg, bias[e], nl));
-        float x1 = fmaf(a2, s1, fmaf(gg, bias[e + 1], nl));
+        const uint64_t s2 = f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+        const uint64_t b2 = bias2[e >> 1];
+        float x0, x1;
+        f2_unpack(f2_fma(a2p, s2, f2_fma(ggp, b2, nlp)), x0, x1);
         if (diag) {
           if (key0 + e > grow) x0 = -INFINITY;
           if (key0 + e + 1 > grow) x1 = -INFINITY;
         }
-        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-        const float dl0 = p0 * (__uint_as_float(dp[e]) - dr);
-        const float dl1 = p1 * (__uint_as_float(dp[e + 1]) - dr);
-        dgain_acc = fmaf(dl0, bias[e], fmaf(dl1, bias[e + 1], dgain_acc));
-        dtz_acc = fmaf(dl0, s0, fmaf(dl1, s1, dtz_acc));
-        pk[e >> 1] = pack_bf16x2(dl0 * as, dl1 * as);
+        const uint64_t p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        const uint64_t dl2 = f2_mul(p2, f2_add(f2_pack(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])), ndrp));
+        dgain2 = f2_fma(dl2, b2, dgain2);
+        dtz2 = f2_fma(dl2, s2, dtz2);
+        float d0, d1;
+        f2_unpack(f2_mul(dl2, asp), d0, d1);
+        pk[e >> 1] = pack_bf16x2(d0, d1);
       }
       tmem_st16(tmem + lane_base + 64 * b + 32 * wg, pk);
       tmem_st_wait();
@@ -309,23 +362,23 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     if (ok && !*abort_flag) ok = warp_wait(o_final, 0, kErrWaitAttention);
     if (!ok) *abort_flag = 1;
     if (ok) {
+      // dQ through a per-warp staging area in the (now idle) K ring
       tc_fence_after();
+      float* stage = reinterpret_cast<float*>(sK) + warp * 1024;
 #pragma unroll 1
       for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
         uint32_t o[32];
         tmem_ld32(tmem + lane_base + Cfg::kColDQ + c0, o);
         tmem_ld_wait();
-        if (row_ok) {
-          float4* dst = reinterpret_cast<float4*>(p.dq + int64_t(grow) * p.hq * D + h * D + c0);
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
-                                 __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
-        }
+        stage_rows32(stage, o);
+        stage_store32(stage, p.dq + h * D + c0, int64_t(p.hq) * D, qb * 128 + q4 * 32, p.m);
       }
     }
     // dgain / dtemp of this (head, row block): fixed-order sums over lanes, then warps
-    float vg = dgain_acc, vt = dtz_acc * ratio_r * p.sm_scale;
+    float g0, g1, t0, t1;
+    f2_unpack(dgain2, g0, g1);
+    f2_unpack(dtz2, t0, t1);
+    float vg = g0 + g1, vt = (t0 + t1) * ratio_r * p.sm_scale;
 #pragma unroll
     for (int off = 16; off; off >>= 1) {
       vg += __shfl_xor_sync(0xffffffffu, vg, off);
@@ -372,7 +425,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
   uint8_t* sV = smem + Cfg::kOffV;
   uint8_t* sQ = smem + Cfg::kOffQ;
   uint8_t* sDO = smem + Cfg::kOffDO;
-  const float4* sPar = reinterpret_cast<const float4*>(smem + Cfg::kOffPar);  // [stage][64 rows] (a2, nl, D_r, as)
+  const float4* sPar = reinterpret_cast<const float4*>(smem + Cfg::kOffPar);  // [stage][32 row pairs][2] float4
   float* red = reinterpret_cast<float*>(smem + Cfg::kOffRed);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBars);
   constexpr int kS = Cfg::kStages;
@@ -387,11 +440,11 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // longest first: key block 0 is seen by every row
-  const int kb = static_cast<int>(blockIdx.x) / p.hkv;
-  const int g = static_cast<int>(blockIdx.x) % p.hkv;
+  const int kb = static_cast<int>(blockIdx.x) / p.hq;
+  const int h = static_cast<int>(blockIdx.x) % p.hq;
+  const int g = h / p.group, u = h % p.group;
   const int key0 = kb * Cfg::BK;
-  const int ntq = (p.m - key0 + BR - 1) / BR;  // row tiles per head
-  const int nt = ntq * p.group;                // tile n: head g * group + n / ntq, rows key0 + 64 (n % ntq)
+  const int nt = (p.m - key0 + BR - 1) / BR;  // row tiles: rows key0 + 64 n
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -435,8 +488,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
           *abort_flag = 1;
           break;
         }
-        const int h = g * p.group + n / ntq;
-        const int row0 = key0 + BR * (n % ntq);
+        const int row0 = key0 + BR * n;
         mbar_arrive_expect_tx(&r_full[s], 2 * Cfg::kRBytes + BR * 16);
         for (int b = 0; b < kDBoxes; ++b) {
           tma_load_2d(sQ + s * Cfg::kRBytes + b * Cfg::kRBlk, &tmQ, &r_full[s], h * D + 64 * b, row0);
@@ -506,12 +558,14 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     const int kl = q4 * 32 + lane, key = key0 + kl;  // this thread's key
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const float bias_c = (p.bias && key < p.m) ? p.bias[key] : 0.0f;
-    float dbias_acc = 0.0f;
+    const float gain = p.gain[h];
+    const float gb2 = gain * kLog2e * bias_c;
+    const uint64_t gb2p = f2_pack(gb2, gb2), gainp = f2_pack(gain, gain);
+    uint64_t dbias2 = 0;  // (even rows, odd rows) partial sums
     bool ok = true;
     for (int n = 0; n < nt; ++n) {
       const int b = n & 1, s = n % kS;
-      const int h = g * p.group + n / ntq;
-      const int i = n % ntq;
+      const int i = n;
       bool rdy = !*abort_flag &&
                  mbar_wait2(&s_full[b], (n >> 1) & 1, &r_full[s], (n / kS) & 1, kErrWaitAttention);
       if (!__all_sync(0xffffffffu, rdy)) {
@@ -523,29 +577,29 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       tmem_ld32(tmem + lane_base + 64 * b + 32 * wg, sr);
       tmem_ld32(tmem + lane_base + Cfg::kColDP + 64 * b + 32 * wg, dp);
       tmem_ld_wait();
-      const float gain = p.gain[h];
-      const float gb2 = gain * kLog2e * bias_c;
+      // (a2, a2', nl, nl') and (-D, -D', as, as') of each row pair of this half
       const float4* par = sPar + s * BR + 32 * wg;
       const int r0 = key0 + BR * i + 32 * wg;  // row of column 0 of this half
       const bool diag = i < 2;                 // rows before key0 + 128 meet the causal mask
       uint32_t pp[16], pd[16];
 #pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        float pv[4], dsv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 c = par[e + u];  // (a2, nl, D_r, as) of the row
-          float x = fmaf(c.x, __uint_as_float(sr[e + u]), gb2 + c.y);
-          if (diag && key > r0 + e + u) x = -INFINITY;
-          pv[u] = ex2_approx(x);
-          const float dl = pv[u] * (__uint_as_float(dp[e + u]) - c.z);
-          dbias_acc = fmaf(gain, dl, dbias_acc);
-          dsv[u] = dl * c.w;
+      for (int e = 0; e < 32; e += 2) {
+        const float4 c0 = par[e], c1 = par[e + 1];
+        const uint64_t s2 = f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(c0.x, c0.y), s2, f2_add(gb2p, f2_pack(c0.z, c0.w))), x0, x1);
+        if (diag) {
+          if (key > r0 + e) x0 = -INFINITY;
+          if (key > r0 + e + 1) x1 = -INFINITY;
         }
-        pp[e >> 1] = pack_bf16x2(pv[0], pv[1]);
-        pp[(e >> 1) + 1] = pack_bf16x2(pv[2], pv[3]);
-        pd[e >> 1] = pack_bf16x2(dsv[0], dsv[1]);
-        pd[(e >> 1) + 1] = pack_bf16x2(dsv[2], dsv[3]);
+        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+        const uint64_t dl2 = f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
+                                                            f2_pack(c1.x, c1.y)));
+        dbias2 = f2_fma(gainp, dl2, dbias2);
+        float d0, d1;
+        f2_unpack(f2_mul(dl2, f2_pack(c1.z, c1.w)), d0, d1);
+        pp[e >> 1] = pack_bf16x2(p0, p1);
+        pd[e >> 1] = pack_bf16x2(d0, d1);
       }
       tmem_st16(tmem + lane_base + 64 * b + 32 * wg, pp);
       tmem_st16(tmem + lane_base + Cfg::kColDP + 64 * b + 32 * wg, pd);
@@ -555,29 +609,105 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     }
     if (ok && !*abort_flag) ok = warp_wait(o_final, 0, kErrWaitAttention);
     if (!ok) *abort_flag = 1;
-    if (ok) {
-      // warpgroup 0 writes dV, warpgroup 1 dK (fp32 rows of this key)
+    // the two warpgroups each summed half of every tile's rows: add them in a fixed order
+    float dbl, dbh;
+    f2_unpack(dbias2, dbl, dbh);
+    const float dbias_acc = dbl + dbh;
+    if (wg == 1) red[kl] = dbias_acc;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (wg == 0 && key < p.m) p.dbias_part[int64_t(h) * p.m + key] = dbias_acc + red[kl];
+    const bool good = !*abort_flag;  // agreed by every elementwise thread (read after the barrier)
+    // (dV, dK) of this head: warpgroup 0 holds the dV columns, warpgroup 1 the dK columns.
+    // With GQA the heads of the group meet here: every CTA but the last (by ticket)
+    // publishes its partial; the last adds all heads' partials in head order.
+    const uint32_t col = wg ? Cfg::kColDK : Cfg::kColDV;
+    float* dst_base = (wg ? p.dk : p.dv) + g * D;  // row 0 of this KV head's columns
+    const int nslots = p.hkv * (p.m_pad / Cfg::BK);
+    const int slot = g * (p.m_pad / Cfg::BK) + kb;
+    int role = 0;  // 0: write the result directly, 1: publish a partial, 2: merge the partials
+    if (good && p.group > 1) {
+      if (threadIdx.x == 0) tmem_slot[2] = atomicAdd(&p.kv_ctr[slot], 1u) == unsigned(p.group - 1) ? 2u : 1u;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      role = static_cast<int>(tmem_slot[2]);
+    }
+    float* part = p.kv_part + (int64_t(slot) * p.group) * Cfg::BK * 2 * D;  // [group][128][2 D]
+    // per-warp staging area in the (now idle) Q ring
+    float* stage = reinterpret_cast<float*>(sQ) + warp * 1024;
+    if (good && role == 1) {
       tc_fence_after();
-      const uint32_t col = wg ? Cfg::kColDK : Cfg::kColDV;
-      float* dst_row = (wg ? p.dk : p.dv) + int64_t(key) * p.hkv * D + g * D;
+      float* mine = part + int64_t(u) * Cfg::BK * 2 * D + (wg ? D : 0);
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
         tmem_ld32(tmem + lane_base + col + c0, o);
         tmem_ld_wait();
-        if (key < p.m) {
-          float4* dst = reinterpret_cast<float4*>(dst_row + c0);
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
-                                 __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+        stage_rows32(stage, o);
+        stage_store32(stage, mine + c0, 2 * D, q4 * 32, Cfg::BK);
+      }
+      __threadfence();
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (threadIdx.x == 0) atomicAdd(&p.kv_ctr[nslots + slot], 1u);
+    }
+    bool merge_ok = true;
+    if (good && role == 2) {
+      // the other heads' CTAs took their tickets before this one, so they are
+      // running; wait (bounded) until all have published
+      if (threadIdx.x == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        uint32_t okw = 1;
+        while (ld_acquire_gpu(&p.kv_ctr[nslots + slot]) < unsigned(p.group - 1)) {
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            raise_error(kErrWaitAttention, 2);
+            okw = 0;
+            break;
+          }
         }
+        tmem_slot[3] = okw;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      merge_ok = tmem_slot[3] != 0;
+    }
+    if (good && role != 1 && merge_ok) {
+      tc_fence_after();
+      const int cc = lane & 7;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + col + c0, o);
+        tmem_ld_wait();
+        stage_rows32(stage, o);
+        if (role == 2) {
+          // sum over the group's heads in head order, on the staged (coalesced)
+          // layout; the eight rows of a head are fetched together
+          float4 acc[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[k] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          for (int w = 0; w < p.group; ++w) {
+            float4 x[8];
+            if (w == u) {
+#pragma unroll
+              for (int k = 0; k < 8; ++k) x[k] = *stage_slot(stage, (lane >> 3) + 4 * k, cc);
+            } else {
+              const float4* src = reinterpret_cast<const float4*>(part + (int64_t(w) * Cfg::BK + q4 * 32) * 2 * D +
+                                                                  (wg ? D : 0) + c0) + cc;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) x[k] = __ldcg(src + ((lane >> 3) + 4 * k) * (2 * D / 4));
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              acc[k].x += x[k].x;
+              acc[k].y += x[k].y;
+              acc[k].z += x[k].z;
+              acc[k].w += x[k].w;
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) *stage_slot(stage, (lane >> 3) + 4 * k, cc) = acc[k];
+          __syncwarp();
+        }
+        stage_store32(stage, dst_base + c0, int64_t(p.hkv) * D, key0 + q4 * 32, p.m);
       }
     }
-    // the two warpgroups each summed half of every tile's rows: add them in a fixed order
-    if (wg == 1) red[kl] = dbias_acc;
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (wg == 0 && key < p.m) p.dbias_part[int64_t(g) * p.m + key] = dbias_acc + red[kl];
   }
   tc_fence_before();
   __syncthreads();

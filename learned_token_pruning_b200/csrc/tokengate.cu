@@ -608,8 +608,10 @@ size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t
     auto al = [](size_t b) { return (b + 255) / 256 * 256; };
     const size_t nkb = static_cast<size_t>((m + tg::kBwdBlk - 1) / tg::kBwdBlk);
     const size_t m_pad = static_cast<size_t>((m + 127) / 128 * 128);
+    const size_t hd = static_cast<size_t>(shape->head_dim > 0 ? shape->head_dim : 128);
     return al(size_t(shape->hq) * m * 4) + al(size_t(shape->hkv) * m * 4) + al(size_t(shape->hq) * nkb * 2 * 4) +
-           al(size_t(shape->hq) * m_pad * 16);
+           al(size_t(shape->hq) * m_pad * 16) + al(size_t(shape->hq) * m_pad * 2 * hd * 4) +
+           al(2 * size_t(shape->hkv) * (m_pad / 128) * 4);
   }
   if (op == TG_OP_DECODE) {
     if (!shape || m <= 0 || shape->hkv <= 0 || shape->hq % shape->hkv) return 0;
@@ -1014,7 +1016,12 @@ int tg_gated_attention_backward(const void* q, int64_t ldq, const void* k, int64
   p.dgt_part = reinterpret_cast<float*>(wb);
   wb += al(size_t(hq) * p.nkb * 2 * 4);
   p.m_pad = static_cast<int>((m + 127) / 128 * 128);
-  p.rowpar = reinterpret_cast<float4*>(wb);
+  p.rowpar = reinterpret_cast<float*>(wb);
+  wb += al(size_t(hq) * p.m_pad * 16);
+  p.kv_part = reinterpret_cast<float*>(wb);
+  wb += al(size_t(hq) * p.m_pad * 2 * head_dim * 4);
+  p.kv_ctr = reinterpret_cast<unsigned*>(wb);
+  p.dbias_nparts = hkv;
   const int nqb = p.nkb;
   // bf16 operands that TMA can read go to the tensor cores
   const bool tc = dtype == TG_BF16 && aligned16(q) && aligned16(k) && aligned16(v) && aligned16(dout) &&
@@ -1039,9 +1046,14 @@ int tg_gated_attention_backward(const void* q, int64_t ldq, const void* k, int64
       if (!rc) rc = set_smem(qk, smem_q);
       if (rc) return rc;
       const int nqb128 = static_cast<int>((m + 127) / 128);
+      // per-head dbias partials in the row-dot region; group tickets start at zero
+      p.dbias_part = p.rowdot;
+      p.dbias_nparts = hq;
+      if (cudaMemsetAsync(p.kv_ctr, 0, 2 * size_t(hkv) * nqb128 * 4, st) != cudaSuccess)
+        return fail(TG_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(cudaGetLastError()));
       prep<<<unsigned((int64_t(p.m_pad) * hq + 7) / 8), 256, 0, st>>>(p);
       if ((rc = check_launch("k_attn_bwd_prep"))) return rc;
-      kv<<<unsigned(hkv * nqb128), tg::kBwdTcThreads, smem_kv, st>>>(tk128, tv128, tq64, tdo64, tpar, p);
+      kv<<<unsigned(hq * nqb128), tg::kBwdTcThreads, smem_kv, st>>>(tk128, tv128, tq64, tdo64, tpar, p);
       if ((rc = check_launch("k_attn_bwd_kv_tc"))) return rc;
       p.nkb = nqb128;  // dgain / dtemp partials per block of 128 rows
       qk<<<unsigned(hq * nqb128), tg::kBwdTcThreads, smem_q, st>>>(tq128, tdo128, tk64, tv64, tb, p);

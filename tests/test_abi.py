@@ -173,11 +173,15 @@ def test_attention_backward_validation_and_workspace(L):
     assert call(ws=ctypes.c_void_p(260)) == 3  # workspace alignment
     al = lambda b: (b + 255) // 256 * 256
     # per query head and row the dO . o row dot, per KV head and key the dbias partial,
-    # per query head and key block of 32 the (dgain, dtemp) partials, and per query
-    # head and row (rounded up to 128) four per-row constants of the tensor-core kernels
+    # per query head and key block of 32 the (dgain, dtemp) partials, and for the
+    # tensor-core kernels per query head and row (rounded up to 128) four per-row
+    # constants and one head's (dV, dK) partial, then two counters per KV head and
+    # key block of 128
     for m in (1, 31, 32, 33, 2064):
-        nkb = (m + 31) // 32
-        m_pad = (m + 127) // 128 * 128
-        assert tg.attention_backward_workspace_bytes(m, 16, 8, 128) == \
-            al(16 * m * 4) + al(8 * m * 4) + al(16 * nkb * 8) + al(16 * m_pad * 16)
+        for dh in (64, 128):
+            nkb = (m + 31) // 32
+            m_pad = (m + 127) // 128 * 128
+            assert tg.attention_backward_workspace_bytes(m, 16, 8, dh) == \
+                al(16 * m * 4) + al(8 * m * 4) + al(16 * nkb * 8) + al(16 * m_pad * 16) + \
+                al(16 * m_pad * 2 * dh * 4) + al(2 * 8 * (m_pad // 128) * 4)
     assert tg.tg_workspace_bytes(tg.TG_OP_ATTENTION_BWD, m=0) == 0
