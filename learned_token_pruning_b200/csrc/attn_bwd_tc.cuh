@@ -124,43 +124,53 @@ __device__ __forceinline__ void stage_store32(float* stage, float* dst, int64_t 
 }
 
 // ---------------------------------------------------------------------------
-// Per-row constants: one warp per (row, head), rows m .. m_pad - 1 masked
+// Per-row constants: one warp per row, all heads (rows m .. m_pad - 1 masked).
+// A 16-byte load per lane covers 256 / D heads (D / 8 lanes each); all loads
+// of the row are issued before the lane-group reductions.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) k_attn_bwd_prep(AttnBwdParams p) {
-  const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (w >= p.m_pad * p.hq) return;  // warp-uniform
-  const int r = w / p.hq, h = w % p.hq;
-  // rows r and r ^ 1 share 8 floats: (a2, a2', nl, nl', -D, -D', as, as')
-  float* dst = p.rowpar + (int64_t(h) * (p.m_pad / 2) + r / 2) * 8 + (r & 1);
+  constexpr int kLanesPerHead = D / 8, kHeadsPerLoad = 32 / kLanesPerHead;
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (r >= p.m_pad) return;  // warp-uniform
+  // rows r and r ^ 1 share 8 floats per head: (a2, a2', nl, nl', -D, -D', as, as')
+  auto dst = [&](int h) { return p.rowpar + (int64_t(h) * (p.m_pad / 2) + r / 2) * 8 + (r & 1); };
   if (r >= p.m) {
-    if (lane == 0) {
-      dst[0] = 0.0f;
-      dst[2] = -INFINITY;
-      dst[4] = 0.0f;
-      dst[6] = 0.0f;
+    for (int h = lane; h < p.hq; h += 32) {
+      float* d = dst(h);
+      d[0] = 0.0f;
+      d[2] = -INFINITY;
+      d[4] = 0.0f;
+      d[6] = 0.0f;
     }
     return;
   }
-  const __nv_bfloat16* go = static_cast<const __nv_bfloat16*>(p.dout) + int64_t(r) * p.lddo + h * D;
-  const __nv_bfloat16* oo = static_cast<const __nv_bfloat16*>(p.o) + int64_t(r) * p.ldo + h * D;
-  float s = 0.0f;
-  if constexpr (D == 128) {
-    const uint2 a = reinterpret_cast<const uint2*>(go)[lane], b = reinterpret_cast<const uint2*>(oo)[lane];
-    s = bf16_lo(a.x) * bf16_lo(b.x) + bf16_hi(a.x) * bf16_hi(b.x) + bf16_lo(a.y) * bf16_lo(b.y) +
-        bf16_hi(a.y) * bf16_hi(b.y);
-  } else {
-    const uint32_t a = reinterpret_cast<const uint32_t*>(go)[lane], b = reinterpret_cast<const uint32_t*>(oo)[lane];
-    s = bf16_lo(a) * bf16_lo(b) + bf16_hi(a) * bf16_hi(b);
-  }
+  const float ratio_r = p.ratio ? p.ratio[r] : 1.0f;
+  const uint4* go = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dout) + int64_t(r) * p.lddo);
+  const uint4* oo = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.o) + int64_t(r) * p.ldo);
+  const int sub = lane % kLanesPerHead;
+  const int niter = (p.hq + kHeadsPerLoad - 1) / kHeadsPerLoad;
+#pragma unroll 4
+  for (int it = 0; it < niter; ++it) {
+    const int h = it * kHeadsPerLoad + lane / kLanesPerHead;
+    const bool hv = h < p.hq;
+    const uint4 a = hv ? go[h * kLanesPerHead + sub] : make_uint4(0, 0, 0, 0);
+    const uint4 b = hv ? oo[h * kLanesPerHead + sub] : make_uint4(0, 0, 0, 0);
+    const float lse = (hv && sub == 0) ? p.lse[int64_t(h) * p.m + r] : 0.0f;
+    const float th = (hv && sub == 0) ? p.temp[h] : 0.0f;
+    float sdot = bf16_lo(a.x) * bf16_lo(b.x) + bf16_hi(a.x) * bf16_hi(b.x) + bf16_lo(a.y) * bf16_lo(b.y) +
+                 bf16_hi(a.y) * bf16_hi(b.y) + bf16_lo(a.z) * bf16_lo(b.z) + bf16_hi(a.z) * bf16_hi(b.z) +
+                 bf16_lo(a.w) * bf16_lo(b.w) + bf16_hi(a.w) * bf16_hi(b.w);
 #pragma unroll
-  for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) {
-    const float as = p.temp[h] * (p.ratio ? p.ratio[r] : 1.0f) * p.sm_scale;
-    dst[0] = as * kLog2e;
-    dst[2] = -p.lse[int64_t(h) * p.m + r] * kLog2e;
-    dst[4] = -s;
-    dst[6] = as;
+    for (int off = kLanesPerHead / 2; off; off >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, off);
+    if (hv && sub == 0) {
+      const float as = th * ratio_r * p.sm_scale;
+      float* d = dst(h);
+      d[0] = as * kLog2e;
+      d[2] = -lse * kLog2e;
+      d[4] = -sdot;
+      d[6] = as;
+    }
   }
 }
 

@@ -1051,7 +1051,7 @@ int tg_gated_attention_backward(const void* q, int64_t ldq, const void* k, int64
       p.dbias_nparts = hq;
       if (cudaMemsetAsync(p.kv_ctr, 0, 2 * size_t(hkv) * nqb128 * 4, st) != cudaSuccess)
         return fail(TG_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(cudaGetLastError()));
-      prep<<<unsigned((int64_t(p.m_pad) * hq + 7) / 8), 256, 0, st>>>(p);
+      prep<<<unsigned((p.m_pad + 7) / 8), 256, 0, st>>>(p);
       if ((rc = check_launch("k_attn_bwd_prep"))) return rc;
       kv<<<unsigned(hq * nqb128), tg::kBwdTcThreads, smem_kv, st>>>(tk128, tv128, tq64, tdo64, tpar, p);
       if ((rc = check_launch("k_attn_bwd_kv_tc"))) return rc;
