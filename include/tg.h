@@ -197,9 +197,15 @@ int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk,
  *   dbias device fp32 [m] or NULL;  dgain, dtemp device fp32 [hq] or NULL
  *   ws    device workspace of tg_workspace_bytes(TG_OP_ATTENTION_BWD, 0, m, 0, 0,
  *         shape) bytes, 16-byte aligned
- * P is recomputed from lse.  CUDA cores, fp32 arithmetic; deterministic
- * (every gradient is written by one thread; cross-block sums go through the
- * workspace in a fixed order).  head_dim in {64, 128}; hq % hkv == 0.
+ * P is recomputed from lse.  bf16 operands with 16-byte aligned bases and row
+ * strides (and 16-byte aligned dq, dk, dv, bias) run on the tensor cores, with
+ * P and dS rounded to bf16 for the MMAs and fp32 accumulation; fp32 operands
+ * and other bf16 layouts run on CUDA cores in fp32.  Deterministic either way:
+ * no atomics on values, every cross-block sum is taken in a fixed order (the
+ * query heads of a KV head add their dk / dv partials in head order).
+ * head_dim in {64, 128}; hq % hkv == 0.  Errors: TG_ERR_INVALID_ARG (null
+ * pointer, m <= 0, bad heads or dtype), TG_ERR_UNSUPPORTED (head_dim, m >= 2^31),
+ * TG_ERR_SHAPE (leading dimension), TG_ERR_WORKSPACE, TG_ERR_ALIGN (workspace).
  */
 int tg_gated_attention_backward(const void* q, int64_t ldq, const void* k, int64_t ldk,
                                 const void* v, int64_t ldv, const void* out, int64_t ldo,
@@ -335,7 +341,7 @@ enum { TG_OP_GATE_SCORE = 0, TG_OP_LAYER = 1, TG_OP_ATTENTION = 2, TG_OP_DECODE 
 /* Workspace bytes needed by an op: TG_OP_GATE_SCORE uses n, d_model and h;
  * TG_OP_LAYER and TG_OP_ATTENTION use m and shape (TG_OP_ATTENTION reads its
  * dtype, hq, hkv and head_dim); TG_OP_DECODE uses m = the cache length and
- * shape's hq, hkv and head_dim; TG_OP_ATTENTION_BWD uses m and shape's hq and hkv.  Returns 0 for an invalid request, and 0 for
+ * shape's hq, hkv and head_dim; TG_OP_ATTENTION_BWD uses m and shape's hq, hkv and head_dim.  Returns 0 for an invalid request, and 0 for
  * TG_OP_ATTENTION when the attention needs no workspace. */
 size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t h, const tg_layer_shape* shape);
 
