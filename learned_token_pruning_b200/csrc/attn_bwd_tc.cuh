@@ -305,8 +305,12 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       }
       for (int j = 0; ok && j < nt; ++j) {
         const bool next = j + 2 < nt;
-        ok = mbar_wait(&ds_full[j & 1], (j >> 1) & 1, kErrWaitAttention) &&
-             (!next || mbar_wait(&kv_full[(j + 2) % kS], ((j + 2) / kS) & 1, kErrWaitAttention));
+        // both barriers tested at once (each test holds back the next MMA issue for a round trip)
+        const bool r0 = mbar_try_wait(smem_u32(&ds_full[j & 1]), (j >> 1) & 1);
+        const bool r1 = !next || mbar_try_wait(smem_u32(&kv_full[(j + 2) % kS]), ((j + 2) / kS) & 1);
+        if (!(r0 && r1))
+          ok = mbar_wait(&ds_full[j & 1], (j >> 1) & 1, kErrWaitAttention) &&
+               (!next || mbar_wait(&kv_full[(j + 2) % kS], ((j + 2) / kS) & 1, kErrWaitAttention));
         if (!ok) break;
         tc_fence_after();
         issue_dq(j);
@@ -552,8 +556,11 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       }
       for (int n = 0; ok && n < nt; ++n) {
         const bool next = n + 2 < nt;
-        ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, kErrWaitAttention) &&
-             (!next || mbar_wait(&r_full[(n + 2) % kS], ((n + 2) / kS) & 1, kErrWaitAttention));
+        const bool r0 = mbar_try_wait(smem_u32(&p_full[n & 1]), (n >> 1) & 1);
+        const bool r1 = !next || mbar_try_wait(smem_u32(&r_full[(n + 2) % kS]), ((n + 2) / kS) & 1);
+        if (!(r0 && r1))
+          ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, kErrWaitAttention) &&
+               (!next || mbar_wait(&r_full[(n + 2) % kS], ((n + 2) / kS) & 1, kErrWaitAttention));
         if (!ok) break;
         tc_fence_after();
         issue_acc(n);
