@@ -11,8 +11,9 @@
 // sum is fp32; nothing is summed by atomics, so reruns are bit-identical.
 //
 // k_attn_bwd_dq_tc: one CTA per (query head h, block of 128 rows), walking the
-//   key tiles of 64 up to the diagonal.  S = Q K^T and dP = dO V^T are SS-MMAs
-//   into double-buffered tensor memory; two warpgroups (one thread per row,
+//   key tiles of 64 up to the diagonal.  Q and dO are copied once into tensor
+//   memory, so S = Q K^T and dP = dO V^T are TS-MMAs (only K and V come from
+//   shared memory) into double-buffered tensor memory; two warpgroups (one thread per row,
 //   each taking 32 of a tile's 64 keys) turn them into dS, written as bf16
 //   pairs over the first 16 columns of their half of the S buffer, and the
 //   MMA thread accumulates dQ += dS K as a TS-MMA (K MN-major from shared
@@ -60,7 +61,8 @@ struct BwdDqCfg {
   static constexpr size_t kData = kOffBars + 256;
   // one CTA per SM, so that its 512-column TMEM allocation never waits
   static constexpr size_t kSmem = 1024 + (kData < 120 * 1024 ? 120 * 1024 : kData);
-  static constexpr uint32_t kColDP = 128, kColDQ = 256;  // S[b] at 64 b, dP[b] at 128 + 64 b
+  // S[b] at 64 b, dP[b] at 128 + 64 b, dQ, then Q and dO as packed bf16 pairs (the A operands)
+  static constexpr uint32_t kColDP = 128, kColDQ = 256, kColQ = 256 + D, kColDO = 256 + D + D / 2;
 };
 
 template <int D>
@@ -201,7 +203,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
   uint64_t* s_full = dq_done + kS;     // [2] S and dP of tile j in buffer j % 2
   uint64_t* ds_full = s_full + 2;      // [2] dS of tile j written (256 arrivals)
   uint64_t* o_final = ds_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 1);
+  uint64_t* qt_ready = o_final + 1;    // Q and dO copied into tensor memory (256 arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qt_ready + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -224,6 +227,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       mbar_init(&ds_full[b], 256);
     }
     mbar_init(o_final, 1);
+    mbar_init(qt_ready, 256);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -270,19 +274,18 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, false, false);
       constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, false, true);
-      const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t ddo0 = sdesc_sw128(smem_u32(sDO), 16, 1024);
       const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dv0 = sdesc_sw128(smem_u32(sV), 16, 1024);
       const uint64_t dkmn0 = sdesc_sw128(smem_u32(sK), Cfg::kKVBlk, 1024);
+      // S = Q K^T and dP = dO V^T take Q and dO from tensor memory (TS): per
+      // MMA only the 64-key K or V slice is read from shared memory
       auto issue_s = [&](int j) {
         const int b = j & 1, s = j % kS;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ao = ((kk >> 2) * Cfg::kQBlk + (kk & 3) * 32) >> 4;
           const uint32_t bo = (s * Cfg::kKVBytes + (kk >> 2) * Cfg::kKVBlk + (kk & 3) * 32) >> 4;
-          umma_ss(tmem + 64 * b, dq0 + ao, dk0 + bo, idesc_s, kk != 0 ? 1u : 0u);
-          umma_ss(tmem + Cfg::kColDP + 64 * b, ddo0 + ao, dv0 + bo, idesc_s, kk != 0 ? 1u : 0u);
+          umma_ts(tmem + 64 * b, tmem + Cfg::kColQ + kk * 8, dk0 + bo, idesc_s, kk != 0 ? 1u : 0u);
+          umma_ts(tmem + Cfg::kColDP + 64 * b, tmem + Cfg::kColDO + kk * 8, dv0 + bo, idesc_s, kk != 0 ? 1u : 0u);
         }
         umma_commit(&s_full[b]);
       };
@@ -294,7 +297,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                   dkmn0 + ((s * Cfg::kKVBytes + kk * 16 * 128) >> 4), idesc_dq, (j | kk) != 0 ? 1u : 0u);
         umma_commit(&dq_done[s]);
       };
-      bool ok = mbar_wait2(q_full, 0, &kv_full[0], 0, kErrWaitAttention);
+      bool ok = mbar_wait2(qt_ready, 0, &kv_full[0], 0, kErrWaitAttention);
       if (ok) {
         tc_fence_after();
         issue_s(0);
@@ -333,6 +336,31 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
                    ggp = f2_pack(gg, gg);
     uint64_t dgain2 = 0, dtz2 = 0;  // (even keys, odd keys) partial sums
     bool ok = true;
+    // warpgroup 0 copies the Q rows, warpgroup 1 the dO rows, from their TMA
+    // tiles (128-byte swizzled boxes of 64 columns) into tensor memory as
+    // packed bf16 pairs: thread = row = TMEM lane
+    if (warp_wait(q_full, 0, kErrWaitAttention)) {
+      const uint8_t* tile = (wg ? sDO : sQ) + row * 128;
+      const uint32_t col = wg ? Cfg::kColDO : Cfg::kColQ;
+#pragma unroll
+      for (int bx = 0; bx < kDBoxes; ++bx) {
+        uint32_t v[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 x = *reinterpret_cast<const uint4*>(tile + bx * Cfg::kQBlk + ((c ^ (row & 7)) << 4));
+          v[4 * c] = x.x;
+          v[4 * c + 1] = x.y;
+          v[4 * c + 2] = x.z;
+          v[4 * c + 3] = x.w;
+        }
+        tmem_st32(tmem + lane_base + col + 32 * bx, v);
+      }
+      tmem_st_wait();
+    } else {
+      ok = false;
+    }
+    tc_fence_before();
+    mbar_arrive(qt_ready);
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1;
       bool rdy = !*abort_flag &&
