@@ -152,26 +152,39 @@ __global__ void __launch_bounds__(256) k_attn_bwd_prep(AttnBwdParams p) {
   const uint4* oo = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.o) + int64_t(r) * p.ldo);
   const int sub = lane % kLanesPerHead;
   const int niter = (p.hq + kHeadsPerLoad - 1) / kHeadsPerLoad;
-#pragma unroll 4
-  for (int it = 0; it < niter; ++it) {
-    const int h = it * kHeadsPerLoad + lane / kLanesPerHead;
-    const bool hv = h < p.hq;
-    const uint4 a = hv ? go[h * kLanesPerHead + sub] : make_uint4(0, 0, 0, 0);
-    const uint4 b = hv ? oo[h * kLanesPerHead + sub] : make_uint4(0, 0, 0, 0);
-    const float lse = (hv && sub == 0) ? p.lse[int64_t(h) * p.m + r] : 0.0f;
-    const float th = (hv && sub == 0) ? p.temp[h] : 0.0f;
-    float sdot = bf16_lo(a.x) * bf16_lo(b.x) + bf16_hi(a.x) * bf16_hi(b.x) + bf16_lo(a.y) * bf16_lo(b.y) +
-                 bf16_hi(a.y) * bf16_hi(b.y) + bf16_lo(a.z) * bf16_lo(b.z) + bf16_hi(a.z) * bf16_hi(b.z) +
-                 bf16_lo(a.w) * bf16_lo(b.w) + bf16_hi(a.w) * bf16_hi(b.w);
+  // chunks of kChunk loads per operand, all issued before any use (the stores
+  // of a chunk would otherwise keep the next chunk's loads behind them)
+  constexpr int kChunk = 8;
+  for (int it0 = 0; it0 < niter; it0 += kChunk) {
+    uint4 a[kChunk], b[kChunk];
+    float lse[kChunk], th[kChunk];
 #pragma unroll
-    for (int off = kLanesPerHead / 2; off; off >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, off);
-    if (hv && sub == 0) {
-      const float as = th * ratio_r * p.sm_scale;
-      float* d = dst(h);
-      d[0] = as * kLog2e;
-      d[2] = -lse * kLog2e;
-      d[4] = -sdot;
-      d[6] = as;
+    for (int c = 0; c < kChunk; ++c) {
+      const int h = (it0 + c) * kHeadsPerLoad + lane / kLanesPerHead;
+      const bool hv = it0 + c < niter && h < p.hq;
+      a[c] = hv ? go[h * kLanesPerHead + sub] : make_uint4(0, 0, 0, 0);           // dO: read again by the MMAs
+      b[c] = hv ? __ldcs(oo + h * kLanesPerHead + sub) : make_uint4(0, 0, 0, 0);  // o: this pass only
+      lse[c] = (hv && sub == 0) ? p.lse[int64_t(h) * p.m + r] : 0.0f;
+      th[c] = (hv && sub == 0) ? p.temp[h] : 0.0f;
+    }
+#pragma unroll
+    for (int c = 0; c < kChunk; ++c) {
+      const int h = (it0 + c) * kHeadsPerLoad + lane / kLanesPerHead;
+      const bool hv = it0 + c < niter && h < p.hq;
+      float sdot = bf16_lo(a[c].x) * bf16_lo(b[c].x) + bf16_hi(a[c].x) * bf16_hi(b[c].x) +
+                   bf16_lo(a[c].y) * bf16_lo(b[c].y) + bf16_hi(a[c].y) * bf16_hi(b[c].y) +
+                   bf16_lo(a[c].z) * bf16_lo(b[c].z) + bf16_hi(a[c].z) * bf16_hi(b[c].z) +
+                   bf16_lo(a[c].w) * bf16_lo(b[c].w) + bf16_hi(a[c].w) * bf16_hi(b[c].w);
+#pragma unroll
+      for (int off = kLanesPerHead / 2; off; off >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, off);
+      if (hv && sub == 0) {
+        const float as = th[c] * ratio_r * p.sm_scale;
+        float* d = dst(h);
+        d[0] = as * kLog2e;
+        d[2] = -lse[c] * kLog2e;
+        d[4] = -sdot;
+        d[6] = as;
+      }
     }
   }
 }
