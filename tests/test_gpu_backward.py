@@ -156,3 +156,26 @@ def test_backward_bf16_unaligned_rows_use_the_cuda_core_kernels(m):
     for n in NAMES:
         scale = max(np.max(np.abs(got[n])), FLOOR)
         assert np.max(np.abs(tc[n] - got[n])) <= 2 * TOL["bf16"] * scale, n
+
+
+def test_backward_kept_rows_of_the_128k_prompt_properties_and_sampled_rows():
+    # 8256 rows (the 128K-token prompt's kept rows) in the bench's configuration:
+    # every gradient finite, the bias gradient summing to zero over keys,
+    # bit-identical reruns, and sampled query rows r against the oracle run on
+    # rows 0 .. r (row r's dq depends only on its causal prefix)
+    m, hq, hkv, dh = 8256, 16, 8, 128
+    q, k, v, do, bias, ratio, gain, temp = _case(m, hq, hkv, dh, "bf16", seed=8256)
+    a = _gpu(q, k, v, do, bias, ratio, gain, temp, "bf16")
+    b = _gpu(q, k, v, do, bias, ratio, gain, temp, "bf16")
+    for n in NAMES:
+        assert np.all(np.isfinite(a[n])), n
+        assert np.array_equal(a[n], b[n]), n
+    assert abs(a["dbias"].sum()) <= 2e-3 * np.abs(a["dbias"]).sum()
+    scale = 1.0 / math.sqrt(dh)
+    for r in (0, 63, 64, 127, 128, 255, 383):
+        sl = slice(0, r + 1)
+        want = O.gated_attention_backward(q[sl], k[sl], v[sl], bias[sl], gain, temp, ratio[sl], scale, do[sl])
+        w = want["dq"][r].reshape(-1)
+        got = a["dq"][r]
+        tol = TOL["bf16"] * max(np.max(np.abs(w)), FLOOR)
+        assert np.max(np.abs(got - w)) <= tol, r
