@@ -13,11 +13,11 @@
 // k_attn_bwd_dq_tc: one CTA per (query head h, block of 128 rows), walking the
 //   key tiles of 64 up to the diagonal.  Q and dO are copied once into tensor
 //   memory, so S = Q K^T and dP = dO V^T are TS-MMAs (only K and V come from
-//   shared memory) into double-buffered tensor memory; two warpgroups (one thread per row,
-//   each taking 32 of a tile's 64 keys) turn them into dS, written as bf16
-//   pairs over the first 16 columns of their half of the S buffer, and the
-//   MMA thread accumulates dQ += dS K as a TS-MMA (K MN-major from shared
-//   memory).  The row's dgain / dtemp contributions are summed on the way.
+//   shared memory) into double-buffered tensor memory; two warpgroups (one
+//   thread per row, each taking 32 of a tile's 64 keys) turn them into dS,
+//   written as bf16 pairs over the first 16 columns of their half of the S
+//   buffer, and the MMA thread accumulates dQ += dS K as a TS-MMA (K MN-major
+//   from shared memory).  The row's dgain / dtemp terms are summed on the way.
 // k_attn_bwd_kv_tc: one CTA per (query head h, block of 128 keys), walking the
 //   query tiles of 64 rows from the diagonal on.
 //   S^T = K Q^T and dP^T = V dO^T (one thread per key), P^T and dS^T as bf16
