@@ -332,16 +332,16 @@ def rope(x, pos, theta: float) -> np.ndarray:
     return np.concatenate([x1 * cos - x2 * sin, x2 * cos + x1 * sin], axis=-1)
 
 
-def decoder_layer(hidden, weights: Dict[str, np.ndarray], *, hq: int, hkv: int, head_dim: int,
-                  pos, bias, ratio, head_gain, head_temp, rope_theta: float, qk_norm: bool,
-                  norm_eps: float = 1e-6, rows: Optional[Sequence[int]] = None) -> np.ndarray:
-    """One Qwen3-shaped decoder layer run on the kept rows only.
+def attention_block(hidden, weights: Dict[str, np.ndarray], *, hq: int, hkv: int, head_dim: int,
+                    pos, bias, ratio, head_gain, head_temp, rope_theta: float, qk_norm: bool,
+                    norm_eps: float = 1e-6, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """The attention half of a Qwen3-shaped decoder layer: the post-attention
+    residual h + Attn(RMSNorm(h)) Wo^T.
 
     RMSNorm -> QKV projection -> (per-head q/k RMSNorm) -> RoPE at the original
-    positions -> token-gated attention -> O projection + residual -> RMSNorm ->
-    SwiGLU MLP + residual.  Linear weights are [out, in]; w_gate_up stacks the
-    gate rows over the up rows.  All float64.  With `rows`, only those output
-    rows are produced (keys and values still come from every row).
+    positions -> token-gated attention -> O projection + residual.  Linear
+    weights are [out, in].  All float64.  With `rows`, only those output rows
+    are produced (keys and values still come from every row).
     """
     h = np.asarray(hidden, dtype=F64)
     mrows = h.shape[0]
@@ -357,12 +357,36 @@ def decoder_layer(hidden, weights: Dict[str, np.ndarray], *, hq: int, hkv: int, 
     q = rope(q, pos, rope_theta)
     k = rope(k, pos, rope_theta)
     a = gated_attention(q, k, v, bias, head_gain, head_temp, ratio, 1.0 / math.sqrt(head_dim), rows=sel)
-    h1 = h[sel] + a.reshape(sel.size, hq * head_dim) @ np.asarray(weights["w_o"], dtype=F64).T
+    return h[sel] + a.reshape(sel.size, hq * head_dim) @ np.asarray(weights["w_o"], dtype=F64).T
+
+
+def mlp_block(hidden, weights: Dict[str, np.ndarray], *, norm_eps: float = 1e-6) -> np.ndarray:
+    """The MLP half of a Qwen3-shaped decoder layer, row by row:
+    h + (SiLU(y Wg^T) * (y Wu^T)) Wd^T with y = RMSNorm(h) (post-attention
+    norm); w_gate_up stacks the gate rows over the up rows.  float64."""
+    h1 = np.asarray(hidden, dtype=F64)
     y = rms_norm(h1, weights["w_post_norm"], norm_eps)
     gu = y @ np.asarray(weights["w_gate_up"], dtype=F64).T
     d_ff = gu.shape[1] // 2
     act = silu(gu[:, :d_ff]) * gu[:, d_ff:]
     return h1 + act @ np.asarray(weights["w_down"], dtype=F64).T
+
+
+def decoder_layer(hidden, weights: Dict[str, np.ndarray], *, hq: int, hkv: int, head_dim: int,
+                  pos, bias, ratio, head_gain, head_temp, rope_theta: float, qk_norm: bool,
+                  norm_eps: float = 1e-6, rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """One Qwen3-shaped decoder layer run on the kept rows only: the attention
+    half (attention_block) followed by the MLP half (mlp_block).
+
+    RMSNorm -> QKV projection -> (per-head q/k RMSNorm) -> RoPE at the original
+    positions -> token-gated attention -> O projection + residual -> RMSNorm ->
+    SwiGLU MLP + residual.  All float64.  With `rows`, only those output rows
+    are produced (keys and values still come from every row).
+    """
+    h1 = attention_block(hidden, weights, hq=hq, hkv=hkv, head_dim=head_dim, pos=pos, bias=bias, ratio=ratio,
+                         head_gain=head_gain, head_temp=head_temp, rope_theta=rope_theta, qk_norm=qk_norm,
+                         norm_eps=norm_eps, rows=rows)
+    return mlp_block(h1, weights, norm_eps=norm_eps)
 
 
 def pruned_prefill_step(hidden, gate: Dict[str, np.ndarray], k: int, layer: Dict[str, np.ndarray], *,
@@ -391,42 +415,57 @@ def pruned_prefill_step(hidden, gate: Dict[str, np.ndarray], k: int, layer: Dict
 
 
 # ---------------------------------------------------------------------------
-# A whole decoder stack  ([R] §4.1 three-stage forward)
+# A whole decoder stack  ([R] §4.1 three-stage forward and Gate module; [K]
+# "tying the mechanism together"; [M] "how does learned token pruning work")
 # ---------------------------------------------------------------------------
 def pruned_prefill_stack(hidden, layers: Sequence[Dict[str, np.ndarray]], heads: Sequence[Dict[str, np.ndarray]],
-                         gate: Dict[str, np.ndarray], k: int, gate_after: int, *, hq: int, hkv: int,
+                         gate: Dict[str, np.ndarray], k: int, gate_layer: int, *, hq: int, hkv: int,
                          head_dim: int, rope_theta: float, qk_norm: bool, norm_eps: float = 1e-6,
                          eps_s: float = 1e-6, pruned: bool = True) -> Dict[str, np.ndarray]:
     """Prefill of one prompt through len(layers) decoder layers.
 
-    [R] §4.1 splits the forward in three: layers below the gate run on every
-    token; the gate scores the tokens, keeps the top-K documents tokens plus
-    the question and compacts them in order; the layers above run on the kept
-    tokens only, with token-gated attention.  Here layers 0 .. gate_after run
-    on all N rows (positions 0..N-1, no gate bias, ratio 1, temperature 1);
-    READING: the gate after layer L scores the residual stream leaving layer L
-    (normalised by gate['norm_w']); layers gate_after+1 .. run on the kept rows
-    with each layer's head gain and temperature (heads[l]).  With pruned=False
-    every layer runs on all rows with no gate: the unpruned stack.
+    [R] §4.1 splits the forward in three: below the gate every token is
+    processed; at gate layer L the gate scores each prunable token from that
+    layer's normalised post-attention residual, the top-K document tokens
+    plus every question token are kept and compacted in order; everything
+    after runs on the kept tokens only, with token-gated attention in the
+    layers above L ([K] and [M] place the scoring in the same spot: after
+    layer L's attention).  So here:
+      layers 0 .. L-1        all N rows (positions 0..N-1, no gate bias,
+                             ratio 1, temperature 1);
+      layer L, attention     all N rows, the same way -> residual h1 (N rows);
+      gate                   scores RMSNorm(h1) * w_post_norm of layer L (READING:
+                             the gate's normalisation is layer L's own
+                             post-attention RMSNorm, the vector layer L's MLP
+                             reads), select, gather the kept rows of h1;
+      layer L, MLP           the kept rows only (row-wise, so the same rows as
+                             running it on all N and gathering afterwards);
+      layers L+1 ..          the kept rows with each layer's head gain and
+                             temperature (heads[l]).
+    With pruned=False every layer runs on all rows with no gate: the unpruned
+    stack.  gate["norm_w"] is not used here (the layer's weight takes its place).
     """
     h = np.asarray(hidden, dtype=F64)
     n = h.shape[0]
     pos = np.arange(n)
     n_layers = len(layers)
     common = dict(hq=hq, hkv=hkv, head_dim=head_dim, rope_theta=rope_theta, qk_norm=qk_norm, norm_eps=norm_eps)
-    n_full = n_layers if not pruned else gate_after + 1
-    for l in range(n_full):
-        h = decoder_layer(h, layers[l], pos=pos, bias=None, ratio=None, head_gain=np.zeros(hq),
-                          head_temp=np.ones(hq), **common)
+    flat = dict(pos=pos, bias=None, ratio=None, head_gain=np.zeros(hq), head_temp=np.ones(hq))
     if not pruned:
+        for l in range(n_layers):
+            h = decoder_layer(h, layers[l], **flat, **common)
         return {"out": h}
+    for l in range(gate_layer):
+        h = decoder_layer(h, layers[l], **flat, **common)
+    h1 = attention_block(h, layers[gate_layer], **flat, **common)
     prunable = gate["prunable"]
-    s = gate_scores(h, gate["norm_w"], norm_eps, gate["w1"], gate["b1"], gate["w2"], gate["b2"], prunable)
+    s = gate_scores(h1, layers[gate_layer]["w_post_norm"], norm_eps, gate["w1"], gate["b1"], gate["w2"], gate["b2"],
+                    prunable)
     s32 = s.astype(np.float32)
     idx = select_kept(s32, prunable, k)
-    g = gather(h, idx, s32, prunable, eps_s)
-    hk = g["hidden_kept"]
-    for l in range(gate_after + 1, n_layers):
+    g = gather(h1, idx, s32, prunable, eps_s)
+    hk = mlp_block(g["hidden_kept"], layers[gate_layer], norm_eps=norm_eps)
+    for l in range(gate_layer + 1, n_layers):
         hk = decoder_layer(hk, layers[l], pos=g["pos"], bias=g["bias"], ratio=g["ratio"],
                            head_gain=heads[l]["head_gain"], head_temp=heads[l]["head_temp"], **common)
-    return {"gate_input": h, "scores": s, "kept_idx": idx, **g, "out": hk}
+    return {"gate_input": h1, "scores": s, "kept_idx": idx, **g, "out": hk}

@@ -498,31 +498,99 @@ def _stack_case(n_layers=4):
     return w, synth.gate_inputs(w), layers, heads
 
 
-def _stack(w, g, layers, heads, k, gate_after, pruned=True):
-    return O.pruned_prefill_stack(g["hidden"], layers, heads, g, k, gate_after, hq=w.hq, hkv=w.hkv,
+def _stack(w, g, layers, heads, k, gate_layer, pruned=True):
+    return O.pruned_prefill_stack(g["hidden"], layers, heads, g, k, gate_layer, hq=w.hq, hkv=w.hkv,
                                   head_dim=w.head_dim, rope_theta=w.rope_theta, qk_norm=True, pruned=pruned)
 
 
 def test_stack_keeping_everything_with_zero_gain_is_the_unpruned_stack():
     w, g, layers, heads = _stack_case()
     flat = [{"head_gain": np.zeros(w.hq), "head_temp": np.ones(w.hq)} for _ in layers]
-    res = _stack(w, g, layers, flat, w.n, gate_after=1)
+    res = _stack(w, g, layers, flat, w.n, gate_layer=1)
     assert list(res["kept_idx"]) == list(range(w.n))
-    full = _stack(w, g, layers, heads, w.n, gate_after=1, pruned=False)
+    full = _stack(w, g, layers, heads, w.n, gate_layer=1, pruned=False)
     np.testing.assert_allclose(res["out"], full["out"], rtol=1e-12, atol=1e-12)
 
 
 def test_stack_gate_at_the_top_gathers_the_unpruned_output():
     w, g, layers, heads = _stack_case(3)
-    res = _stack(w, g, layers, heads, w.k, gate_after=2)
-    full = _stack(w, g, layers, heads, w.k, gate_after=2, pruned=False)
+    res = _stack(w, g, layers, heads, w.k, gate_layer=2)
+    full = _stack(w, g, layers, heads, w.k, gate_layer=2, pruned=False)
     assert len(res["kept_idx"]) == w.k + w.n_question
-    np.testing.assert_array_equal(res["out"], full["out"][res["kept_idx"]])
+    # layer 2's MLP runs on the kept rows only, a row-wise step: equal up to
+    # the summation order of the matmul over fewer rows
+    np.testing.assert_allclose(res["out"], full["out"][res["kept_idx"]], rtol=1e-12, atol=1e-12)
+
+
+def test_stack_layer_mlp_runs_on_the_kept_rows_only():
+    # the gate sits inside layer L (after its attention): with the gate in the
+    # middle of the stack, the kept rows entering layer L+1 are layer L's
+    # unpruned output at those rows (its MLP is row-wise), and the pruned
+    # output differs from the unpruned one (the layers above see fewer keys)
+    w, g, layers, heads = _stack_case(3)
+    res = _stack(w, g, layers, heads, w.k, gate_layer=1)
+    two = _stack(w, g, layers[:2], heads, w.k, gate_layer=1, pruned=False)["out"]
+    idx = res["kept_idx"]
+    hk = O.mlp_block(res["hidden_kept"], layers[1])
+    np.testing.assert_allclose(hk, two[idx], rtol=1e-12, atol=1e-12)
+    full = _stack(w, g, layers, heads, w.k, gate_layer=1, pruned=False)["out"]
+    assert np.max(np.abs(res["out"] - full[idx])) > 1e-3
+
+
+def _hf_chain_gate_input(w, g, layers, gate_layer):
+    """Run transformers Qwen3DecoderLayers 0..gate_layer and capture, with
+    forward hooks, the input and output of layer gate_layer's
+    post_attention_layernorm: its post-attention residual and that residual
+    normalised by the layer's own RMSNorm."""
+    x = torch.from_numpy(np.asarray(g["hidden"], dtype=np.float64))[None]
+    pid = torch.arange(w.n)[None]
+    mask = torch.zeros(w.n, w.n, dtype=torch.float64).masked_fill(
+        ~torch.ones(w.n, w.n, dtype=torch.bool).tril(), float("-inf"))[None, None]
+    seen = {}
+    with torch.no_grad():
+        for l in range(gate_layer + 1):
+            layer, rot = _hf_layer(w, layers[l], w.n)
+            if l == gate_layer:
+                def hook(mod, args, out):
+                    seen["in"] = args[0][0].clone()
+                    seen["out"] = out[0].clone()
+                layer.post_attention_layernorm.register_forward_hook(hook)
+            cos, sin = rot(x, pid)
+            x = layer(x, attention_mask=mask, position_ids=pid, position_embeddings=(cos, sin))
+            x = x[0] if isinstance(x, tuple) else x
+    return seen["in"].numpy(), seen["out"].numpy()
+
+
+@pytest.mark.parametrize("gate_layer", [0, 1, 2])
+def test_stack_gate_reads_the_post_attention_residual_of_its_layer(gate_layer):
+    # [R] §4.1 Gate module / [K] / [M]: the gate scores layer L's normalised
+    # post-attention residual.  Pinned against transformers' Qwen3 layer: the
+    # input of layer L's post_attention_layernorm is the oracle's gate input,
+    # and that norm's output fed to the gate MLP gives the oracle's scores.
+    w, g, layers, heads = _stack_case(3)
+    w = w.replace(k=6)
+    g = dict(g)
+    # a non-trivial post-attention norm weight, so that taking the gate's
+    # normalisation from the wrong place shows
+    rng = np.random.default_rng(11)
+    layers = [dict(lw) for lw in layers]
+    layers[gate_layer]["w_post_norm"] = rng.uniform(0.5, 1.5, w.d_model)
+    res = _stack(w, g, layers, heads, w.k, gate_layer=gate_layer)
+    hf_in, hf_out = _hf_chain_gate_input(w, g, layers, gate_layer)
+    np.testing.assert_allclose(res["gate_input"], hf_in, rtol=1e-5, atol=1e-5)
+    t = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+    u = F.linear(t(hf_out), t(g["w1"]), t(g["b1"]))
+    s_hf = (F.silu(u) @ t(g["w2"]) + float(g["b2"])).numpy()
+    s_hf = np.where(np.asarray(g["prunable"]) != 0, s_hf, 0.0)
+    np.testing.assert_allclose(res["scores"], s_hf, rtol=1e-5, atol=1e-7)
+    # the residual leaving layer L (after its MLP) is a different vector
+    leaving = _stack(w, g, layers[: gate_layer + 1], heads, w.k, gate_layer=0, pruned=False)["out"]
+    assert np.max(np.abs(leaving - res["gate_input"])) > 1e-3
 
 
 def test_unpruned_stack_matches_a_chain_of_transformers_layers():
     w, g, layers, heads = _stack_case(3)
-    ours = _stack(w, g, layers, heads, w.k, gate_after=0, pruned=False)["out"]
+    ours = _stack(w, g, layers, heads, w.k, gate_layer=0, pruned=False)["out"]
     x = torch.from_numpy(np.asarray(g["hidden"], dtype=np.float64))[None]
     pid = torch.arange(w.n)[None]
     mask = torch.zeros(w.n, w.n, dtype=torch.float64).masked_fill(
