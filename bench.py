@@ -33,7 +33,7 @@ METRIC = "gated-prefill tokens/s & TTFT ms at N=16K/128K; attention % bf16 peak"
 L2_FLUSH_BYTES = 256 << 20   # > the 126 MB L2
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch, from
-# an ncu capture of `bench.py --ncu-case` (profiles/ncu_full_gate_attention_swiglu_case.md),
+# an ncu capture of `bench.py --ncu-case` (its summary is kept under profiles/),
 # with the rows that launch processed; scaled to the bench launch by rows.  A
 # record counts only while the SHA-256 of its kernel's sources still matches.
 MEASURED_TRAFFIC = {
@@ -74,14 +74,19 @@ def load_peaks():
 
 
 def workload_work(w, m):
-    """Algorithmic bytes / flops of each call of one step ('roofline')."""
+    """Algorithmic bytes / flops of each call of one step: the gate reads every
+    hidden row once (plus mask, score and W1), the selector its scores and mask
+    and writes the kept indices, the gather reads and writes each kept row
+    (the fused gather + RMSNorm writes it twice), attention counts the kept
+    causal pairs times the two contractions, each GEMM 2*M*K*N."""
     n, dm, h, D, hq, hkv, dff = w.n, w.d_model, w.gate_hidden, w.head_dim, w.hq, w.hkv, w.d_ff
     es = 2 if w.dtype == "bf16" else 4
     qkv = (hq + 2 * hkv) * D
     return {
         "gate_score": {"bytes": n * dm * es + n * 1 + n * 4 + h * dm * es, "flops": 2 * n * dm * h},
         "topk_select": {"bytes": n * 4 + n * 1 + m * 4},
-        "gather": {"bytes": 2 * m * dm * es + m * 4 * 5},
+        "unfused_gather": {"bytes": 2 * m * dm * es + m * 4 * 5},
+        "gather_rmsnorm": {"bytes": 3 * m * dm * es + m * 4 * 5 + dm * 4},
         "attention": {"flops": 2 * D * hq * m * (m + 1)},
         "linear_qkv": {"flops": 2 * m * dm * qkv},
         "linear_o": {"flops": 2 * m * hq * D * dm},
@@ -266,7 +271,7 @@ def config_dict(w, world):
             "kept_rows": w.m, "d_model": w.d_model, "heads": f"{w.hq}/{w.hkv}x{w.head_dim}",
             "gate_mlp": f"{w.d_model}->{w.gate_hidden}->1", "d_ff": w.d_ff, "layers_above_gate": 1,
             "parallelism": f"replicas x{world}", "l2": "flushed (256 MiB write) before every timed step",
-            "launch": "one CUDA graph per step (gate, select, gather, layer)"}
+            "launch": "one CUDA graph per step (gate, select, gather folded into the layer's RMSNorm, layer)"}
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -343,7 +348,9 @@ def run_gpu(args, w):
         if name == "gate_score":
             entry["tflops"] = wk["flops"] / (ms * 1e-3) / 1e12
         kernels[name] = entry
-    dom = max((k for k in kernels if k != "layer_total" and kernels[k]["us"] > 0), key=lambda k: kernels[k]["us"])
+    kernels["unfused_gather"]["in_step"] = False   # tg_gather alone: the step folds it into the layer's RMSNorm
+    dom = max((k for k in kernels if k not in ("gather_layer_total", "unfused_gather") and kernels[k]["us"] > 0),
+              key=lambda k: kernels[k]["us"])
     wk = work[dom]
     traffic = measured_traffic(dom, w.n if dom == "gate_score" else m)
     if "flops" in wk and dom != "gate_score":
@@ -358,11 +365,27 @@ def run_gpu(args, w):
     # ---- end to end through the public API: pinned host inputs in, result back to the host
     e2e = end_to_end(step, w, args, stream, flush, dist, dev, world)
 
-    launches_per_step = 11  # gate(1) + select(1) + gather(1) + layer(rmsnorm, qkv, rope, attn, o, rmsnorm, mlp-up, down)
+    # gate, select, gather + RMSNorm, then qkv, q/k-norm + RoPE, attention, o, RMSNorm, gate/up + SwiGLU, down
+    launches_per_step = 10
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()
         return
+    # ---- the rest of the metric (single GPU only): the 128K-token step and the
+    # 28-layer stack's time to first token at 16K and 128K, pruned and not
+    ttft = {"gated_layer_step_n16384": ms_per_step}
+    att_frac = {f"n{w.n}_m{m}": kernels["attention"].get("frac_bf16_peak")}
+    extras = {}
+    if world == 1 and not args.no_extras:
+        from learned_token_pruning_b200 import synth
+        w128 = synth.long_128k()
+        long = single_layer_step(w128, dev, stream, flush, 10, peaks)
+        ttft["gated_layer_step_n131072"] = long["step_ms"]
+        att_frac[f"n{w128.n}_m{long['kept_rows']}"] = long["attention"]["frac_bf16_peak"]
+        extras["long_context_step"] = long
+        for n_, k_ in ((16384, 2000), (131072, 8192)):
+            r = stack_ttft(n_, k_, [13, 1], 3, dev, stream)
+            ttft[f"stack28_n{n_}"] = r
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         sec, desc, threads = oracle_step_seconds(w)
@@ -372,7 +395,7 @@ def run_gpu(args, w):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) hidden, N(0,0.02) weights)",
         "config": config_dict(w, world),
-        "ttft_ms": {"gated_layer_step": ms_per_step},
+        "ttft_ms": ttft, "attention_frac_bf16_peak": att_frac, **extras,
         "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks, "wall_s": wall,
@@ -399,10 +422,13 @@ def breakdown(step, w, args, stream, flush):
     L = step.layer
     aws_n = tg.attention_workspace_bytes(m, hq, hkv, D, dt)
     aws = torch.empty(max(aws_n, 16), dtype=torch.uint8, device=stream.device) if aws_n else None
+    hk_buf = torch.empty_like(step.hidden_kept)
     calls = {
         "gate_score": step.gate_score,
         "topk_select": step.select,
-        "gather": step.gather,
+        "gather_rmsnorm": lambda: tg.tg_gather_rmsnorm(step.hidden, step.kept, step.scores, step.sumsq,
+                                                       step.n_prunable, step.eps_s, L["w_in_norm"], step.norm_eps,
+                                                       hk_buf, xn, step.pos, step.bias, step.ratio),
         "attention": lambda: tg.tg_gated_attention(qkv[:, :hq * D], qkv[:, hq * D:(hq + hkv) * D],
                                                    qkv[:, (hq + hkv) * D:], D, step.bias, L["head_gain"],
                                                    L["head_temp"], step.ratio, 1.0 / math.sqrt(D), att,
@@ -411,7 +437,8 @@ def breakdown(step, w, args, stream, flush):
         "linear_o": lambda: tg.tg_linear(att, L["w_o"], hres, tg.TG_EPI_RESIDUAL),
         "linear_gate_up_swiglu": lambda: tg.tg_linear(xn, L["w_gate_up"], act, tg.TG_EPI_SWIGLU),
         "linear_down": lambda: tg.tg_linear(act, L["w_down"], hres, tg.TG_EPI_RESIDUAL),
-        "layer_total": step.layer_above,
+        "gather_layer_total": step.gather_layer,
+        "unfused_gather": step.gather,
     }
     step.run()
     torch.cuda.synchronize()
@@ -871,65 +898,119 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
-def run_stack(args):
+def stack_ttft(n, k, gate_layers, reps, dev, stream):
     """Time to first token of a random-init 28-layer Qwen3-1.7B-shaped stack
-    (gate after layer 13, or --gate-after L) against the same stack unpruned,
-    at N = 16K, 64K and 128K: from the layer-0 hidden states in HBM to the last layer's output for
-    the kept rows (embedding, final norm and LM head are not part of the path).
-    One JSON line per N."""
+    with the gate at each layer in `gate_layers` (scoring that layer's
+    post-attention residual), against the same stack unpruned: from the layer-0
+    hidden states in HBM to the last layer's output for the kept rows
+    (embedding, final norm and LM head are not part of the path).  Median of
+    `reps` runs after one untimed run of each.  Returns a dict."""
     import torch
     from learned_token_pruning_b200 import pipeline, synth, tokengate as tg
+    w = synth.full_stack_64k(n=n, k=k, name=f"qwen3_1.7b_stack28_n{n}_k{k}")
+    torch.cuda.reset_peak_memory_stats(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    hidden = torch.randn(n, w.d_model, generator=g, device=dev).to(torch.bfloat16)
+    prunable = torch.ones(n, dtype=torch.uint8, device=dev)
+    prunable[n - w.n_question:] = 0
+    gate = {"w1": (torch.randn(w.gate_hidden, w.d_model, generator=g, device=dev) * 0.02).to(torch.bfloat16),
+            "b1": torch.zeros(w.gate_hidden, device=dev),
+            "w2": torch.randn(w.gate_hidden, generator=g, device=dev) * 0.02, "b2": 0.0}
+    layers, heads = pipeline.stack_weights_on_device(w, w.n_layers, dev)
+    stacks = {L: pipeline.PrunedPrefillStack(w, hidden, prunable, gate, layers, heads, L) for L in gate_layers}
+
+    def timed(st, fn, reps):
+        out = []
+        for _ in range(reps):
+            st.reset()
+            torch.cuda.synchronize(dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            out.append(a.elapsed_time(b))
+        return sorted(out)[len(out) // 2]
+
+    st0 = stacks[gate_layers[0]]
+    for L, st in stacks.items():
+        timed(st, st.run, 1)
+    timed(st0, st0.unpruned, 1)
+    tg.tg_check_device_error()
+    t_full = timed(st0, st0.unpruned, reps)
+    res = {"workload": w.name, "n": n, "k": k, "kept_rows": st0.m, "layers": w.n_layers,
+           "ttft_unpruned_ms": round(t_full, 3), "reps": reps, "gate": {}}
+    for L, st in stacks.items():
+        t = timed(st, st.run, reps)
+        res["gate"][f"layer{L}"] = {"ttft_ms": round(t, 3), "speedup": round(t_full / t, 3),
+                                    "tokens_per_s": n / (t * 1e-3)}
+    tg.tg_check_device_error()
+    res["peak_hbm_gb"] = round(torch.cuda.max_memory_allocated(dev) / 1e9, 3)
+    del stacks, st0, layers, heads, hidden
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_stack(args):
+    """The 28-layer stack TTFT at N = 16K, 64K and 128K (gate at layer 13, or
+    --gate-layer L), pruned against unpruned; one JSON line per N."""
+    import torch
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream(dev)
     sizes = [(16384, 2000), (65536, 4096), (131072, 8192)]
     if args.stack_n:
         sizes = [x for x in sizes if x[0] in args.stack_n]
+    gl = [args.gate_layer] if args.gate_layer is not None else [13]
     for n, k in sizes:
-        w = synth.full_stack_64k(n=n, k=k, name=f"qwen3_1.7b_stack28_n{n}_k{k}")
-        if args.gate_after is not None:
-            # the gate after layer L (TokenGate's own default is the first layer)
-            w = dataclasses.replace(w, gate_after=args.gate_after,
-                                    name=f"qwen3_1.7b_stack28_gate{args.gate_after}_n{n}_k{k}")
-        torch.cuda.reset_peak_memory_stats(dev)
-        g = torch.Generator(device=dev)
-        g.manual_seed(w.seed)
-        hidden = torch.randn(n, w.d_model, generator=g, device=dev).to(torch.bfloat16)
-        prunable = torch.ones(n, dtype=torch.uint8, device=dev)
-        prunable[n - w.n_question:] = 0
-        gate = {"w1": (torch.randn(w.gate_hidden, w.d_model, generator=g, device=dev) * 0.02).to(torch.bfloat16),
-                "b1": torch.zeros(w.gate_hidden, device=dev),
-                "w2": torch.randn(w.gate_hidden, generator=g, device=dev) * 0.02, "b2": 0.0, "norm_w": None}
-        layers, heads = pipeline.stack_weights_on_device(w, w.n_layers, dev)
-        st = pipeline.PrunedPrefillStack(w, hidden, prunable, gate, layers, heads, w.gate_after)
-
-        def timed(fn, reps):
-            out = []
-            for _ in range(reps):
-                st.reset()
-                torch.cuda.synchronize(dev)
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                fn()
-                b.record(stream)
-                torch.cuda.synchronize(dev)
-                out.append(a.elapsed_time(b))
-            return sorted(out)[len(out) // 2]
-
-        timed(st.run, 1)
-        timed(st.unpruned, 1)
-        tg.tg_check_device_error()
-        reps = max(1, min(args.steps, 3))
-        t_pruned = timed(st.run, reps)
-        t_full = timed(st.unpruned, reps)
-        tg.tg_check_device_error()
-        line = {"mode": "stack", "workload": w.name, "n": n, "k": k, "kept_rows": st.m, "layers": w.n_layers,
-                "gate_after_layer": w.gate_after, "ttft_ms": round(t_pruned, 3),
-                "ttft_unpruned_ms": round(t_full, 3), "speedup": round(t_full / t_pruned, 3),
-                "tokens_per_s": n / (t_pruned * 1e-3), "peak_hbm_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 3),
-                "data": "synthetic (seeded on the device: N(0,1) hidden, N(0,0.02) weights)", "reps": reps}
+        r = stack_ttft(n, k, gl, max(1, min(args.steps, 3)), dev, stream)
+        g = r["gate"][f"layer{gl[0]}"]
+        line = {"mode": "stack", "workload": r["workload"], "n": n, "k": k, "kept_rows": r["kept_rows"],
+                "layers": r["layers"], "gate_layer": gl[0], "ttft_ms": g["ttft_ms"],
+                "ttft_unpruned_ms": r["ttft_unpruned_ms"], "speedup": g["speedup"], "tokens_per_s": g["tokens_per_s"],
+                "peak_hbm_gb": r["peak_hbm_gb"],
+                "data": "synthetic (seeded on the device: N(0,1) hidden, N(0,0.02) weights)", "reps": r["reps"]}
         print(json.dumps(line), flush=True)
-        del st, layers, heads, hidden
-        torch.cuda.empty_cache()
+
+
+def single_layer_step(w, dev, stream, flush, reps, peaks):
+    """Median time of the whole gated step (one CUDA graph, L2 flushed before
+    each) on workload w, with the attention call's time and fraction of the
+    measured bf16 peak on its kept causal FLOPs."""
+    import torch
+    from learned_token_pruning_b200 import pipeline, tokengate as tg
+    torch.cuda.reset_peak_memory_stats(dev)
+    step = pipeline.GatedPrefillStep(w, dev)
+    step.capture()
+    for _ in range(3):
+        flush.zero_()
+        step.replay()
+    torch.cuda.synchronize(dev)
+    times = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        times.append(a.elapsed_time(b))
+    tg.tg_check_device_error()
+    ms = sorted(times)[len(times) // 2]
+    br = breakdown(step, w, types.SimpleNamespace(steps=reps), stream, flush)
+    work = workload_work(w, step.m)
+    att_tf = work["attention"]["flops"] / (br["attention"] * 1e-3) / 1e12
+    gate_gbs = work["gate_score"]["bytes"] / (br["gate_score"] * 1e-3) / 1e9
+    res = {"workload": w.name, "n": w.n, "k": w.k, "kept_rows": step.m, "step_ms": round(ms, 4),
+           "tokens_per_s": w.n / (ms * 1e-3), "peak_hbm_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 3),
+           "attention": {"us": round(br["attention"] * 1e3, 2), "tflops": round(att_tf, 1),
+                         "frac_bf16_peak": round(att_tf / peaks["bf16_tflops"], 4)},
+           "gate_score": {"us": round(br["gate_score"] * 1e3, 2), "gbs": round(gate_gbs, 1),
+                          "frac_hbm": round(gate_gbs / peaks["hbm_gbs"], 4)},
+           "reps": reps}
+    del step
+    torch.cuda.empty_cache()
+    return res
 
 
 def main(argv=None):
@@ -948,8 +1029,10 @@ def main(argv=None):
     ap.add_argument("--backward", action="store_true", help="backward of gated attention at the kept-row counts")
     ap.add_argument("--ncu-backward", action="store_true", help="one backward call at 2064 rows (profiling)")
     ap.add_argument("--stack-n", type=int, nargs="*", default=None, help="stack sizes to run (default all)")
-    ap.add_argument("--gate-after", type=int, default=None,
-                    help="stack: the layer whose output the gate scores (default 13)")
+    ap.add_argument("--gate-layer", type=int, default=None,
+                    help="stack: the layer whose post-attention residual the gate scores (default 13)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="default run: skip the 128K step and the 28-layer TTFT figures")
     args = ap.parse_args(argv)
     if args.ncu_case:
         ncu_case()

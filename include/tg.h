@@ -149,6 +149,24 @@ int tg_gather(const void* hidden, int dtype, int64_t n, int32_t d_model,
               void* hidden_kept, int32_t* pos, float* bias, float* ratio, void* stream);
 
 /*
+ * tg_gather fused with a row-wise RMSNorm of the gathered rows: the kept rows
+ * are read once and written twice, as the bit-exact residual copy
+ * hidden_kept[r] = hidden[kept_idx[r]] and as the normalised row
+ *     x_norm[r] = hidden_kept[r] / sqrt(mean(hidden_kept[r]^2) + norm_eps) * norm_w
+ * that the first projection of the layer above reads ([R] §4.1 three-stage
+ * forward: the compacted rows go straight into the layers above the gate).
+ * pos, bias and ratio are written exactly as tg_gather writes them.
+ *   hidden .. ratio   as tg_gather;  norm_w device fp32 [d_model] or NULL (ones)
+ *   x_norm            device dtype [m][d_model] out, 16-byte aligned
+ * The normalised rows are rounded to dtype, as the layer's own RMSNorm does.
+ */
+int tg_gather_rmsnorm(const void* hidden, int dtype, int64_t n, int32_t d_model,
+                      const int32_t* kept_idx, int64_t m,
+                      const float* scores, const float* sumsq, int64_t n_prunable, float seq_eps,
+                      const float* norm_w, float norm_eps, void* hidden_kept, void* x_norm,
+                      int32_t* pos, float* bias, float* ratio, void* stream);
+
+/*
  * Token-gated causal GQA attention over the m kept rows ([R] §4.1 "token-gated
  * attention", "head-wise gain", "temperature scaling"; [K]; [M]).  For query
  * head h, KV head g = h / (hq / hkv), kept row r and key c <= r:
@@ -297,6 +315,51 @@ int tg_pruned_prefill_layer(const tg_layer_weights* weights, const tg_layer_shap
                             void* hidden_kept, const int32_t* pos, const float* bias,
                             const float* ratio, int64_t m, void* ws, size_t ws_bytes, void* stream);
 
+/* Parts of a decoder layer (tg_gather_prefill_layer's `part`). */
+enum { TG_LAYER_ATTENTION = 1, TG_LAYER_MLP = 2, TG_LAYER_FULL = 3 };
+
+/*
+ * The two halves of tg_pruned_prefill_layer, for the gate layer L itself
+ * ([R] §4.1 Gate module and three-stage forward; [K] "tying the mechanism
+ * together"; [M] "how does learned token pruning work": the gate scores layer
+ * L's normalised post-attention residual, so layer L's attention runs on every
+ * token and its MLP, a row-wise step, only on the kept ones):
+ *   tg_layer_attention_block:  h += Attn(RMSNorm(h)) Wo^T   (steps up to the
+ *                              O projection; the post-attention residual)
+ *   tg_layer_mlp_block:        h += (SiLU(y Wg^T) * (y Wu^T)) Wd^T, y = RMSNorm(h)
+ *                              with w_post_norm
+ * Arguments as tg_pruned_prefill_layer (the MLP half reads only w_post_norm,
+ * w_gate_up and w_down; the attention half every other weight), with the
+ * same workspace size.  Calling the two in a row is the whole layer.
+ */
+int tg_layer_attention_block(const tg_layer_weights* weights, const tg_layer_shape* shape, void* hidden,
+                             const int32_t* pos, const float* bias, const float* ratio, int64_t m,
+                             void* ws, size_t ws_bytes, void* stream);
+int tg_layer_mlp_block(const tg_layer_weights* weights, const tg_layer_shape* shape, void* hidden,
+                       int64_t m, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * tg_gather followed by a layer part on the kept rows, with the gather folded
+ * into that part's first RMSNorm ([R] §4.1 three-stage forward: the kept rows
+ * are compacted and go straight into the layers above): one pass reads
+ * hidden[kept_idx[r]], writes it to hidden_kept[r] (bit-exact) together with
+ * pos, bias and ratio exactly as tg_gather does, and writes the normalised row
+ * the part's first projection reads; the rest of the part then runs on the
+ * kept rows as tg_pruned_prefill_layer (part TG_LAYER_FULL: the whole gated
+ * layer above the gate) or tg_layer_mlp_block (part TG_LAYER_MLP: the gate
+ * layer's own MLP half) would.  The result equals tg_gather then that call.
+ *   hidden, n, kept_idx, m, scores, sumsq, n_prunable, seq_eps, hidden_kept,
+ *   pos, bias, ratio   as tg_gather (dtype and d_model from shape); the full
+ *                      layer needs pos; bias / ratio may be NULL (0 / 1 in
+ *                      attention, and not written)
+ *   ws                 as tg_pruned_prefill_layer for m rows
+ */
+int tg_gather_prefill_layer(const tg_layer_weights* weights, const tg_layer_shape* shape, int part,
+                            const void* hidden, int64_t n, const int32_t* kept_idx, int64_t m,
+                            const float* scores, const float* sumsq, int64_t n_prunable, float seq_eps,
+                            void* hidden_kept, int32_t* pos, float* bias, float* ratio,
+                            void* ws, size_t ws_bytes, void* stream);
+
 /*
  * The same layer over a batch of requests whose kept rows are concatenated
  * (varlen batching; [R] §4.1 three-stage forward, per request): rows
@@ -356,10 +419,13 @@ size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t
  *
  * Scratch lives in a fixed array compiled into the library,
  * tg_gate_score_noalloc_scratch_bytes() bytes (2 MiB + 64 KiB) on every device
- * that loads the library, held until the process exits.  Sizes whose scratch
- * would not fit (about n/32 + 2*d_model*h bytes, e.g. n up to 2^20 tokens with
- * d_model*h up to 2^20) are rejected with TG_ERR_UNSUPPORTED before anything
- * is enqueued.  The call allocates and frees nothing.
+ * that loads the library, held until the process exits.  Only the tensor-core
+ * path of tg_gate_score (see there) uses scratch: calls that take it and whose
+ * scratch would not fit (about n/32 + 2*d_model*h bytes, e.g. n up to 2^20
+ * tokens with d_model*h up to 2^20) are rejected with TG_ERR_UNSUPPORTED
+ * before anything is enqueued; calls on the CUDA-core path (fp32, or shapes the
+ * tensor cores do not take) need none and have no size limit from it.  The
+ * call allocates and frees nothing.
  *
  * The first call on each device looks up the array's device address (with
  * that device current) and caches it; make that first call before any stream

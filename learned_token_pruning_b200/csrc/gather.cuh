@@ -167,3 +167,79 @@ __global__ void __launch_bounds__(kGatherBulkThreads) k_gather_bulk(GatherParams
 }
 
 }  // namespace tg
+
+namespace tg {
+
+// ---------------------------------------------------------------------------
+// Gather fused with the first RMSNorm of the layer that reads the kept rows.
+// One warp per kept row r: the source row hidden[idx[r]] is loaded once into
+// registers (every 16-byte load of a lane in flight together), written out
+// unchanged as the residual copy hidden_kept[r] (bit-exact, as k_gather_bulk),
+// and normalised in the same pass, xn[r] = x / sqrt(mean(x^2) + eps) * w,
+// rounded to the row's dtype (the arithmetic and summation order of
+// k_rmsnorm_warp, so the result equals a gather followed by that norm).
+// Lane 0 writes the side outputs pos, bias and ratio as k_gather_bulk does.
+// ---------------------------------------------------------------------------
+template <typename T, int MAXV>
+__global__ void __launch_bounds__(256) k_gather_rmsnorm_warp(GatherParams p, T* __restrict__ xn,
+                                                             const float* __restrict__ w, int d, float norm_eps) {
+  pdl_wait();
+  pdl_launch_dependents();
+  constexpr int V = 16 / sizeof(T);
+  const int lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (r >= p.m) return;  // warp-uniform
+  const int64_t j = p.idx[r];
+  if (j < 0 || j >= p.n) {
+    if (lane == 0) raise_error(kErrGatherIndex, static_cast<uint32_t>(r & 0xffffff));
+    return;
+  }
+  const int nv = d / V;
+  const uint4* xr = reinterpret_cast<const uint4*>(p.hidden + j * p.row_bytes);
+  uint4* cr = reinterpret_cast<uint4*>(p.out + r * p.row_bytes);
+  uint4* yr = reinterpret_cast<uint4*>(xn + r * d);
+  uint4 v[MAXV];
+  float ss = 0.0f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = lane + 32 * i;
+    v[i] = c < nv ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+  }
+  if (lane == 0) gather_side_outputs(p, r, j);
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = lane + 32 * i;
+    if (c < nv) cr[c] = v[i];
+    const T* e = reinterpret_cast<const T*>(&v[i]);
+#pragma unroll
+    for (int t = 0; t < V; ++t) {
+      const float f = to_f32(e[t]);
+      ss = fmaf(f, f, ss);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.0f / sqrtf(ss / static_cast<float>(d) + norm_eps);
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int c = lane + 32 * i;
+    if (c >= nv) continue;
+    float wv[V];
+#pragma unroll
+    for (int t = 0; t < V; t += 4) {
+      const float4 w4 = w ? __ldg(reinterpret_cast<const float4*>(w + c * V + t)) : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+      wv[t] = w4.x;
+      wv[t + 1] = w4.y;
+      wv[t + 2] = w4.z;
+      wv[t + 3] = w4.w;
+    }
+    const T* e = reinterpret_cast<const T*>(&v[i]);
+    uint4 o;
+    T* oe = reinterpret_cast<T*>(&o);
+#pragma unroll
+    for (int t = 0; t < V; ++t) oe[t] = from_f32<T>(to_f32(e[t]) * inv * wv[t]);
+    yr[c] = o;
+  }
+}
+
+}  // namespace tg

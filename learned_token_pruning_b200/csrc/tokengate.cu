@@ -320,6 +320,12 @@ int launch_gate_tc(const void* A, const void* W1, int M, int K, const tg::GatePa
 
 int dtype_size(int dtype) { return dtype == TG_BF16 ? 2 : (dtype == TG_F32 ? 4 : 0); }
 
+// Whether tg_gate_score takes the tensor-core kernel (the only path that uses
+// its workspace); other shapes and fp32 run on CUDA cores without scratch.
+bool gate_uses_tc(const void* hidden, int dtype, int32_t d_model, const void* w1, int32_t h) {
+  return dtype == TG_BF16 && d_model % 8 == 0 && h <= 256 && h % 16 == 0 && aligned16(hidden) && aligned16(w1);
+}
+
 // workspace layout of tg_gate_score (256-byte aligned pieces):
 //   [per-CTA partial sums of s^2][completion counter][W1 scaled by the norm weight, bf16 [h][d]]
 size_t gate_partials_bytes(int64_t n) { return ((static_cast<size_t>((n + 127) / 128) * 4 + 255) / 256) * 256; }
@@ -413,9 +419,28 @@ static size_t layer_buffers_bytes(int64_t m, const tg_layer_shape* S) {
          al(rows * act * es);
 }
 
-static int prefill_layer_impl(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden_kept, const int32_t* pos,
-                       const float* bias, const float* ratio, int64_t m, const int64_t* seg_rows, int32_t nseg,
-                       void* ws, size_t ws_bytes, void* stream);
+// Where the layer's first RMSNorm reads its rows from when the gather is
+// folded into it: hidden_kept[r] = hidden[idx[r]] is written in the same pass
+// (with pos, bias and ratio, as tg_gather writes them).
+struct LayerGather {
+  const void* hidden;
+  int64_t n;
+  const int32_t* idx;
+  const float* scores;
+  const float* sumsq;
+  int64_t n_prunable;
+  float seq_eps;
+  int32_t* pos;
+  float* bias;
+  float* ratio;
+};
+
+static int prefill_layer_impl(const tg_layer_weights* W, const tg_layer_shape* S, int parts, void* hidden_kept,
+                              const int32_t* pos, const float* bias, const float* ratio, int64_t m,
+                              const int64_t* seg_rows, int32_t nseg, const LayerGather* gather, void* ws,
+                              size_t ws_bytes, void* stream);
+static int launch_gather_rmsnorm(const LayerGather& g, int dtype, void* hidden_kept, void* xn, const float* w,
+                                 int64_t m, int d, float eps, cudaStream_t st);
 
 extern "C" {
 
@@ -628,9 +653,7 @@ int tg_gate_score(const void* hidden, int dtype, int64_t n, int32_t d_model, con
   if (n >= (int64_t(1) << 31)) return fail(TG_ERR_UNSUPPORTED, "n must be < 2^31");
   if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "dtype");
   cudaStream_t st = as_stream(stream);
-  const bool tc = dtype == TG_BF16 && d_model % 8 == 0 && h <= 256 && h % 16 == 0 && aligned16(hidden) &&
-                  aligned16(w1);
-  if (tc) {
+  if (gate_uses_tc(hidden, dtype, d_model, w1, h)) {
     const size_t need = gate_ws_bytes(n, d_model, h);
     if (!ws || ws_bytes < need) return fail(TG_ERR_WORKSPACE, "gate score needs %zu workspace bytes", need);
     if (!aligned16(ws)) return fail(TG_ERR_ALIGN, "workspace must be 16-byte aligned");
@@ -1153,7 +1176,52 @@ int tg_gated_decode_attention(const void* q, const void* k, int64_t ldk, const v
 int tg_pruned_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden_kept,
                             const int32_t* pos, const float* bias, const float* ratio, int64_t m, void* ws,
                             size_t ws_bytes, void* stream) {
-  return prefill_layer_impl(W, S, hidden_kept, pos, bias, ratio, m, nullptr, 0, ws, ws_bytes, stream);
+  return prefill_layer_impl(W, S, TG_LAYER_FULL, hidden_kept, pos, bias, ratio, m, nullptr, 0, nullptr, ws, ws_bytes,
+                            stream);
+}
+
+int tg_layer_attention_block(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden, const int32_t* pos,
+                             const float* bias, const float* ratio, int64_t m, void* ws, size_t ws_bytes,
+                             void* stream) {
+  return prefill_layer_impl(W, S, TG_LAYER_ATTENTION, hidden, pos, bias, ratio, m, nullptr, 0, nullptr, ws, ws_bytes,
+                            stream);
+}
+
+int tg_layer_mlp_block(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden, int64_t m, void* ws,
+                       size_t ws_bytes, void* stream) {
+  return prefill_layer_impl(W, S, TG_LAYER_MLP, hidden, nullptr, nullptr, nullptr, m, nullptr, 0, nullptr, ws,
+                            ws_bytes, stream);
+}
+
+int tg_gather_rmsnorm(const void* hidden, int dtype, int64_t n, int32_t d_model, const int32_t* kept_idx, int64_t m,
+                      const float* scores, const float* sumsq, int64_t n_prunable, float seq_eps, const float* norm_w,
+                      float norm_eps, void* hidden_kept, void* x_norm, int32_t* pos, float* bias, float* ratio,
+                      void* stream) {
+  if (!hidden || !kept_idx || !hidden_kept || !x_norm) return fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (bias && (!scores || !sumsq)) return fail(TG_ERR_INVALID_ARG, "bias needs scores and sumsq");
+  if (n <= 0 || m <= 0 || m > n || d_model <= 0) return fail(TG_ERR_INVALID_ARG, "bad sizes");
+  if (bias && n_prunable <= 0) return fail(TG_ERR_INVALID_ARG, "n_prunable must be > 0 for bias");
+  const int es = dtype_size(dtype);
+  if (!es) return fail(TG_ERR_INVALID_ARG, "dtype");
+  if ((int64_t(d_model) * es) % 16 != 0 || !aligned16(hidden) || !aligned16(hidden_kept) || !aligned16(x_norm))
+    return fail(TG_ERR_ALIGN, "rows must be 16-byte multiples on 16-byte aligned buffers");
+  const LayerGather g{hidden, n, kept_idx, scores, sumsq, n_prunable, seq_eps, pos, bias, ratio};
+  return launch_gather_rmsnorm(g, dtype, hidden_kept, x_norm, norm_w, m, d_model, norm_eps, as_stream(stream));
+}
+
+int tg_gather_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, int part, const void* hidden,
+                            int64_t n, const int32_t* kept_idx, int64_t m, const float* scores, const float* sumsq,
+                            int64_t n_prunable, float seq_eps, void* hidden_kept, int32_t* pos, float* bias,
+                            float* ratio, void* ws, size_t ws_bytes, void* stream) {
+  if (part != TG_LAYER_FULL && part != TG_LAYER_MLP) return fail(TG_ERR_INVALID_ARG, "part must be full or MLP");
+  if (!hidden || !kept_idx || !hidden_kept) return fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (part == TG_LAYER_FULL && !pos) return fail(TG_ERR_INVALID_ARG, "the attention half needs pos");
+  if (bias && (!scores || !sumsq)) return fail(TG_ERR_INVALID_ARG, "bias needs scores and sumsq");
+  if (n <= 0 || m <= 0 || m > n) return fail(TG_ERR_INVALID_ARG, "bad sizes");
+  if (bias && n_prunable <= 0) return fail(TG_ERR_INVALID_ARG, "n_prunable must be > 0 for bias");
+  if (!aligned16(hidden) || !aligned16(hidden_kept)) return fail(TG_ERR_ALIGN, "rows must be 16-byte aligned");
+  const LayerGather g{hidden, n, kept_idx, scores, sumsq, n_prunable, seq_eps, pos, bias, ratio};
+  return prefill_layer_impl(W, S, part, hidden_kept, pos, bias, ratio, m, nullptr, 0, &g, ws, ws_bytes, stream);
 }
 
 size_t tg_layer_varlen_workspace_bytes(const tg_layer_shape* shape, const int64_t* seg_rows, int32_t nseg) {
@@ -1178,22 +1246,69 @@ int tg_pruned_prefill_layer_varlen(const tg_layer_weights* W, const tg_layer_sha
   if (seg_rows[0] != 0) return fail(TG_ERR_INVALID_ARG, "seg_rows[0] must be 0");
   for (int32_t r = 0; r < nseg; ++r)
     if (seg_rows[r + 1] < seg_rows[r]) return fail(TG_ERR_INVALID_ARG, "seg_rows must not decrease");
-  return prefill_layer_impl(W, S, hidden_kept, pos, bias, ratio, seg_rows[nseg], seg_rows, nseg, ws, ws_bytes,
-                            stream);
+  return prefill_layer_impl(W, S, TG_LAYER_FULL, hidden_kept, pos, bias, ratio, seg_rows[nseg], seg_rows, nseg,
+                            nullptr, ws, ws_bytes, stream);
 }
 
 }  // extern "C"
 
+static int mlp_half(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden_kept, void* xn, void* act,
+                    int64_t m, void* stream);
+
+// The gather fused with an RMSNorm (k_gather_rmsnorm_warp): rows whose 16-byte
+// vectors fit a warp's registers; other shapes gather first and normalise after.
+static int launch_gather_rmsnorm(const LayerGather& g, int dtype, void* hidden_kept, void* xn, const float* w,
+                                 int64_t m, int d, float eps, cudaStream_t st) {
+  const int es = dtype_size(dtype);
+  tg::GatherParams p{};
+  p.hidden = static_cast<const uint8_t*>(g.hidden);
+  p.n = g.n;
+  p.row_bytes = int64_t(d) * es;
+  p.idx = g.idx;
+  p.m = m;
+  p.scores = g.scores;
+  p.sumsq = g.sumsq;
+  p.n_prunable = g.n_prunable;
+  p.eps = g.seq_eps;
+  p.out = static_cast<uint8_t*>(hidden_kept);
+  p.pos = g.pos;
+  p.bias = g.bias;
+  p.ratio = g.ratio;
+  const int nv = d * es / 16;
+  const dim3 grid(unsigned((m + 7) / 8)), block(256);
+  if (!w || aligned16(w)) {
+    if (dtype == TG_BF16) {
+      auto* y = static_cast<__nv_bfloat16*>(xn);
+      if (nv <= 32 * 4) return launch_pdl("k_gather_rmsnorm_warp", tg::k_gather_rmsnorm_warp<__nv_bfloat16, 4>, grid, block, 0, st, p, y, w, d, eps);
+      if (nv <= 32 * 8) return launch_pdl("k_gather_rmsnorm_warp", tg::k_gather_rmsnorm_warp<__nv_bfloat16, 8>, grid, block, 0, st, p, y, w, d, eps);
+      if (nv <= 32 * 16) return launch_pdl("k_gather_rmsnorm_warp", tg::k_gather_rmsnorm_warp<__nv_bfloat16, 16>, grid, block, 0, st, p, y, w, d, eps);
+    } else {
+      auto* y = static_cast<float*>(xn);
+      if (nv <= 32 * 4) return launch_pdl("k_gather_rmsnorm_warp", tg::k_gather_rmsnorm_warp<float, 4>, grid, block, 0, st, p, y, w, d, eps);
+      if (nv <= 32 * 8) return launch_pdl("k_gather_rmsnorm_warp", tg::k_gather_rmsnorm_warp<float, 8>, grid, block, 0, st, p, y, w, d, eps);
+      if (nv <= 32 * 16) return launch_pdl("k_gather_rmsnorm_warp", tg::k_gather_rmsnorm_warp<float, 16>, grid, block, 0, st, p, y, w, d, eps);
+    }
+  }
+  int rc = tg_gather(g.hidden, dtype, g.n, d, g.idx, m, g.scores, g.sumsq, g.n_prunable, g.seq_eps, hidden_kept, g.pos,
+                     g.bias, g.ratio, st);
+  if (rc) return rc;
+  return dtype == TG_BF16 ? launch_rmsnorm<__nv_bfloat16>(hidden_kept, xn, w, m, d, eps, st)
+                          : launch_rmsnorm<float>(hidden_kept, xn, w, m, d, eps, st);
+}
+
 // One decoder layer over m rows; with seg_rows (host, nseg + 1 offsets) the
 // rows are nseg independent requests and attention runs per request.
-static int prefill_layer_impl(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden_kept, const int32_t* pos,
-                       const float* bias, const float* ratio, int64_t m, const int64_t* seg_rows, int32_t nseg,
-                       void* ws, size_t ws_bytes, void* stream) {
+static int prefill_layer_impl(const tg_layer_weights* W, const tg_layer_shape* S, int parts, void* hidden_kept,
+                              const int32_t* pos, const float* bias, const float* ratio, int64_t m,
+                              const int64_t* seg_rows, int32_t nseg, const LayerGather* gather, void* ws,
+                              size_t ws_bytes, void* stream) {
   if (!W || !S || !hidden_kept) return fail(TG_ERR_INVALID_ARG, "null pointer");
-  if (!W->w_in_norm || !W->w_qkv || !W->w_o || !W->w_post_norm || !W->w_gate_up || !W->w_down || !W->head_gain ||
-      !W->head_temp)
+  const bool do_attn = (parts & TG_LAYER_ATTENTION) != 0, do_mlp = (parts & TG_LAYER_MLP) != 0;
+  if (do_attn && (!W->w_in_norm || !W->w_qkv || !W->w_o || !W->head_gain || !W->head_temp))
     return fail(TG_ERR_INVALID_ARG, "null weight pointer");
-  if (S->qk_norm && (!W->w_q_norm || !W->w_k_norm)) return fail(TG_ERR_INVALID_ARG, "qk_norm needs its weights");
+  if (do_mlp && (!W->w_post_norm || !W->w_gate_up || !W->w_down)) return fail(TG_ERR_INVALID_ARG, "null weight pointer");
+  if (do_attn && !pos) return fail(TG_ERR_INVALID_ARG, "null pointer (pos)");
+  if (do_attn && S->qk_norm && (!W->w_q_norm || !W->w_k_norm)) return fail(TG_ERR_INVALID_ARG, "qk_norm needs its weights");
   if (m <= 0 || S->d_model <= 0 || S->hq <= 0 || S->hkv <= 0 || S->hq % S->hkv || S->d_ff <= 0)
     return fail(TG_ERR_INVALID_ARG, "bad layer shape");
   if (S->head_dim != 64 && S->head_dim != 128) return fail(TG_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
@@ -1227,10 +1342,20 @@ static int prefill_layer_impl(const tg_layer_weights* W, const tg_layer_shape* S
   float* bias_stage = reinterpret_cast<float*>(static_cast<uint8_t*>(attn_ws) + attn_ws_sz);
   const bool bf = S->dtype == TG_BF16;
   int rc;
+  // the first RMSNorm of the parts run here: from the rows in place, or
+  // gathering them from the full sequence in the same pass
+  auto first_norm = [&](const float* w) -> int {
+    if (!gather)
+      return bf ? launch_rmsnorm<__nv_bfloat16>(hidden_kept, xn, w, m, d, S->norm_eps, st)
+                : launch_rmsnorm<float>(hidden_kept, xn, w, m, d, S->norm_eps, st);
+    return launch_gather_rmsnorm(*gather, S->dtype, hidden_kept, xn, w, m, d, S->norm_eps, st);
+  };
+  if (!do_attn) {
+    if ((rc = first_norm(W->w_post_norm))) return rc;
+    return mlp_half(W, S, hidden_kept, xn, act, m, stream);
+  }
   // 1. x = RMSNorm(h)
-  rc = bf ? launch_rmsnorm<__nv_bfloat16>(hidden_kept, xn, W->w_in_norm, m, d, S->norm_eps, st)
-          : launch_rmsnorm<float>(hidden_kept, xn, W->w_in_norm, m, d, S->norm_eps, st);
-  if (rc) return rc;
+  if ((rc = first_norm(W->w_in_norm))) return rc;
   // 2. qkv = x Wqkv^T
   if ((rc = tg_linear(xn, d, W->w_qkv, qkv, qkv_w, S->dtype, m, int32_t(qkv_w), d, TG_EPI_STORE, stream))) return rc;
   // 3. per-head q/k norm and RoPE at the original positions (one warp per row)
@@ -1276,10 +1401,22 @@ static int prefill_layer_impl(const tg_layer_weights* W, const tg_layer_shape* S
   // 5. h += a Wo^T
   if ((rc = tg_linear(att, int64_t(hq) * D, W->w_o, hidden_kept, d, S->dtype, m, d, hq * D, TG_EPI_RESIDUAL, stream)))
     return rc;
+  if (!do_mlp) return TG_OK;
   // 6. y = RMSNorm(h)
   rc = bf ? launch_rmsnorm<__nv_bfloat16>(hidden_kept, xn, W->w_post_norm, m, d, S->norm_eps, st)
           : launch_rmsnorm<float>(hidden_kept, xn, W->w_post_norm, m, d, S->norm_eps, st);
   if (rc) return rc;
+  return mlp_half(W, S, hidden_kept, xn, act, m, stream);
+}
+
+// Steps 7-8 of the layer on rows already normalised into xn: act = SiLU(y Wg^T)
+// * (y Wu^T), h += act Wd^T.
+static int mlp_half(const tg_layer_weights* W, const tg_layer_shape* S, void* hidden_kept, void* xn, void* act,
+                    int64_t m, void* stream) {
+  cudaStream_t st = as_stream(stream);
+  const int d = S->d_model, dff = S->d_ff;
+  const bool bf = S->dtype == TG_BF16;
+  int rc;
   // 7. act = SiLU(y Wg^T) * (y Wu^T)
   if (bf && dff % 128 == 0) {
     if ((rc = tg_linear(xn, d, W->w_gate_up, act, dff, S->dtype, m, dff, d, TG_EPI_SWIGLU, stream))) return rc;
@@ -1352,7 +1489,8 @@ extern "C" {
 int tg_gate_score_noalloc(const void* hidden, int dtype, int64_t n, int32_t d_model, const float* norm_w,
                           float norm_eps, const void* w1, const float* b1, const float* w2, float b2, int32_t h,
                           const uint8_t* prunable, float* scores, float* sumsq, void* stream) {
-  if (n > 0 && d_model > 0 && h > 0) {
+  if (n > 0 && d_model > 0 && h > 0 && gate_uses_tc(hidden, dtype, d_model, w1, h)) {
+    // only the tensor-core path uses scratch; the CUDA-core path needs none
     const size_t need = gate_ws_bytes(n, d_model, h);
     if (need > kNoAllocScratchBytes)
       return fail(TG_ERR_UNSUPPORTED,

@@ -78,12 +78,18 @@ class GatedPrefillStep:
         tg.tg_pruned_prefill_layer(self.W, self.S, self.hidden_kept, self.pos, self.bias, self.ratio, self.ws_layer,
                                    stream)
 
+    def gather_layer(self, stream=None):
+        """The gather folded into the layer above: one pass gathers the kept rows
+        (and pos, bias, ratio) and normalises them for the QKV projection."""
+        tg.tg_gather_prefill_layer(self.W, self.S, tg.TG_LAYER_FULL, self.hidden, self.kept, self.scores, self.sumsq,
+                                   self.n_prunable, self.eps_s, self.hidden_kept, self.pos, self.bias, self.ratio,
+                                   self.ws_layer, stream)
+
     def run(self, stream=None):
         """One whole step; the result is left in self.hidden_kept ([m, d_model])."""
         self.gate_score(stream)
         self.select(stream)
-        self.gather(stream)
-        self.layer_above(stream)
+        self.gather_layer(stream)
         return self.hidden_kept
 
     def capture(self):
@@ -198,21 +204,28 @@ class BatchedPrefillStep:
 
 class PrunedPrefillStack:
     """Prefill of one prompt through a decoder stack, the three-stage forward of
-    "TokenGate and T2Quant: a close reading", §4.1: layers 0 .. gate_after run
-    on all N rows; the gate scores the residual stream leaving layer
-    gate_after, the top-K document tokens and every question token are kept
-    and gathered in order; layers gate_after+1 .. run on the kept rows with
-    token-gated attention.  `unpruned()` runs every layer on all rows with no
-    gate.  Every step is a library call on the current stream.
+    "TokenGate and T2Quant: a close reading", §4.1 (Gate module; [K] "tying the
+    mechanism together" and [M] "how does learned token pruning work" put the
+    scoring in the same place):
+      layers 0 .. L-1      all N rows;
+      layer L, attention   all N rows -> the post-attention residual;
+      gate                 scores that residual normalised by layer L's own
+                           post-attention RMSNorm; top-K document tokens plus
+                           every question token are selected;
+      layer L, MLP         on the kept rows only, with the gather folded into
+                           its RMSNorm;
+      layers L+1 ..        on the kept rows with token-gated attention.
+    `unpruned()` runs every layer on all rows with no gate.  Every step is a
+    library call on the current stream.
 
     layers: per layer a dict of device tensors (tg_layer_weights names, without
     head_gain / head_temp); heads: per layer a dict with device tensors
     head_gain and head_temp (used by the layers above the gate; the layers on
     all rows run with no gate bias and unit temperature)."""
 
-    def __init__(self, w: synth.Workload, hidden, prunable, gate: Dict, layers, heads, gate_after: int,
+    def __init__(self, w: synth.Workload, hidden, prunable, gate: Dict, layers, heads, gate_layer: int,
                  norm_eps: float = 1e-6, eps_s: float = 1e-6):
-        self.w, self.gate_after, self.norm_eps, self.eps_s = w, gate_after, norm_eps, eps_s
+        self.w, self.gate_layer, self.norm_eps, self.eps_s = w, gate_layer, norm_eps, eps_s
         dev = hidden.device
         self.dt = hidden.dtype
         self.hidden0 = hidden
@@ -234,6 +247,8 @@ class PrunedPrefillStack:
         self.ratio = torch.empty(self.m, dtype=torch.float32, device=dev)
         ones = torch.ones(w.hq, dtype=torch.float32, device=dev)
         zeros = torch.zeros(w.hq, dtype=torch.float32, device=dev)
+        # the gate normalises with layer L's post-attention RMSNorm weight
+        self.gate_norm_w = layers[gate_layer]["w_post_norm"]
         self._keep = []  # device tensors the structs point to
         self.full_layers, self.pruned_layers = [], []
         for l, lw in enumerate(layers):
@@ -254,25 +269,35 @@ class PrunedPrefillStack:
         self.h.copy_(self.hidden0)
 
     def full_part(self):
-        for W, S in self.full_layers[: self.gate_after + 1]:
+        """Layers 0 .. L-1 and layer L's attention half on all rows: self.h ends
+        as layer L's post-attention residual, the gate's input."""
+        for W, S in self.full_layers[: self.gate_layer]:
             tg.tg_pruned_prefill_layer(W, S, self.h, self.pos_all, None, None, self.ws_layer)
+        W, S = self.full_layers[self.gate_layer]
+        tg.tg_layer_attention_block(W, S, self.h, self.pos_all, None, None, self.ws_layer)
 
-    def gate_select_gather(self):
+    def gate_select(self):
         g = self.gate
-        tg.tg_gate_score(self.h, g.get("norm_w"), self.norm_eps, g["w1"], g["b1"], g["w2"], g["b2"], self.prunable,
+        tg.tg_gate_score(self.h, self.gate_norm_w, self.norm_eps, g["w1"], g["b1"], g["w2"], g["b2"], self.prunable,
                          self.scores, self.sumsq, self.ws_gate)
         tg.tg_topk_select(self.scores, self.prunable, self.n_prunable, self.w.k, self.kept)
-        tg.tg_gather(self.h, self.kept, self.scores, self.sumsq, self.n_prunable, self.eps_s, self.hk, self.pos,
-                     self.bias, self.ratio)
+
+    def gather_mlp(self):
+        """Gather the kept rows of the residual into self.hk and run layer L's
+        MLP half on them (the gather folded into its RMSNorm)."""
+        W, S = self.full_layers[self.gate_layer]
+        tg.tg_gather_prefill_layer(W, S, tg.TG_LAYER_MLP, self.h, self.kept, self.scores, self.sumsq, self.n_prunable,
+                                   self.eps_s, self.hk, self.pos, self.bias, self.ratio, self.ws_layer)
 
     def pruned_part(self):
-        for W, S in self.pruned_layers[self.gate_after + 1:]:
+        for W, S in self.pruned_layers[self.gate_layer + 1:]:
             tg.tg_pruned_prefill_layer(W, S, self.hk, self.pos, self.bias, self.ratio, self.ws_layer)
 
     def run(self):
         """Layer-0 input in self.h -> kept-row output of the last layer in self.hk."""
         self.full_part()
-        self.gate_select_gather()
+        self.gate_select()
+        self.gather_mlp()
         self.pruned_part()
         return self.hk
 

@@ -48,7 +48,7 @@ class Workload:
     question_first: bool = False
     score_mixture: bool = False   # inject Gaussian-mixture scores for the selector
     n_layers: int = 1             # decoder layers of a whole-stack workload
-    gate_after: int = 0           # the gate scores the residual leaving this layer
+    gate_layer: int = 0           # the gate scores this layer's post-attention residual
 
     @property
     def n_prunable(self) -> int:
@@ -105,7 +105,7 @@ def full_stack_64k(**kw) -> Workload:
     N=65536 with 64 question tokens, K=4096 (TTFT against the unpruned stack)."""
     w = Workload(name="qwen3_1.7b_stack28_n65536_k4096", seed=5, n=65536, n_question=64,
                  d_model=2048, hq=16, hkv=8, head_dim=128, gate_hidden=256, k=4096, dtype="bf16",
-                 d_ff=6144, n_layers=28, gate_after=13)
+                 d_ff=6144, n_layers=28, gate_layer=13)
     return w.replace(**kw) if kw else w
 
 

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(HERE, "libtokengate.so")
 
 TG_F32, TG_BF16 = 0, 1
 TG_OP_GATE_SCORE, TG_OP_LAYER, TG_OP_ATTENTION, TG_OP_DECODE, TG_OP_ATTENTION_BWD = 0, 1, 2, 3, 4
+TG_LAYER_ATTENTION, TG_LAYER_MLP, TG_LAYER_FULL = 1, 2, 3
 STATUS = {0: "TG_OK", 1: "TG_ERR_INVALID_ARG", 2: "TG_ERR_SHAPE", 3: "TG_ERR_ALIGN", 4: "TG_ERR_UNSUPPORTED",
           5: "TG_ERR_WORKSPACE", 6: "TG_ERR_CUDA", 7: "TG_ERR_DEVICE_TIMEOUT", 8: "TG_ERR_DEVICE_CHECK"}
 
@@ -67,6 +68,12 @@ SIGNATURES = {
     "tg_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I32, _I32, ctypes.POINTER(LayerShape)]),
     "tg_gate_score_noalloc": (_INT, [_P, _INT, _I64, _I32, _P, _F, _P, _P, _P, _F, _I32, _P, _P, _P, _P]),
     "tg_gate_score_noalloc_scratch_bytes": (_SZ, []),
+    "tg_gather_rmsnorm": (_INT, [_P, _INT, _I64, _I32, _P, _I64, _P, _P, _I64, _F, _P, _F, _P, _P, _P, _P, _P, _P]),
+    "tg_layer_attention_block": (_INT, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerShape), _P, _P, _P, _P,
+                                        _I64, _P, _SZ, _P]),
+    "tg_layer_mlp_block": (_INT, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerShape), _P, _I64, _P, _SZ, _P]),
+    "tg_gather_prefill_layer": (_INT, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerShape), _INT, _P, _I64, _P,
+                                       _I64, _P, _P, _I64, _F, _P, _P, _P, _P, _P, _SZ, _P]),
 }
 
 _lib = None
@@ -164,6 +171,16 @@ def tg_gather(hidden, kept_idx, scores, sumsq, n_prunable: int, seq_eps: float, 
                          _ptr(sumsq), int(n_prunable), float(seq_eps), _ptr(hidden_kept), _ptr(pos), _ptr(bias),
                          _ptr(ratio), _stream(stream))
     _check("tg_gather", rc)
+
+
+def tg_gather_rmsnorm(hidden, kept_idx, scores, sumsq, n_prunable: int, seq_eps: float, norm_w, norm_eps: float,
+                      hidden_kept, x_norm, pos=None, bias=None, ratio=None, stream=None):
+    """tg_gather plus x_norm = RMSNorm(hidden_kept) * norm_w in the same pass."""
+    n, d = hidden.shape
+    rc = lib().tg_gather_rmsnorm(_ptr(hidden), _dtype(hidden), n, d, _ptr(kept_idx), kept_idx.numel(), _ptr(scores),
+                                 _ptr(sumsq), int(n_prunable), float(seq_eps), _ptr(norm_w), float(norm_eps),
+                                 _ptr(hidden_kept), _ptr(x_norm), _ptr(pos), _ptr(bias), _ptr(ratio), _stream(stream))
+    _check("tg_gather_rmsnorm", rc)
 
 
 def _row_view(t: torch.Tensor):
@@ -277,6 +294,33 @@ def tg_pruned_prefill_layer(W: LayerWeights, S: LayerShape, hidden_kept, pos, bi
     rc = lib().tg_pruned_prefill_layer(ctypes.byref(W), ctypes.byref(S), _ptr(hidden_kept), _ptr(pos), _ptr(bias),
                                        _ptr(ratio), m, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check("tg_pruned_prefill_layer", rc)
+
+
+def tg_layer_attention_block(W: LayerWeights, S: LayerShape, hidden, pos, bias, ratio, ws, stream=None):
+    """hidden += Attn(RMSNorm(hidden)) Wo^T: the post-attention residual, in place."""
+    rc = lib().tg_layer_attention_block(ctypes.byref(W), ctypes.byref(S), _ptr(hidden), _ptr(pos), _ptr(bias),
+                                        _ptr(ratio), hidden.shape[0], _ptr(ws), ws.numel() * ws.element_size(),
+                                        _stream(stream))
+    _check("tg_layer_attention_block", rc)
+
+
+def tg_layer_mlp_block(W: LayerWeights, S: LayerShape, hidden, ws, stream=None):
+    """hidden += SwiGLU MLP of RMSNorm(hidden), in place."""
+    rc = lib().tg_layer_mlp_block(ctypes.byref(W), ctypes.byref(S), _ptr(hidden), hidden.shape[0], _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream))
+    _check("tg_layer_mlp_block", rc)
+
+
+def tg_gather_prefill_layer(W: LayerWeights, S: LayerShape, part: int, hidden, kept_idx, scores, sumsq,
+                            n_prunable: int, seq_eps: float, hidden_kept, pos, bias, ratio, ws, stream=None):
+    """tg_gather into hidden_kept / pos / bias / ratio fused with the first RMSNorm of a layer part
+    (TG_LAYER_FULL or TG_LAYER_MLP), which then runs on the kept rows."""
+    n = hidden.shape[0]
+    rc = lib().tg_gather_prefill_layer(ctypes.byref(W), ctypes.byref(S), int(part), _ptr(hidden), n, _ptr(kept_idx),
+                                       kept_idx.numel(), _ptr(scores), _ptr(sumsq), int(n_prunable), float(seq_eps),
+                                       _ptr(hidden_kept), _ptr(pos), _ptr(bias), _ptr(ratio), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream))
+    _check("tg_gather_prefill_layer", rc)
 
 
 def _seg_array(seg_rows):

@@ -49,3 +49,35 @@ def test_exp2_poly_special_values():
     assert got[0] == 1.0 and got[1] == 2.0 and got[2] == 0.5 and got[3] == 256.0
     assert got[5] == 0.0 and got[6] == 0.0
     assert abs(got[4] / 2.0 ** -126 - 1.0) < 1e-4
+
+
+def remez_exp2_cubic(iters: int = 30):
+    """Minimax (Remez exchange) fit of 2^f on [0, 1] by p(f) = 1 + c1 f + c2 f^2
+    + c3 f^3 for RELATIVE error, with p(0) = 1 fixed so that exact powers of
+    two stay exact.  Three free coefficients: at the optimum the relative error
+    p(f)/2^f - 1 takes its maximum magnitude E with alternating signs at four
+    points of (0, 1].  Each step solves p(x_i)/2^x_i - 1 = (-1)^i E on the
+    current reference points, then moves them to the extremum of each sign run
+    of the error on a fine grid.  Returns (c1, c2, c3, max relative error)."""
+    xs = np.linspace(0.0, 1.0, 200001)[1:]
+    ref = np.array([0.1, 0.4, 0.75, 1.0])
+    for _ in range(iters):
+        a = np.stack([ref, ref ** 2, ref ** 3, -((-1.0) ** np.arange(4)) * 2.0 ** ref], 1)
+        c1, c2, c3, _ = np.linalg.solve(a, 2.0 ** ref - 1.0)
+        err = (1.0 + c1 * xs + c2 * xs ** 2 + c3 * xs ** 3) / 2.0 ** xs - 1.0
+        runs = np.split(np.arange(xs.size), np.flatnonzero(np.diff(np.sign(err))) + 1)
+        ext = [r[np.argmax(np.abs(err[r]))] for r in runs]
+        if len(ext) > 4:
+            ext = sorted(ext, key=lambda i: -abs(err[i]))[:4]
+        if len(ext) == 4:
+            ref = np.sort(xs[ext])
+    return c1, c2, c3, float(np.max(np.abs(err)))
+
+
+def test_exp2_poly_coefficients_are_the_remez_minimax_fit():
+    # the kernel's constants re-derived: a Remez fit must land on them (to the
+    # few float32 ulps the fit was printed with) and its error bound must hold
+    c1, c2, c3, e = remez_exp2_cubic()
+    k1, k2, k3 = _coeffs()
+    assert abs(c1 - k1) < 5e-6 and abs(c2 - k2) < 5e-6 and abs(c3 - k3) < 5e-6
+    assert 8.0e-5 < e < 8.7e-5

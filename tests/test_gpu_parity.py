@@ -461,9 +461,16 @@ def test_pruned_layer_matches_oracle(case):
 
 # ============================================================================ whole step
 
-def _check_step(w, tol, sample_rows=None):
+def _check_step(w, tol, sample_rows=None, graph=False):
     step = pipeline.GatedPrefillStep(w, DEV)
-    step.run()
+    if graph:
+        # the launch configuration bench.py times: one CUDA graph per step,
+        # replayed twice (the second replay starts from the first one's buffers)
+        step.capture()
+        step.replay()
+        step.replay()
+    else:
+        step.run()
     torch.cuda.synchronize()
     gate = synth.gate_inputs(w)
     layer = synth.layer_weights(w)
@@ -481,8 +488,9 @@ def _check_step(w, tol, sample_rows=None):
     g = O.gather(gate["hidden"], idx, s_gpu, gate["prunable"], 1e-6)
     assert np.array_equal(host(step.pos).astype(np.int64), g["pos"])
     assert_close(host(step.bias), g["bias"], 1e-6, 2e-6, "bias")
-    # the layer above the gate on the kept rows
-    out_rows = None if sample_rows is None else np.unique(np.r_[0, 1, idx.size // 2, idx.size - 1])
+    assert_close(host(step.ratio), g["ratio"], 1e-7, 1e-6, "ratio")
+    # the layer above the gate on every kept row
+    out_rows = None
     want = O.decoder_layer(g["hidden_kept"], layer, hq=w.hq, hkv=w.hkv, head_dim=w.head_dim, pos=g["pos"],
                            bias=g["bias"], ratio=g["ratio"], head_gain=hp["head_gain"], head_temp=hp["head_temp"],
                            rope_theta=w.rope_theta, qk_norm=w.qk_norm, rows=out_rows)
@@ -503,12 +511,15 @@ def test_step_qwen3_shape_reduced_n():
     _check_step(w, dict(score=1e-3, layer=LAYER_BF16))
 
 
-def test_step_qwen3_16k_full_size_sampled():
-    # the bench workload itself, in the launch configuration bench.py times
+def test_step_qwen3_16k_full_size():
+    # the bench workload itself, in the launch configuration bench.py times:
+    # scores on sampled rows (the gate MLP is row-wise; its full-size rows are
+    # covered by the gate test), the kept set bit-exact, pos / bias / ratio and
+    # every one of the 2064 layer-output rows against the oracle
     w = synth.qwen3_1p7b_16k()
     rng = np.random.default_rng(0)
     rows = np.unique(np.r_[0, 1, 8191, 8192, 8200, 16319, 16320, 16383, rng.integers(0, w.n, 200)])
-    _check_step(w, dict(score=1e-3, layer=LAYER_BF16), sample_rows=rows)
+    _check_step(w, dict(score=1e-3, layer=LAYER_BF16), sample_rows=rows, graph=True)
 
 
 def test_attention_bf16_zero_gain_ignores_bias():

@@ -26,7 +26,7 @@ def _build(w):
             "b2": float(g["b2"]), "norm_w": None}
     layers, heads = pipeline.stack_weights_from_synth(w, w.n_layers, DEV)
     st = pipeline.PrunedPrefillStack(w, _to(g["hidden"], dt), _to(g["prunable"], torch.uint8), gate, layers, heads,
-                                     w.gate_after)
+                                     w.gate_layer)
     olayers = [synth.layer_weights(w, layer=l) for l in range(w.n_layers)]
     oheads = [synth.head_params(w, seed_offset=100 + l) for l in range(w.n_layers)]
     return st, g, olayers, oheads
@@ -37,12 +37,12 @@ def _common(w):
 
 
 def test_stack_fp32_matches_oracle():
-    w = synth.tiny_f32(n_layers=4, gate_after=1)
+    w = synth.tiny_f32(n_layers=4, gate_layer=1)
     st, g, ol, oh = _build(w)
     st.reset()
     st.run()
     torch.cuda.synchronize()
-    want = O.pruned_prefill_stack(g["hidden"], ol, oh, g, w.k, w.gate_after, **_common(w))
+    want = O.pruned_prefill_stack(g["hidden"], ol, oh, g, w.k, w.gate_layer, **_common(w))
     np.testing.assert_array_equal(st.kept.cpu().numpy(), want["kept_idx"])
     np.testing.assert_allclose(_host(st.hk), want["out"], atol=2e-3, rtol=2e-3)
 
@@ -51,37 +51,50 @@ def test_stack_bf16_parts_match_oracle():
     # bf16 tensor-core path: each part is checked against the oracle fed the
     # GPU's own input to that part, so bf16 rounding upstream cannot move the
     # kept set of the comparison
-    w = synth.tiny_f32(dtype="bf16", qk_norm=True, n_layers=4, gate_after=1)
+    w = synth.tiny_f32(dtype="bf16", qk_norm=True, n_layers=4, gate_layer=1)
     st, g, ol, oh = _build(w)
+    common = _common(w)
+    flat = dict(pos=np.arange(w.n), bias=None, ratio=None, head_gain=np.zeros(w.hq), head_temp=np.ones(w.hq))
     st.reset()
     st.full_part()
     torch.cuda.synchronize()
+    # layers 0 .. L-1 and layer L's attention half: the post-attention residual
     h_gate = _host(st.h)
-    full = O.pruned_prefill_stack(g["hidden"], ol[: w.gate_after + 1], oh, g, w.k, w.gate_after,
-                                  pruned=False, **_common(w))
-    np.testing.assert_allclose(h_gate, full["out"], atol=6e-2, rtol=4e-2)
-    st.gate_select_gather()
+    h = g["hidden"]
+    for l in range(w.gate_layer):
+        h = O.decoder_layer(h, ol[l], **flat, **common)
+    want_h1 = O.attention_block(h, ol[w.gate_layer], **flat, **common)
+    np.testing.assert_allclose(h_gate, want_h1, atol=6e-2, rtol=4e-2)
+    st.gate_select()
     torch.cuda.synchronize()
     s_gpu = st.scores.cpu().numpy()
-    s_or = O.gate_scores(h_gate, g["norm_w"], 1e-6, g["w1"], g["b1"], g["w2"], g["b2"], g["prunable"])
+    # the gate normalises with layer L's post-attention RMSNorm weight
+    s_or = O.gate_scores(h_gate, ol[w.gate_layer]["w_post_norm"], 1e-6, g["w1"], g["b1"], g["w2"], g["b2"],
+                         g["prunable"])
     rms = np.sqrt(np.mean(s_or[g["prunable"] == 1] ** 2))
     assert np.max(np.abs(s_gpu - s_or)) <= 1e-3 * rms
     idx = O.select_kept(s_gpu, g["prunable"], w.k)
     np.testing.assert_array_equal(st.kept.cpu().numpy(), idx)     # bit-exact on the GPU's own scores
+    st.gather_mlp()
+    torch.cuda.synchronize()
     gat = O.gather(h_gate, idx, s_gpu, g["prunable"], 1e-6)
+    np.testing.assert_array_equal(st.pos.cpu().numpy(), gat["pos"])
+    np.testing.assert_allclose(st.bias.cpu().numpy(), gat["bias"], atol=1e-6, rtol=2e-6)
+    np.testing.assert_allclose(st.ratio.cpu().numpy(), gat["ratio"], atol=1e-6, rtol=2e-6)
+    # layer L's MLP half on the kept rows only
     hk0 = _host(st.hk)
-    np.testing.assert_array_equal(hk0, gat["hidden_kept"])
+    np.testing.assert_allclose(hk0, O.mlp_block(gat["hidden_kept"], ol[w.gate_layer]), atol=6e-2, rtol=4e-2)
     st.pruned_part()
     torch.cuda.synchronize()
     out = hk0
-    for l in range(w.gate_after + 1, w.n_layers):
+    for l in range(w.gate_layer + 1, w.n_layers):
         out = O.decoder_layer(out, ol[l], pos=gat["pos"], bias=gat["bias"], ratio=gat["ratio"],
-                              head_gain=oh[l]["head_gain"], head_temp=oh[l]["head_temp"], **_common(w))
+                              head_gain=oh[l]["head_gain"], head_temp=oh[l]["head_temp"], **common)
     np.testing.assert_allclose(_host(st.hk), out, atol=6e-2, rtol=4e-2)
 
 
 def test_stack_keeping_everything_with_zero_gain_is_the_unpruned_stack():
-    w = synth.tiny_f32(dtype="bf16", qk_norm=True, n_layers=4, gate_after=1)
+    w = synth.tiny_f32(dtype="bf16", qk_norm=True, n_layers=4, gate_layer=1)
     w = w.replace(k=w.n)
     st, g, ol, oh = _build(w)
     for hp in st._keep:

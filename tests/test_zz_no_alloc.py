@@ -18,6 +18,7 @@ import pytest
 import torch
 
 from learned_token_pruning_b200 import synth, tokengate as tg
+from oracle import tokengate_oracle as O
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -48,6 +49,15 @@ def _case(n, d, h, dtype, seed, with_norm):
 ])
 def test_noalloc_matches_workspace_entry_point_on_two_calls(n, d, h, dtype, with_norm):
     w, args = _case(n, d, h, dtype, seed=n + d, with_norm=with_norm)
+    g = synth.gate_inputs(w)
+    norm_w = args[1].cpu().numpy() if with_norm else None
+    # a bf16 norm weight is folded into bf16 W1 on the tensor-core path: the
+    # oracle takes the same folded weights (one bf16 rounding of W1 * w_n)
+    w1_eff = g["w1"] * norm_w[None, :] if norm_w is not None else g["w1"]
+    if norm_w is not None and dtype == "bf16":
+        w1_eff = synth.round_to(w1_eff.astype(np.float32), "bf16")
+    want = O.gate_scores(g["hidden"], None, 1e-6, w1_eff, g["b1"], g["w2"], 0.125, g["prunable"])
+    want_rms = math.sqrt(float(np.mean(want ** 2)))
     ref_s = torch.empty(n, device=DEV)
     ref_q = torch.empty(1, device=DEV)
     ws = torch.empty(tg.tg_workspace_bytes(tg.TG_OP_GATE_SCORE, n=n, d_model=d, h=h), dtype=torch.uint8, device=DEV)
@@ -64,6 +74,31 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(n, d, h, dtype, with
         assert np.all(np.isfinite(got))
         assert np.max(np.abs(got - ref)) <= SCORE_TOL * rms
         assert abs(q.item() - ref_q.item()) <= 10 * SCORE_TOL * abs(ref_q.item())
+        # and against the oracle directly
+        assert np.max(np.abs(got - want)) <= SCORE_TOL * want_rms
+        want_q = float(np.sum(want[g["prunable"] != 0] ** 2))
+        assert abs(q.item() - want_q) <= 10 * SCORE_TOL * want_q
+
+
+def test_noalloc_cuda_core_path_has_no_scratch_limit():
+    # fp32 takes the CUDA-core path, which uses no scratch: a size whose
+    # tensor-core scratch (2 * d_model * h bytes of folded W1 = 4 MiB) would
+    # exceed the array is still served
+    n, d, h = 300, 4096, 512
+    assert 2 * d * h > tg.lib().tg_gate_score_noalloc_scratch_bytes()
+    rng = np.random.default_rng(3)
+    hid = rng.standard_normal((n, d)).astype(np.float32)
+    w1 = (rng.standard_normal((h, d)) * 0.02).astype(np.float32)
+    w2 = rng.standard_normal(h).astype(np.float32)
+    mask = np.ones(n, np.uint8)
+    mask[-5:] = 0
+    s = torch.empty(n, device=DEV)
+    q = torch.empty(1, device=DEV)
+    tg.tg_gate_score_noalloc(_dev(hid), None, 1e-6, _dev(w1), None, _dev(w2), 0.0, _dev(mask, torch.uint8), s, q)
+    assert tg.tg_check_device_error() == 0
+    want = O.gate_scores(hid, None, 1e-6, w1, None, w2, 0.0, mask)
+    got = s.cpu().numpy()
+    assert np.max(np.abs(got - want)) <= 1e-4 * math.sqrt(float(np.mean(want ** 2)))
 
 
 def test_noalloc_refuses_sizes_beyond_its_scratch():
