@@ -5,41 +5,52 @@
 // and kept rows c <= r
 //     l_rc = temp_h * ratio_r * sm_scale * (q_r . k_c) + gain_h * bias_c
 //     o_r  = sum_c softmax_c(l_r.) v_c
-// computed in base 2 with the head gain factored out of the row:
-//     x_rc = g_h * y_rc,   y_rc = (a_r / g_h) * S_rc + bias_c,
-//     a_r = temp_h * ratio_r * sm_scale * log2(e),  g_h = gain_h * log2(e),
-// so the raw per-key bias tile, which TMA brings in with each K tile, serves
-// both query heads of the CTA unchanged; the softmax runs on y (max, then
-// exp2(g_h * (y - max))).
+// computed in base 2, x_rc = l_rc * log2(e) = a_r * S'_rc, with
+//     a_r = temp_h * ratio_r * sm_scale * log2(e),   g_h = gain_h * log2(e),
+//     S'_rc = q_r . k_c + u_r * bias_c,   u_r = g_h / a_r.
+// The key bias enters the score MMA itself: each Q K^T gets one more K = 16
+// MMA of E_h F^T, where row r of E_h is (u_hi, u_hi, u_lo, 0 ...) and key row c
+// of F is (b_hi, b_lo, b_hi, 0 ...) (bf16 hi/lo splits of u_r and bias_c, so
+// u_r * bias_c is carried to about 2^-17 relative), so the softmax reads
+// nothing from shared memory, whose bandwidth the score MMAs need.  |a_r| is
+// held at least 1e-30 (a zero content scale then leaves 1e-30 * S, nothing).
 //
 // One CTA owns a 128-row query block of TWO query heads that share a KV head
 // (GQA), so every K/V tile fetched by TMA feeds two score tiles.  Keys come in
-// tiles of 64.
-//   warps 0-3  softmax warpgroup 0 (query head 0), one thread per row
-//   warps 4-7  softmax warpgroup 1 (query head 1)
-//   warp 8     TMA producer (Q once, then K + bias tiles through a 3-stage
-//              ring and V tiles through a 2-stage ring)
+// tiles of 128, so each Q K^T is an M128 N128 MMA (an N64 one is bound by the
+// shared-memory reads of its A operand).
+//   warps 0-3  softmax warpgroup 0 (query head 0), one thread per row; at
+//              the start each thread writes its row of E_0
+//   warps 4-7  softmax warpgroup 1 (query head 1), and E_1
+//   warp 8     TMA producer (Q once; K and V tiles through two-stage rings,
+//              the fp32 bias through a four-stage staging ring) and, all 32
+//              lanes, the conversion of each bias tile into F
 //   warp 9     TMEM allocator and single-thread tcgen05.mma issuer
-// Tensor memory (512 columns): S of each head double-buffered, 4 x 64 columns,
-// then O0 and O1 (D columns each).  S = Q K^T is an SS-MMA into TMEM; the
-// softmax reads S with tcgen05.ld and writes P = exp2(x - m) as bf16 pairs
-// back over the first 32 columns of the same S buffer; O += P V is a TS-MMA
-// (P from tensor memory, V MN-major from shared memory), which leaves the
-// shared-memory port to Q, K and V.  Per key tile j the MMA thread issues
-// P V of tile j for both heads and then Q K^T of tile j + 2 into the S
-// buffers tile j used (in issue order, after P V has read P), so the scores
-// of the next tile are ready when a softmax finishes and the loop is bounded
-// by the slower of the softmax and the tensor core, not by their sum.
+// Tensor memory (512 columns): S0 | S1 (128 columns each), O0 | O1 (D each).
+// S' is an SS-MMA into TMEM; the softmax reads it with tcgen05.ld and writes
+// P = exp2(x - m) as bf16 pairs over the first 64 columns of the same S
+// buffer; O += P V is a TS-MMA (P from tensor memory, V MN-major from shared
+// memory).
 //
-// The MMA thread checks the four barriers a tile needs (V, the P of both
-// heads, K of tile j + 2) at once: each mbarrier check holds back its next
-// tcgen05.mma for a shared-memory round trip while the tensor core's short
-// queue drains.  The softmax does its elementwise arithmetic on packed pairs
-// (fma/add.f32x2, three-input max), which halves its FMA-pipe instructions and
-// leaves issue slots to the MMA thread.  The running row maximum only moves
-// when it grows by more than 8 (log2 units); O is then rescaled in tensor
-// memory by the softmax warps after the previous P V into it has completed.
+// The two heads take turns (ping-pong): per key tile j the MMA thread issues
+//     P0 V(j), Q0 K(j+1)^T, P1 V(j), Q1 K(j+1)^T
+// so while one warpgroup turns its scores into probabilities the tensor core
+// works on the other head, and the loop is bound by the slower of the tensor
+// core (four M128 N128 K128 products per tile) and one head's softmax, not by
+// their sum.  Because the scores of head i for tile j+1 are issued after its
+// P V of tile j, their completion (the s_full barrier) also means that P V is
+// done: the softmax rescales O in place when its running maximum moves
+// without waiting for anything.  The running maximum only moves when it grows
+// by more than 8 (log2 units), so every p stays <= 2^8.
+//
+// Exponentials: two heads of 128 x 128 probabilities per tile are as many
+// MUFU operations (16 per clock per SM) as the tensor core has cycles, so one
+// pair in four off the diagonal is evaluated on the FMA pipe instead
+// (exp2_poly2), leaving the MUFU unit headroom.  The elementwise arithmetic
+// runs on packed pairs (fma/add.f32x2, three-input max).
 #pragma once
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "simt.cuh"
@@ -47,31 +58,32 @@
 namespace tg {
 
 constexpr int kAttnThreads = 320;
-constexpr bool kPolyShare = false;  // evaluate a quarter of the exponentials with exp2_poly
 
 template <int D>
 struct AttnCfg {
-  static constexpr int BM = 128, BN = 64;
+  static constexpr int BM = 128, BN = 128;
   static constexpr int kQBytes = BM * D * 2;     // one query tile
   static constexpr int kKVBytes = BN * D * 2;    // one K or V tile
   static constexpr int kQBlk = BM * 128;         // one 64-column TMA box of a Q tile
   static constexpr int kKVBlk = BN * 128;        // one 64-column TMA box of a K or V tile
-  static constexpr int kPBytes = BM * BN * 2;    // one P tile (128 rows x 64 keys, bf16)
-  static constexpr int kKStages = 3, kVStages = 2;
-  static constexpr int kColO0 = 256, kColO1 = 256 + D;
+  static constexpr int kStages = 2;              // K ring and V ring (and F)
+  static constexpr int kBiasStages = 4;          // fp32 bias staging ring
+  static constexpr int kExtBytes = 128 * 32;     // E_h or one F tile: 128 rows x 16 bf16
+  static constexpr int kColO0 = 2 * BN, kColO1 = 2 * BN + D;
   static constexpr size_t kOffK = 2 * kQBytes;
-  static constexpr size_t kOffV = kOffK + kKStages * kKVBytes;
-  static constexpr size_t kOffP = kOffV + kVStages * kKVBytes;
-  static constexpr size_t kOffBias = kOffP;  // (P lives in tensor memory, over its S columns)
-  static constexpr size_t kOffBars = kOffBias + kKStages * BN * 4;  // 16 barriers + TMEM slot
+  static constexpr size_t kOffV = kOffK + kStages * kKVBytes;
+  static constexpr size_t kOffE = kOffV + kStages * kKVBytes;      // [2 heads][kExtBytes]
+  static constexpr size_t kOffF = kOffE + 2 * kExtBytes;           // [2 stages][kExtBytes]
+  static constexpr size_t kOffBias = kOffF + kStages * kExtBytes;  // [4 stages][BN] fp32
+  static constexpr size_t kOffBars = kOffBias + kBiasStages * BN * 4;  // 19 barriers + TMEM slot
   static constexpr size_t kData = kOffBars + 256;
   // D = 64 is padded so that only one CTA fits on an SM and its 512-column
   // TMEM allocation never waits on a neighbour
   static constexpr size_t kSmem = 1024 + (kData < 120 * 1024 ? 120 * 1024 : kData);
 };
 
-// TMEM column of head h's S buffer b
-__device__ __forceinline__ uint32_t attn_col_s(int h, int b) { return static_cast<uint32_t>((h * 2 + b) * 64); }
+// TMEM column of head h's S buffer (and of its P, over the first BN/2 columns)
+__device__ __forceinline__ uint32_t attn_col_s(int h) { return static_cast<uint32_t>(h * 128); }
 
 struct AttnTcParams {
   int m, hq, hkv, group;
@@ -110,20 +122,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe for x <= 8 (Cody-Waite split x = n + f with n = floor(x)
-// and f in [0, 1); 2^f by the cubic minimax polynomial 1 + c1 f + c2 f^2 + c3 f^3
-// fitted for relative error on [0, 1) (max 8.6e-5); 2^n by adding n to the
-// exponent field).  Inputs below -127 return 0.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -127.0f);
-  const float n = floorf(x);
-  const float f = x - n;
-  float q = fmaf(f, 0.07706519961357117f, 0.22764700651168823f);
-  q = fmaf(q, f, 0.6951163411140442f);
-  q = fmaf(q, f, 1.0f);
-  return __int_as_float(__float_as_int(q) + (static_cast<int>(n) << 23));
-}
-
 // Packed fp32 pairs (two lanes of one 64-bit register): Blackwell executes
 // fma/add.f32x2 as one instruction with per-lane IEEE round-to-nearest, so the
 // results equal two scalar fmaf/adds.
@@ -149,6 +147,36 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// Coefficients of q(u) ~ 2^(u + 1/2) on [-1/2, 1/2]: the cubic minimax
+// polynomial for relative error (Remez exchange; max 7.5e-5).
+constexpr float kExp2C0 = 1.414111852645874f;
+constexpr float kExp2C1 = 0.9804190993309021f;
+constexpr float kExp2C2 = 0.34310394525527954f;
+constexpr float kExp2C3 = 0.07802452147006989f;
+
+// 2^x of a pair on the FMA pipe, given xh = x - 1/2 with x <= 8 (lanes below
+// -126 are clamped there).  Cody-Waite split xh = n + u with n the nearest
+// integer (adding and subtracting 1.5 * 2^23 rounds it into the low mantissa
+// bits) and u in [-1/2, 1/2]; 2^(u + 1/2) = q(u); 2^n by adding n to the
+// exponent field of q, which is the low bits of the rounded sum shifted up
+// by 23.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t xh2) {
+  float a, b;
+  f2_unpack(xh2, a, b);
+  const uint64_t x2 = f2_pack(fmaxf(a, -126.5f), fmaxf(b, -126.5f));
+  const uint64_t t2 = f2_add(x2, f2_pack(12582912.0f, 12582912.0f));
+  const uint64_t n2 = f2_add(t2, f2_pack(-12582912.0f, -12582912.0f));
+  const uint64_t u2 = f2_fma(n2, f2_pack(-1.0f, -1.0f), x2);
+  uint64_t q2 = f2_fma(f2_pack(kExp2C3, kExp2C3), u2, f2_pack(kExp2C2, kExp2C2));
+  q2 = f2_fma(q2, u2, f2_pack(kExp2C1, kExp2C1));
+  q2 = f2_fma(q2, u2, f2_pack(kExp2C0, kExp2C0));
+  float q0, q1, t0, t1;
+  f2_unpack(q2, q0, q1);
+  f2_unpack(t2, t0, t1);
+  return f2_pack(__int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23)),
+                 __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23)));
 }
 
 // Two barrier checks issued back to back, so that their shared-memory round
@@ -309,6 +337,128 @@ __device__ __forceinline__ void attn_epilogue(const AttnTcParams& p, const CUten
   }
 }
 
+// One softmax warpgroup thread's share of a key tile: its query row against
+// the tile's 128 keys, x = a * S' read from tensor memory twice in groups of
+// 32 columns, the next group's load issued before the current group is
+// processed (its wait comes after, so the latency hides behind arithmetic):
+//   pass 1: the row maximum of x (four chains);
+//   lazy rescale: the reference maximum only moves when the row maximum
+//     exceeds it by more than 8, so every p stays <= 2^8; when any row of the
+//     warp moves, the warp rescales its rows of O in tensor memory (the P V
+//     that last wrote O is complete, see the kernel);
+//   pass 2: p = 2^(x - m), the row sum (four chains) and P as bf16 pairs over
+//     S columns already read (the P of keys 32q .. 32q + 31 goes to columns
+//     16q .. 16q + 15).
+// kDiag: the tile crosses the diagonal, keys past the row are masked with
+// -inf and every exponential goes to the MUFU unit (exp2(-inf) = 0 exactly);
+// off the diagonal one pair in four is evaluated on the FMA pipe.
+template <int D, bool kDiag>
+__device__ __forceinline__ void attn_softmax_tile(uint32_t t_s, uint32_t t_o, uint64_t a2, int key0, int grow,
+                                                  bool first, float& m_run, float& l_run) {
+  constexpr int BN = 128, G = BN / 32;
+  const uint64_t zero2 = f2_pack(0.0f, 0.0f);
+  float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  uint32_t buf[2][32];
+  tmem_ld32(t_s, buf[0]);
+  tmem_ld_wait();
+#pragma unroll
+  for (int q = 0; q < G; ++q) {
+    if (q + 1 < G) tmem_ld32(t_s + 32 * (q + 1), buf[(q + 1) & 1]);
+    const uint32_t* r = buf[q & 1];
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+      float l0, h0, l1, h1;
+      f2_unpack(f2_fma(a2, f2_pack(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), zero2), l0, h0);
+      f2_unpack(f2_fma(a2, f2_pack(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])), zero2), l1, h1);
+      if (kDiag) {
+        const int k = key0 + 32 * q + e;
+        if (k > grow) l0 = -INFINITY;
+        if (k + 1 > grow) h0 = -INFINITY;
+        if (k + 2 > grow) l1 = -INFINITY;
+        if (k + 3 > grow) h1 = -INFINITY;
+      }
+      mxv[(e >> 2) & 3] = fmax3(mxv[(e >> 2) & 3], fmaxf(l0, h0), fmaxf(l1, h1));
+    }
+    if (q + 1 < G) tmem_ld_wait();
+  }
+  const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
+  float sc = 1.0f;
+  if (mx - m_run > 8.0f) {  // per row: divergent, so no warp-collective op inside
+    if (!first) sc = ex2_approx(m_run - mx);
+    m_run = mx;
+  }
+  // tcgen05.ld/st are warp-collective (.sync.aligned): the whole warp rescales
+  // its 32 rows if any of them needs it, the others with sc = 1
+  if (__any_sync(0xffffffffu, sc != 1.0f)) {
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t o[32];
+      tmem_ld32(t_o + c0, o);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * sc);
+      tmem_st32(t_o + c0, o);
+    }
+  }
+  const uint64_t nm2 = f2_pack(-m_run, -m_run), nmh2 = f2_pack(-m_run - 0.5f, -m_run - 0.5f);
+  uint64_t sum2[4] = {0, 0, 0, 0};
+  tmem_ld32(t_s, buf[0]);
+  tmem_ld_wait();
+#pragma unroll
+  for (int q = 0; q < G; ++q) {
+    if (q + 1 < G) tmem_ld32(t_s + 32 * (q + 1), buf[(q + 1) & 1]);
+    const uint32_t* r = buf[q & 1];
+    uint32_t pk[16];
+#pragma unroll
+    for (int v = 0; v < 16; ++v) {
+      const int e = 2 * v;  // keys 32q + e and 32q + e + 1
+      const uint64_t s2 = f2_pack(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+      uint64_t p2;
+      if (!kDiag && (v & 3) == 3) {
+        p2 = exp2_poly2(f2_fma(a2, s2, nmh2));
+      } else {
+        float x0, x1;
+        f2_unpack(f2_fma(a2, s2, nm2), x0, x1);
+        if (kDiag) {
+          const int k = key0 + 32 * q + e;
+          if (k > grow) x0 = -INFINITY;
+          if (k + 1 > grow) x1 = -INFINITY;
+        }
+        p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+      }
+      sum2[v & 3] = f2_add(sum2[v & 3], p2);
+      float p0, p1;
+      f2_unpack(p2, p0, p1);
+      pk[v] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(t_s + 16 * q, pk);
+    if (q + 1 < G) tmem_ld_wait();
+  }
+  float a0, a1, b0, b1;
+  f2_unpack(f2_add(sum2[0], sum2[1]), a0, a1);
+  f2_unpack(f2_add(sum2[2], sum2[3]), b0, b1);
+  l_run = l_run * sc + ((a0 + a1) + (b0 + b1));
+}
+
+// bf16 hi/lo split: v ~= hi + lo, both bf16 (rounded to nearest)
+__device__ __forceinline__ void bf16_split(float v, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(v);
+  lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+
+// Row r of a 32-byte-swizzled K = 16 operand tile: (x, y, z, 0 x 13) in bf16
+__device__ __forceinline__ void write_ext_row(uint8_t* tile, int r, __nv_bfloat16 x, __nv_bfloat16 y,
+                                              __nv_bfloat16 z) {
+  __nv_bfloat162 xy, z0;
+  xy.x = x;
+  xy.y = y;
+  z0.x = z;
+  z0.y = __float2bfloat16_rn(0.0f);
+  *reinterpret_cast<uint4*>(tile + sw32_offset(r, 0)) =
+      make_uint4(*reinterpret_cast<uint32_t*>(&xy), *reinterpret_cast<uint32_t*>(&z0), 0u, 0u);
+  *reinterpret_cast<uint4*>(tile + sw32_offset(r, 1)) = make_uint4(0u, 0u, 0u, 0u);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -320,17 +470,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   extern __shared__ uint8_t attn_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(attn_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                     // [2 heads][kQBytes]
-  uint8_t* sK = smem + Cfg::kOffK;        // [3 stages][kKVBytes]
+  uint8_t* sK = smem + Cfg::kOffK;        // [2 stages][kKVBytes]
   uint8_t* sV = smem + Cfg::kOffV;        // [2 stages][kKVBytes]
-  float* sBias = reinterpret_cast<float*>(smem + Cfg::kOffBias);  // [3 stages][BN]
+  uint8_t* sE = smem + Cfg::kOffE;        // [2 heads][kExtBytes]   rows (u_hi, u_hi, u_lo)
+  uint8_t* sF = smem + Cfg::kOffF;        // [2 stages][kExtBytes]  key rows (b_hi, b_lo, b_hi)
+  float* sBias = reinterpret_cast<float*>(smem + Cfg::kOffBias);  // [4 stages][BN] fp32
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBars);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;      // [3]  K tile j (stage j % 3) and its bias tile
-  uint64_t* v_full = bars + 4;      // [2]  V tile j (stage j % 2)
-  uint64_t* pv_done = bars + 6;     // [4]  P V of tile j (both heads) complete, slot j % 4
-  uint64_t* s_full = bars + 10;     // [head * 2 + buffer]
-  uint64_t* p_full = bars + 14;     // [head * 2 + buffer]  (128 arrivals: the warpgroup)
-  uint64_t* o_final = bars + 18;
+  uint64_t* k_full = bars + 1;      // [2]  K tile j and F tile j in stage j % 2 (TMA bytes + the converter)
+  uint64_t* k_free = bars + 3;      // [2]  both heads' Q K^T of that tile complete
+  uint64_t* v_full = bars + 5;      // [2]  V tile j in stage j % 2
+  uint64_t* v_free = bars + 7;      // [2]  both heads' P V of that tile complete
+  uint64_t* s_full = bars + 9;      // [head]  S' of the head's current tile (and every earlier MMA) complete
+  uint64_t* p_full = bars + 11;     // [head]  P written (128 arrivals: the warpgroup)
+  uint64_t* o_final = bars + 13;
+  uint64_t* b_full = bars + 14;     // [4]  fp32 bias tile j in staging stage j % 4
+  uint64_t* e_full = bars + 18;     // E_0 and E_1 written (256 arrivals)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
@@ -351,23 +506,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int pair = static_cast<int>(blockIdx.x) % per_tile;
   const int g = pair / pairs_per_kv;
   const int h0 = g * p.group + 2 * (pair % pairs_per_kv);
-  // causal: key tiles 0 .. (128t + 127) / 64, and none past the last kept row;
-  // a split block takes the first or the second half of them
-  const int nt_all = min(2 * t + 2, (p.m + BN - 1) / BN);
+  // causal: key tiles 0 .. t (rows 128t .. 128t + 127), and none past the last
+  // kept row; a split block takes the first or the second half of them
+  const int nt_all = min(t + 1, (p.m + BN - 1) / BN);
   const int j0 = part_code == 2 ? nt_all / 2 : 0;
   const int j1 = part_code == 1 ? nt_all / 2 : nt_all;
   const int nt = j1 - j0;  // key tiles of this CTA; local tile i is global tile j0 + i
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < Cfg::kKStages; ++s) mbar_init(&k_full[s], 1);
-    for (int s = 0; s < 2; ++s) mbar_init(&v_full[s], 1);
-    for (int s = 0; s < 4; ++s) mbar_init(&pv_done[s], 1);
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 2);
+      mbar_init(&k_free[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_free[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
     }
+    for (int s = 0; s < Cfg::kBiasStages; ++s) mbar_init(&b_full[s], 1);
     mbar_init(o_final, 1);
+    mbar_init(e_full, 256);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -375,8 +533,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  if (!p.has_bias)
-    for (int i = threadIdx.x; i < Cfg::kKStages * BN; i += kAttnThreads) sBias[i] = 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -385,7 +541,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   pdl_launch_dependents();
 
   if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer + F conversion
+    bool ok = true;
     if (lane == 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
@@ -395,27 +552,63 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int i = 0; i < 2; ++i)
         for (int b = 0; b < kDBoxes; ++b)
           tma_load_2d(sQ + i * Cfg::kQBytes + b * Cfg::kQBlk, &tmQ, q_full, (h0 + i) * D + 64 * b, t * 128);
-      for (int j = 0; j < nt; ++j) {
-        // K stage j % 3 held tile j - 3, V stage j % 2 held tile j - 2: both
-        // are free once the P V of that tile has completed
-        if (j >= 3 && !mbar_wait(&pv_done[(j - 3) & 3], ((j - 3) >> 2) & 1, kErrWaitAttention)) {
-          *abort_flag = 1;
-          break;
+      if (p.has_bias)
+        for (int j = 0; j < 2 && j < nt; ++j) {
+          mbar_arrive_expect_tx(&b_full[j], BN * 4);
+          tma_load_1d(sBias + j * BN, &tmBias, &b_full[j], (j0 + j) * BN);
         }
-        const int ks = j % 3, vs = j & 1;
-        mbar_arrive_expect_tx(&k_full[ks], Cfg::kKVBytes + (p.has_bias ? BN * 4 : 0));
-        for (int b = 0; b < kDBoxes; ++b)
-          tma_load_2d(sK + ks * Cfg::kKVBytes + b * Cfg::kKVBlk, &tmK, &k_full[ks], g * D + 64 * b, (j0 + j) * BN);
-        if (p.has_bias) tma_load_1d(sBias + ks * BN, &tmBias, &k_full[ks], (j0 + j) * BN);
-        if (j >= 2 && !mbar_wait(&pv_done[(j - 2) & 3], ((j - 2) >> 2) & 1, kErrWaitAttention)) {
-          *abort_flag = 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&v_full[vs], Cfg::kKVBytes);
-        for (int b = 0; b < kDBoxes; ++b)
-          tma_load_2d(sV + vs * Cfg::kKVBytes + b * Cfg::kKVBlk, &tmV, &v_full[vs], g * D + 64 * b, (j0 + j) * BN);
-      }
     }
+    for (int j = 0; j < nt; ++j) {
+      // stage j % 2 held tile j - 2: K (and F) are free once both heads'
+      // Q K^T of that tile completed, V once both P V did
+      const int s = j & 1;
+      const uint32_t fph = ((j - 2) >> 1) & 1;
+      if (lane == 0) {
+        if (j >= 2 && !mbar_wait(&k_free[s], fph, kErrWaitAttention)) {
+          ok = false;
+        } else {
+          mbar_arrive_expect_tx(&k_full[s], Cfg::kKVBytes);
+          for (int b = 0; b < kDBoxes; ++b)
+            tma_load_2d(sK + s * Cfg::kKVBytes + b * Cfg::kKVBlk, &tmK, &k_full[s], g * D + 64 * b, (j0 + j) * BN);
+          if (j >= 2 && !mbar_wait(&v_free[s], fph, kErrWaitAttention)) {
+            ok = false;
+          } else {
+            mbar_arrive_expect_tx(&v_full[s], Cfg::kKVBytes);
+            for (int b = 0; b < kDBoxes; ++b)
+              tma_load_2d(sV + s * Cfg::kKVBytes + b * Cfg::kKVBlk, &tmV, &v_full[s], g * D + 64 * b,
+                          (j0 + j) * BN);
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      if (p.has_bias) {
+        // F(j) from the fp32 bias tile: lane l converts keys 4l .. 4l + 3
+        const int bs = j & 3;
+        if (!warp_wait(&b_full[bs], (j >> 2) & 1, kErrWaitAttention)) {
+          ok = false;
+          break;
+        }
+        const float4 b4 = *reinterpret_cast<const float4*>(sBias + bs * BN + 4 * lane);
+        const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+        uint8_t* f = sF + s * Cfg::kExtBytes;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          __nv_bfloat16 hi, lo;
+          bf16_split(bv[u], hi, lo);
+          write_ext_row(f, 4 * lane + u, hi, lo, hi);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        // staging stage (j + 2) % 4 last held tile j - 2, converted two steps ago
+        if (lane == 0 && j + 2 < nt) {
+          mbar_arrive_expect_tx(&b_full[(j + 2) & 3], BN * 4);
+          tma_load_1d(sBias + ((j + 2) & 3) * BN, &tmBias, &b_full[(j + 2) & 3], (j0 + j + 2) * BN);
+        }
+      }
+      if (lane == 0) mbar_arrive(&k_full[s]);  // F(j) written (or no bias to add)
+    }
+    if (!ok) *abort_flag = 1;
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -426,68 +619,69 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dv0 = sdesc_sw128(smem_u32(sV), Cfg::kKVBlk, 1024);
+      const uint64_t de0 = sdesc_sw32(smem_u32(sE)), df0 = sdesc_sw32(smem_u32(sF));
+      const bool ext = p.has_bias != 0;
       auto issue_qk = [&](int h, int j) {
-        const uint64_t da = dq0 + (h * Cfg::kQBytes >> 4), db = dk0 + ((j % 3) * Cfg::kKVBytes >> 4);
-        const uint32_t d_tmem = tmem + attn_col_s(h, j & 1);
+        const uint64_t da = dq0 + (h * Cfg::kQBytes >> 4), db = dk0 + ((j & 1) * Cfg::kKVBytes >> 4);
+        const uint32_t d_tmem = tmem + attn_col_s(h);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           umma_ss(d_tmem, da + (((kk >> 2) * Cfg::kQBlk + (kk & 3) * 32) >> 4),
                   db + (((kk >> 2) * Cfg::kKVBlk + (kk & 3) * 32) >> 4), idesc_qk, kk != 0 ? 1u : 0u);
-        umma_commit(&s_full[2 * h + (j & 1)]);
+        // + E_h F(j)^T: the key bias times u_r
+        if (ext)
+          umma_ss(d_tmem, de0 + ((h * Cfg::kExtBytes) >> 4), df0 + (((j & 1) * Cfg::kExtBytes) >> 4), idesc_qk, 1u);
+        umma_commit(&s_full[h]);
       };
       auto issue_pv = [&](int h, int j) {
-        // A = P from tensor memory (two bf16 keys per column, over the S columns of tile j)
-        const uint32_t pa = tmem + attn_col_s(h, j & 1);
+        // A = P from tensor memory (two bf16 keys per column, over the S columns)
+        const uint32_t pa = tmem + attn_col_s(h);
         const uint64_t db = dv0 + ((j & 1) * Cfg::kKVBytes >> 4);
         const uint32_t d_tmem = tmem + (h ? Cfg::kColO1 : Cfg::kColO0);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
           umma_ts(d_tmem, pa + kk * 8, db + ((kk * 16 * 128) >> 4), idesc_pv, (j | kk) != 0 ? 1u : 0u);
       };
-      // the scores of tiles 0 and 1 first
-      bool ok = mbar_wait2(q_full, 0, &k_full[0], 0, kErrWaitAttention);
+      // the scores of tile 0 for both heads first
+      bool ok = mbar_wait2(q_full, 0, &k_full[0], 0, kErrWaitAttention) && mbar_wait(e_full, 0, kErrWaitAttention);
       if (ok) {
         tc_fence_after();
         issue_qk(0, 0);
         issue_qk(1, 0);
+        umma_commit(&k_free[0]);
       }
-      if (ok && nt > 1 && (ok = mbar_wait(&k_full[1], 0, kErrWaitAttention))) {
-        tc_fence_after();
-        issue_qk(0, 1);
-        issue_qk(1, 1);
-      }
-      // per tile j: P V of tile j for head 0, then head 1, then the scores of
-      // tile j + 2 into the S buffers whose tile j the softmax has read (its
-      // p_full arrival comes after its S loads completed)
-      // Each barrier check of this thread holds back its next MMA issue for a
-      // shared-memory round trip (~150-250 cycles), during which the tensor
-      // core's short queue drains; so all four barriers a tile needs (V, the P
-      // of both heads, K of tile j + 2) are checked at once, and the tile's
-      // twenty-four MMAs then issue back to back.
+      // per tile j: P0 V(j) and Q0 K(j+1)^T once V(j), P0(j) and K(j+1) are
+      // there (checked together: each barrier check holds back the next MMA
+      // issue for a shared-memory round trip); then P1 V(j) and Q1 K(j+1)^T
+      // once P1(j) is.  Q_i K(j+1)^T overwrites S_i / P_i after P_i V(j) has
+      // read P_i (tcgen05 MMAs of one thread run in issue order).
       for (int j = 0; ok && j < nt; ++j) {
-        const uint32_t ph = (j >> 1) & 1;
-        const bool next = j + 2 < nt;
+        const int s = j & 1;
+        const uint32_t vph = (j >> 1) & 1, pph = j & 1;
+        const bool next = j + 1 < nt;
+        uint64_t* kb = &k_full[(j + 1) & 1];
+        const uint32_t kph = ((j + 1) >> 1) & 1;
         {
-          uint64_t* kb = &k_full[(j + 2) % 3];
-          const uint32_t kph = ((j + 2) / 3) & 1;
-          const bool r0 = mbar_try_wait(smem_u32(&v_full[j & 1]), ph);
-          const bool r1 = mbar_try_wait(smem_u32(&p_full[j & 1]), ph);
-          const bool r2 = mbar_try_wait(smem_u32(&p_full[2 + (j & 1)]), ph);
-          const bool r3 = !next || mbar_try_wait(smem_u32(kb), kph);
-          if (!(r0 && r1 && r2 && r3)) {
-            ok = mbar_wait2(&v_full[j & 1], ph, &p_full[j & 1], ph, kErrWaitAttention) &&
-                 mbar_wait(&p_full[2 + (j & 1)], ph, kErrWaitAttention) &&
+          const bool r0 = mbar_try_wait(smem_u32(&v_full[s]), vph);
+          const bool r1 = mbar_try_wait(smem_u32(&p_full[0]), pph);
+          const bool r2 = !next || mbar_try_wait(smem_u32(kb), kph);
+          if (!(r0 && r1 && r2)) {
+            ok = mbar_wait2(&v_full[s], vph, &p_full[0], pph, kErrWaitAttention) &&
                  (!next || mbar_wait(kb, kph, kErrWaitAttention));
             if (!ok) break;
           }
         }
         tc_fence_after();
         issue_pv(0, j);
+        if (next) issue_qk(0, j + 1);
+        if (!mbar_try_wait(smem_u32(&p_full[1]), pph) && !(ok = mbar_wait(&p_full[1], pph, kErrWaitAttention)))
+          break;
+        tc_fence_after();
         issue_pv(1, j);
-        umma_commit(&pv_done[j & 3]);
+        umma_commit(&v_free[s]);
         if (next) {
-          issue_qk(0, j + 2);
-          issue_qk(1, j + 2);
+          issue_qk(1, j + 1);
+          umma_commit(&k_free[(j + 1) & 1]);
         }
       }
       if (ok) umma_commit(o_final);
@@ -500,133 +694,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int row = q4 * 32 + lane;     // row inside the query tile
     const int grow = t * 128 + row;
     const int h = h0 + wg;
+    const uint32_t colS = attn_col_s(wg);
     const uint32_t colO = wg ? Cfg::kColO1 : Cfg::kColO0;
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
-    const float a_row = grow < p.m ? p.temp[h] * (p.ratio ? p.ratio[grow] : 1.0f) * p.scale_log2 : 0.0f;
-    // g > 0 always (a zero gain leaves the bias term at 1e-20 * bias, i.e. nothing)
-    const float gg = fmaxf(p.gain[h] * kLog2e, 1e-20f);
-    const float a_y = a_row / gg;
-    const uint64_t ay2 = f2_pack(a_y, a_y), gg2 = f2_pack(gg, gg);
-    float m_run = -INFINITY, l_run = 0.0f;  // running max of y, running sum of exp2(g * (y - m_run))
+    // x = a * S' with S' = q . k + u * bias, u = g / a (|a| held >= 1e-30)
+    float a_row = grow < p.m ? p.temp[h] * (p.ratio ? p.ratio[grow] : 1.0f) * p.scale_log2 : 0.0f;
+    if (fabsf(a_row) < 1e-30f) a_row = 1e-30f;
+    {
+      __nv_bfloat16 uh, ul;
+      bf16_split(p.gain[h] * kLog2e / a_row, uh, ul);
+      write_ext_row(sE + wg * Cfg::kExtBytes, row, uh, uh, ul);
+      fence_proxy_async_smem();
+      mbar_arrive(e_full);
+    }
+    const uint64_t a2 = f2_pack(a_row, a_row);
+    float m_run = -INFINITY, l_run = 0.0f;  // running max of x, running sum of exp2(x - m_run)
     bool ok = true;
 
-    for (int j = 0; j < nt; ++j) {
-      const int b = j & 1;
-      const uint32_t ph = (j >> 1) & 1;
-      // S of tile j and its bias tile (it rides with K); P goes over the S
-      // columns, which the P V of tile j - 2 had read before the Q K^T of
-      // tile j wrote them
-      bool rdy = !*abort_flag && mbar_wait2(&s_full[2 * wg + b], ph, &k_full[j % 3], (j / 3) & 1, kErrWaitAttention);
-      if (!__all_sync(0xffffffffu, rdy)) {
-        ok = false;
-        break;
-      }
+    // one key tile: wait for its scores (the s_full phase completes once per
+    // tile), turn them into P, hand P over once the S loads, the P stores and
+    // any O rescale are done
+    auto tile = [&](int j, auto diag) -> bool {
+      bool rdy = !*abort_flag && mbar_wait(&s_full[wg], j & 1, kErrWaitAttention);
+      if (!__all_sync(0xffffffffu, rdy)) return false;
       tc_fence_after();
-      uint32_t s0[32], s1[32];
-      tmem_ld32(tmem + lane_base + attn_col_s(wg, b), s0);
-      tmem_ld32(tmem + lane_base + attn_col_s(wg, b) + 32, s1);
-      tmem_ld_wait();
-      const float* bias = sBias + (j % 3) * BN;
-      // Pass 1: y = a_y * S + bias on pairs, and the row maximum (four
-      // independent chains); the causal mask only touches the key tiles that
-      // cross the diagonal.
-      uint64_t y2[BN / 2];
-      const int key0 = (j0 + j) * BN;
-      const bool diag = key0 + BN - 1 > t * 128;  // warp-uniform
-      float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      auto logits = [&](const uint32_t(&r)[32], int c0) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 b4 = *reinterpret_cast<const float4*>(bias + c0 + e);
-          const int i = (c0 + e) >> 1;
-          y2[i] = f2_fma(ay2, f2_pack(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), f2_pack(b4.x, b4.y));
-          y2[i + 1] = f2_fma(ay2, f2_pack(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])), f2_pack(b4.z, b4.w));
-          if (diag) {
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              float lo, hi;
-              f2_unpack(y2[i + u], lo, hi);
-              const int c = key0 + c0 + e + 2 * u;
-              if (c > grow) lo = -INFINITY;
-              if (c + 1 > grow) hi = -INFINITY;
-              y2[i + u] = f2_pack(lo, hi);
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            float lo, hi;
-            f2_unpack(y2[i + u], lo, hi);
-            mxv[(i + u) & 3] = fmax3(mxv[(i + u) & 3], lo, hi);
-          }
-        }
-      };
-      logits(s0, 0);
-      logits(s1, 32);
-      const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
-      // lazy rescaling: the reference maximum only moves when the row maximum
-      // exceeds it by more than 8 in log2 units, so every p stays <= 2^8
-      // (per row: the branch is divergent, so it holds no warp-collective op)
-      float sc = 1.0f;
-      if (gg * (mx - m_run) > 8.0f) {
-        if (j > 0) sc = ex2_approx(gg * (m_run - mx));
-        m_run = mx;
-      }
-      const float nm = -gg * m_run;
-      const uint64_t nm2 = f2_pack(nm, nm);
-      // Pass 2: p = 2^(g*y - g*m), partial sums on pairs, P as bf16 pairs into
-      // tensor memory over the first 32 columns of this tile's S buffer
-      uint64_t sum2[2] = {0, 0};
-      uint32_t pk[BN / 2];
-#pragma unroll
-      for (int i = 0; i < BN / 2; ++i) {
-        float x0, x1;
-        f2_unpack(f2_fma(gg2, y2[i], nm2), x0, x1);
-        float p0, p1;
-        if (kPolyShare && (i & 3) == 3) {
-          p0 = exp2_poly(x0);
-          p1 = exp2_poly(x1);
-        } else {
-          p0 = ex2_approx(x0);
-          p1 = ex2_approx(x1);
-        }
-        sum2[i & 1] = f2_add(sum2[i & 1], f2_pack(p0, p1));
-        pk[i] = pack_bf16x2(p0, p1);
-      }
-      tmem_st32(tmem + lane_base + attn_col_s(wg, b), pk);
-      float sa, sb, sc2, sd;
-      f2_unpack(sum2[0], sa, sb);
-      f2_unpack(sum2[1], sc2, sd);
-      l_run = l_run * sc + ((sa + sb) + (sc2 + sd));
-      // tcgen05.ld/st are warp-collective (.sync.aligned): the whole warp
-      // rescales its 32 rows if any of them needs it, the others with sc = 1
-      if (__any_sync(0xffffffffu, sc != 1.0f)) {
-        // O holds the sum over tiles < j once the P V of tile j - 1 is done;
-        // the P V of tile j is not issued before p_full below
-        if (!warp_wait(&pv_done[(j - 1) & 3], ((j - 1) >> 2) & 1, kErrWaitAttention)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_base + colO + c0, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * sc);
-          tmem_st32(tmem + lane_base + colO + c0, o);
-        }
-      }
-      // the S loads, the P store and any O rescale are complete: hand P over
+      attn_softmax_tile<D, decltype(diag)::value>(tmem + lane_base + colS, tmem + lane_base + colO, a2,
+                                                  (j0 + j) * BN, grow, j == 0, m_run, l_run);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[2 * wg + b]);
-    }
+      mbar_arrive(&p_full[wg]);
+      return true;
+    };
+    // only global tile t crosses the diagonal (keys 128t .. 128t + 127), and
+    // when this CTA has it, it is its last tile; the masked variant of the
+    // tile is kept out of the loop so that the two are compiled apart
+    const bool has_diag = j1 == t + 1;
+    for (int j = 0; ok && j < nt - (has_diag ? 1 : 0); ++j) ok = tile(j, std::false_type{});
+    if (ok && has_diag) ok = tile(nt - 1, std::true_type{});
     if (ok && !*abort_flag) ok = warp_wait(o_final, 0, kErrWaitAttention);
     // every softmax thread ends here, so the named barriers below see all 256
     if (!ok) *abort_flag = 1;
     attn_epilogue<D>(p, &tmO, sK, tmem, lane_base, colO, wg, row, grow, h, t, part_code, (t - p.ts) * per_tile + pair, ok,
-                     m_run, l_run, gg, abort_flag, &s_last, &s_ready);
+                     m_run, l_run, 1.0f, abort_flag, &s_last, &s_ready);
   }
   tc_fence_before();
   __syncthreads();

@@ -406,6 +406,23 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
+// K-major operand tile of 16 bf16 (32 bytes) per row in the 32-byte swizzle
+// layout: 8-row atoms of 256 bytes (SBO), the two 16-byte chunks of row r
+// stored at positions c ^ ((r >> 2) & 1).
+__device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1u) << 16;           // LBO (unused: the tile is one atom wide in K)
+  d |= static_cast<uint64_t>(256u >> 4) << 32;    // SBO: 8 rows x 32 bytes
+  d |= 1ull << 46;  // descriptor version for sm_100
+  d |= 6ull << 61;  // SWIZZLE_32B
+  return d;
+}
+// byte offset of 16-byte chunk c of row r in such a tile
+__host__ __device__ constexpr uint32_t sw32_offset(int r, int c) {
+  return static_cast<uint32_t>((r >> 3) * 256 + (r & 7) * 32 + ((c ^ ((r >> 2) & 1)) << 4));
+}
+
 // kind::f16 instruction descriptor: bf16 x bf16 -> fp32, dense.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                                   // D format: f32

@@ -488,7 +488,7 @@ int tg_check_device_error(void* stream, uint32_t* detail) {
 // fixed cost.  The plan splits the k longest blocks for the k whose simulated
 // longest-first schedule on the SMs ends first (k = 0: no split), and launches
 // the CTAs longest first.
-constexpr int kAttnCtaFixed = 4;
+constexpr int kAttnCtaFixed = 2;
 
 struct AttnPlan {
   int T = 0, per_tile = 0, ts = 0;
@@ -536,7 +536,7 @@ int64_t attn_makespan(const std::vector<AttnItem>& it, int per_tile, int sms, in
 }
 
 AttnPlan attn_plan_compute(int64_t m, int hkv, int group, int head_dim, int sms) {
-  constexpr int bn = 64;  // key-tile width of k_attn_tc
+  constexpr int bn = tg::AttnCfg<128>::BN;  // key-tile width of k_attn_tc
   AttnPlan pl;
   pl.T = static_cast<int>((m + 127) / 128);
   pl.per_tile = hkv * (group / 2);
@@ -545,7 +545,7 @@ AttnPlan attn_plan_compute(int64_t m, int hkv, int group, int head_dim, int sms)
   // fixed cost per CTA in key tiles, and the fewest tiles a split block may have
   // (each half keeps a visible key in every row)
   const int fixed = kAttnCtaFixed;
-  const int min_split = 4;
+  const int min_split = 2;
   sms = std::max(sms, 1);
   // only short launches gain from splitting: at most about two waves of CTAs,
   // and blocks of at least 4 tiles (each half keeps a visible key per row)
@@ -861,14 +861,15 @@ int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk, c
     int rc = make_map(&tq, q, uint64_t(hq) * head_dim, uint64_t(m), uint64_t(ldq) * 2, 128);
     // the output tile of a head is stored by TMA from shared memory, 128 rows x 64 columns per box
     if (!rc) rc = make_map(&to, out, uint64_t(hq) * head_dim, uint64_t(m), uint64_t(ldo) * 2, 128);
-    // keys and values come in tiles of 64 rows (AttnCfg::BN)
-    if (!rc) rc = make_map(&tk, k, uint64_t(hkv) * head_dim, uint64_t(m), uint64_t(ldk) * 2, 64);
-    if (!rc) rc = make_map(&tv, v, uint64_t(hkv) * head_dim, uint64_t(m), uint64_t(ldv) * 2, 64);
+    // keys and values come in tiles of AttnCfg::BN = 128 rows
+    constexpr int kBN = tg::AttnCfg<128>::BN;
+    if (!rc) rc = make_map(&tk, k, uint64_t(hkv) * head_dim, uint64_t(m), uint64_t(ldk) * 2, kBN);
+    if (!rc) rc = make_map(&tv, v, uint64_t(hkv) * head_dim, uint64_t(m), uint64_t(ldv) * 2, kBN);
     if (rc) return rc;
     p.has_bias = bias != nullptr;
     if (bias) {
       if (!aligned16(bias)) return fail(TG_ERR_ALIGN, "bias must be 16-byte aligned");
-      if ((rc = make_map_1d_f32(&tb, bias, uint64_t(m), 64))) return rc;
+      if ((rc = make_map_1d_f32(&tb, bias, uint64_t(m), kBN))) return rc;
     }
     // key-range split of the longest row blocks when a workspace is given
     const AttnPlan& pl = attn_plan(m, hkv, group, head_dim, sm_count());
