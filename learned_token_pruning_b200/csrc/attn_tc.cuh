@@ -157,7 +157,8 @@ constexpr float kExp2C2 = 0.34310394525527954f;
 constexpr float kExp2C3 = 0.07802452147006989f;
 
 // 2^x of a pair on the FMA pipe, given xh = x - 1/2 with x <= 8 (lanes below
-// -126 are clamped there).  Cody-Waite split xh = n + u with n the nearest
+// -125 are clamped there, so every result is a normal float).  Cody-Waite
+// split xh = n + u with n the nearest
 // integer (adding and subtracting 1.5 * 2^23 rounds it into the low mantissa
 // bits) and u in [-1/2, 1/2]; 2^(u + 1/2) = q(u); 2^n by adding n to the
 // exponent field of q, which is the low bits of the rounded sum shifted up
@@ -165,7 +166,7 @@ constexpr float kExp2C3 = 0.07802452147006989f;
 __device__ __forceinline__ uint64_t exp2_poly2(uint64_t xh2) {
   float a, b;
   f2_unpack(xh2, a, b);
-  const uint64_t x2 = f2_pack(fmaxf(a, -126.5f), fmaxf(b, -126.5f));
+  const uint64_t x2 = f2_pack(fmaxf(a, -125.5f), fmaxf(b, -125.5f));
   const uint64_t t2 = f2_add(x2, f2_pack(12582912.0f, 12582912.0f));
   const uint64_t n2 = f2_add(t2, f2_pack(-12582912.0f, -12582912.0f));
   const uint64_t u2 = f2_fma(n2, f2_pack(-1.0f, -1.0f), x2);
