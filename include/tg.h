@@ -77,6 +77,20 @@ const char* tg_last_error(void);
 int tg_check_device_error(void* stream, uint32_t* detail);
 
 /*
+ * For tests of the timeout path only (the TokenGate pages have no counterpart).
+ * Waits on a flag in global memory that another CTA sets -- the attention
+ * kernel's split-merge ready count, where the second half of a split query
+ * block waits for the first half's partial result -- give up after
+ * limit_ns nanoseconds (default 1 s) and wait for the count to reach
+ * merge_ready_target (default: the protocol's own value).  A test sets a
+ * short limit and a target no CTA reaches, so the wait runs out: the waiting
+ * CTA then writes no output, records TG_ERR_DEVICE_TIMEOUT in the device error
+ * word (read with tg_check_device_error) and returns; the context stays
+ * usable.  0 restores a default.  Applies to the current device; synchronous.
+ */
+int tg_debug_set_flag_wait(uint64_t limit_ns, uint32_t merge_ready_target);
+
+/*
  * Gate scores ([R] §4.1 "Gate module"; [M] "how does learned token pruning
  * work"): for every token j,
  *     x_j = RMSNorm(h_j) * norm_w            (eps = norm_eps)

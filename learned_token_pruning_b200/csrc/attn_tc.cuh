@@ -241,13 +241,15 @@ __device__ __forceinline__ void attn_epilogue(const AttnTcParams& p, const CUten
         // bounded wait for the first half's ready value (it is resident and
         // past its own count, so it gets there without this CTA's help)
         bool ready = false;
+        const uint32_t target = g_merge_ready_target;
+        const uint64_t limit = g_flag_wait_limit_ns;
         const uint64_t t0 = globaltimer_ns();
         for (uint32_t i = 0;; ++i) {
-          if (ld_acquire_gpu(&p.counters[slot]) >= 6u) {
+          if (ld_acquire_gpu(&p.counters[slot]) >= target) {
             ready = true;
             break;
           }
-          if ((i & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) break;
+          if ((i & 63u) == 63u && globaltimer_ns() - t0 > limit) break;
         }
         if (!ready) {
           raise_error(kErrWaitAttention, 2);

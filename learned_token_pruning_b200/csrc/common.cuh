@@ -55,6 +55,15 @@ __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepc
 // a few milliseconds, so one second only expires on a genuine bug.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;
 
+// Waits on a flag in global memory that another CTA sets (the attention
+// kernel's split-merge ready count) read their limit and the value they wait
+// for from here, so that a test can make such a wait run out on purpose
+// (tg_debug_set_flag_wait): a short limit and a target no CTA reaches.  The
+// defaults are kWaitLimitNs and the protocol's own value.
+constexpr uint32_t kMergeReadyTarget = 6;
+__device__ uint64_t g_flag_wait_limit_ns = kWaitLimitNs;
+__device__ uint32_t g_merge_ready_target = kMergeReadyTarget;
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

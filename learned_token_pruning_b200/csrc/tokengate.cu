@@ -314,7 +314,9 @@ int launch_gate_tc(const void* A, const void* W1, int M, int K, const tg::GatePa
   p.M = M;
   p.K = K;
   p.hidden = static_cast<const __nv_bfloat16*>(A);
-  return launch_pdl("k_gate_tc", tg::k_gate_tc<BN>, dim3((M + tg::kGateBM - 1) / tg::kGateBM), dim3(tg::kGateThreads),
+  // persistent: one CTA per SM (or per tile when there are fewer tiles)
+  const int tiles = (M + tg::kGateBM - 1) / tg::kGateBM;
+  return launch_pdl("k_gate_tc", tg::k_gate_tc<BN>, dim3(tiles < sm_count() ? tiles : sm_count()), dim3(tg::kGateThreads),
                     Cfg::kSmem, st, ta, tb, p);
 }
 
@@ -462,6 +464,15 @@ const char* tg_status_string(int status) {
 }
 
 const char* tg_last_error(void) { return g_last_error; }
+
+int tg_debug_set_flag_wait(uint64_t limit_ns, uint32_t merge_ready_target) {
+  const uint64_t lim = limit_ns ? limit_ns : tg::kWaitLimitNs;
+  const uint32_t tgt = merge_ready_target ? merge_ready_target : tg::kMergeReadyTarget;
+  cudaError_t e = cudaMemcpyToSymbol(tg::g_flag_wait_limit_ns, &lim, sizeof(lim));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(tg::g_merge_ready_target, &tgt, sizeof(tgt));
+  if (e != cudaSuccess) return fail(TG_ERR_CUDA, "tg_debug_set_flag_wait: %s", cudaGetErrorString(e));
+  return TG_OK;
+}
 
 int tg_check_device_error(void* stream, uint32_t* detail) {
   cudaError_t e = cudaStreamSynchronize(as_stream(stream));

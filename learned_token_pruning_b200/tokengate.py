@@ -68,6 +68,7 @@ SIGNATURES = {
     "tg_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I32, _I32, ctypes.POINTER(LayerShape)]),
     "tg_gate_score_noalloc": (_INT, [_P, _INT, _I64, _I32, _P, _F, _P, _P, _P, _F, _I32, _P, _P, _P, _P]),
     "tg_gate_score_noalloc_scratch_bytes": (_SZ, []),
+    "tg_debug_set_flag_wait": (_INT, [ctypes.c_uint64, ctypes.c_uint32]),
     "tg_gather_rmsnorm": (_INT, [_P, _INT, _I64, _I32, _P, _I64, _P, _P, _I64, _F, _P, _F, _P, _P, _P, _P, _P, _P]),
     "tg_layer_attention_block": (_INT, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerShape), _P, _P, _P, _P,
                                         _I64, _P, _SZ, _P]),
@@ -132,6 +133,11 @@ def tg_check_device_error(stream=None) -> int:
     rc = lib().tg_check_device_error(_stream(stream), ctypes.byref(word))
     _check("tg_check_device_error", rc)
     return word.value
+
+
+def tg_debug_set_flag_wait(limit_ns: int = 0, merge_ready_target: int = 0):
+    """Test hook: limit (ns) and target of the device's waits on flags set by other CTAs (0 = defaults)."""
+    _check("tg_debug_set_flag_wait", lib().tg_debug_set_flag_wait(int(limit_ns), int(merge_ready_target)))
 
 
 def tg_workspace_bytes(op: int, n: int = 0, m: int = 0, d_model: int = 0, h: int = 0,
