@@ -180,14 +180,6 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t xh2) {
                  __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23)));
 }
 
-// Two barrier checks issued back to back, so that their shared-memory round
-// trips overlap; falls back to the bounded waits when either is still open.
-__device__ __forceinline__ bool mbar_wait2(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, uint32_t site) {
-  const bool r0 = mbar_try_wait(smem_u32(b0), p0);
-  const bool r1 = mbar_try_wait(smem_u32(b1), p1);
-  if (r0 && r1) return true;
-  return mbar_wait(b0, p0, site) && mbar_wait(b1, p1, site);
-}
 
 // Epilogue of one softmax warpgroup (128 rows of one query head, O in tensor
 // memory at column colO, complete once o_final has been observed): normalise

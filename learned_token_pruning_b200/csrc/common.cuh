@@ -130,6 +130,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   }
 }
 
+// Two barrier checks issued back to back, so that their shared-memory round
+// trips overlap; falls back to the bounded waits when either is still open.
+__device__ __forceinline__ bool mbar_wait2(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, uint32_t site) {
+  const bool r0 = mbar_try_wait(smem_u32(b0), p0);
+  const bool r1 = mbar_try_wait(smem_u32(b1), p1);
+  if (r0 && r1) return true;
+  return mbar_wait(b0, p0, site) && mbar_wait(b1, p1, site);
+}
+
 // Warp-uniform bounded wait: every lane waits on the barrier itself (so each
 // one acquires what the barrier guards) and the verdict is agreed on by vote,
 // so a warp never splits over a later warp-collective instruction.

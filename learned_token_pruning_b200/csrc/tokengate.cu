@@ -499,7 +499,7 @@ int tg_check_device_error(void* stream, uint32_t* detail) {
 // fixed cost.  The plan splits the k longest blocks for the k whose simulated
 // longest-first schedule on the SMs ends first (k = 0: no split), and launches
 // the CTAs longest first.
-constexpr int kAttnCtaFixed = 2;
+constexpr int kAttnCtaFixed = 4;
 
 struct AttnPlan {
   int T = 0, per_tile = 0, ts = 0;
