@@ -85,6 +85,8 @@ def workload_work(w, m):
     return {
         "gate_score": {"bytes": n * dm * es + n * 1 + n * 4 + h * dm * es, "flops": 2 * n * dm * h},
         "topk_select": {"bytes": n * 4 + n * 1 + m * 4},
+        # the fused call: the gate's bytes plus the selector's (scores and mask read back, indices written)
+        "gate_score_select": {"bytes": n * dm * es + n * 1 + n * 4 + h * dm * es + n * 4 + n * 1 + m * 4},
         "unfused_gather": {"bytes": 2 * m * dm * es + m * 4 * 5},
         "gather_rmsnorm": {"bytes": 3 * m * dm * es + m * 4 * 5 + dm * 4},
         "attention": {"flops": 2 * D * hq * m * (m + 1)},
@@ -348,9 +350,12 @@ def run_gpu(args, w):
         if name == "gate_score":
             entry["tflops"] = wk["flops"] / (ms * 1e-3) / 1e12
         kernels[name] = entry
-    kernels["unfused_gather"]["in_step"] = False   # tg_gather alone: the step folds it into the layer's RMSNorm
-    dom = max((k for k in kernels if k not in ("gather_layer_total", "unfused_gather") and kernels[k]["us"] > 0),
-              key=lambda k: kernels[k]["us"])
+    # calls timed alone that the step runs fused: tg_gather (folded into the
+    # layer's first RMSNorm), tg_gate_score and tg_topk_select (tg_gate_score_select)
+    for k in ("unfused_gather", "gate_score", "topk_select"):
+        kernels[k]["in_step"] = False
+    not_dom = ("gather_layer_total", "unfused_gather", "gate_score", "topk_select")
+    dom = max((k for k in kernels if k not in not_dom and kernels[k]["us"] > 0), key=lambda k: kernels[k]["us"])
     wk = work[dom]
     traffic = measured_traffic(dom, w.n if dom == "gate_score" else m)
     if "flops" in wk and dom != "gate_score":
@@ -365,7 +370,8 @@ def run_gpu(args, w):
     # ---- end to end through the public API: pinned host inputs in, result back to the host
     e2e = end_to_end(step, w, args, stream, flush, dist, dev, world)
 
-    # gate, select, gather + RMSNorm, then qkv, q/k-norm + RoPE, attention, o, RMSNorm, gate/up + SwiGLU, down
+    # gate (with the selector's first-digit histogram), select, gather + RMSNorm,
+    # then qkv, q/k-norm + RoPE, attention, o, RMSNorm, gate/up + SwiGLU, down
     launches_per_step = 10
     if rank != 0:
         if dist is not None:
@@ -424,6 +430,7 @@ def breakdown(step, w, args, stream, flush):
     aws = torch.empty(max(aws_n, 16), dtype=torch.uint8, device=stream.device) if aws_n else None
     hk_buf = torch.empty_like(step.hidden_kept)
     calls = {
+        "gate_score_select": step.gate_select,
         "gate_score": step.gate_score,
         "topk_select": step.select,
         "gather_rmsnorm": lambda: tg.tg_gather_rmsnorm(step.hidden, step.kept, step.scores, step.sumsq,
@@ -1001,12 +1008,16 @@ def single_layer_step(w, dev, stream, flush, reps, peaks):
     work = workload_work(w, step.m)
     att_tf = work["attention"]["flops"] / (br["attention"] * 1e-3) / 1e12
     gate_gbs = work["gate_score"]["bytes"] / (br["gate_score"] * 1e-3) / 1e9
+    gs_gbs = work["gate_score_select"]["bytes"] / (br["gate_score_select"] * 1e-3) / 1e9
     res = {"workload": w.name, "n": w.n, "k": w.k, "kept_rows": step.m, "step_ms": round(ms, 4),
            "tokens_per_s": w.n / (ms * 1e-3), "peak_hbm_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 3),
            "attention": {"us": round(br["attention"] * 1e3, 2), "tflops": round(att_tf, 1),
                          "frac_bf16_peak": round(att_tf / peaks["bf16_tflops"], 4)},
            "gate_score": {"us": round(br["gate_score"] * 1e3, 2), "gbs": round(gate_gbs, 1),
                           "frac_hbm": round(gate_gbs / peaks["hbm_gbs"], 4)},
+           "gate_score_select": {"us": round(br["gate_score_select"] * 1e3, 2), "gbs": round(gs_gbs, 1),
+                                 "frac_hbm": round(gs_gbs / peaks["hbm_gbs"], 4)},
+           "topk_select": {"us": round(br["topk_select"] * 1e3, 2)},
            "reps": reps}
     del step
     torch.cuda.empty_cache()

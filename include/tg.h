@@ -143,6 +143,28 @@ int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int6
                    int64_t k, int32_t* kept_idx, int64_t m, void* stream);
 
 /*
+ * tg_gate_score followed by tg_topk_select, with the selection's first radix
+ * pass folded into the scoring kernel ([R] §4.1 "Gate module" and "Top-K
+ * selector"): when the tensor cores score and the prompt is long enough for
+ * the cluster selector (n > 4096), the scoring kernel's epilogue also counts
+ * the order-preserving keys of the prunable scores by their top 11 bits, and
+ * the selector reads its first digit off that histogram and resolves the
+ * remaining 21 bits in two passes (11 and 10 bits) instead of four of 8.
+ * The outputs equal tg_gate_score then tg_topk_select on the same stream:
+ * scores, sumsq and the kept indices (bit-exact, ascending).
+ *   arguments        as tg_gate_score and tg_topk_select (m = min(k,
+ *                    n_prunable) + n - n_prunable)
+ *   ws               device workspace of tg_workspace_bytes(TG_OP_GATE_SELECT,
+ *                    n, 0, d_model, h, NULL) bytes, 16-byte aligned
+ */
+int tg_gate_score_select(const void* hidden, int dtype, int64_t n, int32_t d_model,
+                         const float* norm_w, float norm_eps,
+                         const void* w1, const float* b1, const float* w2, float b2, int32_t h,
+                         const uint8_t* prunable, int64_t n_prunable, int64_t k,
+                         float* scores, float* sumsq, int32_t* kept_idx, int64_t m,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Compaction of the kept rows ([R] §4.1 three-stage forward: pruned tokens
  * never enter the layers above L) plus the per-row inputs of gated attention:
  *     hidden_kept[r] = hidden[kept_idx[r]]            (bit-exact copy)
@@ -413,9 +435,10 @@ enum { TG_EPI_STORE = 0, TG_EPI_RESIDUAL = 1, TG_EPI_SWIGLU = 2 };
 int tg_linear(const void* x, int64_t ldx, const void* w, void* y, int64_t ldy, int dtype,
               int64_t m, int32_t n_out, int32_t k_in, int epilogue, void* stream);
 
-enum { TG_OP_GATE_SCORE = 0, TG_OP_LAYER = 1, TG_OP_ATTENTION = 2, TG_OP_DECODE = 3, TG_OP_ATTENTION_BWD = 4 };
+enum { TG_OP_GATE_SCORE = 0, TG_OP_LAYER = 1, TG_OP_ATTENTION = 2, TG_OP_DECODE = 3, TG_OP_ATTENTION_BWD = 4,
+       TG_OP_GATE_SELECT = 5 };
 
-/* Workspace bytes needed by an op: TG_OP_GATE_SCORE uses n, d_model and h;
+/* Workspace bytes needed by an op: TG_OP_GATE_SCORE and TG_OP_GATE_SELECT use n, d_model and h;
  * TG_OP_LAYER and TG_OP_ATTENTION use m and shape (TG_OP_ATTENTION reads its
  * dtype, hq, hkv and head_dim); TG_OP_DECODE uses m = the cache length and
  * shape's hq, hkv and head_dim; TG_OP_ATTENTION_BWD uses m and shape's hq, hkv and head_dim.  Returns 0 for an invalid request, and 0 for

@@ -455,6 +455,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool a_mn_ma
 // ---------------------------------------------------------------------------
 // Small numeric helpers
 // ---------------------------------------------------------------------------
+// Order-preserving integer key of an fp32 score for the top-K selection:
+// larger score = larger key, -0 and +0 map to the same key, NaN below -inf.
+__device__ __forceinline__ uint32_t order_key(float s) {
+  uint32_t b = __float_as_uint(s);
+  if ((b & 0x7fffffffu) > 0x7f800000u) return 0u;  // NaN: lowest key
+  if (b == 0x80000000u) b = 0u;                     // -0 ranks with +0
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 

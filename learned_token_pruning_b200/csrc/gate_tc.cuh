@@ -47,7 +47,10 @@ struct GateParams {
   float* partials;    // [gridDim.x]
   uint32_t* counter;  // zero on entry
   float* sumsq;
+  uint32_t* key_hist; // [2048] or null: counts of order_key(s) >> 21 over prunable tokens, zero on entry
 };
+
+constexpr int kGateHistBins = 2048;
 
 template <int BN>
 struct GateCfg {
@@ -56,7 +59,8 @@ struct GateCfg {
   static constexpr int kBBox = BN < 128 ? BN : 128;  // rows per W1 TMA box
   static constexpr int kAccCols = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
   static constexpr int kTmemCols = 2 * kAccCols;   // two accumulators
-  static constexpr size_t kSmem = 1024 + kGateStages * (kABytes + kBBytes) + 256 + 2 * BN * 4 + 2 * 2 * 128 * 4 + 64;
+  static constexpr size_t kSmem =
+      1024 + kGateStages * (kABytes + kBBytes) + 256 + 2 * BN * 4 + 2 * 2 * 128 * 4 + 64 + kGateHistBins * 4;
 };
 
 template <int BN>
@@ -82,6 +86,7 @@ __global__ void __launch_bounds__(kGateThreads, 1)
   float* s_ss = s_w2 + BN;        // [2][128] row sums of h^2 per tile parity
   float* s_half = s_ss + 2 * 128; // [2][128] second-half partial dot products
   float* s_red = s_half + 2 * 128;  // 4 warp partials + broadcast slot
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(s_red + 16);  // [kGateHistBins] this CTA's key histogram
 
   __shared__ int s_stop[2];  // [tile parity] an epilogue warp saw its wait fail
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -233,6 +238,8 @@ __global__ void __launch_bounds__(kGateThreads, 1)
       s_b1[c] = (c < p.N && p.b1) ? p.b1[c] : 0.0f;
       s_w2[c] = c < p.N ? p.w2[c] : 0.0f;
     }
+    if (p.key_hist)
+      for (int c = et; c < kGateHistBins; c += 256) s_hist[c] = 0u;
     asm volatile("bar.sync 1, 256;" ::: "memory");
     float cta_sq = 0.0f;  // this CTA's sum of s^2, tile by tile in order (thread 0 of the group)
     bool stopped = false;
@@ -274,9 +281,18 @@ __global__ void __launch_bounds__(kGateThreads, 1)
       asm volatile("bar.sync 1, 256;" ::: "memory");
       if (half == 0) {
         float s = 0.0f;
+        bool pr = false;
         if (grow < p.M) {
-          s = p.prunable[grow] ? (acc + s_half[b * 128 + row]) + p.b2 : 0.0f;
+          pr = p.prunable[grow] != 0;
+          s = pr ? (acc + s_half[b * 128 + row]) + p.b2 : 0.0f;
           p.scores[grow] = s;
+        }
+        if (p.key_hist) {
+          // the selector's first radix digit (key bits 31..21) over prunable
+          // tokens; lanes holding the same digit add once
+          const uint32_t bin = pr ? (order_key(s) >> 21) : 0xffffffffu;
+          const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+          if (pr && lane == __ffs(peers) - 1) atomicAdd(&s_hist[bin], static_cast<uint32_t>(__popc(peers)));
         }
         // fixed-order reduction of s^2 over this tile's rows, added to the
         // CTA's running sum in tile order
@@ -288,6 +304,12 @@ __global__ void __launch_bounds__(kGateThreads, 1)
         if (row == 0) cta_sq += (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);
         asm volatile("bar.sync 2, 128;" ::: "memory");
       }
+    }
+    if (p.key_hist && !stopped) {
+      // this CTA's histogram into the global one (integer adds: the order does not matter)
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      for (int c = et; c < kGateHistBins; c += 256)
+        if (s_hist[c]) atomicAdd(&p.key_hist[c], s_hist[c]);
     }
     if (half == 0 && !stopped) {
       if (row == 0) {

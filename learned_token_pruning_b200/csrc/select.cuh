@@ -7,15 +7,23 @@
 // integer keys that order fp32 scores totally:
 //   -0 and +0 map to the same key, NaN maps below -inf, larger score = larger key.
 //
-// One launch, one thread-block cluster of up to kSelCluster CTAs (the host
-// picks the smallest cluster whose slices fit the per-CTA key cache, so short
-// prompts run in a single CTA with no cluster-wide barrier).  Each CTA owns a
-// contiguous slice of the tokens and, when it fits, keeps its keys in shared
-// memory for every pass.  Four 8-bit radix passes find the threshold key T and
-// how many ties at T must be kept; the per-pass histograms are merged through
-// distributed shared memory.  A last ordered pass writes the kept indices in
-// ascending order, breaking ties at T towards the lower index, using one
-// exclusive block scan per chunk and cluster-wide prefix counts.
+// Longer prompts take one thread-block cluster of up to kSelCluster CTAs, each
+// owning a contiguous slice of the tokens with its keys cached in shared
+// memory.  The threshold key T (the kp-th largest prunable key) is found in
+// two steps:
+//   1. its top 11 bits d1, from a histogram of (key >> 21) over the prunable
+//      tokens: the gate-score kernel's, or one the CTAs build and merge
+//      through distributed shared memory;
+//   2. its low 21 bits, among the candidates (the keys whose top 11 bits are
+//      d1, usually a few percent of the tokens): every CTA gathers all
+//      candidates into its own shared memory and finds the bits with three
+//      7-bit radix passes that need only block-level barriers.
+// Should the candidates not fit, the low bits take three cluster-wide radix
+// passes instead.  Each CTA then counts its tokens kept outright (key > T, or
+// non-prunable) and its ties at T, pushes both counts into every CTA's shared
+// memory, and after one cluster barrier writes its kept indices in ascending
+// order (ties at T towards the lower index), thread t owning the consecutive
+// tokens [t*kpt, (t+1)*kpt) of the slice so that one block scan places them.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -29,14 +37,13 @@ namespace cg = cooperative_groups;
 constexpr int kSelCluster = 16;  // 16 needs the non-portable cluster size (the host falls back to 8)
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr size_t kSelCacheBytes = 200 * 1024;  // dynamic smem for the key cache
-
-__device__ __forceinline__ uint32_t order_key(float s) {
-  uint32_t b = __float_as_uint(s);
-  if ((b & 0x7fffffffu) > 0x7f800000u) return 0u;  // NaN: lowest key
-  if (b == 0x80000000u) b = 0u;                     // -0 ranks with +0
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
+constexpr int kSelStride = kSelThreads + 1;  // words per row of the key cache [kpt][kSelStride]
+constexpr int kSelMaxKpt = 32;               // cached slices hold up to kSelMaxKpt tokens per thread
+constexpr int kSelOwnCap = 8192;             // candidate keys one CTA can publish
+constexpr int kSelAllCap = 16384;            // candidate keys one CTA can gather
+constexpr size_t kSelCandBytes = static_cast<size_t>(kSelOwnCap + kSelAllCap) * 4;
+constexpr int kSelTopBits = 11;              // first digit: key bits 31..21
+constexpr int kSelLowBits = 7;               // the other 21 bits: three digits of 7
 
 struct SelectParams {
   const float* scores;
@@ -47,8 +54,15 @@ struct SelectParams {
   int32_t* out;
   int64_t m;
   int64_t slice;  // tokens per CTA
-  int cached;     // 1 if each slice's keys fit the shared-memory cache
+  int kpt;        // tokens per thread: a power of two with kpt * kSelThreads >= slice
+  int cached;     // 1 if the slice's keys and flags are kept in shared memory (kpt <= kSelMaxKpt)
+  const uint32_t* hist_top;  // [2048] counts of (key >> 21) over prunable tokens, or null
 };
+
+// dynamic shared memory of k_topk_select
+__host__ __device__ constexpr size_t select_smem_bytes(int kpt, int cached) {
+  return kSelCandBytes + (cached ? ((static_cast<size_t>(kpt) * kSelStride * 5 + 15) / 16) * 16 : 0);
+}
 
 // Exclusive scan over the block of one 32-bit value per thread; returns the
 // exclusive prefix and writes the block total to *total.
@@ -80,168 +94,361 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   return r;
 }
 
+// One warp over 128 bins, lane l holding the counts of bins 127-4l .. 124-4l
+// (highest first) in v[0..3]: the bin holding the rem-th largest key and the
+// count of keys in the bins above it go to s_pick[0], s_pick[1].  Lane 0 sets
+// s_pick to (0, 0) first, so counts that cannot hold rem leave an in-range digit.
+__device__ __forceinline__ void warp_pick_low_digit(const uint32_t v[4], uint32_t rem, uint32_t* s_pick) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) {
+    s_pick[0] = 0;
+    s_pick[1] = 0;
+  }
+  __syncwarp();
+  const uint32_t c = v[0] + v[1] + v[2] + v[3];
+  uint32_t incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const uint32_t above = incl - c;
+  if (above < rem && rem <= incl) {
+    uint32_t a = above;
+    int u = 0;
+    for (; u < 3 && a + v[u] < rem; ++u) a += v[u];
+    s_pick[0] = static_cast<uint32_t>(127 - 4 * lane - u);
+    s_pick[1] = a;
+  }
+}
+
 __global__ void __launch_bounds__(kSelThreads, 1) k_topk_select(SelectParams p) {
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ __align__(16) uint8_t sel_smem[];
-  __shared__ uint32_t hist[256];
+  __shared__ __align__(16) uint32_t hist[1 << kSelTopBits];  // this CTA's first-digit counts
+  __shared__ uint32_t lhist[1 << kSelLowBits];
   __shared__ uint32_t warp_sums[kSelWarps + 1];
-  __shared__ uint32_t info[4];      // this CTA's: prunable count, non-prunable count, gt count, eq count
-  __shared__ uint32_t s_pick[2];    // chosen digit, keys above the chosen digit (cluster-wide)
+  __shared__ uint32_t info_a[kSelCluster][2];  // written by rank r into every rank: its prunable count, its candidates
+  __shared__ uint32_t info_b[kSelCluster][2];  // written by rank r into every rank: tokens it keeps outright, its ties at T
+  __shared__ uint32_t s_pick[2];
+  __shared__ uint32_t s_ncand;
+  __shared__ uint32_t s_off[kSelCluster];
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
   const int nranks = static_cast<int>(cluster.num_blocks());
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t lo = static_cast<int64_t>(rank) * p.slice;
   const int64_t hi = min(p.n, lo + p.slice);
   const int64_t len = hi > lo ? hi - lo : 0;
+  const int kpt = p.kpt;
+  const int kshift = __ffs(kpt) - 1;
+  const bool top = p.hist_top != nullptr;
 
-  uint32_t* keys = reinterpret_cast<uint32_t*>(sel_smem);
-  uint8_t* flags = sel_smem + (p.cached ? p.slice * 4 : 0);
+  uint32_t* own_cand = reinterpret_cast<uint32_t*>(sel_smem);  // [kSelOwnCap] read by every rank
+  uint32_t* all_cand = own_cand + kSelOwnCap;                   // [kSelAllCap]
+  uint32_t* keys = all_cand + kSelAllCap;                       // [kpt][kSelStride]: token t*kpt + j at j*kSelStride + t
+  uint8_t* flags = reinterpret_cast<uint8_t*>(keys + static_cast<size_t>(kpt) * kSelStride);
 
-  auto load_key = [&](int64_t i, uint32_t& key, bool& f) {
+  // token i = tid*kpt + j of the slice (the caller checks i < len)
+  auto load_own = [&](int j, uint32_t& key, bool& f) {
     if (p.cached) {
-      key = keys[i];
-      f = flags[i] != 0;
+      const int s = j * kSelStride + tid;
+      key = keys[s];
+      f = flags[s] != 0;
     } else {
-      const int64_t j = lo + i;
-      f = p.prunable[j] != 0;
-      key = f ? order_key(p.scores[j]) : 0u;
+      const int64_t g = lo + static_cast<int64_t>(tid) * kpt + j;
+      f = p.prunable[g] != 0;
+      key = f ? order_key(p.scores[g]) : 0u;
     }
   };
 
-  // ---- pass 0: keys, flags and the prunable count of this slice
-  uint32_t cnt = 0;
-  for (int64_t i = tid; i < len; i += kSelThreads) {
-    const int64_t j = lo + i;
-    const bool f = p.prunable[j] != 0;
-    const uint32_t key = f ? order_key(p.scores[j]) : 0u;
-    if (p.cached) {
-      keys[i] = key;
-      flags[i] = f ? 1 : 0;
-    }
-    cnt += f ? 1u : 0u;
-  }
-  uint32_t tot;
-  block_exclusive_scan(cnt, warp_sums, &tot);
   if (tid == 0) {
-    info[0] = tot;
-    info[1] = static_cast<uint32_t>(len) - tot;
+    s_ncand = 0;
+    s_pick[0] = 0;
+    s_pick[1] = 0;
   }
-  cluster.sync();
+  // the first-digit counts, four bins a thread with the highest first: thread
+  // t holds bins 2047-4t .. 2044-4t
+  uint32_t hv[4] = {0u, 0u, 0u, 0u};
+  if (top) {
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(p.hist_top) + (kSelThreads - 1 - tid));
+    hv[0] = q.w;
+    hv[1] = q.z;
+    hv[2] = q.y;
+    hv[3] = q.x;
+  } else {
+    for (int b = tid; b < (1 << kSelTopBits); b += kSelThreads) hist[b] = 0;
+  }
+  __syncthreads();
 
-  int64_t np_total = 0;
-  for (int r = 0; r < nranks; ++r) np_total += *cluster.map_shared_rank(&info[0], r);
-  if (tid == 0 && rank == 0 && np_total != p.n_prunable) raise_error(kErrMaskCount, 1);
-
-  const int64_t kp = min(p.k, np_total);
-  // mode 0: keep no prunable token; 1: keep all of them; 2: threshold select
-  const int mode = kp <= 0 ? 0 : (kp >= np_total ? 1 : 2);
-
-  uint32_t thr = 0, need_eq = 0, local_gt = 0, local_eq = 0;
-  if (mode == 2) {
-    uint32_t prefix = 0, pmask = 0;
-    uint32_t remaining = static_cast<uint32_t>(kp);
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      if (tid < 256) hist[tid] = 0;
-      __syncthreads();
-      // warp-aggregated histogram: lanes holding the same digit add once
-      // (early digits of real scores crowd into a few bins)
-      for (int64_t base = 0; base < len; base += kSelThreads) {
-        const int64_t i = base + tid;
-        uint32_t key = 0;
-        bool f = false;
-        if (i < len) load_key(i, key, f);
-        const bool valid = f && (key & pmask) == prefix;
-        const uint32_t bin = valid ? ((key >> shift) & 255u) : 0xffffffffu;
+  // ---- load the slice (coalesced, four rounds of loads in flight): keys and
+  // flags into the cache, the prunable count and, without the gate's
+  // histogram, this CTA's first-digit counts
+  uint32_t cnt = 0;
+  for (int64_t base = 0; base < len; base += 4 * kSelThreads) {
+    float sc[4];
+    uint8_t pf[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = base + u * kSelThreads + tid;
+      sc[u] = i < len ? __ldg(p.scores + lo + i) : 0.0f;
+      pf[u] = i < len ? __ldg(p.prunable + lo + i) : uint8_t(0);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = base + u * kSelThreads + tid;
+      const bool f = pf[u] != 0;
+      const uint32_t key = f ? order_key(sc[u]) : 0u;
+      if (p.cached && i < len) {
+        const int s = static_cast<int>(i & (kpt - 1)) * kSelStride + static_cast<int>(i >> kshift);
+        keys[s] = key;
+        flags[s] = f ? 1 : 0;
+      }
+      cnt += f ? 1u : 0u;
+      if (!top) {
+        // lanes holding the same digit add once (scores crowd into a few bins)
+        const uint32_t bin = f ? (key >> (32 - kSelTopBits)) : 0xffffffffu;
         const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-        if (valid && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+        if (f && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
       }
-      cluster.sync();
-      // merged histogram, scanned from the top bin down
-      uint32_t tot_b = 0, own_b = 0;
-      if (tid < 256) {
-        const int b = 255 - tid;  // thread 0 holds the top bin
-        own_b = hist[b];
-        for (int r = 0; r < nranks; ++r) tot_b += cluster.map_shared_rank(hist, r)[b];
+    }
+  }
+  uint32_t np_cta;
+  block_exclusive_scan(cnt, warp_sums, &np_cta);
+
+  if (!top) {
+    cluster.sync();  // every CTA's first-digit counts are complete
+    uint4 q[kSelCluster];
+#pragma unroll
+    for (int r = 0; r < kSelCluster; ++r)
+      if (r < nranks) q[r] = reinterpret_cast<const uint4*>(cluster.map_shared_rank(hist, r))[kSelThreads - 1 - tid];
+#pragma unroll
+    for (int r = 0; r < kSelCluster; ++r)
+      if (r < nranks) {
+        hv[0] += q[r].w;
+        hv[1] += q[r].z;
+        hv[2] += q[r].y;
+        hv[3] += q[r].x;
       }
-      uint32_t total_all;
-      const uint32_t above = block_exclusive_scan(tid < 256 ? tot_b : 0u, warp_sums, &total_all);
-      if (tid < 256 && above < remaining && remaining <= above + tot_b) {
-        s_pick[0] = 255u - tid;
-        s_pick[1] = above;
+  }
+
+  // ---- the first digit: kp = min(k, prunable tokens), the counts summing to the latter
+  const uint32_t c4 = hv[0] + hv[1] + hv[2] + hv[3];
+  uint32_t np_total;
+  const uint32_t above4 = block_exclusive_scan(c4, warp_sums, &np_total);
+  const uint32_t kp = static_cast<uint32_t>(min(p.k, static_cast<int64_t>(np_total)));
+  // mode 0: keep no prunable token; 1: keep all of them; 2: threshold select
+  const int mode = kp == 0 ? 0 : (kp >= np_total ? 1 : 2);
+  if (mode == 2 && above4 < kp && kp <= above4 + c4) {
+    uint32_t a = above4;
+    int u = 0;
+    for (; u < 3 && a + hv[u] < kp; ++u) a += hv[u];
+    s_pick[0] = static_cast<uint32_t>((1 << kSelTopBits) - 1 - 4 * tid - u);
+    s_pick[1] = a;
+  }
+  __syncthreads();
+  const uint32_t d1 = s_pick[0];
+  uint32_t rem = mode == 2 ? kp - s_pick[1] : 0u;  // rank of T among the keys whose first digit is d1
+
+  // ---- this CTA's candidates
+  if (mode == 2) {
+    for (int j = 0; j < kpt; ++j) {
+      bool c = false;
+      uint32_t key = 0;
+      if (static_cast<int64_t>(tid) * kpt + j < len) {
+        bool f;
+        load_own(j, key, f);
+        c = f && (key >> (32 - kSelTopBits)) == d1;
+      }
+      const uint32_t bal = __ballot_sync(0xffffffffu, c);
+      if (bal) {
+        const int leader = __ffs(bal) - 1;
+        uint32_t b0 = 0;
+        if (lane == leader) b0 = atomicAdd(&s_ncand, static_cast<uint32_t>(__popc(bal)));
+        b0 = __shfl_sync(0xffffffffu, b0, leader);
+        const uint32_t pos = b0 + static_cast<uint32_t>(__popc(bal & ((1u << lane) - 1u)));
+        if (c && pos < static_cast<uint32_t>(kSelOwnCap)) own_cand[pos] = key;
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < nranks) {
+    uint32_t* dst = cluster.map_shared_rank(&info_a[0][0], tid);
+    dst[rank * 2 + 0] = np_cta;
+    dst[rank * 2 + 1] = s_ncand;
+  }
+  cluster.sync();  // (A) counts and candidates published; the first-digit counts read
+
+  uint32_t np_sum = 0, ncand = 0;
+  bool over = false;
+  for (int r = 0; r < nranks; ++r) {
+    if (tid == 0) s_off[r] = ncand;  // where rank r's candidates start in the gathered list
+    np_sum += info_a[r][0];
+    over = over || info_a[r][1] > static_cast<uint32_t>(kSelOwnCap);
+    ncand += info_a[r][1];
+  }
+  over = over || ncand > static_cast<uint32_t>(kSelAllCap);
+  if (tid == 0 && rank == 0 && (static_cast<int64_t>(np_sum) != p.n_prunable || np_sum != np_total))
+    raise_error(kErrMaskCount, 1);
+
+  // ---- the low 21 bits of T
+  uint32_t thr = 0, need_eq = 0;
+  if (mode == 2) {
+    uint32_t prefix = d1 << (32 - kSelTopBits), pmask = ((1u << kSelTopBits) - 1u) << (32 - kSelTopBits);
+    if (!over) {
+      // gather every rank's candidates (four remote loads in flight a thread)
+      // and count their next digit
+      if (tid < (1 << kSelLowBits)) lhist[tid] = 0;
+      __syncthreads();  // lhist zeroed, s_off written
+      for (uint32_t base = 0; base < ncand; base += 4 * kSelThreads) {
+        uint32_t v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t idx = base + u * kSelThreads + tid;
+          v[u] = 0;
+          if (idx < ncand) {
+            int r = 0;
+            for (int t = 1; t < nranks; ++t)
+              if (s_off[t] <= idx) r = t;
+            v[u] = cluster.map_shared_rank(own_cand, r)[idx - s_off[r]];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t idx = base + u * kSelThreads + tid;
+          if (idx < ncand) {
+            all_cand[idx] = v[u];
+            atomicAdd(&lhist[(v[u] >> 14) & 127u], 1u);
+          }
+        }
       }
       __syncthreads();
-      const uint32_t digit = s_pick[0];
-      // keys of this slice strictly above the chosen digit (under the current prefix)
-      uint32_t mine = (tid < 256 && (255u - tid) > digit) ? own_b : 0u;
-      uint32_t gt_pass;
-      block_exclusive_scan(mine, warp_sums, &gt_pass);
-      local_gt += gt_pass;
-      if (pass == 3) local_eq = hist[digit];
-      remaining -= s_pick[1];
-      prefix |= digit << shift;
-      pmask |= 0xffu << shift;
-      cluster.sync();  // every CTA has read the remote histograms
+      for (int pass = 0; pass < 3; ++pass) {
+        const int shift = 14 - kSelLowBits * pass;
+        if (pass > 0) {
+          if (tid < (1 << kSelLowBits)) lhist[tid] = 0;
+          __syncthreads();
+          for (uint32_t idx = tid; idx < ncand; idx += kSelThreads) {
+            const uint32_t v = all_cand[idx];
+            if ((v & pmask) == prefix) atomicAdd(&lhist[(v >> shift) & 127u], 1u);
+          }
+          __syncthreads();
+        }
+        if (warp == 0) {
+          uint32_t v[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) v[u] = lhist[127 - 4 * lane - u];
+          warp_pick_low_digit(v, rem, s_pick);
+        }
+        __syncthreads();
+        rem -= s_pick[1];
+        prefix |= s_pick[0] << shift;
+        pmask |= 127u << shift;
+        __syncthreads();  // s_pick read before the next pass rewrites it
+      }
+    } else {
+      // too many candidates: the low bits by cluster-wide passes over the
+      // cached keys, the counts merged through distributed shared memory
+      for (int pass = 0; pass < 3; ++pass) {
+        const int shift = 14 - kSelLowBits * pass;
+        if (tid < (1 << kSelLowBits)) hist[tid] = 0;
+        __syncthreads();
+        for (int j = 0; j < kpt; ++j) {
+          if (static_cast<int64_t>(tid) * kpt + j < len) {
+            uint32_t key;
+            bool f;
+            load_own(j, key, f);
+            if (f && (key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 127u], 1u);
+          }
+        }
+        cluster.sync();
+        if (warp == 0) {
+          uint32_t v[4] = {0u, 0u, 0u, 0u};
+          for (int r = 0; r < nranks; ++r) {
+            const uint32_t* rh = cluster.map_shared_rank(hist, r);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] += rh[127 - 4 * lane - u];
+          }
+          warp_pick_low_digit(v, rem, s_pick);
+        }
+        __syncthreads();
+        rem -= s_pick[1];
+        prefix |= s_pick[0] << shift;
+        pmask |= 127u << shift;
+        cluster.sync();  // every rank has read the remote counts (and s_pick)
+      }
     }
     thr = prefix;
-    need_eq = remaining;
+    need_eq = rem;  // ties at T to keep
   }
 
-  if (tid == 0) {
-    info[2] = mode == 1 ? info[0] : local_gt;
-    info[3] = local_eq;
-  }
-  cluster.sync();
-
-  // cluster-wide prefixes for this CTA
-  uint32_t eq_before = 0, kept_before = 0;
-  {
-    uint32_t eq_acc = 0;
-    for (int r = 0; r < nranks; ++r) {
-      const uint32_t* ri = cluster.map_shared_rank(info, r);
-      const uint32_t np_r = ri[1], gt_r = ri[2], eq_r = ri[3];
-      const uint32_t tie_keep = eq_acc >= need_eq ? 0u : min(eq_r, need_eq - eq_acc);
-      if (r < rank) {
-        kept_before += np_r + (mode == 0 ? 0u : gt_r) + tie_keep;
-        eq_before += eq_r;
-      }
-      eq_acc += eq_r;
+  // ---- this thread's tokens kept outright and its ties at T
+  auto classify = [&](int j, bool& ngt, bool& eq) {
+    uint32_t key;
+    bool f;
+    load_own(j, key, f);
+    ngt = !f || mode == 1 || (mode == 2 && key > thr);
+    eq = f && mode == 2 && key == thr;
+  };
+  uint32_t n_gt = 0, n_eq = 0;
+  for (int j = 0; j < kpt; ++j) {
+    if (static_cast<int64_t>(tid) * kpt + j < len) {
+      bool ngt, eq;
+      classify(j, ngt, eq);
+      n_gt += ngt ? 1u : 0u;
+      n_eq += eq ? 1u : 0u;
     }
   }
-  cluster.sync();  // remote reads done before any CTA may exit
+  uint32_t gt_ex, eq_ex, gt_cta, eq_cta;
+  if (kpt * kSelThreads < 65536) {
+    uint32_t tot;
+    const uint32_t ex = block_exclusive_scan(n_eq | (n_gt << 16), warp_sums, &tot);
+    gt_ex = ex >> 16;
+    eq_ex = ex & 0xffffu;
+    gt_cta = tot >> 16;
+    eq_cta = tot & 0xffffu;
+  } else {
+    gt_ex = block_exclusive_scan(n_gt, warp_sums, &gt_cta);
+    eq_ex = block_exclusive_scan(n_eq, warp_sums, &eq_cta);
+  }
+  if (tid < nranks) {
+    uint32_t* dst = cluster.map_shared_rank(&info_b[0][0], tid);
+    dst[rank * 2 + 0] = gt_cta;
+    dst[rank * 2 + 1] = eq_cta;
+  }
+  cluster.sync();  // (B) the counts are in; no remote access after this
 
-  // ---- ordered compaction pass
-  uint32_t e0 = eq_before;  // ties at T preceding this chunk (cluster-wide)
-  uint32_t kept_run = kept_before;
-  for (int64_t base = 0; base < len; base += kSelThreads) {
-    const int64_t i = base + tid;
-    bool ngt = false, eq = false;
+  // cluster-wide prefixes: tokens kept by lower ranks, ties at T in lower ranks
+  uint32_t kept_before = 0, eq_before = 0, eq_acc = 0;
+  for (int r = 0; r < nranks; ++r) {
+    const uint32_t gt_r = info_b[r][0], eq_r = info_b[r][1];
+    if (r < rank) {
+      kept_before += gt_r + (min(eq_acc + eq_r, need_eq) - min(eq_acc, need_eq));
+      eq_before += eq_r;
+    }
+    eq_acc += eq_r;
+  }
+
+  // ---- ordered compaction: this thread's kept tokens in index order
+  uint32_t e0 = eq_before + eq_ex;  // ties at T before this thread's tokens (cluster-wide)
+  uint32_t pos = kept_before + gt_ex + (min(e0, need_eq) - min(eq_before, need_eq));
+  for (int j = 0; j < kpt; ++j) {
+    const int64_t i = static_cast<int64_t>(tid) * kpt + j;
     if (i < len) {
-      uint32_t key;
-      bool f;
-      load_key(i, key, f);
-      ngt = !f || mode == 1 || (mode == 2 && key > thr);
-      eq = f && mode == 2 && key == thr;
-    }
-    uint32_t chunk_tot;
-    const uint32_t ex = block_exclusive_scan((eq ? 1u : 0u) | ((ngt ? 1u : 0u) << 16), warp_sums, &chunk_tot);
-    const uint32_t eq_ex = ex & 0xffffu, ngt_ex = ex >> 16;
-    const uint32_t g_eq = e0 + eq_ex;
-    const bool keep = ngt || (eq && g_eq < need_eq);
-    if (keep) {
-      const uint32_t pos = kept_run + ngt_ex + (min(g_eq, need_eq) - min(e0, need_eq));
-      if (pos < p.m) {
-        p.out[pos] = static_cast<int32_t>(lo + i);
-      } else {
-        raise_error(kErrSelectOverflow, 1);
+      bool ngt, eq;
+      classify(j, ngt, eq);
+      if (ngt || (eq && e0 < need_eq)) {
+        if (pos < p.m) {
+          p.out[pos] = static_cast<int32_t>(lo + i);
+        } else {
+          raise_error(kErrSelectOverflow, 1);
+        }
+        ++pos;
       }
+      if (eq) ++e0;
     }
-    const uint32_t eq_tot = chunk_tot & 0xffffu, ngt_tot = chunk_tot >> 16;
-    kept_run += ngt_tot + (min(e0 + eq_tot, need_eq) - min(e0, need_eq));
-    e0 += eq_tot;
   }
 }
 

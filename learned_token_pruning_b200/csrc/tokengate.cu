@@ -334,6 +334,10 @@ size_t gate_partials_bytes(int64_t n) { return ((static_cast<size_t>((n + 127) /
 size_t gate_ws_bytes(int64_t n, int32_t d, int32_t h) {
   return gate_partials_bytes(n) + 256 + ((static_cast<size_t>(d) * h * 2 + 255) / 256) * 256;
 }
+// tg_gate_score_select: the gate's workspace, then the selector's first-digit histogram
+size_t gate_select_ws_bytes(int64_t n, int32_t d, int32_t h) {
+  return gate_ws_bytes(n, d, h) + tg::kGateHistBins * sizeof(uint32_t);
+}
 
 }  // namespace
 
@@ -375,7 +379,7 @@ bool select_cluster16_ok() {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(16);
     cfg.blockDim = dim3(tg::kSelThreads);
-    cfg.dynamicSmemBytes = tg::kSelCacheBytes;
+    cfg.dynamicSmemBytes = tg::select_smem_bytes(tg::kSelMaxKpt, 1);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 16;
@@ -385,7 +389,7 @@ bool select_cluster16_ok() {
     cfg.numAttrs = 1;
     int clusters = 0;
     good = cudaFuncSetAttribute(tg::k_topk_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(tg::kSelCacheBytes)) == cudaSuccess &&
+                                static_cast<int>(tg::select_smem_bytes(tg::kSelMaxKpt, 1))) == cudaSuccess &&
            cudaOccupancyMaxActiveClusters(&clusters, tg::k_topk_select, &cfg) == cudaSuccess && clusters >= 1;
   }
   cudaGetLastError();  // a refused query leaves no sticky error behind
@@ -443,6 +447,12 @@ static int prefill_layer_impl(const tg_layer_weights* W, const tg_layer_shape* S
                               size_t ws_bytes, void* stream);
 static int launch_gather_rmsnorm(const LayerGather& g, int dtype, void* hidden_kept, void* xn, const float* w,
                                  int64_t m, int d, float eps, cudaStream_t st);
+static int gate_score_impl(const void* hidden, int dtype, int64_t n, int32_t d_model, const float* norm_w,
+                           float norm_eps, const void* w1, const float* b1, const float* w2, float b2, int32_t h,
+                           const uint8_t* prunable, float* scores, float* sumsq, void* ws, size_t ws_bytes,
+                           uint32_t* key_hist, void* stream);
+static int topk_select_impl(const float* scores, const uint8_t* prunable, int64_t n, int64_t n_prunable, int64_t k,
+                            int32_t* kept_idx, int64_t m, const uint32_t* hist_top, void* stream);
 
 extern "C" {
 
@@ -631,6 +641,7 @@ DecodePlan decode_plan(int64_t length, int hkv, int group, int head_dim) {
 
 size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t h, const tg_layer_shape* shape) {
   if (op == TG_OP_GATE_SCORE) return (n > 0 && d_model > 0 && h > 0) ? gate_ws_bytes(n, d_model, h) : 0;
+  if (op == TG_OP_GATE_SELECT) return (n > 0 && d_model > 0 && h > 0) ? gate_select_ws_bytes(n, d_model, h) : 0;
   if (op == TG_OP_LAYER) {
     if (!shape || m <= 0 || !dtype_size(shape->dtype)) return 0;
     return layer_buffers_bytes(m, shape) + attn_ws_bytes(m, shape->hq, shape->hkv, shape->head_dim, shape->dtype);
@@ -659,6 +670,20 @@ size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t
 int tg_gate_score(const void* hidden, int dtype, int64_t n, int32_t d_model, const float* norm_w, float norm_eps,
                   const void* w1, const float* b1, const float* w2, float b2, int32_t h, const uint8_t* prunable,
                   float* scores, float* sumsq, void* ws, size_t ws_bytes, void* stream) {
+  return gate_score_impl(hidden, dtype, n, d_model, norm_w, norm_eps, w1, b1, w2, b2, h, prunable, scores, sumsq, ws,
+                         ws_bytes, nullptr, stream);
+}
+
+}  // extern "C"
+
+// tg_gate_score; with key_hist (device [2048], zeroed by the caller on the
+// stream) the tensor-core kernel also counts order_key(s) >> 21 over the
+// prunable tokens (the selector's first digit).  Returns TG_ERR_UNSUPPORTED
+// with key_hist on the CUDA-core path, which does not build it.
+static int gate_score_impl(const void* hidden, int dtype, int64_t n, int32_t d_model, const float* norm_w,
+                           float norm_eps, const void* w1, const float* b1, const float* w2, float b2, int32_t h,
+                           const uint8_t* prunable, float* scores, float* sumsq, void* ws, size_t ws_bytes,
+                           uint32_t* key_hist, void* stream) {
   if (!hidden || !w1 || !w2 || !prunable || !scores || !sumsq) return fail(TG_ERR_INVALID_ARG, "null pointer");
   if (n <= 0 || d_model <= 0 || h <= 0) return fail(TG_ERR_INVALID_ARG, "n, d_model and h must be positive");
   if (n >= (int64_t(1) << 31)) return fail(TG_ERR_UNSUPPORTED, "n must be < 2^31");
@@ -694,11 +719,13 @@ int tg_gate_score(const void* hidden, int dtype, int64_t n, int32_t d_model, con
     p.partials = partials;
     p.counter = counter;
     p.sumsq = sumsq;
+    p.key_hist = key_hist;
     const int nn = static_cast<int>(n);
     if (h <= 64) return launch_gate_tc<64>(hidden, w1_eff, nn, d_model, p, st);
     if (h <= 128) return launch_gate_tc<128>(hidden, w1_eff, nn, d_model, p, st);
     return launch_gate_tc<256>(hidden, w1_eff, nn, d_model, p, st);
   }
+  if (key_hist) return fail(TG_ERR_UNSUPPORTED, "the key histogram comes only from the tensor-core gate kernel");
   if (h > 1024) return fail(TG_ERR_UNSUPPORTED, "h > 1024");
   const unsigned blocks = static_cast<unsigned>((n + 7) / 8);
   if (dtype == TG_F32)
@@ -715,8 +742,19 @@ int tg_gate_score(const void* hidden, int dtype, int64_t n, int32_t d_model, con
   return check_launch("k_sumsq_ordered");
 }
 
+extern "C" {
+
 int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int64_t n_prunable, int64_t k,
                    int32_t* kept_idx, int64_t m, void* stream) {
+  return topk_select_impl(scores, prunable, n, n_prunable, k, kept_idx, m, nullptr, stream);
+}
+
+}  // extern "C"
+
+// tg_topk_select; with hist_top (device [2048] counts of order_key >> 21 over
+// the prunable tokens) the cluster selector starts from that histogram.
+static int topk_select_impl(const float* scores, const uint8_t* prunable, int64_t n, int64_t n_prunable, int64_t k,
+                            int32_t* kept_idx, int64_t m, const uint32_t* hist_top, void* stream) {
   if (!scores || !prunable || (!kept_idx && m > 0)) return fail(TG_ERR_INVALID_ARG, "null pointer");
   if (n <= 0 || n_prunable < 0 || n_prunable > n) return fail(TG_ERR_INVALID_ARG, "bad n / n_prunable");
   if (k < 0) return fail(TG_ERR_INVALID_ARG, "k must be >= 0");
@@ -732,6 +770,7 @@ int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int6
   p.k = k;
   p.out = kept_idx;
   p.m = m;
+  p.hist_top = nullptr;
   if (n <= tg::kSelSmallBest) {
     // short prompt: one CTA, keys resident in shared memory
     const int need = static_cast<int>((n + tg::kSelSmallThreads - 1) / tg::kSelSmallThreads);
@@ -759,17 +798,18 @@ int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int6
                           st, p, vec);
     }
   }
-  // cluster of 2 .. 16 CTAs: about kSelSlice tokens per CTA, and slices that fit the key cache
+  // cluster of 2 .. 16 CTAs of about kSelSlice tokens each, while the cluster can grow
   int csize = 1;
-  while (csize < tg::kSelCluster && ((n + csize - 1) / csize > tg::kSelSlice ||
-                                     static_cast<size_t>((n + csize - 1) / csize) * 5 > tg::kSelCacheBytes))
-    csize *= 2;
+  while (csize < tg::kSelCluster && (n + csize - 1) / csize > tg::kSelSlice) csize *= 2;
   if (csize > 8 && !select_cluster16_ok()) csize = 8;
   p.slice = (n + csize - 1) / csize;
-  const size_t cache = static_cast<size_t>(p.slice) * 5;
-  p.cached = cache <= tg::kSelCacheBytes ? 1 : 0;
-  const size_t smem = p.cached ? ((cache + 15) / 16) * 16 : 0;
-  int rc = set_smem(tg::k_topk_select, smem > 0 ? smem : 16);
+  int kpt = 1;
+  while (static_cast<int64_t>(kpt) * tg::kSelThreads < p.slice) kpt *= 2;
+  p.kpt = kpt;
+  p.cached = kpt <= tg::kSelMaxKpt ? 1 : 0;
+  p.hist_top = hist_top;
+  const size_t smem = tg::select_smem_bytes(kpt, p.cached);
+  int rc = set_smem(tg::k_topk_select, smem);
   if (rc) return rc;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(csize);
@@ -789,6 +829,40 @@ int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int6
   if (e != cudaSuccess) return fail(TG_ERR_CUDA, "k_topk_select launch: %s", cudaGetErrorString(e));
   return check_launch("k_topk_select");
 }
+
+extern "C" {
+
+int tg_gate_score_select(const void* hidden, int dtype, int64_t n, int32_t d_model, const float* norm_w,
+                         float norm_eps, const void* w1, const float* b1, const float* w2, float b2, int32_t h,
+                         const uint8_t* prunable, int64_t n_prunable, int64_t k, float* scores, float* sumsq,
+                         int32_t* kept_idx, int64_t m, void* ws, size_t ws_bytes, void* stream) {
+  if (!scores || !prunable || (!kept_idx && m > 0)) return fail(TG_ERR_INVALID_ARG, "null pointer");
+  if (n <= 0 || n_prunable < 0 || n_prunable > n) return fail(TG_ERR_INVALID_ARG, "bad n / n_prunable");
+  if (k < 0) return fail(TG_ERR_INVALID_ARG, "k must be >= 0");
+  const int64_t want = (k < n_prunable ? k : n_prunable) + (n - n_prunable);
+  if (m != want) return fail(TG_ERR_SHAPE, "m = %lld but min(k, n_prunable) + n - n_prunable = %lld",
+                             static_cast<long long>(m), static_cast<long long>(want));
+  const size_t need = gate_select_ws_bytes(n, d_model, h);
+  if (!ws || ws_bytes < need) return fail(TG_ERR_WORKSPACE, "gate score + select needs %zu workspace bytes", need);
+  if (!aligned16(ws)) return fail(TG_ERR_ALIGN, "workspace must be 16-byte aligned");
+  cudaStream_t st = as_stream(stream);
+  // the selector's first-digit histogram rides with the gate kernel when the
+  // tensor cores score and the cluster selector runs (longer prompts)
+  uint32_t* hist = nullptr;
+  if (n > tg::kSelSmallBest && gate_uses_tc(hidden, dtype, d_model, w1, h)) {
+    hist = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + gate_ws_bytes(n, d_model, h));
+    if (cudaMemsetAsync(hist, 0, tg::kGateHistBins * sizeof(uint32_t), st) != cudaSuccess)
+      return fail(TG_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(cudaGetLastError()));
+  }
+  int rc = gate_score_impl(hidden, dtype, n, d_model, norm_w, norm_eps, w1, b1, w2, b2, h, prunable, scores, sumsq,
+                           ws, ws_bytes, hist, stream);
+  if (rc) return rc;
+  return topk_select_impl(scores, prunable, n, n_prunable, k, kept_idx, m, hist, stream);
+}
+
+}  // extern "C"
+
+extern "C" {
 
 int tg_gather(const void* hidden, int dtype, int64_t n, int32_t d_model, const int32_t* kept_idx, int64_t m,
               const float* scores, const float* sumsq, int64_t n_prunable, float seq_eps, void* hidden_kept,

@@ -46,7 +46,8 @@ class GatedPrefillStep:
         self.b2 = float(gate["b2"])
         self.scores = torch.empty(w.n, dtype=torch.float32, device=dev)
         self.sumsq = torch.empty(1, dtype=torch.float32, device=dev)
-        gws = tg.tg_workspace_bytes(tg.TG_OP_GATE_SCORE, n=w.n, d_model=w.d_model, h=w.gate_hidden)
+        # the fused gate + select workspace also serves tg_gate_score alone
+        gws = tg.tg_workspace_bytes(tg.TG_OP_GATE_SELECT, n=w.n, d_model=w.d_model, h=w.gate_hidden)
         self.ws_gate = torch.empty(max(gws, 16), dtype=torch.uint8, device=dev)
         self.m = min(w.k, self.n_prunable) + (w.n - self.n_prunable)
         self.kept = torch.empty(self.m, dtype=torch.int32, device=dev)
@@ -70,6 +71,13 @@ class GatedPrefillStep:
     def select(self, stream=None):
         tg.tg_topk_select(self.scores, self.prunable, self.n_prunable, self.w.k, self.kept, stream)
 
+    def gate_select(self, stream=None):
+        """Gate scores and the top-K selection, the selection's first radix pass
+        folded into the scoring kernel."""
+        tg.tg_gate_score_select(self.hidden, self.norm_w, self.norm_eps, self.w1, self.b1, self.w2, self.b2,
+                                self.prunable, self.n_prunable, self.w.k, self.scores, self.sumsq, self.kept,
+                                self.ws_gate, stream)
+
     def gather(self, stream=None):
         tg.tg_gather(self.hidden, self.kept, self.scores, self.sumsq, self.n_prunable, self.eps_s, self.hidden_kept,
                      self.pos, self.bias, self.ratio, stream)
@@ -87,8 +95,7 @@ class GatedPrefillStep:
 
     def run(self, stream=None):
         """One whole step; the result is left in self.hidden_kept ([m, d_model])."""
-        self.gate_score(stream)
-        self.select(stream)
+        self.gate_select(stream)
         self.gather_layer(stream)
         return self.hidden_kept
 
@@ -237,7 +244,7 @@ class PrunedPrefillStack:
         self.pos_all = torch.arange(w.n, dtype=torch.int32, device=dev)
         self.scores = torch.empty(w.n, dtype=torch.float32, device=dev)
         self.sumsq = torch.empty(1, dtype=torch.float32, device=dev)
-        self.ws_gate = torch.empty(max(tg.tg_workspace_bytes(tg.TG_OP_GATE_SCORE, n=w.n, d_model=w.d_model,
+        self.ws_gate = torch.empty(max(tg.tg_workspace_bytes(tg.TG_OP_GATE_SELECT, n=w.n, d_model=w.d_model,
                                                              h=gate["w1"].shape[0]), 16), dtype=torch.uint8,
                                    device=dev)
         self.kept = torch.empty(self.m, dtype=torch.int32, device=dev)
@@ -278,9 +285,9 @@ class PrunedPrefillStack:
 
     def gate_select(self):
         g = self.gate
-        tg.tg_gate_score(self.h, self.gate_norm_w, self.norm_eps, g["w1"], g["b1"], g["w2"], g["b2"], self.prunable,
-                         self.scores, self.sumsq, self.ws_gate)
-        tg.tg_topk_select(self.scores, self.prunable, self.n_prunable, self.w.k, self.kept)
+        tg.tg_gate_score_select(self.h, self.gate_norm_w, self.norm_eps, g["w1"], g["b1"], g["w2"], g["b2"],
+                                self.prunable, self.n_prunable, self.w.k, self.scores, self.sumsq, self.kept,
+                                self.ws_gate)
 
     def gather_mlp(self):
         """Gather the kept rows of the residual into self.hk and run layer L's

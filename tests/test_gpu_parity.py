@@ -120,6 +120,23 @@ def test_select_beyond_shared_memory_cache():
     assert np.array_equal(gpu_select(s, mask, k), O.select_kept(s, mask, k))
 
 
+@pytest.mark.parametrize("exact_ties", [False, True])
+def test_select_threshold_bin_too_full_for_the_candidate_lists(exact_ties):
+    # every score in [1, 1.25): all 131008 prunable keys share the first
+    # 11-bit digit, more than a CTA can gather, so the low bits are found by
+    # cluster-wide passes instead
+    n = 131072
+    rng = np.random.default_rng(11)
+    s = (1.0 + 0.25 * rng.random(n)).astype(np.float32)
+    if exact_ties:
+        s = (np.floor(s * 4096) / 4096).astype(np.float32)
+    mask = np.ones(n, np.uint8)
+    mask[-64:] = 0
+    n_p = n - 64
+    for k in (1, 8192, n_p // 2, n_p - 1):
+        assert np.array_equal(gpu_select(s, mask, k), O.select_kept(s, mask, k)), k
+
+
 def test_select_planted_block_kept():
     rng = np.random.default_rng(9)
     n = 20000
@@ -138,6 +155,17 @@ def test_select_mask_count_mismatch_reports_device_error():
     # caller claims 990 prunable tokens although all 1000 are: m = 10 + 10
     kept = torch.zeros(20, dtype=torch.int32, device=DEV)
     tg.tg_topk_select(d(s), d(mask, torch.uint8), 990, 10, kept)
+    with pytest.raises(tg.TokenGateError) as e:
+        tg.tg_check_device_error()
+    assert e.value.status == 8
+
+
+def test_select_mask_count_mismatch_reports_device_error_cluster():
+    n = 20000                               # the cluster selector
+    s = np.arange(n, dtype=np.float32)
+    mask = np.ones(n, np.uint8)
+    kept = torch.zeros(200, dtype=torch.int32, device=DEV)
+    tg.tg_topk_select(d(s), d(mask, torch.uint8), n - 100, 100, kept)
     with pytest.raises(tg.TokenGateError) as e:
         tg.tg_check_device_error()
     assert e.value.status == 8
@@ -229,6 +257,80 @@ def test_gate_score_is_deterministic():
     a = _gpu_scores(w, g, False)
     b = _gpu_scores(w, g, False)
     assert np.array_equal(a[0], b[0]) and a[1] == b[1]
+
+
+def _fused_vs_separate(w, g, k):
+    dt = synth.torch_dtype(w.dtype)
+    n = w.n
+    n_p = int(g["prunable"].sum())
+    m = min(k, n_p) + n - n_p
+    hid, w1 = d(g["hidden"], dt), d(g["w1"], dt)
+    b1, w2 = d(g["b1"]), d(g["w2"])
+    mask = d(g["prunable"], torch.uint8)
+    ws = torch.empty(tg.tg_workspace_bytes(tg.TG_OP_GATE_SELECT, n=n, d_model=w.d_model, h=w.gate_hidden),
+                     dtype=torch.uint8, device=DEV)
+    out = []
+    for fused in (True, False):
+        sc = torch.full((n,), float("nan"), device=DEV)
+        sq = torch.full((1,), float("nan"), device=DEV)
+        kept = torch.full((max(m, 1),), -1, dtype=torch.int32, device=DEV)
+        if fused:
+            tg.tg_gate_score_select(hid, None, 1e-6, w1, b1, w2, float(g["b2"]), mask, n_p, k, sc, sq, kept[:m], ws)
+        else:
+            tg.tg_gate_score(hid, None, 1e-6, w1, b1, w2, float(g["b2"]), mask, sc, sq, ws)
+            tg.tg_topk_select(sc, mask, n_p, k, kept[:m])
+        torch.cuda.synchronize()
+        out.append((sc, sq, kept[:m]))
+    (sf, qf, kf), (ss, qs, ks) = out
+    assert torch.equal(sf, ss) and torch.equal(qf, qs)          # the same scoring kernel
+    assert torch.equal(kf, ks)                                   # bit-exact kept indices
+    want = O.select_kept(host(sf), g["prunable"], k)
+    assert np.array_equal(host(kf).astype(np.int64), want)       # and the oracle's selection on those scores
+    return host(sf)
+
+
+@pytest.mark.parametrize("n,dm,k", [
+    (1000, 512, 100),      # one-CTA selector: no histogram
+    (5000, 512, 600),      # cluster selector from the gate's histogram
+    (16384, 2048, 2000),   # the 16K-token step
+    (40000, 512, 3000),
+    (16384, 512, 0),       # keep only the question
+    (16384, 512, 20000),   # keep everything
+])
+def test_gate_score_select_equals_separate_calls(n, dm, k):
+    w, g = _gate_case(n, dm, 256, "bf16", seed=n + k)
+    _fused_vs_separate(w, g, k)
+
+
+def test_gate_score_select_exact_ties_at_the_threshold():
+    # 400 copies of one hidden row; its entries are 0 or +-1/8, so the row's
+    # sum of squares is exact in any summation order and the copies score
+    # bit-identically wherever they sit in a tile.  The budget puts the
+    # threshold inside that group, so the kept set depends on breaking the
+    # ties towards the lower index
+    n, dm = 20000, 512
+    w, g = _gate_case(n, dm, 256, "bf16", seed=77)
+    rng = np.random.default_rng(77)
+    dup = rng.choice(np.flatnonzero(g["prunable"]), 400, replace=False)
+    g = dict(g)
+    g["hidden"] = g["hidden"].copy()
+    g["hidden"][dup] = np.round(np.clip(g["hidden"][dup[0]], -1, 1)) * 0.125
+    s = _fused_vs_separate(w, g, 1000)              # any budget: scores first
+    above = int(np.sum(s[g["prunable"] != 0] > s[dup[0]]))
+    assert np.all(s[dup] == s[dup[0]])
+    _fused_vs_separate(w, g, above + 150)
+
+
+def test_gate_score_select_all_scores_tied():
+    # every prunable row the same (entries 0 or +-1/8): one score, one bin,
+    # more candidates than a CTA can gather; the budget splits the tie
+    n, dm = 40000, 512
+    w, g = _gate_case(n, dm, 256, "bf16", seed=78)
+    g = dict(g)
+    row = np.round(np.clip(g["hidden"][0], -1, 1)) * 0.125
+    g["hidden"] = np.broadcast_to(row, g["hidden"].shape).astype(g["hidden"].dtype).copy()
+    s = _fused_vs_separate(w, g, 3000)
+    assert np.unique(s[g["prunable"] != 0]).size == 1
 
 
 # ============================================================================ attention
