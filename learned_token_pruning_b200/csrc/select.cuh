@@ -127,13 +127,14 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_topk_select(SelectParams p) 
   pdl_launch_dependents();
   extern __shared__ __align__(16) uint8_t sel_smem[];
   __shared__ __align__(16) uint32_t hist[1 << kSelTopBits];  // this CTA's first-digit counts
-  __shared__ uint32_t lhist[1 << kSelLowBits];
+  __shared__ uint32_t lhist[3][1 << kSelLowBits];  // the candidates' counts, one array per low digit
   __shared__ uint32_t warp_sums[kSelWarps + 1];
   __shared__ uint32_t info_a[kSelCluster][2];  // written by rank r into every rank: its prunable count, its candidates
   __shared__ uint32_t info_b[kSelCluster][2];  // written by rank r into every rank: tokens it keeps outright, its ties at T
   __shared__ uint32_t s_pick[2];
   __shared__ uint32_t s_ncand;
   __shared__ uint32_t s_off[kSelCluster];
+  __shared__ uint32_t s_lpick[3][2];
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
@@ -169,6 +170,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_topk_select(SelectParams p) 
     s_pick[0] = 0;
     s_pick[1] = 0;
   }
+  if (tid < 3 * (1 << kSelLowBits)) (&lhist[0][0])[tid] = 0;
+  if (tid < 6) (&s_lpick[0][0])[tid] = 0;
   // the first-digit counts, four bins a thread with the highest first: thread
   // t holds bins 2047-4t .. 2044-4t
   uint32_t hv[4] = {0u, 0u, 0u, 0u};
@@ -181,33 +184,82 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_topk_select(SelectParams p) 
   } else {
     for (int b = tid; b < (1 << kSelTopBits); b += kSelThreads) hist[b] = 0;
   }
-  __syncthreads();
-
-  // ---- load the slice (coalesced, four rounds of loads in flight): keys and
-  // flags into the cache, the prunable count and, without the gate's
-  // histogram, this CTA's first-digit counts
-  uint32_t cnt = 0;
-  for (int64_t base = 0; base < len; base += 4 * kSelThreads) {
-    float sc[4];
-    uint8_t pf[4];
+  // the first round of the slice's loads goes out before anything waits
+  float sc[4];
+  uint8_t pf[4];
+  auto issue = [&](int64_t base) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int64_t i = base + u * kSelThreads + tid;
       sc[u] = i < len ? __ldg(p.scores + lo + i) : 0.0f;
       pf[u] = i < len ? __ldg(p.prunable + lo + i) : uint8_t(0);
     }
+  };
+  issue(0);
+  __syncthreads();
+
+  // ---- the first digit from the counts: kp = min(k, prunable tokens), the
+  // counts summing to the latter; mode 0: keep no prunable token, 1: keep all
+  // of them, 2: threshold select
+  uint32_t np_total = 0, kp = 0, d1 = 0, rem = 0;
+  int mode = 0;
+  auto first_digit = [&]() {
+    const uint32_t c4 = hv[0] + hv[1] + hv[2] + hv[3];
+    const uint32_t above4 = block_exclusive_scan(c4, warp_sums, &np_total);
+    kp = static_cast<uint32_t>(min(p.k, static_cast<int64_t>(np_total)));
+    mode = kp == 0 ? 0 : (kp >= np_total ? 1 : 2);
+    if (mode == 2 && above4 < kp && kp <= above4 + c4) {
+      uint32_t a = above4;
+      int u = 0;
+      for (; u < 3 && a + hv[u] < kp; ++u) a += hv[u];
+      s_pick[0] = static_cast<uint32_t>((1 << kSelTopBits) - 1 - 4 * tid - u);
+      s_pick[1] = a;
+    }
+    __syncthreads();
+    d1 = s_pick[0];
+    rem = mode == 2 ? kp - s_pick[1] : 0u;  // rank of T among the keys whose first digit is d1
+  };
+  // warp-aggregated append of this lane's key to the CTA's candidate list
+  auto append = [&](bool c, uint32_t key) {
+    const uint32_t bal = __ballot_sync(0xffffffffu, c);
+    if (bal) {
+      const int leader = __ffs(bal) - 1;
+      uint32_t b0 = 0;
+      if (lane == leader) b0 = atomicAdd(&s_ncand, static_cast<uint32_t>(__popc(bal)));
+      b0 = __shfl_sync(0xffffffffu, b0, leader);
+      const uint32_t pos = b0 + static_cast<uint32_t>(__popc(bal & ((1u << lane) - 1u)));
+      if (c && pos < static_cast<uint32_t>(kSelOwnCap)) own_cand[pos] = key;
+    }
+  };
+  if (top) first_digit();
+
+  // ---- load the slice (coalesced, the next round in flight while one is
+  // processed): keys and flags into the cache, the prunable count, and either
+  // the candidates (first digit known) or this CTA's first-digit counts
+  uint32_t cnt = 0;
+  for (int64_t base = 0; base < len; base += 4 * kSelThreads) {
+    float csc[4];
+    uint8_t cpf[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      csc[u] = sc[u];
+      cpf[u] = pf[u];
+    }
+    if (base + 4 * kSelThreads < len) issue(base + 4 * kSelThreads);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int64_t i = base + u * kSelThreads + tid;
-      const bool f = pf[u] != 0;
-      const uint32_t key = f ? order_key(sc[u]) : 0u;
+      const bool f = cpf[u] != 0;
+      const uint32_t key = f ? order_key(csc[u]) : 0u;
       if (p.cached && i < len) {
         const int s = static_cast<int>(i & (kpt - 1)) * kSelStride + static_cast<int>(i >> kshift);
         keys[s] = key;
         flags[s] = f ? 1 : 0;
       }
       cnt += f ? 1u : 0u;
-      if (!top) {
+      if (top) {
+        if (mode == 2) append(f && (key >> (32 - kSelTopBits)) == d1, key);
+      } else {
         // lanes holding the same digit add once (scores crowd into a few bins)
         const uint32_t bin = f ? (key >> (32 - kSelTopBits)) : 0xffffffffu;
         const uint32_t peers = __match_any_sync(0xffffffffu, bin);
@@ -232,44 +284,18 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_topk_select(SelectParams p) 
         hv[2] += q[r].y;
         hv[3] += q[r].x;
       }
-  }
-
-  // ---- the first digit: kp = min(k, prunable tokens), the counts summing to the latter
-  const uint32_t c4 = hv[0] + hv[1] + hv[2] + hv[3];
-  uint32_t np_total;
-  const uint32_t above4 = block_exclusive_scan(c4, warp_sums, &np_total);
-  const uint32_t kp = static_cast<uint32_t>(min(p.k, static_cast<int64_t>(np_total)));
-  // mode 0: keep no prunable token; 1: keep all of them; 2: threshold select
-  const int mode = kp == 0 ? 0 : (kp >= np_total ? 1 : 2);
-  if (mode == 2 && above4 < kp && kp <= above4 + c4) {
-    uint32_t a = above4;
-    int u = 0;
-    for (; u < 3 && a + hv[u] < kp; ++u) a += hv[u];
-    s_pick[0] = static_cast<uint32_t>((1 << kSelTopBits) - 1 - 4 * tid - u);
-    s_pick[1] = a;
-  }
-  __syncthreads();
-  const uint32_t d1 = s_pick[0];
-  uint32_t rem = mode == 2 ? kp - s_pick[1] : 0u;  // rank of T among the keys whose first digit is d1
-
-  // ---- this CTA's candidates
-  if (mode == 2) {
-    for (int j = 0; j < kpt; ++j) {
-      bool c = false;
-      uint32_t key = 0;
-      if (static_cast<int64_t>(tid) * kpt + j < len) {
-        bool f;
-        load_own(j, key, f);
-        c = f && (key >> (32 - kSelTopBits)) == d1;
-      }
-      const uint32_t bal = __ballot_sync(0xffffffffu, c);
-      if (bal) {
-        const int leader = __ffs(bal) - 1;
-        uint32_t b0 = 0;
-        if (lane == leader) b0 = atomicAdd(&s_ncand, static_cast<uint32_t>(__popc(bal)));
-        b0 = __shfl_sync(0xffffffffu, b0, leader);
-        const uint32_t pos = b0 + static_cast<uint32_t>(__popc(bal & ((1u << lane) - 1u)));
-        if (c && pos < static_cast<uint32_t>(kSelOwnCap)) own_cand[pos] = key;
+    first_digit();
+    // this CTA's candidates, from the cache
+    if (mode == 2) {
+      for (int j = 0; j < kpt; ++j) {
+        bool c = false;
+        uint32_t key = 0;
+        if (static_cast<int64_t>(tid) * kpt + j < len) {
+          bool f;
+          load_own(j, key, f);
+          c = f && (key >> (32 - kSelTopBits)) == d1;
+        }
+        append(c, key);
       }
     }
   }
@@ -299,9 +325,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_topk_select(SelectParams p) 
     uint32_t prefix = d1 << (32 - kSelTopBits), pmask = ((1u << kSelTopBits) - 1u) << (32 - kSelTopBits);
     if (!over) {
       // gather every rank's candidates (four remote loads in flight a thread)
-      // and count their next digit
-      if (tid < (1 << kSelLowBits)) lhist[tid] = 0;
-      __syncthreads();  // lhist zeroed, s_off written
+      // and count their next digit; each pass has its own zeroed counts and pick
+      __syncthreads();  // s_off written
       for (uint32_t base = 0; base < ncand; base += 4 * kSelThreads) {
         uint32_t v[4];
 #pragma unroll
@@ -320,7 +345,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_topk_select(SelectParams p) 
           const uint32_t idx = base + u * kSelThreads + tid;
           if (idx < ncand) {
             all_cand[idx] = v[u];
-            atomicAdd(&lhist[(v[u] >> 14) & 127u], 1u);
+            atomicAdd(&lhist[0][(v[u] >> 14) & 127u], 1u);
           }
         }
       }
@@ -328,25 +353,22 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_topk_select(SelectParams p) 
       for (int pass = 0; pass < 3; ++pass) {
         const int shift = 14 - kSelLowBits * pass;
         if (pass > 0) {
-          if (tid < (1 << kSelLowBits)) lhist[tid] = 0;
-          __syncthreads();
           for (uint32_t idx = tid; idx < ncand; idx += kSelThreads) {
             const uint32_t v = all_cand[idx];
-            if ((v & pmask) == prefix) atomicAdd(&lhist[(v >> shift) & 127u], 1u);
+            if ((v & pmask) == prefix) atomicAdd(&lhist[pass][(v >> shift) & 127u], 1u);
           }
           __syncthreads();
         }
         if (warp == 0) {
           uint32_t v[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) v[u] = lhist[127 - 4 * lane - u];
-          warp_pick_low_digit(v, rem, s_pick);
+          for (int u = 0; u < 4; ++u) v[u] = lhist[pass][127 - 4 * lane - u];
+          warp_pick_low_digit(v, rem, s_lpick[pass]);
         }
         __syncthreads();
-        rem -= s_pick[1];
-        prefix |= s_pick[0] << shift;
+        rem -= s_lpick[pass][1];
+        prefix |= s_lpick[pass][0] << shift;
         pmask |= 127u << shift;
-        __syncthreads();  // s_pick read before the next pass rewrites it
       }
     } else {
       // too many candidates: the low bits by cluster-wide passes over the

@@ -330,14 +330,15 @@ bool gate_uses_tc(const void* hidden, int dtype, int32_t d_model, const void* w1
 
 // workspace layout of tg_gate_score (256-byte aligned pieces):
 //   [per-CTA partial sums of s^2][completion counter][W1 scaled by the norm weight, bf16 [h][d]]
+// and of tg_gate_score_select, the selector's first-digit histogram right
+// after the counter so that one memset clears both:
+//   [partial sums][completion counter][histogram, 2048 x u32][scaled W1]
 size_t gate_partials_bytes(int64_t n) { return ((static_cast<size_t>((n + 127) / 128) * 4 + 255) / 256) * 256; }
+constexpr size_t kGateHistBytes = tg::kGateHistBins * sizeof(uint32_t);
 size_t gate_ws_bytes(int64_t n, int32_t d, int32_t h) {
   return gate_partials_bytes(n) + 256 + ((static_cast<size_t>(d) * h * 2 + 255) / 256) * 256;
 }
-// tg_gate_score_select: the gate's workspace, then the selector's first-digit histogram
-size_t gate_select_ws_bytes(int64_t n, int32_t d, int32_t h) {
-  return gate_ws_bytes(n, d, h) + tg::kGateHistBins * sizeof(uint32_t);
-}
+size_t gate_select_ws_bytes(int64_t n, int32_t d, int32_t h) { return gate_ws_bytes(n, d, h) + kGateHistBytes; }
 
 }  // namespace
 
@@ -450,7 +451,7 @@ static int launch_gather_rmsnorm(const LayerGather& g, int dtype, void* hidden_k
 static int gate_score_impl(const void* hidden, int dtype, int64_t n, int32_t d_model, const float* norm_w,
                            float norm_eps, const void* w1, const float* b1, const float* w2, float b2, int32_t h,
                            const uint8_t* prunable, float* scores, float* sumsq, void* ws, size_t ws_bytes,
-                           uint32_t* key_hist, void* stream);
+                           bool with_hist, void* stream);
 static int topk_select_impl(const float* scores, const uint8_t* prunable, int64_t n, int64_t n_prunable, int64_t k,
                             int32_t* kept_idx, int64_t m, const uint32_t* hist_top, void* stream);
 
@@ -671,36 +672,39 @@ int tg_gate_score(const void* hidden, int dtype, int64_t n, int32_t d_model, con
                   const void* w1, const float* b1, const float* w2, float b2, int32_t h, const uint8_t* prunable,
                   float* scores, float* sumsq, void* ws, size_t ws_bytes, void* stream) {
   return gate_score_impl(hidden, dtype, n, d_model, norm_w, norm_eps, w1, b1, w2, b2, h, prunable, scores, sumsq, ws,
-                         ws_bytes, nullptr, stream);
+                         ws_bytes, false, stream);
 }
 
 }  // extern "C"
 
-// tg_gate_score; with key_hist (device [2048], zeroed by the caller on the
-// stream) the tensor-core kernel also counts order_key(s) >> 21 over the
-// prunable tokens (the selector's first digit).  Returns TG_ERR_UNSUPPORTED
-// with key_hist on the CUDA-core path, which does not build it.
+// tg_gate_score; with_hist (the tg_gate_score_select workspace layout) has the
+// tensor-core kernel also count order_key(s) >> 21 over the prunable tokens
+// (the selector's first digit) into the workspace's histogram.  Returns
+// TG_ERR_UNSUPPORTED with with_hist on the CUDA-core path, which does not
+// build it.
 static int gate_score_impl(const void* hidden, int dtype, int64_t n, int32_t d_model, const float* norm_w,
                            float norm_eps, const void* w1, const float* b1, const float* w2, float b2, int32_t h,
                            const uint8_t* prunable, float* scores, float* sumsq, void* ws, size_t ws_bytes,
-                           uint32_t* key_hist, void* stream) {
+                           bool with_hist, void* stream) {
   if (!hidden || !w1 || !w2 || !prunable || !scores || !sumsq) return fail(TG_ERR_INVALID_ARG, "null pointer");
   if (n <= 0 || d_model <= 0 || h <= 0) return fail(TG_ERR_INVALID_ARG, "n, d_model and h must be positive");
   if (n >= (int64_t(1) << 31)) return fail(TG_ERR_UNSUPPORTED, "n must be < 2^31");
   if (dtype != TG_F32 && dtype != TG_BF16) return fail(TG_ERR_INVALID_ARG, "dtype");
   cudaStream_t st = as_stream(stream);
   if (gate_uses_tc(hidden, dtype, d_model, w1, h)) {
-    const size_t need = gate_ws_bytes(n, d_model, h);
+    const size_t need = with_hist ? gate_select_ws_bytes(n, d_model, h) : gate_ws_bytes(n, d_model, h);
     if (!ws || ws_bytes < need) return fail(TG_ERR_WORKSPACE, "gate score needs %zu workspace bytes", need);
     if (!aligned16(ws)) return fail(TG_ERR_ALIGN, "workspace must be 16-byte aligned");
     float* partials = static_cast<float*>(ws);
-    uint32_t* counter = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + gate_partials_bytes(n));
-    cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(uint32_t), st);
+    uint8_t* counter_at = static_cast<uint8_t*>(ws) + gate_partials_bytes(n);
+    uint32_t* counter = reinterpret_cast<uint32_t*>(counter_at);
+    uint32_t* key_hist = with_hist ? reinterpret_cast<uint32_t*>(counter_at + 256) : nullptr;
+    cudaError_t e = cudaMemsetAsync(counter, 0, with_hist ? 256 + kGateHistBytes : sizeof(uint32_t), st);
     if (e != cudaSuccess) return fail(TG_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
     const void* w1_eff = w1;
     if (norm_w) {
       // RMSNorm(h) * w_n feeds W1, so (h * w_n) W1^T = h (W1 diag(w_n))^T: fold the weight into W1
-      __nv_bfloat16* w1f = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + gate_partials_bytes(n) + 256);
+      __nv_bfloat16* w1f = reinterpret_cast<__nv_bfloat16*>(counter_at + 256 + (with_hist ? kGateHistBytes : 0));
       const int64_t total = int64_t(h) * d_model;
       tg::k_fold_norm<<<unsigned((total + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w1), norm_w,
                                                                    w1f, total, d_model);
@@ -725,7 +729,7 @@ static int gate_score_impl(const void* hidden, int dtype, int64_t n, int32_t d_m
     if (h <= 128) return launch_gate_tc<128>(hidden, w1_eff, nn, d_model, p, st);
     return launch_gate_tc<256>(hidden, w1_eff, nn, d_model, p, st);
   }
-  if (key_hist) return fail(TG_ERR_UNSUPPORTED, "the key histogram comes only from the tensor-core gate kernel");
+  if (with_hist) return fail(TG_ERR_UNSUPPORTED, "the key histogram comes only from the tensor-core gate kernel");
   if (h > 1024) return fail(TG_ERR_UNSUPPORTED, "h > 1024");
   const unsigned blocks = static_cast<unsigned>((n + 7) / 8);
   if (dtype == TG_F32)
@@ -845,17 +849,13 @@ int tg_gate_score_select(const void* hidden, int dtype, int64_t n, int32_t d_mod
   const size_t need = gate_select_ws_bytes(n, d_model, h);
   if (!ws || ws_bytes < need) return fail(TG_ERR_WORKSPACE, "gate score + select needs %zu workspace bytes", need);
   if (!aligned16(ws)) return fail(TG_ERR_ALIGN, "workspace must be 16-byte aligned");
-  cudaStream_t st = as_stream(stream);
   // the selector's first-digit histogram rides with the gate kernel when the
   // tensor cores score and the cluster selector runs (longer prompts)
-  uint32_t* hist = nullptr;
-  if (n > tg::kSelSmallBest && gate_uses_tc(hidden, dtype, d_model, w1, h)) {
-    hist = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + gate_ws_bytes(n, d_model, h));
-    if (cudaMemsetAsync(hist, 0, tg::kGateHistBins * sizeof(uint32_t), st) != cudaSuccess)
-      return fail(TG_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(cudaGetLastError()));
-  }
+  const bool with_hist = n > tg::kSelSmallBest && gate_uses_tc(hidden, dtype, d_model, w1, h);
+  const uint32_t* hist =
+      with_hist ? reinterpret_cast<const uint32_t*>(static_cast<uint8_t*>(ws) + gate_partials_bytes(n) + 256) : nullptr;
   int rc = gate_score_impl(hidden, dtype, n, d_model, norm_w, norm_eps, w1, b1, w2, b2, h, prunable, scores, sumsq,
-                           ws, ws_bytes, hist, stream);
+                           ws, ws_bytes, with_hist, stream);
   if (rc) return rc;
   return topk_select_impl(scores, prunable, n, n_prunable, k, kept_idx, m, hist, stream);
 }
