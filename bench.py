@@ -37,12 +37,12 @@ L2_FLUSH_BYTES = 256 << 20   # > the 126 MB L2
 # with the rows that launch processed; scaled to the bench launch by rows.  A
 # record counts only while the SHA-256 of its kernel's sources still matches.
 MEASURED_TRAFFIC = {
-    "linear_gate_up_swiglu": {"bytes": 58852352 + 7237120, "rows": 2064, "sources": ("gemm_tc.cuh", "common.cuh"),
-                              "sha256": "8d1b356a43a10dd74230fca02bba39aef170ea447c87b34d34d4ade57fcc10bb"},
-    "gate_score": {"bytes": 269859328 + 5020160, "rows": 65536, "sources": ("gate_tc.cuh", "common.cuh"),
-                   "sha256": "182595c9d81cb684ae20b148a60c168d96dd5af5e795460977a043d60dfe59c2"},
-    "attention": {"bytes": 16979200 + 22016, "rows": 2064, "sources": ("attn_tc.cuh", "common.cuh"),
-                  "sha256": "21ae350b717df6dfc56a267bb6fa0b545ef7dec309bd2ae1d29d96743d7d6616"},
+    "linear_gate_up_swiglu": {"bytes": 58823680 + 8841472, "rows": 2064, "sources": ("gemm_tc.cuh", "common.cuh"),
+                              "sha256": "527a8b39fc28c7c0d19969704ccff730efd0618e8420255ad1f826e8c2b07b6b"},
+    "gate_score": {"bytes": 269954048 + 3879936, "rows": 65536, "sources": ("gate_tc.cuh", "common.cuh"),
+                   "sha256": "f6182c664cb45b9dc872a44326e2295b8f4a0020cdb639898ff52988753ef2cd"},
+    "attention": {"bytes": 17001728 + 0, "rows": 2064, "sources": ("attn_tc.cuh", "common.cuh"),
+                  "sha256": "6907c5c56acd338f3ea57e63415f7402285bb8c64e1f489ddcfd4e954540ae5c"},
 }
 
 
@@ -568,40 +568,47 @@ def end_to_end(step, w, args, stream, flush, dist, dev, world):
 
 
 def ncu_case():
-    """One launch each of the path's kernels at the bench shapes, for profiler
-    captures (the gate score at N = 65536 so its input exceeds L2; select and
-    gather on the 16K-token prefix with K = 2048 and 16 question tokens)."""
+    """One launch each of the path's kernels, for profiler captures: the fused
+    gate score + select at N = 65536 (K = 8192; its input exceeds L2), the
+    gather folded into RMSNorm on the 16K-token prefix (K = 2048, 16 question
+    tokens), gated attention at m = 2064 and at m = 8256, and the SwiGLU GEMM
+    at 2064 rows."""
     import torch
     from learned_token_pruning_b200 import tokengate as tg
     torch.manual_seed(0)
     dev = "cuda"
-    n, d, h = 65536, 2048, 256
+    n, d, h, kb = 65536, 2048, 256, 8192
     hid = torch.randn(n, d, device=dev).to(torch.bfloat16)
     w1 = (torch.randn(h, d, device=dev) * 0.02).to(torch.bfloat16)
     w2 = torch.randn(h, device=dev) * 0.02
     mask = torch.ones(n, dtype=torch.uint8, device=dev)
     mask[-64:] = 0
     sc, sq = torch.empty(n, device=dev), torch.empty(1, device=dev)
-    ws = torch.empty(tg.tg_workspace_bytes(tg.TG_OP_GATE_SCORE, n=n, d_model=d, h=h), dtype=torch.uint8, device=dev)
-    tg.tg_gate_score(hid, None, 1e-6, w1, torch.zeros(h, device=dev), w2, 0.0, mask, sc, sq, ws)
+    ws = torch.empty(tg.tg_workspace_bytes(tg.TG_OP_GATE_SELECT, n=n, d_model=d, h=h), dtype=torch.uint8, device=dev)
+    kept64 = torch.empty(kb + 64, dtype=torch.int32, device=dev)
+    tg.tg_gate_score_select(hid, None, 1e-6, w1, torch.zeros(h, device=dev), w2, 0.0, mask, n - 64, kb, sc, sq,
+                            kept64, ws)
     n16, nq, k = 16384, 16, 2048
     mask16 = torch.ones(n16, dtype=torch.uint8, device=dev)
     mask16[-nq:] = 0
     kept = torch.empty(k + nq, dtype=torch.int32, device=dev)
     tg.tg_topk_select(sc[:n16].contiguous(), mask16, n16 - nq, k, kept)
     hk = torch.empty(k + nq, d, dtype=torch.bfloat16, device=dev)
-    tg.tg_gather(hid[:n16], kept, sc[:n16].contiguous(), sq, n16 - nq, 1e-6, hk,
-                 torch.empty(k + nq, dtype=torch.int32, device=dev), torch.empty(k + nq, device=dev),
-                 torch.empty(k + nq, device=dev))
-    m, hq, hkv, D = 2064, 16, 8, 128
-    qkv = torch.randn(m, (hq + 2 * hkv) * D, device=dev).to(torch.bfloat16)
-    out = torch.empty(m, hq * D, dtype=torch.bfloat16, device=dev)
-    aws_n = tg.attention_workspace_bytes(m, hq, hkv, D, torch.bfloat16)
-    aws = torch.empty(max(aws_n, 16), dtype=torch.uint8, device=dev) if aws_n else None
-    tg.tg_gated_attention(qkv[:, :hq * D], qkv[:, hq * D:(hq + hkv) * D], qkv[:, (hq + hkv) * D:], D,
-                          torch.randn(m, device=dev), torch.rand(hq, device=dev) + 0.5,
-                          torch.rand(hq, device=dev) * 0.4 + 0.8, torch.rand(m, device=dev), 1 / math.sqrt(D), out,
-                          ws=aws)
+    xn = torch.empty_like(hk)
+    tg.tg_gather_rmsnorm(hid[:n16], kept, sc[:n16].contiguous(), sq, n16 - nq, 1e-6, torch.ones(d, device=dev), 1e-6,
+                         hk, xn, torch.empty(k + nq, dtype=torch.int32, device=dev), torch.empty(k + nq, device=dev),
+                         torch.empty(k + nq, device=dev))
+    hq, hkv, D = 16, 8, 128
+    for m in (2064, 8256):
+        qkv = torch.randn(m, (hq + 2 * hkv) * D, device=dev).to(torch.bfloat16)
+        out = torch.empty(m, hq * D, dtype=torch.bfloat16, device=dev)
+        aws_n = tg.attention_workspace_bytes(m, hq, hkv, D, torch.bfloat16)
+        aws = torch.empty(max(aws_n, 16), dtype=torch.uint8, device=dev) if aws_n else None
+        tg.tg_gated_attention(qkv[:, :hq * D], qkv[:, hq * D:(hq + hkv) * D], qkv[:, (hq + hkv) * D:], D,
+                              torch.randn(m, device=dev), torch.rand(hq, device=dev) + 0.5,
+                              torch.rand(hq, device=dev) * 0.4 + 0.8, torch.rand(m, device=dev), 1 / math.sqrt(D),
+                              out, ws=aws)
+    m = 2064
     x = torch.randn(m, 2048, device=dev).to(torch.bfloat16)
     wgu = (torch.randn(2 * 6144, 2048, device=dev) * 0.02).to(torch.bfloat16)
     act = torch.empty(m, 6144, dtype=torch.bfloat16, device=dev)
