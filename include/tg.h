@@ -224,9 +224,14 @@ int tg_gather_rmsnorm(const void* hidden, int dtype, int64_t n, int32_t d_model,
  *        blocks are split over two CTAs whose partial results meet in ws; with
  *        ws NULL (or smaller than required) nothing is split.  The size depends
  *        on the SM count of the current device and is 0 when no split is made.
- * head_dim in {64, 128}; hq % hkv == 0.  bf16 with an even hq / hkv runs on the
- * tcgen05 tensor cores (fp32 softmax and accumulation); fp32 and odd groups
- * run on CUDA cores in full fp32.
+ * head_dim in {64, 128}; hq % hkv == 0.  bf16 with an even group size hq / hkv
+ * runs on the tcgen05 tensor cores (fp32 softmax and accumulation): each CTA
+ * there serves two query heads of one KV head, so that every K/V tile it loads
+ * feeds two score tiles.  fp32 inputs, and bf16 with an odd group size (1, 3,
+ * 5, ...: MHA included), run on a CUDA-core kernel in full fp32 instead -- the
+ * same results within the attention tolerance, but tens of times slower at the
+ * workloads' sizes (it is there for correctness, not speed).  The split
+ * workspace is ignored on that path.
  */
 int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk,
                        const void* v, int64_t ldv, int dtype, int64_t m,
