@@ -7,23 +7,27 @@
 // into the SM once.
 //
 // A persistent kernel: one CTA per SM walks the 128-token tiles t = blockIdx.x,
-// blockIdx.x + gridDim.x, ...  TMA streams 128x64 tiles of H and BNx64 tiles of
-// W1 (128-byte swizzle) through a STAGES-deep ring that runs on across tile
-// boundaries; one thread issues tcgen05.mma (M=128, N=BN, K=16) into one of
-// two fp32 TMEM accumulators (2 x BN columns), so the epilogue of tile i runs
-// while the MMAs of tile i+1 stream.  Four row-norm warps sum h^2 of the
-// tile's rows from the same shared-memory stages (one thread per row; the
-// swizzle only permutes the 16-byte chunks inside a row's 128-byte line, which
-// a sum does not see); a stage goes back to the producer once the MMAs and
-// these warps have both read it.  Eight epilogue warps, two per TMEM lane
-// quarter, each take half of a row's BN accumulator columns, apply 1/rms, b1,
-// SiLU and w2, and the halves are added through shared memory.  Sum over
-// prunable rows of s^2: per CTA over its tiles in order, then over the CTAs in
-// a fixed order by the last CTA to finish (deterministic).
+// blockIdx.x + gridDim.x, ...  TMA streams 128x64 tiles of H through a
+// kGateHStages-deep ring and BNx64 tiles of W1 through a kGateWStages-deep one
+// (128-byte swizzle), both running on across tile boundaries, each fed by its
+// own producer thread: the hidden rows come from DRAM, whose latency under a
+// full GPU's load needs about 100 KB in flight per SM, while W1 (read by every
+// tile) comes from L2.  One thread issues tcgen05.mma (M=128, N=BN, K=16)
+// into one of two fp32 TMEM accumulators (2 x BN columns), so the epilogue of
+// tile i runs while the MMAs of tile i+1 stream.  Four row-norm warps sum h^2
+// of the tile's rows from the same shared-memory stages (one thread per row;
+// the swizzle only permutes the 16-byte chunks inside a row's 128-byte line,
+// which a sum does not see); a hidden-row stage goes back to its producer
+// once the MMAs and these warps have both read it.  Eight epilogue warps, two
+// per TMEM lane quarter, each take half of a row's BN accumulator columns,
+// apply 1/rms, b1, SiLU and w2, and the halves are added through shared
+// memory.  Sum over prunable rows of s^2: per CTA over its tiles in order,
+// then over the CTAs in a fixed order by the last CTA to finish
+// (deterministic).
 //
-// Warp roles (448 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
-// issuer, warps 2-5 row norms, warps 6-13 epilogue (warp w reads TMEM lanes
-// 32*(w%4)..+31).
+// Warp roles (480 threads): warp 0 hidden-row producer, warp 1 TMEM allocator
+// + MMA issuer, warps 2-5 row norms, warps 6-13 epilogue (warp w reads TMEM
+// lanes 32*(w%4)..+31), warp 14 W1 producer.
 #pragma once
 
 #include "common.cuh"
@@ -32,8 +36,9 @@ namespace tg {
 
 constexpr int kGateBM = 128;
 constexpr int kGateBK = 64;
-constexpr int kGateThreads = 448;
-constexpr int kGateStages = 4;
+constexpr int kGateThreads = 480;
+constexpr int kGateHStages = 7;  // hidden-state ring (from DRAM: the deep one)
+constexpr int kGateWStages = 3;  // W1 ring (from L2)
 
 struct GateParams {
   int M, N, K;        // tokens, gate hidden width h, d_model
@@ -52,6 +57,13 @@ struct GateParams {
 
 constexpr int kGateHistBins = 2048;
 
+static_assert(kGateBK == 64, "the MMA loop issues four K = 16 MMAs per 64-column k-step");
+
+// tcgen05.commit to an mbarrier given by its shared-memory address
+__device__ __forceinline__ void gate_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 template <int BN>
 struct GateCfg {
   static constexpr int kABytes = kGateBM * kGateBK * 2;
@@ -59,8 +71,8 @@ struct GateCfg {
   static constexpr int kBBox = BN < 128 ? BN : 128;  // rows per W1 TMA box
   static constexpr int kAccCols = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
   static constexpr int kTmemCols = 2 * kAccCols;   // two accumulators
-  static constexpr size_t kSmem =
-      1024 + kGateStages * (kABytes + kBBytes) + 256 + 2 * BN * 4 + 2 * 2 * 128 * 4 + 64 + kGateHistBins * 4;
+  static constexpr size_t kSmem = 1024 + kGateHStages * kABytes + kGateWStages * kBBytes + 256 + 2 * BN * 4 +
+                                  2 * 2 * 128 * 4 + 64 + kGateHistBins * 4;
 };
 
 template <int BN>
@@ -68,20 +80,22 @@ __global__ void __launch_bounds__(kGateThreads, 1)
     k_gate_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               GateParams p) {
   using Cfg = GateCfg<BN>;
-  constexpr int STAGES = kGateStages;
+  constexpr int HST = kGateHStages, WST = kGateWStages;
   extern __shared__ uint8_t gate_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gate_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * Cfg::kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * Cfg::kBBytes);
-  uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;   // [2] accumulator b holds a finished tile
+  uint8_t* sB = smem + HST * Cfg::kABytes;
+  uint64_t* hfull = reinterpret_cast<uint64_t*>(sB + WST * Cfg::kBBytes);  // [HST] hidden rows landed
+  uint64_t* hempty = hfull + HST;  // [HST] the MMAs and the four row-norm warps have read them
+  uint64_t* wfull = hempty + HST;  // [WST] W1 tile landed
+  uint64_t* wempty = wfull + WST;  // [WST] the MMAs have read it
+  uint64_t* acc_full = wempty + WST;     // [2] accumulator b holds a finished tile
   uint64_t* acc_empty = acc_full + 2;    // [2] the epilogue has read accumulator b (256 arrivals)
   uint64_t* ss_full = acc_empty + 2;     // [2] row sums of squares of the tile in buffer b (128 arrivals)
   uint64_t* ss_free = ss_full + 2;       // [2] the epilogue has read them (256 arrivals)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ss_free + 2);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  float* s_b1 = reinterpret_cast<float*>(smem + STAGES * (Cfg::kABytes + Cfg::kBBytes) + 256);
+  float* s_b1 = reinterpret_cast<float*>(smem + HST * Cfg::kABytes + WST * Cfg::kBBytes + 256);
   float* s_w2 = s_b1 + BN;
   float* s_ss = s_w2 + BN;        // [2][128] row sums of h^2 per tile parity
   float* s_half = s_ss + 2 * 128; // [2][128] second-half partial dot products
@@ -96,9 +110,13 @@ __global__ void __launch_bounds__(kGateThreads, 1)
   const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);  // the MMA commit and the four row-norm warps
+    for (int s = 0; s < HST; ++s) {
+      mbar_init(&hfull[s], 1);
+      mbar_init(&hempty[s], 1 + 4);  // the MMA commit and the four row-norm warps
+    }
+    for (int s = 0; s < WST; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], 1);  // the MMA commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -121,62 +139,95 @@ __global__ void __launch_bounds__(kGateThreads, 1)
   pdl_wait();
   pdl_launch_dependents();
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (runs across tiles)
+  if (warp == 0 || warp == 14) {
+    // ------------------------------------------------------------ TMA producers (run across tiles)
+    // Warp 0 streams the hidden rows through the deep ring, warp 14 the W1
+    // tiles through the short one, each as far ahead as its own ring allows.
+    // Every CTA needs all of W1: walking K from a tile-dependent start spreads
+    // the concurrent W1 reads over different L2 lines instead of having every
+    // SM hit the same k-tile at once.  (Only the fp32 summation order changes.)
     if (lane == 0) {
-      prefetch_tmap(&tmA);
-      prefetch_tmap(&tmB);
+      const bool hid = warp == 0;
+      prefetch_tmap(hid ? &tmA : &tmB);
+      const int nst = hid ? HST : WST;
       int g = 0;  // k-steps issued so far
       for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
         const int tile = blockIdx.x + i * gridDim.x;
-        // Every CTA needs all of W1: walking K from a tile-dependent start
-        // spreads the concurrent W1 reads over different L2 lines instead of
-        // having every SM hit the same k-tile at once.  (Only the fp32
-        // summation order changes.)
         const int kofs = tile % num_k;
         for (int kt = 0; kt < num_k; ++kt, ++g) {
-          const int s = g % STAGES;
-          const uint32_t ph = (g / STAGES) & 1;
-          if (!mbar_wait(&empty[s], ph ^ 1, kErrWaitGemm)) {
+          const int s = g % nst;
+          const uint32_t ph = (g / nst) & 1;
+          if (!mbar_wait(hid ? &hempty[s] : &wempty[s], ph ^ 1, kErrWaitGemm)) {
             *abort_flag = 1;
             break;
           }
           const int kx = ((kt + kofs) % num_k) * kGateBK;
-          mbar_arrive_expect_tx(&full[s], Cfg::kABytes + Cfg::kBBytes);
-          tma_load_2d(sA + s * Cfg::kABytes, &tmA, &full[s], kx, tile * kGateBM);
+          if (hid) {
+            mbar_arrive_expect_tx(&hfull[s], Cfg::kABytes);
+            tma_load_2d(sA + s * Cfg::kABytes, &tmA, &hfull[s], kx, tile * kGateBM);
+          } else {
+            mbar_arrive_expect_tx(&wfull[s], Cfg::kBBytes);
 #pragma unroll
-          for (int hb = 0; hb < BN / Cfg::kBBox; ++hb)
-            tma_load_2d(sB + s * Cfg::kBBytes + hb * Cfg::kBBox * 128, &tmB, &full[s], kx, hb * Cfg::kBBox);
+            for (int hb = 0; hb < BN / Cfg::kBBox; ++hb)
+              tma_load_2d(sB + s * Cfg::kBBytes + hb * Cfg::kBBox * 128, &tmB, &wfull[s], kx, hb * Cfg::kBBox);
+          }
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // A barrier check holds back the next tcgen05.mma for its shared-memory
+    // round trip, and the tensor core's issue queue is short, so the rings of
+    // k-step g + 1 are checked between the second and third MMA of k-step g,
+    // while the first two run; the loop keeps its slot and phase counters
+    // incrementally and reads the abort flag once per tile.
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kGateBM, BN, false, false);
-      int g = 0;
-      bool ok = true;
+      // descriptors of stage 0 and barrier addresses, advanced by adding
+      // offsets (16-byte units in a descriptor's address field, which cannot
+      // carry out of it: shared memory is below 256 KB)
+      const uint64_t da0 = sdesc_sw128(smem_u32(sA), 16, 1024), db0 = sdesc_sw128(smem_u32(sB), 16, 1024);
+      constexpr uint32_t kAUnits = Cfg::kABytes >> 4, kBUnits = Cfg::kBBytes >> 4;
+      const uint32_t hfull_a = smem_u32(hfull), hempty_a = smem_u32(hempty);
+      const uint32_t wfull_a = smem_u32(wfull), wempty_a = smem_u32(wempty);
+      int sh = 0, sw = 0;          // ring slots of the current k-step
+      uint32_t phh = 0, phw = 0;   // and their phases
+      uint32_t oa = 0, ob = 0;     // descriptor offsets of those slots
+      bool ok = my_tiles == 0 || mbar_wait2(&hfull[0], 0, &wfull[0], 0, kErrWaitGemm);
       for (int i = 0; i < my_tiles && ok; ++i) {
         const int b = i & 1;
         // accumulator b last held tile i - 2: free once its epilogue read it
-        if (i >= 2 && !(ok = mbar_wait(&acc_empty[b], ((i - 2) >> 1) & 1, kErrWaitGemm))) break;
+        if (*abort_flag || (i >= 2 && !mbar_wait(&acc_empty[b], ((i - 2) >> 1) & 1, kErrWaitGemm))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t acc = tmem + b * Cfg::kAccCols;
-        for (int kt = 0; kt < num_k; ++kt, ++g) {
-          const int s = g % STAGES;
-          const uint32_t ph = (g / STAGES) & 1;
-          if (*abort_flag || !mbar_wait(&full[s], ph, kErrWaitGemm)) {
-            ok = false;
-            break;
+        const int checks = i == my_tiles - 1 ? num_k - 1 : num_k;  // k-steps followed by another
+        for (int kt = 0; kt < num_k; ++kt) {
+          const uint64_t da = da0 + oa, db = db0 + ob;
+          const int nsh = sh + 1 == HST ? 0 : sh + 1, nsw = sw + 1 == WST ? 0 : sw + 1;
+          const uint32_t nphh = nsh == 0 ? phh ^ 1u : phh, nphw = nsw == 0 ? phw ^ 1u : phw;
+          umma_ss(acc, da, db, idesc, kt != 0 ? 1u : 0u);
+          umma_ss(acc, da + 2, db + 2, idesc, 1u);
+          if (kt < checks) {
+            const bool rh = mbar_try_wait(hfull_a + nsh * 8, nphh);
+            const bool rw = mbar_try_wait(wfull_a + nsw * 8, nphw);
+            if (!(rh && rw))
+              ok = mbar_wait(&hfull[nsh], nphh, kErrWaitGemm) && mbar_wait(&wfull[nsw], nphw, kErrWaitGemm);
+            tc_fence_after();
           }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + s * Cfg::kABytes);
-          const uint32_t b0 = smem_u32(sB + s * Cfg::kBBytes);
-#pragma unroll
-          for (int kk = 0; kk < kGateBK / 16; ++kk)
-            umma_ss(acc, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), idesc,
-                    (kt | kk) != 0 ? 1u : 0u);
-          umma_commit(&empty[s]);
+          umma_ss(acc, da + 4, db + 4, idesc, 1u);
+          umma_ss(acc, da + 6, db + 6, idesc, 1u);
+          gate_commit(hempty_a + sh * 8);
+          gate_commit(wempty_a + sw * 8);
+          sh = nsh;
+          sw = nsw;
+          phh = nphh;
+          phw = nphw;
+          oa = nsh == 0 ? 0u : oa + kAUnits;
+          ob = nsw == 0 ? 0u : ob + kBUnits;
+          if (!ok) break;
         }
         if (ok) umma_commit(&acc_full[b]);
       }
@@ -194,9 +245,9 @@ __global__ void __launch_bounds__(kGateThreads, 1)
       float ss = 0.0f;
       bool ok = true;
       for (int kt = 0; kt < num_k; ++kt, ++g) {
-        const int s = g % STAGES;
-        const uint32_t ph = (g / STAGES) & 1;
-        if (*abort_flag || !warp_wait(&full[s], ph, kErrWaitGemm)) {
+        const int s = g % HST;
+        const uint32_t ph = (g / HST) & 1;
+        if (*abort_flag || !warp_wait(&hfull[s], ph, kErrWaitGemm)) {
           ok = false;
           break;
         }
@@ -212,7 +263,7 @@ __global__ void __launch_bounds__(kGateThreads, 1)
           }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);  // release: the reads above come first
+        if (lane == 0) mbar_arrive(&hempty[s]);  // release: the reads above come first
       }
       if (!ok) {
         *abort_flag = 1;
@@ -227,7 +278,7 @@ __global__ void __launch_bounds__(kGateThreads, 1)
       mbar_arrive(&ss_full[b]);
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 6-13)
+    // ------------------------------------------------------------ epilogue (warps 6-13; 14 is a producer)
     const int q = warp & 3;
     const int half = (warp - 6) >> 2;  // 0: columns [0, BN/2), 1: [BN/2, BN)
     const int row = q * 32 + lane;
