@@ -336,6 +336,8 @@ def run_gpu(args, w):
     br = breakdown(step, w, args, stream, flush)
     kernels = {}
     for name, ms in br.items():
+        if name.startswith("_"):
+            continue
         wk = work.get(name, {})
         entry = {"us": ms * 1e3}
         if ms <= 0:             # serialised replays (under a profiler) can leave no difference to time
@@ -348,7 +350,10 @@ def run_gpu(args, w):
             gbs = wk["bytes"] / (ms * 1e-3) / 1e9
             entry.update({"gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"]})
         if name == "gate_score":
+            # 256 flop per byte of hidden state: its tensor ceiling is as
+            # close as its HBM one, so both fractions are given
             entry["tflops"] = wk["flops"] / (ms * 1e-3) / 1e12
+            entry["frac_bf16_peak"] = entry["tflops"] / peaks["bf16_tflops"]
         kernels[name] = entry
     # calls timed alone that the step runs fused: tg_gather (folded into the
     # layer's first RMSNorm), tg_gate_score and tg_topk_select (tg_gate_score_select)
@@ -472,20 +477,29 @@ def breakdown(step, w, args, stream, flush):
         return a.elapsed_time(b) / reps
 
     # each call is timed as (L2 flush + call) minus (L2 flush): cold L2 like
-    # the step, without the flush and without launch gaps
+    # the step, without the flush and without launch gaps.  A call whose input
+    # alone is larger than L2 (the gate at 128K tokens reads 512 MiB) finds
+    # none of it there anyway; it runs back to back without the flush, whose
+    # dirty lines it would otherwise write back to HBM inside its own time.
+    l2_bytes = torch.cuda.get_device_properties(stream.device).L2_cache_size
+    work = workload_work(w, m)
     g_flush = graph_of(lambda: flush.zero_())
     t_flush = replay_ms(g_flush)
     out = {}
     for name, fn in calls.items():
         fn()
         torch.cuda.synchronize()
+        if work.get(name, {}).get("bytes", 0) > l2_bytes:
+            g = graph_of(fn)
+            out[name] = replay_ms(g)
+            out.setdefault("_unflushed", []).append(name)
+        else:
+            def body(fn=fn):
+                flush.zero_()
+                fn()
 
-        def body(fn=fn):
-            flush.zero_()
-            fn()
-
-        g = graph_of(body)
-        out[name] = max(replay_ms(g) - t_flush, 0.0)
+            g = graph_of(body)
+            out[name] = max(replay_ms(g) - t_flush, 0.0)
         del g
     del g_flush
     return out
@@ -893,12 +907,13 @@ def run_sweep(args):
         br = breakdown(step, w, types.SimpleNamespace(steps=max(args.steps, 5)), stream, flush)
         calls = {}
         for name, ms in br.items():
+            if name.startswith("_"):
+                continue
             e = {"us": round(ms * 1e3, 2)}
             wk = work.get(name, {})
             if "flops" in wk:
                 e["tflops"] = round(wk["flops"] / (ms * 1e-3) / 1e12, 1)
-                if name not in ("gate_score",):
-                    e["frac_bf16_peak"] = round(e["tflops"] / peaks["bf16_tflops"], 3)
+                e["frac_bf16_peak"] = round(e["tflops"] / peaks["bf16_tflops"], 3)
             if "bytes" in wk:
                 e["gbs"] = round(wk["bytes"] / (ms * 1e-3) / 1e9, 1)
                 e["frac_hbm"] = round(e["gbs"] / peaks["hbm_gbs"], 3)
@@ -906,7 +921,9 @@ def run_sweep(args):
         line = {"mode": "sweep", "workload": w.name, "n": w.n, "k": w.k, "kept_rows": step.m,
                 "step_ms": round(step_ms, 4), "tokens_per_s": w.n / (step_ms * 1e-3),
                 "peak_hbm_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 3), "calls": calls,
-                "l2": "flushed before every timed step"}
+                "l2": "step: flushed before each; calls: flushed before each, except "
+                      + (", ".join(br.get("_unflushed", [])) or "none")
+                      + " (input larger than L2: back to back, no flush)"}
         print(json.dumps(line), flush=True)
         del step
         torch.cuda.empty_cache()
@@ -1015,16 +1032,21 @@ def single_layer_step(w, dev, stream, flush, reps, peaks):
     work = workload_work(w, step.m)
     att_tf = work["attention"]["flops"] / (br["attention"] * 1e-3) / 1e12
     gate_gbs = work["gate_score"]["bytes"] / (br["gate_score"] * 1e-3) / 1e9
+    gate_tf = work["gate_score"]["flops"] / (br["gate_score"] * 1e-3) / 1e12
     gs_gbs = work["gate_score_select"]["bytes"] / (br["gate_score_select"] * 1e-3) / 1e9
     res = {"workload": w.name, "n": w.n, "k": w.k, "kept_rows": step.m, "step_ms": round(ms, 4),
            "tokens_per_s": w.n / (ms * 1e-3), "peak_hbm_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 3),
            "attention": {"us": round(br["attention"] * 1e3, 2), "tflops": round(att_tf, 1),
                          "frac_bf16_peak": round(att_tf / peaks["bf16_tflops"], 4)},
            "gate_score": {"us": round(br["gate_score"] * 1e3, 2), "gbs": round(gate_gbs, 1),
-                          "frac_hbm": round(gate_gbs / peaks["hbm_gbs"], 4)},
+                          "frac_hbm": round(gate_gbs / peaks["hbm_gbs"], 4), "tflops": round(gate_tf, 1),
+                          "frac_bf16_peak": round(gate_tf / peaks["bf16_tflops"], 4)},
            "gate_score_select": {"us": round(br["gate_score_select"] * 1e3, 2), "gbs": round(gs_gbs, 1),
                                  "frac_hbm": round(gs_gbs / peaks["hbm_gbs"], 4)},
            "topk_select": {"us": round(br["topk_select"] * 1e3, 2)},
+           "l2": "step: flushed (256 MiB write) before each; calls: flushed before each, except "
+                 + (", ".join(br.get("_unflushed", [])) or "none")
+                 + " (input larger than L2: back to back, no flush)",
            "reps": reps}
     del step
     torch.cuda.empty_cache()

@@ -35,6 +35,8 @@ struct GatherParams {
   int32_t* pos;
   float* bias;
   float* ratio;
+  uint32_t* zero;  // k_gather_rmsnorm_warp: words cleared by block 0 for a later kernel (or null)
+  int zero_n;
 };
 
 __global__ void __launch_bounds__(kGatherThreads) k_gather(GatherParams p) {
@@ -185,6 +187,8 @@ __global__ void __launch_bounds__(256) k_gather_rmsnorm_warp(GatherParams p, T* 
                                                              const float* __restrict__ w, int d, float norm_eps) {
   pdl_wait();
   pdl_launch_dependents();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < p.zero_n; i += blockDim.x) p.zero[i] = 0u;
   constexpr int V = 16 / sizeof(T);
   const int lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);

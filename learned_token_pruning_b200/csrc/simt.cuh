@@ -348,9 +348,14 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope(T* __restrict__ qkv, int64
 // ---------------------------------------------------------------------------
 template <typename T, int MAXV>
 __global__ void __launch_bounds__(256) k_rmsnorm_warp(const T* __restrict__ x, T* __restrict__ y,
-                                                      const float* __restrict__ w, int64_t m, int d, float eps) {
+                                                      const float* __restrict__ w, int64_t m, int d, float eps,
+                                                      uint32_t* zero, int zero_n) {
   pdl_wait();
   pdl_launch_dependents();
+  // words a later kernel needs cleared (its counters), done here so that no
+  // memset sits between kernels and breaks their programmatic launches
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < zero_n; i += blockDim.x) zero[i] = 0u;
   constexpr int V = 16 / sizeof(T);
   const int lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);

@@ -344,8 +344,16 @@ size_t gate_select_ws_bytes(int64_t n, int32_t d, int32_t h) { return gate_ws_by
 
 // RMSNorm of m rows: one warp per row when the row fits in a warp's registers
 // (and the weight is 16-byte aligned), else one block per row.
+// words of a later kernel's workspace (counters) that the launched kernel
+// clears as a side job
+struct ZeroSpan {
+  uint32_t* p = nullptr;
+  int n = 0;
+};
+
 template <typename T>
-int launch_rmsnorm(const void* x, void* y, const float* w, int64_t m, int d, float eps, cudaStream_t st) {
+int launch_rmsnorm(const void* x, void* y, const float* w, int64_t m, int d, float eps, cudaStream_t st,
+                   ZeroSpan z = ZeroSpan{}) {
   constexpr int V = 16 / sizeof(T);
   const int nv = d / V;
   const T* xa = static_cast<const T*>(x);
@@ -353,15 +361,20 @@ int launch_rmsnorm(const void* x, void* y, const float* w, int64_t m, int d, flo
   const unsigned blocks = static_cast<unsigned>((m + 7) / 8);
   if (!w || aligned16(w)) {
     if (nv <= 32 * 4) {
-      return launch_pdl("k_rmsnorm_warp", tg::k_rmsnorm_warp<T, 4>, dim3(blocks), dim3(256), 0, st, xa, ya, w, m, d, eps);
+      return launch_pdl("k_rmsnorm_warp", tg::k_rmsnorm_warp<T, 4>, dim3(blocks), dim3(256), 0, st, xa, ya, w, m, d, eps,
+                        z.p, z.n);
     }
     if (nv <= 32 * 8) {
-      return launch_pdl("k_rmsnorm_warp", tg::k_rmsnorm_warp<T, 8>, dim3(blocks), dim3(256), 0, st, xa, ya, w, m, d, eps);
+      return launch_pdl("k_rmsnorm_warp", tg::k_rmsnorm_warp<T, 8>, dim3(blocks), dim3(256), 0, st, xa, ya, w, m, d, eps,
+                        z.p, z.n);
     }
     if (nv <= 32 * 16) {
-      return launch_pdl("k_rmsnorm_warp", tg::k_rmsnorm_warp<T, 16>, dim3(blocks), dim3(256), 0, st, xa, ya, w, m, d, eps);
+      return launch_pdl("k_rmsnorm_warp", tg::k_rmsnorm_warp<T, 16>, dim3(blocks), dim3(256), 0, st, xa, ya, w, m, d, eps,
+                        z.p, z.n);
     }
   }
+  if (z.n && cudaMemsetAsync(z.p, 0, size_t(z.n) * 4, st) != cudaSuccess)
+    return fail(TG_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(cudaGetLastError()));
   return launch_pdl("k_rmsnorm", tg::k_rmsnorm<T>, dim3(unsigned(m)), dim3(256), 0, st, xa, ya, w, d, eps);
 }
 
@@ -447,7 +460,7 @@ static int prefill_layer_impl(const tg_layer_weights* W, const tg_layer_shape* S
                               const int64_t* seg_rows, int32_t nseg, const LayerGather* gather, void* ws,
                               size_t ws_bytes, void* stream);
 static int launch_gather_rmsnorm(const LayerGather& g, int dtype, void* hidden_kept, void* xn, const float* w,
-                                 int64_t m, int d, float eps, cudaStream_t st);
+                                 int64_t m, int d, float eps, cudaStream_t st, ZeroSpan z);
 static int gate_score_impl(const void* hidden, int dtype, int64_t n, int32_t d_model, const float* norm_w,
                            float norm_eps, const void* w1, const float* b1, const float* w2, float b2, int32_t h,
                            const uint8_t* prunable, float* scores, float* sumsq, void* ws, size_t ws_bytes,
@@ -907,10 +920,14 @@ int tg_gather(const void* hidden, int dtype, int64_t n, int32_t d_model, const i
   return launch_pdl("k_gather", tg::k_gather, dim3(blocks), dim3(tg::kGatherThreads), 0, as_stream(stream), p);
 }
 
-int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk, const void* v, int64_t ldv, int dtype,
-                       int64_t m, int32_t hq, int32_t hkv, int32_t head_dim, const float* bias,
-                       const float* head_gain, const float* head_temp, const float* ratio, float sm_scale, void* out,
-                       int64_t ldo, float* lse, void* ws, size_t ws_bytes, void* stream) {
+// tg_gated_attention; counters_zeroed: the caller has already cleared the
+// split-merge counters in ws (attn_counter_span) in an earlier kernel on the
+// stream, so no memset is issued here
+static int gated_attention_impl(const void* q, int64_t ldq, const void* k, int64_t ldk, const void* v, int64_t ldv,
+                                int dtype, int64_t m, int32_t hq, int32_t hkv, int32_t head_dim, const float* bias,
+                                const float* head_gain, const float* head_temp, const float* ratio, float sm_scale,
+                                void* out, int64_t ldo, float* lse, void* ws, size_t ws_bytes, void* stream,
+                                bool counters_zeroed) {
   if (!q || !k || !v || !out || !head_gain || !head_temp) return fail(TG_ERR_INVALID_ARG, "null pointer");
   if (m <= 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0) return fail(TG_ERR_INVALID_ARG, "bad m / heads");
   if (m >= (int64_t(1) << 31)) return fail(TG_ERR_UNSUPPORTED, "m must be < 2^31");
@@ -970,7 +987,7 @@ int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk, c
       p.counters = reinterpret_cast<unsigned*>(wb + pl.ctr_off);
       std::fill(std::begin(work.item), std::end(work.item), uint16_t(0));
       std::copy(pl.items.begin(), pl.items.end(), work.item);
-      if (cudaMemsetAsync(p.counters, 0, pl.bytes - pl.ctr_off, st) != cudaSuccess)
+      if (!counters_zeroed && cudaMemsetAsync(p.counters, 0, pl.bytes - pl.ctr_off, st) != cudaSuccess)
         return fail(TG_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(cudaGetLastError()));
     }
     const int items = p.use_table ? static_cast<int>(pl.items.size()) : p.num_qtiles;
@@ -1014,6 +1031,27 @@ int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk, c
     else tg::k_attn_simt<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(p);
   }
   return check_launch("k_attn_simt");
+}
+
+int tg_gated_attention(const void* q, int64_t ldq, const void* k, int64_t ldk, const void* v, int64_t ldv, int dtype,
+                       int64_t m, int32_t hq, int32_t hkv, int32_t head_dim, const float* bias,
+                       const float* head_gain, const float* head_temp, const float* ratio, float sm_scale, void* out,
+                       int64_t ldo, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  return gated_attention_impl(q, ldq, k, ldk, v, ldv, dtype, m, hq, hkv, head_dim, bias, head_gain, head_temp, ratio,
+                              sm_scale, out, ldo, lse, ws, ws_bytes, stream, false);
+}
+
+// The split-merge counters a tensor-core attention call over m rows would use
+// in ws (empty when it splits nothing or takes the CUDA-core path)
+static ZeroSpan attn_counter_span(int64_t m, int32_t hq, int32_t hkv, int32_t head_dim, int dtype, void* ws,
+                                  size_t ws_bytes) {
+  ZeroSpan z;
+  if (dtype != TG_BF16 || hkv <= 0 || hq % hkv || (hq / hkv) % 2 || !ws || !aligned16(ws)) return z;
+  const AttnPlan& pl = attn_plan(m, hkv, hq / hkv, head_dim, sm_count());
+  if (!pl.table || ws_bytes < pl.bytes) return z;
+  z.p = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + pl.ctr_off);
+  z.n = static_cast<int>((pl.bytes - pl.ctr_off) / 4);
+  return z;
 }
 
 int tg_linear(const void* x, int64_t ldx, const void* w, void* y, int64_t ldy, int dtype, int64_t m, int32_t n_out,
@@ -1292,7 +1330,8 @@ int tg_gather_rmsnorm(const void* hidden, int dtype, int64_t n, int32_t d_model,
   if ((int64_t(d_model) * es) % 16 != 0 || !aligned16(hidden) || !aligned16(hidden_kept) || !aligned16(x_norm))
     return fail(TG_ERR_ALIGN, "rows must be 16-byte multiples on 16-byte aligned buffers");
   const LayerGather g{hidden, n, kept_idx, scores, sumsq, n_prunable, seq_eps, pos, bias, ratio};
-  return launch_gather_rmsnorm(g, dtype, hidden_kept, x_norm, norm_w, m, d_model, norm_eps, as_stream(stream));
+  return launch_gather_rmsnorm(g, dtype, hidden_kept, x_norm, norm_w, m, d_model, norm_eps, as_stream(stream),
+                               ZeroSpan{});
 }
 
 int tg_gather_prefill_layer(const tg_layer_weights* W, const tg_layer_shape* S, int part, const void* hidden,
@@ -1344,9 +1383,11 @@ static int mlp_half(const tg_layer_weights* W, const tg_layer_shape* S, void* hi
 // The gather fused with an RMSNorm (k_gather_rmsnorm_warp): rows whose 16-byte
 // vectors fit a warp's registers; other shapes gather first and normalise after.
 static int launch_gather_rmsnorm(const LayerGather& g, int dtype, void* hidden_kept, void* xn, const float* w,
-                                 int64_t m, int d, float eps, cudaStream_t st) {
+                                 int64_t m, int d, float eps, cudaStream_t st, ZeroSpan z) {
   const int es = dtype_size(dtype);
   tg::GatherParams p{};
+  p.zero = z.p;
+  p.zero_n = z.n;
   p.hidden = static_cast<const uint8_t*>(g.hidden);
   p.n = g.n;
   p.row_bytes = int64_t(d) * es;
@@ -1378,8 +1419,8 @@ static int launch_gather_rmsnorm(const LayerGather& g, int dtype, void* hidden_k
   int rc = tg_gather(g.hidden, dtype, g.n, d, g.idx, m, g.scores, g.sumsq, g.n_prunable, g.seq_eps, hidden_kept, g.pos,
                      g.bias, g.ratio, st);
   if (rc) return rc;
-  return dtype == TG_BF16 ? launch_rmsnorm<__nv_bfloat16>(hidden_kept, xn, w, m, d, eps, st)
-                          : launch_rmsnorm<float>(hidden_kept, xn, w, m, d, eps, st);
+  return dtype == TG_BF16 ? launch_rmsnorm<__nv_bfloat16>(hidden_kept, xn, w, m, d, eps, st, z)
+                          : launch_rmsnorm<float>(hidden_kept, xn, w, m, d, eps, st, z);
 }
 
 // One decoder layer over m rows; with seg_rows (host, nseg + 1 offsets) the
@@ -1430,18 +1471,23 @@ static int prefill_layer_impl(const tg_layer_weights* W, const tg_layer_shape* S
   int rc;
   // the first RMSNorm of the parts run here: from the rows in place, or
   // gathering them from the full sequence in the same pass
-  auto first_norm = [&](const float* w) -> int {
+  auto first_norm = [&](const float* w, ZeroSpan z) -> int {
     if (!gather)
-      return bf ? launch_rmsnorm<__nv_bfloat16>(hidden_kept, xn, w, m, d, S->norm_eps, st)
-                : launch_rmsnorm<float>(hidden_kept, xn, w, m, d, S->norm_eps, st);
-    return launch_gather_rmsnorm(*gather, S->dtype, hidden_kept, xn, w, m, d, S->norm_eps, st);
+      return bf ? launch_rmsnorm<__nv_bfloat16>(hidden_kept, xn, w, m, d, S->norm_eps, st, z)
+                : launch_rmsnorm<float>(hidden_kept, xn, w, m, d, S->norm_eps, st, z);
+    return launch_gather_rmsnorm(*gather, S->dtype, hidden_kept, xn, w, m, d, S->norm_eps, st, z);
   };
   if (!do_attn) {
-    if ((rc = first_norm(W->w_post_norm))) return rc;
+    if ((rc = first_norm(W->w_post_norm, ZeroSpan{}))) return rc;
     return mlp_half(W, S, hidden_kept, xn, act, m, stream);
   }
+  // the attention split-merge counters of a single request are cleared by the
+  // layer's first kernel, so no memset node sits between the q/k-norm kernel
+  // and attention (it would stop attention's launch from overlapping it)
+  const ZeroSpan attn_ctr =
+      seg_rows ? ZeroSpan{} : attn_counter_span(m, hq, hkv, D, S->dtype, attn_ws_sz ? attn_ws : nullptr, attn_ws_sz);
   // 1. x = RMSNorm(h)
-  if ((rc = first_norm(W->w_in_norm))) return rc;
+  if ((rc = first_norm(W->w_in_norm, attn_ctr))) return rc;
   // 2. qkv = x Wqkv^T
   if ((rc = tg_linear(xn, d, W->w_qkv, qkv, qkv_w, S->dtype, m, int32_t(qkv_w), d, TG_EPI_STORE, stream))) return rc;
   // 3. per-head q/k norm and RoPE at the original positions (one warp per row)
@@ -1478,10 +1524,10 @@ static int prefill_layer_impl(const tg_layer_weights* W, const tg_layer_shape* S
         return fail(TG_ERR_CUDA, "bias staging copy: %s", cudaGetErrorString(cudaGetLastError()));
       br = bias_stage;
     }
-    if ((rc = tg_gated_attention(qb, qkv_w, qb + int64_t(hq) * D * es, qkv_w, qb + int64_t(hq + hkv) * D * es, qkv_w,
-                                 S->dtype, mr, hq, hkv, D, br, W->head_gain, W->head_temp,
-                                 ratio ? ratio + r0 : nullptr, 1.0f / sqrtf(float(D)), ab, int64_t(hq) * D, nullptr,
-                                 attn_ws_sz ? attn_ws : nullptr, attn_ws_sz, stream)))
+    if ((rc = gated_attention_impl(qb, qkv_w, qb + int64_t(hq) * D * es, qkv_w, qb + int64_t(hq + hkv) * D * es,
+                                   qkv_w, S->dtype, mr, hq, hkv, D, br, W->head_gain, W->head_temp,
+                                   ratio ? ratio + r0 : nullptr, 1.0f / sqrtf(float(D)), ab, int64_t(hq) * D, nullptr,
+                                   attn_ws_sz ? attn_ws : nullptr, attn_ws_sz, stream, attn_ctr.n > 0)))
       return rc;
   }
   // 5. h += a Wo^T
