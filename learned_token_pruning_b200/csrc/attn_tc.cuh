@@ -347,12 +347,14 @@ __device__ __forceinline__ void attn_epilogue(const AttnTcParams& p, const CUten
 // kDiag: the tile crosses the diagonal, keys past the row are masked with
 // -inf and every exponential goes to the MUFU unit (exp2(-inf) = 0 exactly);
 // off the diagonal one pair in four is evaluated on the FMA pipe.
-template <int D, bool kDiag>
-__device__ __forceinline__ void attn_softmax_tile(uint32_t t_s, uint32_t t_o, uint64_t a2, int key0, int grow,
-                                                  bool first, float& m_run, float& l_run) {
+// The tile's second pass: P = exp2(a S' - m) for the row's maximum m (nm2 =
+// -m, nmh2 = -m - 1/2 for the FMA-pipe form) written back as bf16 pairs over
+// the first 64 columns of the same S buffer; returns the row sum of P.
+template <bool kDiag>
+__device__ __forceinline__ float attn_exp_pass(uint32_t t_s, uint64_t a2, uint64_t nm2, uint64_t nmh2, int key0,
+                                               int grow) {
   constexpr int BN = 128, G = BN / 32;
-  const uint64_t zero2 = f2_pack(0.0f, 0.0f);
-  float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  uint64_t sum2[4] = {0, 0, 0, 0};
   uint32_t buf[2][32];
   tmem_ld32(t_s, buf[0]);
   tmem_ld_wait();
@@ -360,23 +362,82 @@ __device__ __forceinline__ void attn_softmax_tile(uint32_t t_s, uint32_t t_o, ui
   for (int q = 0; q < G; ++q) {
     if (q + 1 < G) tmem_ld32(t_s + 32 * (q + 1), buf[(q + 1) & 1]);
     const uint32_t* r = buf[q & 1];
+    uint32_t pk[16];
 #pragma unroll
-    for (int e = 0; e < 32; e += 4) {
-      float l0, h0, l1, h1;
-      f2_unpack(f2_fma(a2, f2_pack(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), zero2), l0, h0);
-      f2_unpack(f2_fma(a2, f2_pack(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])), zero2), l1, h1);
+    for (int v = 0; v < 16; ++v) {
+      const int e = 2 * v;  // keys 32q + e and 32q + e + 1
+      float s0 = __uint_as_float(r[e]), s1 = __uint_as_float(r[e + 1]);
       if (kDiag) {
         const int k = key0 + 32 * q + e;
-        if (k > grow) l0 = -INFINITY;
-        if (k + 1 > grow) h0 = -INFINITY;
-        if (k + 2 > grow) l1 = -INFINITY;
-        if (k + 3 > grow) h1 = -INFINITY;
+        if (k > grow) s0 = -INFINITY;
+        if (k + 1 > grow) s1 = -INFINITY;
       }
-      mxv[(e >> 2) & 3] = fmax3(mxv[(e >> 2) & 3], fmaxf(l0, h0), fmaxf(l1, h1));
+      const uint64_t s2 = f2_pack(s0, s1);
+      uint64_t p2;
+      if (!kDiag && (v & 3) == 3) {
+        p2 = exp2_poly2(f2_fma(a2, s2, nmh2));
+      } else {
+        float x0, x1;
+        f2_unpack(f2_fma(a2, s2, nm2), x0, x1);
+        p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+      }
+      sum2[v & 3] = f2_add(sum2[v & 3], p2);
+      float p0, p1;
+      f2_unpack(p2, p0, p1);
+      pk[v] = pack_bf16x2(p0, p1);
     }
+    tmem_st16(t_s + 16 * q, pk);
     if (q + 1 < G) tmem_ld_wait();
   }
-  const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
+  float a0, a1, b0, b1;
+  f2_unpack(f2_add(sum2[0], sum2[1]), a0, a1);
+  f2_unpack(f2_add(sum2[2], sum2[3]), b0, b1);
+  return (a0 + a1) + (b0 + b1);
+}
+
+template <int D, bool kDiag>
+__device__ __forceinline__ void attn_softmax_tile(uint32_t t_s, uint32_t t_o, uint64_t a2, int key0, int grow,
+                                                  bool first, float& m_run, float& l_run) {
+  constexpr int BN = 128, G = BN / 32;
+  float a, a_hi;
+  f2_unpack(a2, a, a_hi);
+  // The tile's maximum of x = a S': for a > 0 it is a * max(S') exactly (the
+  // rounding of a product is monotonic in the other factor), which saves the
+  // scaling of every element in this pass; otherwise the scaled values.
+  float mx;
+  {
+    const bool raw = __all_sync(0xffffffffu, a > 0.0f);
+    const uint64_t zero2 = f2_pack(0.0f, 0.0f);
+    float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    uint32_t buf[2][32];
+    tmem_ld32(t_s, buf[0]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int q = 0; q < G; ++q) {
+      if (q + 1 < G) tmem_ld32(t_s + 32 * (q + 1), buf[(q + 1) & 1]);
+      const uint32_t* r = buf[q & 1];
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        float l0 = __uint_as_float(r[e]), h0 = __uint_as_float(r[e + 1]);
+        float l1 = __uint_as_float(r[e + 2]), h1 = __uint_as_float(r[e + 3]);
+        if (!raw) {
+          f2_unpack(f2_fma(a2, f2_pack(l0, h0), zero2), l0, h0);
+          f2_unpack(f2_fma(a2, f2_pack(l1, h1), zero2), l1, h1);
+        }
+        if (kDiag) {
+          const int k = key0 + 32 * q + e;
+          if (k > grow) l0 = -INFINITY;
+          if (k + 1 > grow) h0 = -INFINITY;
+          if (k + 2 > grow) l1 = -INFINITY;
+          if (k + 3 > grow) h1 = -INFINITY;
+        }
+        mxv[(e >> 2) & 3] = fmax3(mxv[(e >> 2) & 3], fmaxf(l0, h0), fmaxf(l1, h1));
+      }
+      if (q + 1 < G) tmem_ld_wait();
+    }
+    mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
+    if (raw) mx = a * mx;
+  }
   float sc = 1.0f;
   if (mx - m_run > 8.0f) {  // per row: divergent, so no warp-collective op inside
     if (!first) sc = ex2_approx(m_run - mx);
@@ -395,44 +456,9 @@ __device__ __forceinline__ void attn_softmax_tile(uint32_t t_s, uint32_t t_o, ui
       tmem_st32(t_o + c0, o);
     }
   }
-  const uint64_t nm2 = f2_pack(-m_run, -m_run), nmh2 = f2_pack(-m_run - 0.5f, -m_run - 0.5f);
-  uint64_t sum2[4] = {0, 0, 0, 0};
-  tmem_ld32(t_s, buf[0]);
-  tmem_ld_wait();
-#pragma unroll
-  for (int q = 0; q < G; ++q) {
-    if (q + 1 < G) tmem_ld32(t_s + 32 * (q + 1), buf[(q + 1) & 1]);
-    const uint32_t* r = buf[q & 1];
-    uint32_t pk[16];
-#pragma unroll
-    for (int v = 0; v < 16; ++v) {
-      const int e = 2 * v;  // keys 32q + e and 32q + e + 1
-      const uint64_t s2 = f2_pack(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
-      uint64_t p2;
-      if (!kDiag && (v & 3) == 3) {
-        p2 = exp2_poly2(f2_fma(a2, s2, nmh2));
-      } else {
-        float x0, x1;
-        f2_unpack(f2_fma(a2, s2, nm2), x0, x1);
-        if (kDiag) {
-          const int k = key0 + 32 * q + e;
-          if (k > grow) x0 = -INFINITY;
-          if (k + 1 > grow) x1 = -INFINITY;
-        }
-        p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
-      }
-      sum2[v & 3] = f2_add(sum2[v & 3], p2);
-      float p0, p1;
-      f2_unpack(p2, p0, p1);
-      pk[v] = pack_bf16x2(p0, p1);
-    }
-    tmem_st16(t_s + 16 * q, pk);
-    if (q + 1 < G) tmem_ld_wait();
-  }
-  float a0, a1, b0, b1;
-  f2_unpack(f2_add(sum2[0], sum2[1]), a0, a1);
-  f2_unpack(f2_add(sum2[2], sum2[3]), b0, b1);
-  l_run = l_run * sc + ((a0 + a1) + (b0 + b1));
+  const float sum =
+      attn_exp_pass<kDiag>(t_s, a2, f2_pack(-m_run, -m_run), f2_pack(-m_run - 0.5f, -m_run - 0.5f), key0, grow);
+  l_run = l_run * sc + sum;
 }
 
 // bf16 hi/lo split: v ~= hi + lo, both bf16 (rounded to nearest)
