@@ -43,6 +43,7 @@ MEASURED_TRAFFIC = {
                    "sha256": "119cea418d54f0b167a567331415219d357f7a3e836c5eeb503578c143718edb"},
     "attention": {"bytes": 17002240 + 0, "rows": 2064, "sources": ("attn_tc.cuh", "common.cuh"),
                   "sha256": "dea1b84a1dcf77b3a2579da49c6d3c8937eb553f075a054d4d52c78a1f465801"},
+}
 
 
 # ----------------------------------------------------------------------------- helpers (host only)
