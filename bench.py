@@ -359,6 +359,8 @@ def run_gpu(args, w):
     # layer's first RMSNorm), tg_gate_score and tg_topk_select (tg_gate_score_select)
     for k in ("unfused_gather", "gate_score", "topk_select"):
         kernels[k]["in_step"] = False
+    # what the selector adds inside the fused call (started from the gate's histogram)
+    kernels["gate_score_select"]["select_us_beyond_gate"] = kernels["gate_score_select"]["us"] - kernels["gate_score"]["us"]
     not_dom = ("gather_layer_total", "unfused_gather", "gate_score", "topk_select")
     dom = max((k for k in kernels if k not in not_dom and kernels[k]["us"] > 0), key=lambda k: kernels[k]["us"])
     wk = work[dom]
