@@ -302,6 +302,36 @@ def test_gate_score_select_equals_separate_calls(n, dm, k):
     _fused_vs_separate(w, g, k)
 
 
+@pytest.mark.parametrize("dtype,dm,h,norm_w", [
+    ("f32", 256, 64, False),     # CUDA-core gate: the cluster selector builds its own first digit
+    ("bf16", 2048, 256, True),   # the norm weight folded into W1, histogram from the gate
+])
+def test_gate_score_select_other_gate_paths(dtype, dm, h, norm_w):
+    n, k = 9000, 1500
+    w, g = _gate_case(n, dm, h, dtype, seed=31, norm_w=norm_w)
+    dt = synth.torch_dtype(w.dtype)
+    n_p = int(g["prunable"].sum())
+    m = min(k, n_p) + n - n_p
+    args = [d(g["hidden"], dt), d(g["norm_w"]) if norm_w else None, 1e-6, d(g["w1"], dt), d(g["b1"]), d(g["w2"]),
+            float(g["b2"]), d(g["prunable"], torch.uint8)]
+    ws = torch.empty(tg.tg_workspace_bytes(tg.TG_OP_GATE_SELECT, n=n, d_model=dm, h=h), dtype=torch.uint8, device=DEV)
+    sc, sq = torch.empty(n, device=DEV), torch.empty(1, device=DEV)
+    kept = torch.empty(m, dtype=torch.int32, device=DEV)
+    tg.tg_gate_score_select(*args, n_p, k, sc, sq, kept, ws)
+    sc2, sq2 = torch.empty(n, device=DEV), torch.empty(1, device=DEV)
+    kept2 = torch.empty(m, dtype=torch.int32, device=DEV)
+    tg.tg_gate_score(*args, sc2, sq2, ws)
+    tg.tg_topk_select(sc2, args[-1], n_p, k, kept2)
+    torch.cuda.synchronize()
+    assert torch.equal(sc, sc2) and torch.equal(sq, sq2) and torch.equal(kept, kept2)
+    assert np.array_equal(host(kept).astype(np.int64), O.select_kept(host(sc), g["prunable"], k))
+    want = O.gate_scores(g["hidden"], g["norm_w"] if norm_w else None, 1e-6, g["w1"], g["b1"], g["w2"], g["b2"],
+                         g["prunable"])
+    rms = math.sqrt(np.mean(want ** 2))
+    tol = 1e-4 if dtype == "f32" else 1e-2
+    assert np.max(np.abs(host(sc) - want)) <= tol * rms
+
+
 def test_gate_score_select_exact_ties_at_the_threshold():
     # 400 copies of one hidden row; its entries are 0 or +-1/8, so the row's
     # sum of squares is exact in any summation order and the copies score
