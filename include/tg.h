@@ -144,25 +144,35 @@ int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int6
 
 /*
  * tg_gate_score followed by tg_topk_select, with the selection's first radix
- * pass folded into the scoring kernel ([R] §4.1 "Gate module" and "Top-K
+ * digit counted by the scoring kernel ([R] §4.1 "Gate module" and "Top-K
  * selector"): when the tensor cores score and the prompt is long enough for
  * the cluster selector (n > 4096), the scoring kernel's epilogue also counts
  * the order-preserving keys of the prunable scores by their top 11 bits, and
- * the selector reads its first digit off that histogram and resolves the
- * remaining 21 bits in two passes (11 and 10 bits) instead of four of 8.
- * The outputs equal tg_gate_score then tg_topk_select on the same stream:
- * scores, sumsq and the kept indices (bit-exact, ascending).
+ * the selector reads the threshold's first digit off that histogram instead
+ * of building one.  The outputs equal tg_gate_score then tg_topk_select on
+ * the same stream: scores, sumsq and the kept indices (bit-exact, ascending).
  *   arguments        as tg_gate_score and tg_topk_select (m = min(k,
  *                    n_prunable) + n - n_prunable)
  *   ws               device workspace of tg_workspace_bytes(TG_OP_GATE_SELECT,
  *                    n, 0, d_model, h, NULL) bytes, 16-byte aligned
+ *   flags            0, or TG_WS_KEPT_ZERO: the caller promises that ws is
+ *                    zero-filled or exactly as the previous successful call
+ *                    with this flag left it; the call then issues no memset
+ *                    (a memset between two kernels ends their programmatic
+ *                    launch overlap) and leaves the counters it uses at zero
+ *                    again.  After a call that reported an error, clear ws
+ *                    (or pass 0) before the next one.  With 0 the contents of
+ *                    ws on entry do not matter.
+ * Errors: those of tg_gate_score and tg_topk_select; TG_ERR_INVALID_ARG for an
+ * unknown flag.
  */
+#define TG_WS_KEPT_ZERO 1u
 int tg_gate_score_select(const void* hidden, int dtype, int64_t n, int32_t d_model,
-                         const float* norm_w, float norm_eps,
-                         const void* w1, const float* b1, const float* w2, float b2, int32_t h,
-                         const uint8_t* prunable, int64_t n_prunable, int64_t k,
-                         float* scores, float* sumsq, int32_t* kept_idx, int64_t m,
-                         void* ws, size_t ws_bytes, void* stream);
+                         const float* norm_w, float norm_eps, const void* w1, const float* b1,
+                         const float* w2, float b2, int32_t h, const uint8_t* prunable,
+                         int64_t n_prunable, int64_t k, float* scores, float* sumsq,
+                         int32_t* kept_idx, int64_t m, void* ws, size_t ws_bytes, uint32_t flags,
+                         void* stream);
 
 /*
  * Compaction of the kept rows ([R] §4.1 three-stage forward: pruned tokens

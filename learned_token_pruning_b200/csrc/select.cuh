@@ -57,6 +57,7 @@ struct SelectParams {
   int kpt;        // tokens per thread: a power of two with kpt * kSelThreads >= slice
   int cached;     // 1 if the slice's keys and flags are kept in shared memory (kpt <= kSelMaxKpt)
   const uint32_t* hist_top;  // [2048] counts of (key >> 21) over prunable tokens, or null
+  uint32_t* hist_clear;      // hist_top again when it is to be left zeroed for the next call, or null
 };
 
 // dynamic shared memory of k_topk_select
@@ -306,6 +307,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_topk_select(SelectParams p) 
     dst[rank * 2 + 1] = s_ncand;
   }
   cluster.sync();  // (A) counts and candidates published; the first-digit counts read
+  // every rank has read the gate's histogram: leave it zeroed for the next call
+  if (rank == 0 && p.hist_clear)
+    for (int b = tid; b < (1 << kSelTopBits); b += kSelThreads) p.hist_clear[b] = 0u;
 
   uint32_t np_sum = 0, ncand = 0;
   bool over = false;

@@ -464,9 +464,10 @@ static int launch_gather_rmsnorm(const LayerGather& g, int dtype, void* hidden_k
 static int gate_score_impl(const void* hidden, int dtype, int64_t n, int32_t d_model, const float* norm_w,
                            float norm_eps, const void* w1, const float* b1, const float* w2, float b2, int32_t h,
                            const uint8_t* prunable, float* scores, float* sumsq, void* ws, size_t ws_bytes,
-                           bool with_hist, void* stream);
+                           bool with_hist, void* stream, bool ws_clean = false);
 static int topk_select_impl(const float* scores, const uint8_t* prunable, int64_t n, int64_t n_prunable, int64_t k,
-                            int32_t* kept_idx, int64_t m, const uint32_t* hist_top, void* stream);
+                            int32_t* kept_idx, int64_t m, const uint32_t* hist_top, void* stream,
+                            uint32_t* hist_clear = nullptr);
 
 extern "C" {
 
@@ -698,7 +699,7 @@ int tg_gate_score(const void* hidden, int dtype, int64_t n, int32_t d_model, con
 static int gate_score_impl(const void* hidden, int dtype, int64_t n, int32_t d_model, const float* norm_w,
                            float norm_eps, const void* w1, const float* b1, const float* w2, float b2, int32_t h,
                            const uint8_t* prunable, float* scores, float* sumsq, void* ws, size_t ws_bytes,
-                           bool with_hist, void* stream) {
+                           bool with_hist, void* stream, bool ws_clean) {
   if (!hidden || !w1 || !w2 || !prunable || !scores || !sumsq) return fail(TG_ERR_INVALID_ARG, "null pointer");
   if (n <= 0 || d_model <= 0 || h <= 0) return fail(TG_ERR_INVALID_ARG, "n, d_model and h must be positive");
   if (n >= (int64_t(1) << 31)) return fail(TG_ERR_UNSUPPORTED, "n must be < 2^31");
@@ -712,8 +713,13 @@ static int gate_score_impl(const void* hidden, int dtype, int64_t n, int32_t d_m
     uint8_t* counter_at = static_cast<uint8_t*>(ws) + gate_partials_bytes(n);
     uint32_t* counter = reinterpret_cast<uint32_t*>(counter_at);
     uint32_t* key_hist = with_hist ? reinterpret_cast<uint32_t*>(counter_at + 256) : nullptr;
-    cudaError_t e = cudaMemsetAsync(counter, 0, with_hist ? 256 + kGateHistBytes : sizeof(uint32_t), st);
-    if (e != cudaSuccess) return fail(TG_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+    // (ws_clean: the counter and histogram are zero already, as the previous
+    // call left them: the last CTA resets the counter, the selector clears
+    // the histogram after reading it)
+    if (!ws_clean) {
+      cudaError_t e = cudaMemsetAsync(counter, 0, with_hist ? 256 + kGateHistBytes : sizeof(uint32_t), st);
+      if (e != cudaSuccess) return fail(TG_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+    }
     const void* w1_eff = w1;
     if (norm_w) {
       // RMSNorm(h) * w_n feeds W1, so (h * w_n) W1^T = h (W1 diag(w_n))^T: fold the weight into W1
@@ -771,7 +777,8 @@ int tg_topk_select(const float* scores, const uint8_t* prunable, int64_t n, int6
 // tg_topk_select; with hist_top (device [2048] counts of order_key >> 21 over
 // the prunable tokens) the cluster selector starts from that histogram.
 static int topk_select_impl(const float* scores, const uint8_t* prunable, int64_t n, int64_t n_prunable, int64_t k,
-                            int32_t* kept_idx, int64_t m, const uint32_t* hist_top, void* stream) {
+                            int32_t* kept_idx, int64_t m, const uint32_t* hist_top, void* stream,
+                            uint32_t* hist_clear) {
   if (!scores || !prunable || (!kept_idx && m > 0)) return fail(TG_ERR_INVALID_ARG, "null pointer");
   if (n <= 0 || n_prunable < 0 || n_prunable > n) return fail(TG_ERR_INVALID_ARG, "bad n / n_prunable");
   if (k < 0) return fail(TG_ERR_INVALID_ARG, "k must be >= 0");
@@ -825,6 +832,7 @@ static int topk_select_impl(const float* scores, const uint8_t* prunable, int64_
   p.kpt = kpt;
   p.cached = kpt <= tg::kSelMaxKpt ? 1 : 0;
   p.hist_top = hist_top;
+  p.hist_clear = hist_top ? hist_clear : nullptr;
   const size_t smem = tg::select_smem_bytes(kpt, p.cached);
   int rc = set_smem(tg::k_topk_select, smem);
   if (rc) return rc;
@@ -852,7 +860,9 @@ extern "C" {
 int tg_gate_score_select(const void* hidden, int dtype, int64_t n, int32_t d_model, const float* norm_w,
                          float norm_eps, const void* w1, const float* b1, const float* w2, float b2, int32_t h,
                          const uint8_t* prunable, int64_t n_prunable, int64_t k, float* scores, float* sumsq,
-                         int32_t* kept_idx, int64_t m, void* ws, size_t ws_bytes, void* stream) {
+                         int32_t* kept_idx, int64_t m, void* ws, size_t ws_bytes, uint32_t flags, void* stream) {
+  if (flags & ~uint32_t(TG_WS_KEPT_ZERO)) return fail(TG_ERR_INVALID_ARG, "unknown flags");
+  const bool ws_clean = (flags & TG_WS_KEPT_ZERO) != 0;
   if (!scores || !prunable || (!kept_idx && m > 0)) return fail(TG_ERR_INVALID_ARG, "null pointer");
   if (n <= 0 || n_prunable < 0 || n_prunable > n) return fail(TG_ERR_INVALID_ARG, "bad n / n_prunable");
   if (k < 0) return fail(TG_ERR_INVALID_ARG, "k must be >= 0");
@@ -865,12 +875,12 @@ int tg_gate_score_select(const void* hidden, int dtype, int64_t n, int32_t d_mod
   // the selector's first-digit histogram rides with the gate kernel when the
   // tensor cores score and the cluster selector runs (longer prompts)
   const bool with_hist = n > tg::kSelSmallBest && gate_uses_tc(hidden, dtype, d_model, w1, h);
-  const uint32_t* hist =
-      with_hist ? reinterpret_cast<const uint32_t*>(static_cast<uint8_t*>(ws) + gate_partials_bytes(n) + 256) : nullptr;
+  uint32_t* hist =
+      with_hist ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + gate_partials_bytes(n) + 256) : nullptr;
   int rc = gate_score_impl(hidden, dtype, n, d_model, norm_w, norm_eps, w1, b1, w2, b2, h, prunable, scores, sumsq,
-                           ws, ws_bytes, with_hist, stream);
+                           ws, ws_bytes, with_hist, stream, ws_clean);
   if (rc) return rc;
-  return topk_select_impl(scores, prunable, n, n_prunable, k, kept_idx, m, hist, stream);
+  return topk_select_impl(scores, prunable, n, n_prunable, k, kept_idx, m, hist, stream, ws_clean ? hist : nullptr);
 }
 
 }  // extern "C"

@@ -46,9 +46,11 @@ class GatedPrefillStep:
         self.b2 = float(gate["b2"])
         self.scores = torch.empty(w.n, dtype=torch.float32, device=dev)
         self.sumsq = torch.empty(1, dtype=torch.float32, device=dev)
-        # the fused gate + select workspace also serves tg_gate_score alone
         gws = tg.tg_workspace_bytes(tg.TG_OP_GATE_SELECT, n=w.n, d_model=w.d_model, h=w.gate_hidden)
-        self.ws_gate = torch.empty(max(gws, 16), dtype=torch.uint8, device=dev)
+        self.ws_gate = torch.empty(max(gws, 16), dtype=torch.uint8, device=dev)  # tg_gate_score alone
+        # the fused call's own workspace, zero-filled once: each call leaves its
+        # counters at zero again, so no memset precedes the gate kernel
+        self.ws_gate_sel = torch.zeros(max(gws, 16), dtype=torch.uint8, device=dev)
         self.m = min(w.k, self.n_prunable) + (w.n - self.n_prunable)
         self.kept = torch.empty(self.m, dtype=torch.int32, device=dev)
         self.hidden_kept = torch.empty(self.m, w.d_model, dtype=dt, device=dev)
@@ -76,7 +78,7 @@ class GatedPrefillStep:
         folded into the scoring kernel."""
         tg.tg_gate_score_select(self.hidden, self.norm_w, self.norm_eps, self.w1, self.b1, self.w2, self.b2,
                                 self.prunable, self.n_prunable, self.w.k, self.scores, self.sumsq, self.kept,
-                                self.ws_gate, stream)
+                                self.ws_gate_sel, stream, flags=tg.TG_WS_KEPT_ZERO)
 
     def gather(self, stream=None):
         tg.tg_gather(self.hidden, self.kept, self.scores, self.sumsq, self.n_prunable, self.eps_s, self.hidden_kept,
@@ -244,7 +246,8 @@ class PrunedPrefillStack:
         self.pos_all = torch.arange(w.n, dtype=torch.int32, device=dev)
         self.scores = torch.empty(w.n, dtype=torch.float32, device=dev)
         self.sumsq = torch.empty(1, dtype=torch.float32, device=dev)
-        self.ws_gate = torch.empty(max(tg.tg_workspace_bytes(tg.TG_OP_GATE_SELECT, n=w.n, d_model=w.d_model,
+        # zero-filled once: each fused call leaves its counters at zero again
+        self.ws_gate = torch.zeros(max(tg.tg_workspace_bytes(tg.TG_OP_GATE_SELECT, n=w.n, d_model=w.d_model,
                                                              h=gate["w1"].shape[0]), 16), dtype=torch.uint8,
                                    device=dev)
         self.kept = torch.empty(self.m, dtype=torch.int32, device=dev)
@@ -287,7 +290,7 @@ class PrunedPrefillStack:
         g = self.gate
         tg.tg_gate_score_select(self.h, self.gate_norm_w, self.norm_eps, g["w1"], g["b1"], g["w2"], g["b2"],
                                 self.prunable, self.n_prunable, self.w.k, self.scores, self.sumsq, self.kept,
-                                self.ws_gate)
+                                self.ws_gate, flags=tg.TG_WS_KEPT_ZERO)
 
     def gather_mlp(self):
         """Gather the kept rows of the residual into self.hk and run layer L's

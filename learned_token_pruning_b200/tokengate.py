@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(HERE, "libtokengate.so")
 
 TG_F32, TG_BF16 = 0, 1
 TG_OP_GATE_SCORE, TG_OP_LAYER, TG_OP_ATTENTION, TG_OP_DECODE, TG_OP_ATTENTION_BWD, TG_OP_GATE_SELECT = 0, 1, 2, 3, 4, 5
+TG_WS_KEPT_ZERO = 1
 TG_LAYER_ATTENTION, TG_LAYER_MLP, TG_LAYER_FULL = 1, 2, 3
 STATUS = {0: "TG_OK", 1: "TG_ERR_INVALID_ARG", 2: "TG_ERR_SHAPE", 3: "TG_ERR_ALIGN", 4: "TG_ERR_UNSUPPORTED",
           5: "TG_ERR_WORKSPACE", 6: "TG_ERR_CUDA", 7: "TG_ERR_DEVICE_TIMEOUT", 8: "TG_ERR_DEVICE_CHECK"}
@@ -69,7 +70,7 @@ SIGNATURES = {
     "tg_gate_score_noalloc": (_INT, [_P, _INT, _I64, _I32, _P, _F, _P, _P, _P, _F, _I32, _P, _P, _P, _P]),
     "tg_gate_score_noalloc_scratch_bytes": (_SZ, []),
     "tg_gate_score_select": (_INT, [_P, _INT, _I64, _I32, _P, _F, _P, _P, _P, _F, _I32, _P, _I64, _I64, _P, _P, _P,
-                                     _I64, _P, _SZ, _P]),
+                                     _I64, _P, _SZ, ctypes.c_uint32, _P]),
     "tg_debug_set_flag_wait": (_INT, [ctypes.c_uint64, ctypes.c_uint32]),
     "tg_gather_rmsnorm": (_INT, [_P, _INT, _I64, _I32, _P, _I64, _P, _P, _I64, _F, _P, _F, _P, _P, _P, _P, _P, _P]),
     "tg_layer_attention_block": (_INT, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerShape), _P, _P, _P, _P,
@@ -167,14 +168,15 @@ def tg_gate_score_noalloc(hidden, norm_w, norm_eps, w1, b1, w2, b2, prunable, sc
 
 
 def tg_gate_score_select(hidden, norm_w, norm_eps, w1, b1, w2, b2, prunable, n_prunable: int, k: int, scores, sumsq,
-                         kept_idx, ws, stream=None):
-    """tg_gate_score then tg_topk_select, the selector's first radix pass folded into the scoring kernel."""
+                         kept_idx, ws, stream=None, flags: int = 0):
+    """tg_gate_score then tg_topk_select, the selector's first radix digit counted by the scoring kernel.
+    flags=TG_WS_KEPT_ZERO: ws is zero-filled or as the previous such call left it (no memset is issued)."""
     n, d = hidden.shape
     h = w1.shape[0]
     rc = lib().tg_gate_score_select(_ptr(hidden), _dtype(hidden), n, d, _ptr(norm_w), float(norm_eps), _ptr(w1),
                                     _ptr(b1), _ptr(w2), float(b2), h, _ptr(prunable), int(n_prunable), int(k),
                                     _ptr(scores), _ptr(sumsq), _ptr(kept_idx), kept_idx.numel(), _ptr(ws),
-                                    ws.numel() * ws.element_size(), _stream(stream))
+                                    ws.numel() * ws.element_size(), int(flags), _stream(stream))
     _check("tg_gate_score_select", rc)
 
 

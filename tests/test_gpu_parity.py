@@ -332,6 +332,36 @@ def test_gate_score_select_other_gate_paths(dtype, dm, h, norm_w):
     assert np.max(np.abs(host(sc) - want)) <= tol * rms
 
 
+def test_gate_score_select_kept_zero_workspace_across_calls():
+    # TG_WS_KEPT_ZERO: no memset; each call must leave the gate's counter and
+    # the selector's histogram at zero, so calls on alternating inputs through
+    # one zero-filled workspace equal calls without the flag
+    n, dm, h, k = 20000, 512, 256, 3000
+    cases = [_gate_case(n, dm, h, "bf16", seed=s) for s in (41, 42)]
+    n_p = int(cases[0][1]["prunable"].sum())
+    m = min(k, n_p) + n - n_p
+    nbytes = tg.tg_workspace_bytes(tg.TG_OP_GATE_SELECT, n=n, d_model=dm, h=h)
+    ws_kept = torch.zeros(nbytes, dtype=torch.uint8, device=DEV)
+    ws_plain = torch.full((nbytes,), 0xA5, dtype=torch.uint8, device=DEV)   # contents do not matter without the flag
+    part = (((n + 127) // 128) * 4 + 255) // 256 * 256     # the counter slot, then the histogram
+    for rep in range(4):
+        w, g = cases[rep % 2]
+        args = [d(g["hidden"], torch.bfloat16), None, 1e-6, d(g["w1"], torch.bfloat16), d(g["b1"]), d(g["w2"]),
+                float(g["b2"]), d(g["prunable"], torch.uint8), n_p, k]
+        out = []
+        for ws, flags in ((ws_kept, tg.TG_WS_KEPT_ZERO), (ws_plain, 0)):
+            sc, sq = torch.empty(n, device=DEV), torch.empty(1, device=DEV)
+            kept = torch.empty(m, dtype=torch.int32, device=DEV)
+            tg.tg_gate_score_select(*args, sc, sq, kept, ws, flags=flags)
+            out.append((sc, sq, kept))
+        torch.cuda.synchronize()
+        assert torch.equal(out[0][0], out[1][0]) and torch.equal(out[0][1], out[1][1])
+        assert torch.equal(out[0][2], out[1][2])
+        assert int(ws_kept[part:part + 256 + 8192].count_nonzero()) == 0
+    with pytest.raises(tg.TokenGateError):
+        tg.tg_gate_score_select(*args, sc, sq, kept, ws_kept, flags=2)
+
+
 def test_gate_score_select_exact_ties_at_the_threshold():
     # 400 copies of one hidden row; its entries are 0 or +-1/8, so the row's
     # sum of squares is exact in any summation order and the copies score
