@@ -281,4 +281,290 @@ __global__ void __launch_bounds__(kDecThreads) k_decode_attn(DecodeParams p) {
   if (threadIdx.x == 0) p.counters[g] = 0u;  // ready for the next call
 }
 
+
+// ---------------------------------------------------------------------------
+// bf16 cache: the same computation with the cache rows streamed through
+// shared memory by TMA, so the bytes in flight no longer depend on registers
+// or on the phase the warps are in.  CTA (g, j) takes KV head g and a chunk of
+// rows (one wave: about one CTA per SM over all KV heads).  Warp 8 loads
+// 64-row tiles of K and V (128-byte swizzled boxes of 64 head dimensions)
+// into a ring of 128 KB; warps 0-7 take each tile in three steps:
+//   logits: four lanes per key, lane qq holding 16-byte chunks qq, qq + 4, ...
+//     of the key row (the swizzle spreads a warp's eight keys over all banks);
+//   online softmax per head (warp u for head u): tile maximum, running
+//     maximum M and sum l, p = 2^(x - M), rescale factor 2^(M_old - M);
+//   P V: thread (key slice, head, 16-byte group of dimensions) rescales its
+//     accumulators and adds the slice's rows of the tile.
+// The slices are added in slice order at the end, and (M, l, O) of the chunk
+// go to the same workspace layout and chunk-order merge as above.
+constexpr int kDtRows = 64;        // cache rows per tile
+constexpr int kDtThreads = 288;    // 8 compute warps + 1 producer warp
+constexpr int kDtCompute = 256;
+constexpr int kDtRingBytes = 128 * 1024;
+
+template <int D>
+struct DecTmaCfg {
+  static constexpr int kBoxes = D / 64;                      // 64-dimension boxes per row
+  static constexpr int kBoxBytes = kDtRows * 128;
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;      // K or V tile
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kStages = kDtRingBytes / kStageBytes;  // 4 (D = 128) or 8 (D = 64)
+  static constexpr size_t kFloats = static_cast<size_t>(kDecMaxGroup) * D      // s_q
+                                    + 2 * kDecMaxGroup * kDtRows               // s_x, two tiles
+                                    + 24                                       // s_alpha, s_stat
+                                    + kDtCompute * 8                           // s_pv
+                                    + 2 * kDecMaxGroup * kDecMaxChunks;        // merge
+  static constexpr size_t kSmem = 1024 + kDtRingBytes + kFloats * 4 + 2 * kStages * 8;
+};
+
+template <int D, int G>
+__global__ void __launch_bounds__(kDtThreads, 1)
+    k_decode_tma(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, DecodeParams p) {
+  using Cfg = DecTmaCfg<D>;
+  constexpr int R = kDtRows, S = Cfg::kStages;
+  extern __shared__ uint8_t dec_smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dec_smem_raw) + 1023) & ~uintptr_t(1023));
+  float* s_q = reinterpret_cast<float*>(ring + kDtRingBytes);  // [G][D] query rows scaled by a_h
+  float* s_x = s_q + kDecMaxGroup * D;                         // [2][G][R] logits, then p, per tile parity
+  float* s_alpha = s_x + 2 * kDecMaxGroup * R;                 // [8] rescale factor of the tile per head
+  float* s_stat = s_alpha + 8;                                 // [G][2] (M, l) of the chunk
+  float* s_pv = s_alpha + 24;                                  // [slices][G * D]
+  float* s_merge = s_pv + kDtCompute * 8;                      // [2][G][nchunks]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_merge + 2 * kDecMaxGroup * kDecMaxChunks);
+  uint64_t* empty = full + S;
+  __shared__ int s_last;
+  // a compute warp's wait ran out: set before a tile's first named barrier,
+  // read by every compute warp after it, so all of them leave together
+  __shared__ volatile int s_stop;
+  __shared__ volatile int s_pstop;  // the producer's wait ran out
+
+  const int g = blockIdx.x / p.nchunks, j = blockIdx.x % p.nchunks;
+  const int c0 = j * p.chunk, c1 = min(c0 + p.chunk, p.length), nk = c1 - c0;
+  const int ntiles = (nk + R - 1) / R;
+  const int h0 = g * G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kDtCompute / 32);
+    }
+    s_stop = 0;
+    s_pstop = 0;
+    fence_mbar_init();
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+  const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(p.q);
+  for (int i = threadIdx.x; i < G * D; i += kDtThreads) {
+    const int u = i / D, d = i % D;
+    s_q[i] = __bfloat162float(qp[static_cast<int64_t>(h0 + u) * D + d]) * (p.temp[h0 + u] * p.ratio_scale_log2);
+  }
+  __syncthreads();
+
+  // P V mapping: PAIRS (head, 16-byte dimension group) per slice, SL slices
+  constexpr int DG = D / 8;
+  constexpr int PAIRS = G * DG;
+  constexpr int SL = kDtCompute / PAIRS;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+  const int pair = threadIdx.x % PAIRS, slice = threadIdx.x / PAIRS;
+  const int pu = pair / DG, pdg = pair % DG;
+  float m_run = -INFINITY, l_run = 0.0f;  // warp u < G: head u's running maximum and sum
+
+  if (warp == kDtCompute / 32) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      for (int t = 0; t < ntiles; ++t) {
+        const int st = t % S;
+        if (!mbar_wait(&empty[st], ((t / S) & 1) ^ 1, kErrWaitAttention)) {
+          s_pstop = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[st], Cfg::kStageBytes);
+        uint8_t* dst = ring + st * Cfg::kStageBytes;
+        const int y = c0 + t * R;  // rows past the cache read as zeros
+#pragma unroll
+        for (int b = 0; b < Cfg::kBoxes; ++b) {
+          tma_load_2d(dst + b * Cfg::kBoxBytes, &tmK, &full[st], g * D + b * 64, y);
+          tma_load_2d(dst + Cfg::kTileBytes + b * Cfg::kBoxBytes, &tmV, &full[st], g * D + b * 64, y);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ compute warps
+    constexpr int NM = D / 32;  // 16-byte chunks per lane per key
+    constexpr bool kQReg = G * D / 4 <= 64;
+    const int kr = threadIdx.x >> 2, qq = threadIdx.x & 3;
+    float qreg[kQReg ? G : 1][kQReg ? D / 4 : 1];
+    if constexpr (kQReg) {
+#pragma unroll
+      for (int u = 0; u < G; ++u)
+#pragma unroll
+        for (int m = 0; m < NM; ++m)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) qreg[u][m * 8 + e] = s_q[u * D + 8 * (qq + 4 * m) + e];
+    }
+    float gbias[G];
+#pragma unroll
+    for (int u = 0; u < G; ++u) gbias[u] = p.gain[h0 + u] * kLog2e;
+    float b_next = (p.bias && kr < nk) ? __ldg(p.bias + c0 + kr) : 0.0f;
+    for (int t = 0; t < ntiles; ++t) {
+      const int st = t % S;
+      const bool ok = warp_wait(&full[st], (t / S) & 1, kErrWaitAttention);
+      if (!ok && lane == 0) s_stop = 1;
+      const uint8_t* kt = ring + st * Cfg::kStageBytes;
+      float* sx = s_x + (t & 1) * (kDecMaxGroup * R);
+      // logits
+      float xa[G];
+#pragma unroll
+      for (int u = 0; u < G; ++u) xa[u] = 0.0f;
+#pragma unroll
+      for (int m = 0; m < NM; ++m) {
+        const int c = qq + 4 * m;
+        const uint4 w = *reinterpret_cast<const uint4*>(kt + (c >> 3) * Cfg::kBoxBytes + kr * 128 +
+                                                        (((c & 7) ^ (kr & 7)) << 4));
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float k0 = bf16_lo(ww[h]), k1 = bf16_hi(ww[h]);
+#pragma unroll
+          for (int u = 0; u < G; ++u) {
+            const float q0 = kQReg ? qreg[kQReg ? u : 0][kQReg ? m * 8 + 2 * h : 0] : s_q[u * D + 8 * c + 2 * h];
+            const float q1 = kQReg ? qreg[kQReg ? u : 0][kQReg ? m * 8 + 2 * h + 1 : 0] : s_q[u * D + 8 * c + 2 * h + 1];
+            xa[u] = fmaf(q0, k0, xa[u]);
+            xa[u] = fmaf(q1, k1, xa[u]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < G; ++u) {
+        xa[u] += __shfl_xor_sync(0xffffffffu, xa[u], 1);
+        xa[u] += __shfl_xor_sync(0xffffffffu, xa[u], 2);
+      }
+      const int key = t * R + kr;
+      if (qq == 0) {
+#pragma unroll
+        for (int u = 0; u < G; ++u) sx[u * R + kr] = key < nk ? fmaf(gbias[u], b_next, xa[u]) : -INFINITY;
+      }
+      {
+        const int kn = key + R;
+        b_next = (p.bias && kn < nk) ? __ldg(p.bias + c0 + kn) : 0.0f;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (s_stop) break;
+      // online softmax, warp u for head u
+      if (warp < G) {
+        const float x0 = sx[warp * R + lane], x1 = sx[warp * R + lane + 32];
+        float tm = fmaxf(x0, x1);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, o));
+        const float m_new = fmaxf(m_run, tm);
+        const float alpha = exp2f(m_run - m_new);
+        const float p0 = exp2f(x0 - m_new), p1 = exp2f(x1 - m_new);
+        sx[warp * R + lane] = p0;
+        sx[warp * R + lane + 32] = p1;
+        float ts = p0 + p1;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) ts += __shfl_xor_sync(0xffffffffu, ts, o);
+        l_run = fmaf(l_run, alpha, ts);
+        m_run = m_new;
+        if (lane == 0) s_alpha[warp] = alpha;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      // P V
+      if (slice < SL) {
+        const float a = s_alpha[pu];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] *= a;
+        const uint8_t* vt = kt + Cfg::kTileBytes + (pdg >> 3) * Cfg::kBoxBytes;
+        const float* pp = sx + pu * R;
+#pragma unroll 4
+        for (int c = slice; c < R; c += SL) {
+          const float pc = pp[c];
+          const uint4 w = *reinterpret_cast<const uint4*>(vt + c * 128 + (((pdg & 7) ^ (c & 7)) << 4));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            acc[2 * h] = fmaf(pc, bf16_lo(ww[h]), acc[2 * h]);
+            acc[2 * h + 1] = fmaf(pc, bf16_hi(ww[h]), acc[2 * h + 1]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);  // this warp's reads of the stage are done
+    }
+    if (warp < G && lane == 0) {
+      s_stat[2 * warp] = m_run;
+      s_stat[2 * warp + 1] = l_run;
+    }
+    if (!s_stop && slice < SL) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s_pv[slice * (G * D) + pu * D + pdg * 8 + e] = acc[e];
+    }
+  }
+  __syncthreads();
+  if (s_stop || s_pstop) return;  // a wait ran out (recorded in the error word)
+
+  // the chunk's unnormalised O (slices added in slice order), M and l
+  float* part = p.part + (static_cast<size_t>(g) * p.nchunks + j) * G * (D + 2);
+  for (int i = threadIdx.x; i < G * D; i += kDtThreads) {
+    float o = 0.0f;
+    for (int sl = 0; sl < SL; ++sl) o += s_pv[sl * (G * D) + i];
+    part[(i / D) * (D + 2) + (i % D)] = o;
+  }
+  if (threadIdx.x < G) {
+    part[threadIdx.x * (D + 2) + D] = s_stat[2 * threadIdx.x];
+    part[threadIdx.x * (D + 2) + D + 1] = s_stat[2 * threadIdx.x + 1];
+  }
+
+  // the last CTA of KV head g merges the chunks in chunk order
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(&p.counters[g], 1u) == static_cast<unsigned>(p.nchunks - 1) ? 1 : 0;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int nc = p.nchunks;
+  const float* gpart = p.part + static_cast<size_t>(g) * nc * G * (D + 2);
+  float* s_m = s_merge;                 // [G][nc] chunk maxima, then weights
+  float* s_l = s_merge + G * nc;        // [G][nc] chunk sums
+  for (int i = threadIdx.x; i < G * nc; i += kDtThreads) {
+    const int u = i / nc, jj = i % nc;
+    s_m[i] = __ldcg(gpart + (jj * G + u) * (D + 2) + D);
+    s_l[i] = __ldcg(gpart + (jj * G + u) * (D + 2) + D + 1);
+  }
+  __syncthreads();
+  if (threadIdx.x < G) {
+    const int u = threadIdx.x;
+    float mx = -INFINITY;
+    for (int jj = 0; jj < nc; ++jj) mx = fmaxf(mx, s_m[u * nc + jj]);
+    float l = 0.0f;
+    for (int jj = 0; jj < nc; ++jj) {
+      const float w = exp2f(s_m[u * nc + jj] - mx);
+      s_m[u * nc + jj] = w;
+      l = fmaf(s_l[u * nc + jj], w, l);
+    }
+    const float inv = 1.0f / l;
+    for (int jj = 0; jj < nc; ++jj) s_m[u * nc + jj] *= inv;
+    if (p.lse) p.lse[h0 + u] = (mx + log2f(l)) * kLn2;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < G * D; i += kDtThreads) {
+    const int u = i / D, d = i % D;
+    const float* po = gpart + u * (D + 2) + d;
+    float o0 = 0.0f, o1 = 0.0f;
+    int jj = 0;
+    for (; jj + 2 <= nc; jj += 2) {
+      o0 = fmaf(s_m[u * nc + jj], __ldcg(po + jj * G * (D + 2)), o0);
+      o1 = fmaf(s_m[u * nc + jj + 1], __ldcg(po + (jj + 1) * G * (D + 2)), o1);
+    }
+    for (; jj < nc; ++jj) o0 = fmaf(s_m[u * nc + jj], __ldcg(po + jj * G * (D + 2)), o0);
+    static_cast<__nv_bfloat16*>(p.out)[static_cast<int64_t>(h0 + u) * D + d] = from_f32<__nv_bfloat16>(o0 + o1);
+  }
+  if (threadIdx.x == 0) p.counters[g] = 0u;  // ready for the next call
+}
+
 }  // namespace tg

@@ -426,6 +426,36 @@ int launch_decode(int group, dim3 grid, cudaStream_t st, const tg::DecodeParams&
   }
 }
 
+// TMA decode kernel: tensor maps of the KV head columns of K and V (64-row
+// boxes of 64 dimensions, 128-byte swizzle; rows past the cache read as zeros)
+template <int D, int G>
+int launch_decode_tma_g(dim3 grid, cudaStream_t st, const tg::DecodeParams& p) {
+  using Cfg = tg::DecTmaCfg<D>;
+  CUtensorMap tk, tv;
+  const uint64_t cols = static_cast<uint64_t>(p.hkv) * D;
+  int rc = make_map(&tk, p.k, cols, static_cast<uint64_t>(p.length), static_cast<uint64_t>(p.ldk) * 2, tg::kDtRows);
+  if (rc) return rc;
+  rc = make_map(&tv, p.v, cols, static_cast<uint64_t>(p.length), static_cast<uint64_t>(p.ldv) * 2, tg::kDtRows);
+  if (rc) return rc;
+  rc = set_smem(tg::k_decode_tma<D, G>, Cfg::kSmem);
+  if (rc) return rc;
+  return launch_pdl("k_decode_tma", tg::k_decode_tma<D, G>, grid, dim3(tg::kDtThreads), Cfg::kSmem, st, tk, tv, p);
+}
+
+template <int D>
+int launch_decode_tma(int group, dim3 grid, cudaStream_t st, const tg::DecodeParams& p) {
+  switch (group) {
+    case 1: return launch_decode_tma_g<D, 1>(grid, st, p);
+    case 2: return launch_decode_tma_g<D, 2>(grid, st, p);
+    case 3: return launch_decode_tma_g<D, 3>(grid, st, p);
+    case 4: return launch_decode_tma_g<D, 4>(grid, st, p);
+    case 5: return launch_decode_tma_g<D, 5>(grid, st, p);
+    case 6: return launch_decode_tma_g<D, 6>(grid, st, p);
+    case 7: return launch_decode_tma_g<D, 7>(grid, st, p);
+    default: return launch_decode_tma_g<D, 8>(grid, st, p);
+  }
+}
+
 // the layer's own buffers (normed rows, qkv, attention output, MLP activation)
 static size_t layer_buffers_bytes(int64_t m, const tg_layer_shape* S) {
   const int es = dtype_size(S->dtype);
@@ -639,19 +669,44 @@ struct DecodePlan {
   size_t part_bytes = 0, bytes = 0;
 };
 
-DecodePlan decode_plan(int64_t length, int hkv, int group, int head_dim) {
+// TG_DECODE_SIMT=1 in the environment sends bf16 decode to the CUDA-core
+// kernel too (read at every call, so a test can run both kernels in one process).
+bool force_simt_decode() {
+  const char* e = std::getenv("TG_DECODE_SIMT");
+  return e && e[0] == '1';
+}
+
+// tma: the bf16 kernel that streams the cache through shared memory (one CTA
+// per SM over all KV heads, chunks of whole 64-row tiles); otherwise about two
+// CTAs per SM with chunks of at most kDecMaxChunk rows.  Both keep at most
+// kDecMaxChunks chunks per KV head.
+DecodePlan decode_plan(int64_t length, int hkv, int group, int head_dim, bool tma) {
   DecodePlan pl;
   if (length <= 0 || hkv <= 0 || group <= 0) return pl;
   const int64_t sms = sm_count();
-  int64_t chunk = (length * hkv + 2 * sms - 1) / (2 * sms);
-  chunk = std::max<int64_t>(chunk, (length + tg::kDecMaxChunks - 1) / tg::kDecMaxChunks);  // <= 256 chunks
-  chunk = std::min<int64_t>(std::max<int64_t>((chunk + 63) / 64 * 64, 64), tg::kDecMaxChunk);
+  int64_t chunk;
+  if (tma) {
+    const int64_t per_head = std::max<int64_t>(1, std::min<int64_t>(sms / hkv, tg::kDecMaxChunks));
+    chunk = (length + per_head - 1) / per_head;
+    chunk = std::max<int64_t>((chunk + tg::kDtRows - 1) / tg::kDtRows * tg::kDtRows, tg::kDtRows);
+  } else {
+    chunk = (length * hkv + 2 * sms - 1) / (2 * sms);
+    chunk = std::max<int64_t>(chunk, (length + tg::kDecMaxChunks - 1) / tg::kDecMaxChunks);  // <= 256 chunks
+    chunk = std::min<int64_t>(std::max<int64_t>((chunk + 63) / 64 * 64, 64), tg::kDecMaxChunk);
+  }
   pl.chunk = static_cast<int>(chunk);
   pl.nchunks = static_cast<int>((length + chunk - 1) / chunk);
   auto al = [](size_t b) { return (b + 255) / 256 * 256; };
   pl.part_bytes = al(static_cast<size_t>(hkv) * pl.nchunks * group * (head_dim + 2) * sizeof(float));
   pl.bytes = pl.part_bytes + al(static_cast<size_t>(hkv) * sizeof(uint32_t));
   return pl;
+}
+
+// workspace that covers either decode kernel (the query does not see the
+// pointers that decide between them)
+size_t decode_ws_bytes(int64_t length, int hkv, int group, int head_dim) {
+  return std::max(decode_plan(length, hkv, group, head_dim, false).bytes,
+                  decode_plan(length, hkv, group, head_dim, true).bytes);
 }
 
 size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t h, const tg_layer_shape* shape) {
@@ -677,7 +732,7 @@ size_t tg_workspace_bytes(int op, int64_t n, int64_t m, int32_t d_model, int32_t
   }
   if (op == TG_OP_DECODE) {
     if (!shape || m <= 0 || shape->hkv <= 0 || shape->hq % shape->hkv) return 0;
-    return decode_plan(m, shape->hkv, shape->hq / shape->hkv, shape->head_dim).bytes;
+    return decode_ws_bytes(m, shape->hkv, shape->hq / shape->hkv, shape->head_dim);
   }
   return 0;
 }
@@ -1274,8 +1329,12 @@ int tg_gated_decode_attention(const void* q, const void* k, int64_t ldk, const v
   if (!aligned16(k) || !aligned16(v) || (ldk * es) % 16 || (ldv * es) % 16)
     return fail(TG_ERR_ALIGN, "cache rows need 16-byte alignment");
   const int group = hq / hkv;
-  const DecodePlan pl = decode_plan(length, hkv, group, head_dim);
-  if (!ws || ws_bytes < pl.bytes) return fail(TG_ERR_WORKSPACE, "decode attention needs %zu workspace bytes", pl.bytes);
+  // bf16 caches stream through shared memory by TMA (16-byte aligned rows,
+  // checked above); fp32 caches take the CUDA-core kernel
+  const bool tma = dtype == TG_BF16 && !force_simt_decode();
+  const DecodePlan pl = decode_plan(length, hkv, group, head_dim, tma);
+  const size_t need = decode_ws_bytes(length, hkv, group, head_dim);
+  if (!ws || ws_bytes < need) return fail(TG_ERR_WORKSPACE, "decode attention needs %zu workspace bytes", need);
   if (!aligned16(ws)) return fail(TG_ERR_ALIGN, "workspace must be 16-byte aligned");
   cudaStream_t st = as_stream(stream);
   tg::DecodeParams p{};
@@ -1301,6 +1360,7 @@ int tg_gated_decode_attention(const void* q, const void* k, int64_t ldk, const v
   if (cudaMemsetAsync(p.counters, 0, pl.bytes - pl.part_bytes, st) != cudaSuccess)
     return fail(TG_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(cudaGetLastError()));
   const dim3 grid(static_cast<unsigned>(hkv * pl.nchunks));
+  if (tma) return head_dim == 128 ? launch_decode_tma<128>(group, grid, st, p) : launch_decode_tma<64>(group, grid, st, p);
   if (dtype == TG_BF16)
     return head_dim == 128 ? launch_decode<__nv_bfloat16, 128>(group, grid, st, p)
                            : launch_decode<__nv_bfloat16, 64>(group, grid, st, p);

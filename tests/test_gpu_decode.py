@@ -1,8 +1,10 @@
-"""Decode over the gated KV cache: the CUDA kernel against the CPU oracle on the
+"""Decode over the gated KV cache: the CUDA kernels against the CPU oracle on the
 same seeded inputs, element by element (small caches, ragged chunk tails, every
-GQA group size the kernel takes, both head dims and dtypes), and at the cache
+GQA group size the kernels take, both head dims and dtypes), and at the cache
 lengths of the workloads (kept rows of the 16K and 128K prompts plus generated
-tokens) on every output."""
+tokens) on every output.  bf16 caches take the kernel that streams the cache
+through shared memory by TMA; TG_DECODE_SIMT=1 sends them to the CUDA-core
+kernel that fp32 caches use, and a few cases run that way too."""
 import math
 
 import numpy as np
@@ -131,3 +133,27 @@ def test_decode_continues_prefill_attention():
 def test_decode_maximum_cache_length():
     # 262144 rows: 256 chunks of 1024 keys per KV head, the most one call takes
     _check(262144, 4, 2, 128, "bf16", seed=3)
+
+
+@pytest.fixture
+def cuda_core_decode(monkeypatch):
+    monkeypatch.setenv("TG_DECODE_SIMT", "1")
+
+
+@pytest.mark.parametrize("length,hq,hkv,dh", [(1, 16, 8, 128), (1000, 16, 8, 64), (2065, 16, 8, 128),
+                                              (517, 8, 1, 128), (517, 6, 2, 128)])
+def test_decode_bf16_through_the_cuda_core_kernel(cuda_core_decode, length, hq, hkv, dh):
+    _check(length, hq, hkv, dh, "bf16", seed=length + hq)
+
+
+@pytest.mark.parametrize("length", [64 * 18 * 3 + 1, 64 * 18 * 3, 64 * 18 * 3 - 1])
+def test_decode_chunk_boundaries_of_the_streaming_kernel(length):
+    # 8 KV heads share the SMs: chunks of whole 64-row tiles, a last chunk of
+    # one row, exactly full, and one row short
+    _check(length, 16, 8, 128, "bf16", seed=length)
+
+
+@pytest.mark.parametrize("hq,hkv,dh", [(8, 1, 64), (12, 2, 64), (14, 2, 128), (10, 2, 128)])
+def test_decode_group_sizes_streaming_kernel(hq, hkv, dh):
+    # query rows from registers (group x head_dim / 4 <= 64) or from shared memory, slices that leave threads idle
+    _check(1333, hq, hkv, dh, "bf16", seed=hq * 100 + hkv * 10 + dh)
