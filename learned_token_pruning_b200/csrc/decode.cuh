@@ -287,16 +287,20 @@ __global__ void __launch_bounds__(kDecThreads) k_decode_attn(DecodeParams p) {
 // shared memory by TMA, so the bytes in flight no longer depend on registers
 // or on the phase the warps are in.  CTA (g, j) takes KV head g and a chunk of
 // rows (one wave: about one CTA per SM over all KV heads).  Warp 8 loads
-// 64-row tiles of K and V (128-byte swizzled boxes of 64 head dimensions)
-// into a ring of 128 KB; warps 0-7 take each tile in three steps:
+// 64-row tiles of K and V (128-byte swizzled boxes of 64 head dimensions),
+// and the tile's 64 key biases, into a ring of 128 KB (a bias read by the
+// threads themselves one tile ahead would wait on DRAM under the full load);
+// warps 0-7 take each tile in two steps:
 //   logits: four lanes per key, lane qq holding 16-byte chunks qq, qq + 4, ...
 //     of the key row (the swizzle spreads a warp's eight keys over all banks);
-//   online softmax per head (warp u for head u): tile maximum, running
-//     maximum M and sum l, p = 2^(x - M), rescale factor 2^(M_old - M);
-//   P V: thread (key slice, head, 16-byte group of dimensions) rescales its
-//     accumulators and adds the slice's rows of the tile.
-// The slices are added in slice order at the end, and (M, l, O) of the chunk
-// go to the same workspace layout and chunk-order merge as above.
+//   P V: thread (key slice, head, 16-byte group of dimensions) keeps an
+//     online softmax over its own slice of the keys (running maximum M and
+//     sum l; the tile's slice maximum, the rescale factor 2^(M_old - M),
+//     p = 2^(x - M)) and adds p v of the slice's rows of the tile.
+// One named barrier per tile (logits before P V).  At the end the slices are
+// rescaled to the largest slice maximum and added in slice order, and (M, l,
+// O) of the chunk go to the same workspace layout and chunk-order merge as
+// above.
 constexpr int kDtRows = 64;        // cache rows per tile
 constexpr int kDtThreads = 288;    // 8 compute warps + 1 producer warp
 constexpr int kDtCompute = 256;
@@ -311,31 +315,35 @@ struct DecTmaCfg {
   static constexpr int kStages = kDtRingBytes / kStageBytes;  // 4 (D = 128) or 8 (D = 64)
   static constexpr size_t kFloats = static_cast<size_t>(kDecMaxGroup) * D      // s_q
                                     + 2 * kDecMaxGroup * kDtRows               // s_x, two tiles
-                                    + 24                                       // s_alpha, s_stat
+                                    + 64                                       // s_ml
                                     + kDtCompute * 8                           // s_pv
                                     + 2 * kDecMaxGroup * kDecMaxChunks;        // merge
-  static constexpr size_t kSmem = 1024 + kDtRingBytes + kFloats * 4 + 2 * kStages * 8;
+  static constexpr int kBiasBytes = kDtRows * 4;            // the tile's key biases
+  static constexpr size_t kSmem = 1024 + kDtRingBytes + kStages * kBiasBytes + kFloats * 4 + 2 * kStages * 8;
 };
 
 template <int D, int G>
 __global__ void __launch_bounds__(kDtThreads, 1)
-    k_decode_tma(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, DecodeParams p) {
+    k_decode_tma(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmBias, DecodeParams p) {
   using Cfg = DecTmaCfg<D>;
   constexpr int R = kDtRows, S = Cfg::kStages;
   extern __shared__ uint8_t dec_smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dec_smem_raw) + 1023) & ~uintptr_t(1023));
-  float* s_q = reinterpret_cast<float*>(ring + kDtRingBytes);  // [G][D] query rows scaled by a_h
+  float* s_bias = reinterpret_cast<float*>(ring + kDtRingBytes);  // [S][R] key biases per stage
+  float* s_q = s_bias + S * R;                                 // [G][D] query rows scaled by a_h
   float* s_x = s_q + kDecMaxGroup * D;                         // [2][G][R] logits, then p, per tile parity
-  float* s_alpha = s_x + 2 * kDecMaxGroup * R;                 // [8] rescale factor of the tile per head
-  float* s_stat = s_alpha + 8;                                 // [G][2] (M, l) of the chunk
-  float* s_pv = s_alpha + 24;                                  // [slices][G * D]
+  float* s_ml = s_x + 2 * kDecMaxGroup * R;                    // [slices][G][2] (M, l) per slice and head
+  float* s_pv = s_ml + 64;                                     // [slices][G * D]
   float* s_merge = s_pv + kDtCompute * 8;                      // [2][G][nchunks]
   uint64_t* full = reinterpret_cast<uint64_t*>(s_merge + 2 * kDecMaxGroup * kDecMaxChunks);
   uint64_t* empty = full + S;
   __shared__ int s_last;
-  // a compute warp's wait ran out: set before a tile's first named barrier,
-  // read by every compute warp after it, so all of them leave together
-  __shared__ volatile int s_stop;
+  // [tile parity] a compute warp's wait for tile t ran out: set before tile
+  // t's named barrier and read by every compute warp right after it (a set
+  // for tile t + 2 needs every warp past tile t + 1's barrier), so all of
+  // them leave at the same tile
+  __shared__ volatile int s_stop[2];
   __shared__ volatile int s_pstop;  // the producer's wait ran out
 
   const int g = blockIdx.x / p.nchunks, j = blockIdx.x % p.nchunks;
@@ -348,7 +356,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], kDtCompute / 32);
     }
-    s_stop = 0;
+    s_stop[0] = s_stop[1] = 0;
     s_pstop = 0;
     fence_mbar_init();
   }
@@ -365,27 +373,29 @@ __global__ void __launch_bounds__(kDtThreads, 1)
   constexpr int DG = D / 8;
   constexpr int PAIRS = G * DG;
   constexpr int SL = kDtCompute / PAIRS;
-  float acc[8];
+  float2 acc[4];  // dimensions 8 pdg + 2h, 8 pdg + 2h + 1
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+  for (int h = 0; h < 4; ++h) acc[h] = make_float2(0.0f, 0.0f);
   const int pair = threadIdx.x % PAIRS, slice = threadIdx.x / PAIRS;
   const int pu = pair / DG, pdg = pair % DG;
-  float m_run = -INFINITY, l_run = 0.0f;  // warp u < G: head u's running maximum and sum
+  float m_run = -INFINITY, l_run = 0.0f;  // running maximum and sum of this thread's key slice and head
 
   if (warp == kDtCompute / 32) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
+      if (p.bias) prefetch_tmap(&tmBias);
       for (int t = 0; t < ntiles; ++t) {
         const int st = t % S;
         if (!mbar_wait(&empty[st], ((t / S) & 1) ^ 1, kErrWaitAttention)) {
           s_pstop = 1;
           break;
         }
-        mbar_arrive_expect_tx(&full[st], Cfg::kStageBytes);
+        mbar_arrive_expect_tx(&full[st], Cfg::kStageBytes + (p.bias ? Cfg::kBiasBytes : 0));
         uint8_t* dst = ring + st * Cfg::kStageBytes;
         const int y = c0 + t * R;  // rows past the cache read as zeros
+        if (p.bias) tma_load_1d(s_bias + st * R, &tmBias, &full[st], y);
 #pragma unroll
         for (int b = 0; b < Cfg::kBoxes; ++b) {
           tma_load_2d(dst + b * Cfg::kBoxBytes, &tmK, &full[st], g * D + b * 64, y);
@@ -410,17 +420,16 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     float gbias[G];
 #pragma unroll
     for (int u = 0; u < G; ++u) gbias[u] = p.gain[h0 + u] * kLog2e;
-    float b_next = (p.bias && kr < nk) ? __ldg(p.bias + c0 + kr) : 0.0f;
     for (int t = 0; t < ntiles; ++t) {
       const int st = t % S;
       const bool ok = warp_wait(&full[st], (t / S) & 1, kErrWaitAttention);
-      if (!ok && lane == 0) s_stop = 1;
+      if (!ok && lane == 0) s_stop[t & 1] = 1;
       const uint8_t* kt = ring + st * Cfg::kStageBytes;
       float* sx = s_x + (t & 1) * (kDecMaxGroup * R);
-      // logits
-      float xa[G];
+      // logits (per head an fp32 pair of partial sums over even and odd dimensions)
+      float2 xa2[G];
 #pragma unroll
-      for (int u = 0; u < G; ++u) xa[u] = 0.0f;
+      for (int u = 0; u < G; ++u) xa2[u] = make_float2(0.0f, 0.0f);
 #pragma unroll
       for (int m = 0; m < NM; ++m) {
         const int c = qq + 4 * m;
@@ -434,90 +443,92 @@ __global__ void __launch_bounds__(kDtThreads, 1)
           for (int u = 0; u < G; ++u) {
             const float q0 = kQReg ? qreg[kQReg ? u : 0][kQReg ? m * 8 + 2 * h : 0] : s_q[u * D + 8 * c + 2 * h];
             const float q1 = kQReg ? qreg[kQReg ? u : 0][kQReg ? m * 8 + 2 * h + 1 : 0] : s_q[u * D + 8 * c + 2 * h + 1];
-            xa[u] = fmaf(q0, k0, xa[u]);
-            xa[u] = fmaf(q1, k1, xa[u]);
+            xa2[u] = ffma2(make_float2(q0, q1), make_float2(k0, k1), xa2[u]);
           }
         }
       }
 #pragma unroll
+      float xa[G];
+#pragma unroll
       for (int u = 0; u < G; ++u) {
+        xa[u] = xa2[u].x + xa2[u].y;
         xa[u] += __shfl_xor_sync(0xffffffffu, xa[u], 1);
         xa[u] += __shfl_xor_sync(0xffffffffu, xa[u], 2);
       }
       const int key = t * R + kr;
       if (qq == 0) {
+        const float b = p.bias ? s_bias[st * R + kr] : 0.0f;
 #pragma unroll
-        for (int u = 0; u < G; ++u) sx[u * R + kr] = key < nk ? fmaf(gbias[u], b_next, xa[u]) : -INFINITY;
-      }
-      {
-        const int kn = key + R;
-        b_next = (p.bias && kn < nk) ? __ldg(p.bias + c0 + kn) : 0.0f;
+        for (int u = 0; u < G; ++u) sx[u * R + kr] = key < nk ? fmaf(gbias[u], b, xa[u]) : -INFINITY;
       }
       asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (s_stop) break;
-      // online softmax, warp u for head u
-      if (warp < G) {
-        const float x0 = sx[warp * R + lane], x1 = sx[warp * R + lane + 32];
-        float tm = fmaxf(x0, x1);
-#pragma unroll
-        for (int o = 16; o; o >>= 1) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, o));
-        const float m_new = fmaxf(m_run, tm);
-        const float alpha = exp2f(m_run - m_new);
-        const float p0 = exp2f(x0 - m_new), p1 = exp2f(x1 - m_new);
-        sx[warp * R + lane] = p0;
-        sx[warp * R + lane + 32] = p1;
-        float ts = p0 + p1;
-#pragma unroll
-        for (int o = 16; o; o >>= 1) ts += __shfl_xor_sync(0xffffffffu, ts, o);
-        l_run = fmaf(l_run, alpha, ts);
-        m_run = m_new;
-        if (lane == 0) s_alpha[warp] = alpha;
-      }
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      // P V
+      if (s_stop[t & 1]) break;
+      // P V, each thread with its own online softmax over its slice of the
+      // keys (running maximum M and sum l per slice and head, no barrier
+      // between the two steps; the slices are merged like chunks at the end)
       if (slice < SL) {
-        const float a = s_alpha[pu];
+        const float* xx = sx + pu * R;
+        float tmax = -INFINITY;
+#pragma unroll 4
+        for (int c = slice; c < R; c += SL) tmax = fmaxf(tmax, xx[c]);
+        const float m_new = fmaxf(m_run, tmax);
+        const float m_use = m_new == -INFINITY ? 0.0f : m_new;  // no key of the slice yet: all weights 0
+        const float alpha = ex2_approx(m_run - m_use);
+        m_run = m_new;
+        l_run *= alpha;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] *= a;
+        for (int h = 0; h < 4; ++h) {
+          acc[h].x *= alpha;
+          acc[h].y *= alpha;
+        }
         const uint8_t* vt = kt + Cfg::kTileBytes + (pdg >> 3) * Cfg::kBoxBytes;
-        const float* pp = sx + pu * R;
 #pragma unroll 4
         for (int c = slice; c < R; c += SL) {
-          const float pc = pp[c];
+          const float pc = ex2_approx(xx[c] - m_use);
+          l_run += pc;
           const uint4 w = *reinterpret_cast<const uint4*>(vt + c * 128 + (((pdg & 7) ^ (c & 7)) << 4));
           const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            acc[2 * h] = fmaf(pc, bf16_lo(ww[h]), acc[2 * h]);
-            acc[2 * h + 1] = fmaf(pc, bf16_hi(ww[h]), acc[2 * h + 1]);
-          }
+          for (int h = 0; h < 4; ++h) acc[h] = ffma2(make_float2(pc, pc), make_float2(bf16_lo(ww[h]), bf16_hi(ww[h])), acc[h]);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);  // this warp's reads of the stage are done
     }
-    if (warp < G && lane == 0) {
-      s_stat[2 * warp] = m_run;
-      s_stat[2 * warp + 1] = l_run;
-    }
-    if (!s_stop && slice < SL) {
+    if (!(s_stop[0] | s_stop[1]) && slice < SL) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) s_pv[slice * (G * D) + pu * D + pdg * 8 + e] = acc[e];
+      for (int h = 0; h < 4; ++h) {
+        s_pv[slice * (G * D) + pu * D + pdg * 8 + 2 * h] = acc[h].x;
+        s_pv[slice * (G * D) + pu * D + pdg * 8 + 2 * h + 1] = acc[h].y;
+      }
+      if (pdg == 0) {
+        s_ml[(slice * G + pu) * 2] = m_run;
+        s_ml[(slice * G + pu) * 2 + 1] = l_run;
+      }
     }
   }
   __syncthreads();
-  if (s_stop || s_pstop) return;  // a wait ran out (recorded in the error word)
+  if (s_stop[0] | s_stop[1] | s_pstop) return;  // a wait ran out (recorded in the error word)
 
-  // the chunk's unnormalised O (slices added in slice order), M and l
+  // the chunk's (M, l, unnormalised O): the slices rescaled to the largest
+  // slice maximum and added in slice order
   float* part = p.part + (static_cast<size_t>(g) * p.nchunks + j) * G * (D + 2);
   for (int i = threadIdx.x; i < G * D; i += kDtThreads) {
+    const int u = i / D;
+    float mx = -INFINITY;
+    for (int sl = 0; sl < SL; ++sl) mx = fmaxf(mx, s_ml[(sl * G + u) * 2]);
     float o = 0.0f;
-    for (int sl = 0; sl < SL; ++sl) o += s_pv[sl * (G * D) + i];
-    part[(i / D) * (D + 2) + (i % D)] = o;
+    for (int sl = 0; sl < SL; ++sl) o = fmaf(exp2f(s_ml[(sl * G + u) * 2] - mx), s_pv[sl * (G * D) + i], o);
+    part[u * (D + 2) + (i % D)] = o;
   }
   if (threadIdx.x < G) {
-    part[threadIdx.x * (D + 2) + D] = s_stat[2 * threadIdx.x];
-    part[threadIdx.x * (D + 2) + D + 1] = s_stat[2 * threadIdx.x + 1];
+    const int u = threadIdx.x;
+    float mx = -INFINITY;
+    for (int sl = 0; sl < SL; ++sl) mx = fmaxf(mx, s_ml[(sl * G + u) * 2]);
+    float l = 0.0f;
+    for (int sl = 0; sl < SL; ++sl) l = fmaf(exp2f(s_ml[(sl * G + u) * 2] - mx), s_ml[(sl * G + u) * 2 + 1], l);
+    part[u * (D + 2) + D] = mx;
+    part[u * (D + 2) + D + 1] = l;
   }
 
   // the last CTA of KV head g merges the chunks in chunk order

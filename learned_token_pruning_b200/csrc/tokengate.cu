@@ -431,15 +431,21 @@ int launch_decode(int group, dim3 grid, cudaStream_t st, const tg::DecodeParams&
 template <int D, int G>
 int launch_decode_tma_g(dim3 grid, cudaStream_t st, const tg::DecodeParams& p) {
   using Cfg = tg::DecTmaCfg<D>;
-  CUtensorMap tk, tv;
+  CUtensorMap tk, tv, tb;
   const uint64_t cols = static_cast<uint64_t>(p.hkv) * D;
   int rc = make_map(&tk, p.k, cols, static_cast<uint64_t>(p.length), static_cast<uint64_t>(p.ldk) * 2, tg::kDtRows);
   if (rc) return rc;
   rc = make_map(&tv, p.v, cols, static_cast<uint64_t>(p.length), static_cast<uint64_t>(p.ldv) * 2, tg::kDtRows);
   if (rc) return rc;
+  if (p.bias) {
+    rc = make_map_1d_f32(&tb, p.bias, static_cast<uint64_t>(p.length), tg::kDtRows);
+    if (rc) return rc;
+  } else {
+    tb = tk;  // not read
+  }
   rc = set_smem(tg::k_decode_tma<D, G>, Cfg::kSmem);
   if (rc) return rc;
-  return launch_pdl("k_decode_tma", tg::k_decode_tma<D, G>, grid, dim3(tg::kDtThreads), Cfg::kSmem, st, tk, tv, p);
+  return launch_pdl("k_decode_tma", tg::k_decode_tma<D, G>, grid, dim3(tg::kDtThreads), Cfg::kSmem, st, tk, tv, tb, p);
 }
 
 template <int D>
@@ -1330,8 +1336,9 @@ int tg_gated_decode_attention(const void* q, const void* k, int64_t ldk, const v
     return fail(TG_ERR_ALIGN, "cache rows need 16-byte alignment");
   const int group = hq / hkv;
   // bf16 caches stream through shared memory by TMA (16-byte aligned rows,
-  // checked above); fp32 caches take the CUDA-core kernel
-  const bool tma = dtype == TG_BF16 && !force_simt_decode();
+  // checked above, and a 16-byte aligned bias vector); fp32 caches take the
+  // CUDA-core kernel
+  const bool tma = dtype == TG_BF16 && (!bias || aligned16(bias)) && !force_simt_decode();
   const DecodePlan pl = decode_plan(length, hkv, group, head_dim, tma);
   const size_t need = decode_ws_bytes(length, hkv, group, head_dim);
   if (!ws || ws_bytes < need) return fail(TG_ERR_WORKSPACE, "decode attention needs %zu workspace bytes", need);

@@ -157,3 +157,21 @@ def test_decode_chunk_boundaries_of_the_streaming_kernel(length):
 def test_decode_group_sizes_streaming_kernel(hq, hkv, dh):
     # query rows from registers (group x head_dim / 4 <= 64) or from shared memory, slices that leave threads idle
     _check(1333, hq, hkv, dh, "bf16", seed=hq * 100 + hkv * 10 + dh)
+
+
+def test_decode_unaligned_bias_vector_takes_the_cuda_core_kernel():
+    # a bias vector that starts off a 16-byte boundary cannot be a TMA source
+    length, hq, hkv, dh = 700, 16, 8, 128
+    q, k, v, bias, gain, temp = _case(length, hq, hkv, dh, "bf16", seed=11)
+    dt = torch.bfloat16
+    kd = torch.from_numpy(k.reshape(length, -1)).to(DEV, dt)
+    vd = torch.from_numpy(v.reshape(length, -1)).to(DEV, dt)
+    bd = torch.from_numpy(np.concatenate([[0.0], bias]).astype(np.float32)).to(DEV)[1:]
+    assert bd.data_ptr() % 16 != 0
+    out = torch.empty(hq, dh, dtype=dt, device=DEV)
+    ws = torch.empty(tg.decode_workspace_bytes(length, hq, hkv, dh), dtype=torch.uint8, device=DEV)
+    tg.tg_gated_decode_attention(torch.from_numpy(q).to(DEV, dt), kd, vd, dh, bd, torch.from_numpy(gain).to(DEV),
+                                 torch.from_numpy(temp).to(DEV), 0.8, 1.0 / math.sqrt(dh), out, ws)
+    assert tg.tg_check_device_error() == 0
+    want = O.gated_decode_attention(q, k, v, bias, gain, temp, 0.8, 1.0 / math.sqrt(dh))
+    np.testing.assert_allclose(out.float().cpu().numpy(), want, **ATTN_BF16)
