@@ -800,7 +800,7 @@ def ncu_backward_case():
 def ncu_decode_case():
     """One decode-attention call on a 131137-row cache (16/8 heads x 128, bf16;
     the unpruned 128K-token prompt's cache) after a warm-up call, each after an
-    L2 flush, for profiler captures of k_decode_attn."""
+    L2 flush, for profiler captures of the decode kernel (k_decode_tma for a bf16 cache)."""
     import torch
     from learned_token_pruning_b200 import tokengate as tg
     dev, hq, hkv, dh, length = "cuda", 16, 8, 128, 131137
