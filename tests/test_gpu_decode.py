@@ -175,3 +175,44 @@ def test_decode_unaligned_bias_vector_takes_the_cuda_core_kernel():
     assert tg.tg_check_device_error() == 0
     want = O.gated_decode_attention(q, k, v, bias, gain, temp, 0.8, 1.0 / math.sqrt(dh))
     np.testing.assert_allclose(out.float().cpu().numpy(), want, **ATTN_BF16)
+
+
+def test_decode_graph_replays_and_a_reused_workspace():
+    # the chunk-merge counters: a workspace of garbage, one call replayed from a
+    # CUDA graph, and eager calls of another cache length on the same workspace
+    # in between
+    hq, hkv, dh = 16, 8, 128
+    dt = torch.bfloat16
+    ws = torch.full((tg.decode_workspace_bytes(5000, hq, hkv, dh),), 0xA5, dtype=torch.uint8, device=DEV)
+    cases = []
+    for length, seed in ((5000, 21), (1300, 22)):
+        q, k, v, bias, gain, temp = _case(length, hq, hkv, dh, "bf16", seed=seed)
+        want = O.gated_decode_attention(q, k, v, bias, gain, temp, 0.85, 1.0 / math.sqrt(dh))
+        dev = [torch.from_numpy(q).to(DEV, dt), torch.from_numpy(k.reshape(length, -1)).to(DEV, dt),
+               torch.from_numpy(v.reshape(length, -1)).to(DEV, dt), torch.from_numpy(bias).to(DEV),
+               torch.from_numpy(gain).to(DEV), torch.from_numpy(temp).to(DEV),
+               torch.empty(hq, dh, dtype=dt, device=DEV)]
+        cases.append((dev, want))
+
+    def call(dev):
+        q, k, v, b, g, t, out = dev
+        tg.tg_gated_decode_attention(q, k, v, dh, b, g, t, 0.85, 1.0 / math.sqrt(dh), out, ws)
+
+    def check(i):
+        torch.cuda.synchronize()
+        assert tg.tg_check_device_error() == 0
+        np.testing.assert_allclose(cases[i][0][-1].float().cpu().numpy(), cases[i][1], **ATTN_BF16)
+
+    call(cases[0][0])
+    check(0)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call(cases[0][0])
+    for _ in range(3):
+        cases[0][0][-1].zero_()
+        graph.replay()
+        check(0)
+        cases[1][0][-1].zero_()
+        call(cases[1][0])
+        check(1)
+    del graph
