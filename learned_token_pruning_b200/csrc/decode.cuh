@@ -24,6 +24,7 @@
 //      result does not depend on which CTA finished when.
 #pragma once
 
+#include "attn_tc.cuh"  // packed fp32 pairs (f2_*) and ex2_approx, shared with the attention kernel
 #include "common.cuh"
 #include "simt.cuh"
 
@@ -301,6 +302,14 @@ __global__ void __launch_bounds__(kDecThreads) k_decode_attn(DecodeParams p) {
 // rescaled to the largest slice maximum and added in slice order, and (M, l,
 // O) of the chunk go to the same workspace layout and chunk-order merge as
 // above.
+// Two fp32 fused multiply-adds in one instruction on float2 values
+// (fma.rn.f32x2): per lane exactly fmaf(a, b, c).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  f2_unpack(f2_fma(f2_pack(a.x, a.y), f2_pack(b.x, b.y), f2_pack(c.x, c.y)), d.x, d.y);
+  return d;
+}
+
 constexpr int kDtRows = 64;        // cache rows per tile
 constexpr int kDtThreads = 288;    // 8 compute warps + 1 producer warp
 constexpr int kDtCompute = 256;
@@ -447,7 +456,6 @@ __global__ void __launch_bounds__(kDtThreads, 1)
           }
         }
       }
-#pragma unroll
       float xa[G];
 #pragma unroll
       for (int u = 0; u < G; ++u) {
