@@ -307,7 +307,11 @@ int tg_gated_attention_backward(const void* q, int64_t ldq, const void* k, int64
  *          merged in it).  The size depends on the SM count of the device.
  * head_dim in {64, 128}; hq % hkv == 0 with at most 8 query heads per KV head;
  * length <= 262144; cache rows 16-byte aligned.  bf16 or fp32 inputs, fp32 arithmetic on the
- * CUDA cores (the step reads the cache once and is bound by memory).
+ * CUDA cores (the step reads the cache once and is bound by memory).  A bf16
+ * cache with bias NULL or 16-byte aligned streams through shared memory by TMA
+ * (one CTA per SM over all KV heads); fp32 caches, an unaligned bias, or
+ * TG_DECODE_SIMT=1 in the environment take the split-KV kernel that loads the
+ * cache into registers.  Both give the same results within fp32 rounding.
  */
 int tg_gated_decode_attention(const void* q, const void* k, int64_t ldk, const void* v, int64_t ldv,
                               int dtype, int64_t length, int32_t hq, int32_t hkv, int32_t head_dim,
