@@ -399,6 +399,14 @@ def run_gpu(args, w):
         for n_, k_ in ((16384, 2000), (131072, 8192)):
             r = stack_ttft(n_, k_, [13, 1], 3, dev, stream)
             ttft[f"stack28_n{n_}"] = r
+        # decode over the gated cache (off the step; the same records as --decode)
+        dec = {}
+        try:
+            run_decode(args, emit=lambda r: dec.__setitem__(
+                r["workload"], {k: r[k] for k in ("cache_rows", "us", "gbs", "frac_hbm")}))
+        except Exception as e:  # the line still prints; the record says why decode is missing
+            dec = {"error": f"{type(e).__name__}: {e}"}
+        extras["decode"] = dec
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         sec, desc, threads = oracle_step_seconds(w)
@@ -634,11 +642,12 @@ def ncu_case():
     print("ncu case done")
 
 
-def run_decode(args):
+def run_decode(args, emit=None):
     """Decode over the gated KV cache (one new token's attention over the kept
     rows plus the tokens generated so far), per call, L2 flushed before each:
-    one JSON line per cache length with the time, the cache bytes read per call
-    and their rate against the measured HBM copy bandwidth."""
+    one record per cache length with the time, the cache bytes read per call
+    and their rate against the measured HBM copy bandwidth, printed as a JSON
+    line or, with `emit`, passed to it."""
     import torch
     from learned_token_pruning_b200 import tokengate as tg
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -696,10 +705,14 @@ def run_decode(args):
         tg.tg_check_device_error()
         nbytes = 2 * length * hkv * dh * 2 + length * 4
         gbs = nbytes / (ms * 1e-3) / 1e9
-        print(json.dumps({"mode": "decode", "workload": name, "cache_rows": length, "kept_prompt_rows": m_kept,
-                          "prompt_tokens": n_prompt, "step": t, "us": ms * 1e3, "cache_bytes": nbytes, "gbs": gbs,
-                          "frac_hbm": gbs / peaks["hbm_gbs"], "peak_source": peaks["source"],
-                          "l2": "flushed before every call", "ratio": ratio}), flush=True)
+        rec = {"mode": "decode", "workload": name, "cache_rows": length, "kept_prompt_rows": m_kept,
+               "prompt_tokens": n_prompt, "step": t, "us": ms * 1e3, "cache_bytes": nbytes, "gbs": gbs,
+               "frac_hbm": gbs / peaks["hbm_gbs"], "peak_source": peaks["source"],
+               "l2": "flushed before every call", "ratio": ratio}
+        if emit is None:
+            print(json.dumps(rec), flush=True)
+        else:
+            emit(rec)
 
 
 def run_backward(args):
