@@ -399,14 +399,7 @@ def run_gpu(args, w):
         for n_, k_ in ((16384, 2000), (131072, 8192)):
             r = stack_ttft(n_, k_, [13, 1], 3, dev, stream)
             ttft[f"stack28_n{n_}"] = r
-        # decode over the gated cache (off the step; the same records as --decode)
-        dec = {}
-        try:
-            run_decode(args, emit=lambda r: dec.__setitem__(
-                r["workload"], {k: r[k] for k in ("cache_rows", "us", "gbs", "frac_hbm")}))
-        except Exception as e:  # the line still prints; the record says why decode is missing
-            dec = {"error": f"{type(e).__name__}: {e}"}
-        extras["decode"] = dec
+        extras["decode"] = decode_extras(args)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         sec, desc, threads = oracle_step_seconds(w)
@@ -713,6 +706,19 @@ def run_decode(args, emit=None):
             print(json.dumps(rec), flush=True)
         else:
             emit(rec)
+
+
+def decode_extras(args, run=None):
+    """Decode over the gated cache for the default JSON line (off the step; the
+    same measurement as --decode): per workload its cache rows, time, GB/s and
+    HBM fraction.  A failure there leaves {"error": ...} and the line still prints."""
+    run = run_decode if run is None else run
+    dec = {}
+    try:
+        run(args, emit=lambda r: dec.__setitem__(r["workload"], {k: r[k] for k in ("cache_rows", "us", "gbs", "frac_hbm")}))
+    except Exception as e:
+        dec = {"error": f"{type(e).__name__}: {e}"}
+    return dec
 
 
 def run_backward(args):

@@ -70,3 +70,25 @@ def test_traffic_record_scales_by_rows_and_goes_stale(monkeypatch):
     monkeypatch.setitem(bench.MEASURED_TRAFFIC, "probe", dict(rec, bytes=1000, rows=10, sha256="0" * 64))
     assert bench.measured_traffic("probe", 40) is None
     assert bench.measured_traffic("no such kernel", 40) is None
+
+
+def test_decode_extras_collects_each_workload_and_survives_a_failure():
+    sys.path.insert(0, ROOT)
+    import bench
+    args = types.SimpleNamespace(steps=2, warmup=3)
+
+    def fake_run(a, emit):
+        assert a is args
+        for name, rows, us in (("w_small", 2129, 14.8), ("w_large", 131137, 119.0)):
+            emit({"mode": "decode", "workload": name, "cache_rows": rows, "us": us, "gbs": 1.0e3 / us,
+                  "frac_hbm": 0.5, "ratio": 0.9, "l2": "flushed"})
+
+    dec = bench.decode_extras(args, run=fake_run)
+    assert set(dec) == {"w_small", "w_large"}
+    assert dec["w_large"] == {"cache_rows": 131137, "us": 119.0, "gbs": 1.0e3 / 119.0, "frac_hbm": 0.5}
+
+    def failing_run(a, emit):
+        emit({"workload": "w_small", "cache_rows": 1, "us": 1.0, "gbs": 1.0, "frac_hbm": 0.1})
+        raise RuntimeError("no device")
+
+    assert bench.decode_extras(args, run=failing_run) == {"error": "RuntimeError: no device"}
